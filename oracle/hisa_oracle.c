@@ -1,0 +1,476 @@
+/*
+ * HISA CPU oracle.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product library calls, links or
+ * loads this file; only the tests, the package's smoke check and the bench's
+ * CPU-baseline leg do.  It shares no code, header or table with the CUDA path.
+ *
+ * It computes, slowly and in double precision, what the HISA indexer computes:
+ *
+ *   HISA: Efficient Hierarchical Indexing for Fine-Grained Sparse Attention
+ *   (gptget.net summary, "Methodology"; Chinese summary, "方法详解" / method
+ *   details; arXiv abstract):
+ *     1. split the length-L prefix into contiguous blocks of size B and
+ *        mean-pool each block's keys into one block representative;
+ *     2. score every representative with the original indexer and keep the
+ *        top-m blocks (block-level coarse filter);
+ *     3. score every token of the kept blocks with the original indexer
+ *        (token-level refinement);
+ *     4. keep the final top-k tokens; their indices go to the sparse
+ *        attention operator.
+ *   The flat DSA scan (blog "Hierarchical Indexing Makes Sparse Attention
+ *   Actually Fast", "How Fine-Grained Sparse Attention Works Today") scores
+ *   every prefix token and keeps the top-k.
+ *
+ * The indexer score of a key x for one query row is
+ *     score(q, x) = sum_h w_h * max(0, q_h . x)      over the H indexer heads,
+ * the lightning-indexer form (the pages only call it a lightweight
+ * dot-product scorer).  Readings where the pages are silent:
+ *   - causal: a key at position s is visible to a query at t iff s <= t;
+ *   - the trailing block is pooled over its visible tokens only;
+ *   - the query's own block is always kept and counts inside m;
+ *   - ties go to the lower index (tokens) and the lower block id (blocks);
+ *   - output: the selected indices in ascending order, then -1 padding;
+ *   - e4m3 keys are dequantised as fl32(e4m3 value * scale), the fp32
+ *     product, and used in double from there.
+ *
+ * Parity pins: the tests check this file against exact rational brute force
+ * on tiny inputs, closed-form pooled means, the B = 1 identity, one-hot score
+ * cases and the m >= #blocks == flat-scan identity.
+ *
+ * Rows are independent; they are spread over POSIX threads.  A library sort
+ * (qsort) is the only borrowed step.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+enum { KEY_BF16 = 0, KEY_E4M3 = 1 };
+
+typedef struct {
+    const void* keys;    /* [batch, cap, d] bf16 bits or e4m3 codes */
+    const float* scale;  /* [batch, cap] (e4m3 only) */
+    int dtype, batch, cap, d;
+} cache_t;
+
+/* ---------------------------------------------------------------- values */
+
+static double bf16_value(uint16_t bits) {
+    uint32_t u = (uint32_t)bits << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* OCP e4m3 ("fn"): 1 sign, 4 exponent (bias 7), 3 mantissa bits, no inf. */
+static double e4m3_value(uint8_t c) {
+    int sgn = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m, -9);
+    else v = ldexp(1.0 + m / 8.0, e - 7);
+    return sgn ? -v : v;
+}
+
+/* Key row s of sequence b as the indexer sees it. */
+static void key_row(const cache_t* c, int b, long s, double* x) {
+    size_t base = ((size_t)b * c->cap + (size_t)s) * c->d;
+    if (c->dtype == KEY_BF16) {
+        const uint16_t* k = (const uint16_t*)c->keys + base;
+        for (int e = 0; e < c->d; ++e) x[e] = bf16_value(k[e]);
+    } else {
+        const uint8_t* k = (const uint8_t*)c->keys + base;
+        float sc = c->scale[(size_t)b * c->cap + (size_t)s];
+        for (int e = 0; e < c->d; ++e) {
+            /* one fp32 rounding of the exact product, then double */
+            float v = (float)(e4m3_value(k[e]) * (double)sc);
+            x[e] = (double)v;
+        }
+    }
+}
+
+/* ---------------------------------------------------------- the indexer */
+
+/* q_h . x with four interleaved partial sums (fixed order, double). */
+static double dot(const double* a, const double* x, int d) {
+    double s0 = 0, s1 = 0, s2 = 0, s3 = 0;
+    int e = 0;
+    for (; e + 4 <= d; e += 4) {
+        s0 += a[e] * x[e];
+        s1 += a[e + 1] * x[e + 1];
+        s2 += a[e + 2] * x[e + 2];
+        s3 += a[e + 3] * x[e + 3];
+    }
+    for (; e < d; ++e) s0 += a[e] * x[e];
+    return (s0 + s1) + (s2 + s3);
+}
+
+/* score(q, x) = sum_h w_h * ReLU(q_h . x) */
+static double indexer_score(const double* q, const double* w, int H, int d, const double* x) {
+    double acc = 0.0;
+    for (int h = 0; h < H; ++h) {
+        double z = dot(q + (size_t)h * d, x, d);
+        acc += w[h] * (z > 0.0 ? z : 0.0);
+    }
+    return acc;
+}
+
+/* Step 1: block representative = mean of the block's visible keys
+ * (tokens j*B .. min((j+1)*B, n) - 1). */
+static void pool_block(const cache_t* c, int b, int B, long j, long n, double* mu, double* tmp) {
+    long s0 = j * (long)B, s1 = s0 + B < n ? s0 + B : n;
+    for (int e = 0; e < c->d; ++e) mu[e] = 0.0;
+    for (long s = s0; s < s1; ++s) {
+        key_row(c, b, s, tmp);
+        for (int e = 0; e < c->d; ++e) mu[e] += tmp[e];
+    }
+    for (int e = 0; e < c->d; ++e) mu[e] /= (double)(s1 - s0);
+}
+
+/* ------------------------------------------------------------ selection */
+
+typedef struct { double v; long i; } scored_t;
+
+/* higher value first; equal values: lower index first */
+static int by_value_then_index(const void* pa, const void* pb) {
+    const scored_t* a = (const scored_t*)pa;
+    const scored_t* b = (const scored_t*)pb;
+    if (a->v > b->v) return -1;
+    if (a->v < b->v) return 1;
+    return (a->i > b->i) - (a->i < b->i);
+}
+
+static int by_index(const void* pa, const void* pb) {
+    long a = ((const scored_t*)pa)->i, b = ((const scored_t*)pb)->i;
+    return (a > b) - (a < b);
+}
+
+/* Keep the first k of `items` under (value desc, index asc); write them in
+ * ascending index order into idx/val (padding -1 / NaN up to k). */
+static void keep_top(scored_t* items, long n, int k, int32_t* idx, double* val) {
+    qsort(items, (size_t)n, sizeof(scored_t), by_value_then_index);
+    long kept = n < k ? n : k;
+    qsort(items, (size_t)kept, sizeof(scored_t), by_index);
+    for (long r = 0; r < k; ++r) {
+        idx[r] = r < kept ? (int32_t)items[r].i : -1;
+        if (val) val[r] = r < kept ? items[r].v : NAN;
+    }
+}
+
+/* ------------------------------------------------------------ threading */
+
+typedef void (*row_fn)(void* ctx, int row, void* scratch);
+
+typedef struct {
+    row_fn fn;
+    void* ctx;
+    int n_rows, n_threads, tid;
+    size_t scratch_bytes;
+    int failed;
+} worker_t;
+
+static void* worker_main(void* p) {
+    worker_t* w = (worker_t*)p;
+    void* scratch = malloc(w->scratch_bytes);
+    if (!scratch) { w->failed = 1; return NULL; }
+    for (int r = w->tid; r < w->n_rows; r += w->n_threads) w->fn(w->ctx, r, scratch);
+    free(scratch);
+    return NULL;
+}
+
+static int for_rows(row_fn fn, void* ctx, int n_rows, int n_threads, size_t scratch_bytes) {
+    if (n_threads < 1) n_threads = 1;
+    if (n_threads > n_rows) n_threads = n_rows > 0 ? n_rows : 1;
+    worker_t* ws = (worker_t*)calloc((size_t)n_threads, sizeof(worker_t));
+    pthread_t* th = (pthread_t*)calloc((size_t)n_threads, sizeof(pthread_t));
+    if (!ws || !th) { free(ws); free(th); return 3; }
+    int rc = 0;
+    for (int t = 0; t < n_threads; ++t) {
+        ws[t] = (worker_t){fn, ctx, n_rows, n_threads, t, scratch_bytes, 0};
+        if (pthread_create(&th[t], NULL, worker_main, &ws[t]) != 0) {
+            worker_main(&ws[t]);   /* run inline if a thread cannot start */
+            th[t] = 0;
+        }
+    }
+    for (int t = 0; t < n_threads; ++t) {
+        if (th[t]) pthread_join(th[t], NULL);
+        if (ws[t].failed) rc = 3;
+    }
+    free(ws);
+    free(th);
+    return rc;
+}
+
+/* ---------------------------------------------------------- query rows */
+
+typedef struct {
+    cache_t c;
+    int B;
+    const int32_t* lens;
+    const uint16_t* Q;    /* [n_q, H, d] bf16 */
+    const float* w;       /* [n_q, H] */
+    const int32_t* q_seq;
+    const int32_t* q_pos; /* NULL: last position of the sequence */
+    int n_q, H, m, k, nbmax;
+    /* HISA outputs */
+    int32_t* idx; double* score;
+    int32_t* blocks; int32_t* nblocks; double* block_scores; int64_t* counts;
+    /* refine inputs */
+    const int32_t* in_blocks; const int32_t* in_nblocks; int mm;
+    double* cand_scores;
+    /* flat output */
+    double* all_scores;
+    int bad;
+} job_t;
+
+static long row_position(const job_t* J, int i, int* b_out) {
+    int b = J->q_seq[i];
+    *b_out = b;
+    if (b < 0 || b >= J->c.batch) return -1;
+    long t = J->q_pos ? J->q_pos[i] : (long)J->lens[b] - 1;
+    if (t < 0 || t >= J->lens[b] || J->lens[b] > J->c.cap) return -1;
+    return t;
+}
+
+static void load_query(const job_t* J, int i, double* q, double* w) {
+    const uint16_t* Qi = J->Q + (size_t)i * J->H * J->c.d;
+    for (int x = 0; x < J->H * J->c.d; ++x) q[x] = bf16_value(Qi[x]);
+    for (int h = 0; h < J->H; ++h) w[h] = (double)J->w[(size_t)i * J->H + h];
+}
+
+static size_t row_scratch_bytes(int H, int d, long n_items) {
+    return sizeof(double) * ((size_t)H * d + H + 2 * (size_t)d) + sizeof(scored_t) * (size_t)n_items;
+}
+
+/* Token-level refinement on a given set of blocks (steps 3-4). */
+static void refine_blocks(const job_t* J, int i, int b, long t, const double* q, const double* w,
+                          const int32_t* blk, int nblk, scored_t* items, double* x,
+                          int32_t* idx, double* val, double* cand) {
+    long n = 0;
+    for (int r = 0; r < nblk; ++r) {
+        for (int o = 0; o < J->B; ++o) {
+            long s = (long)blk[r] * J->B + o;
+            double v = NAN;
+            if (blk[r] >= 0 && s <= t) {
+                key_row(&J->c, b, s, x);
+                v = indexer_score(q, w, J->H, J->c.d, x);
+                items[n].v = v;
+                items[n].i = s;
+                ++n;
+            }
+            if (cand) cand[(size_t)r * J->B + o] = v;
+        }
+    }
+    keep_top(items, n, J->k, idx, val);
+}
+
+static void hisa_row(void* ctx, int i, void* scratch) {
+    job_t* J = (job_t*)ctx;
+    int H = J->H, d = J->c.d, B = J->B, b;
+    long t = row_position(J, i, &b);
+    int32_t* idx = J->idx + (size_t)i * J->k;
+    double* val = J->score ? J->score + (size_t)i * J->k : NULL;
+    int32_t* blocks = J->blocks ? J->blocks + (size_t)i * J->m : NULL;
+    if (t < 0) {
+        J->bad = 1;
+        for (int r = 0; r < J->k; ++r) { idx[r] = -1; if (val) val[r] = NAN; }
+        return;
+    }
+    double* q = (double*)scratch;
+    double* w = q + (size_t)H * d;
+    double* mu = w + H;
+    double* x = mu + d;
+    scored_t* items = (scored_t*)(x + d);
+
+    load_query(J, i, q, w);
+    long n_t = t + 1;
+    long nb = (n_t + B - 1) / B;
+
+    /* steps 1-2: pool every visible block, score the representatives */
+    double* S = J->block_scores ? J->block_scores + (size_t)i * J->nbmax : NULL;
+    if (S) for (int j = 0; j < J->nbmax; ++j) S[j] = NAN;
+    for (long j = 0; j < nb; ++j) {
+        pool_block(&J->c, b, B, j, n_t, mu, x);
+        double sj = indexer_score(q, w, H, d, mu);
+        if (S) S[j] = sj;
+        items[j].v = sj;
+        items[j].i = j;
+    }
+    /* keep the own block (nb-1) plus the best m-1 of the others */
+    int32_t chosen[4096];
+    int n_chosen;
+    if (nb <= J->m) {
+        n_chosen = (int)nb;
+        for (int j = 0; j < n_chosen; ++j) chosen[j] = j;
+    } else {
+        qsort(items, (size_t)(nb - 1), sizeof(scored_t), by_value_then_index);
+        n_chosen = J->m;
+        for (int r = 0; r < J->m - 1; ++r) chosen[r] = (int32_t)items[r].i;
+        chosen[J->m - 1] = (int32_t)(nb - 1);
+        /* ascending block order */
+        for (int a = 1; a < n_chosen; ++a)
+            for (int c2 = a; c2 > 0 && chosen[c2 - 1] > chosen[c2]; --c2) {
+                int32_t tmp = chosen[c2]; chosen[c2] = chosen[c2 - 1]; chosen[c2 - 1] = tmp;
+            }
+    }
+    if (blocks) for (int r = 0; r < J->m; ++r) blocks[r] = r < n_chosen ? chosen[r] : -1;
+    if (J->nblocks) J->nblocks[i] = n_chosen;
+    if (J->counts) {
+        J->counts[2 * (size_t)i] = nb;                          /* block scores */
+        J->counts[2 * (size_t)i + 1] = (int64_t)n_chosen * B;   /* token slots */
+    }
+    /* steps 3-4 */
+    refine_blocks(J, i, b, t, q, w, chosen, n_chosen, items, x, idx, val, NULL);
+}
+
+static void refine_row(void* ctx, int i, void* scratch) {
+    job_t* J = (job_t*)ctx;
+    int H = J->H, d = J->c.d, b;
+    long t = row_position(J, i, &b);
+    int32_t* idx = J->idx + (size_t)i * J->k;
+    double* val = J->score ? J->score + (size_t)i * J->k : NULL;
+    double* cand = J->cand_scores ? J->cand_scores + (size_t)i * J->mm * J->B : NULL;
+    int nblk = J->in_nblocks[i];
+    if (t < 0 || nblk < 0 || nblk > J->mm) {
+        J->bad = 1;
+        for (int r = 0; r < J->k; ++r) { idx[r] = -1; if (val) val[r] = NAN; }
+        return;
+    }
+    double* q = (double*)scratch;
+    double* w = q + (size_t)H * d;
+    double* x = w + H + d;
+    scored_t* items = (scored_t*)(x + d);
+    load_query(J, i, q, w);
+    if (cand) for (long s = 0; s < (long)J->mm * J->B; ++s) cand[s] = NAN;
+    refine_blocks(J, i, b, t, q, w, J->in_blocks + (size_t)i * J->mm, nblk, items, x, idx, val, cand);
+}
+
+/* Flat scan: every visible token is a candidate. */
+static void flat_row(void* ctx, int i, void* scratch) {
+    job_t* J = (job_t*)ctx;
+    int H = J->H, d = J->c.d, b;
+    long t = row_position(J, i, &b);
+    int32_t* idx = J->idx + (size_t)i * J->k;
+    double* val = J->score ? J->score + (size_t)i * J->k : NULL;
+    double* all = J->all_scores ? J->all_scores + (size_t)i * J->c.cap : NULL;
+    if (t < 0) {
+        J->bad = 1;
+        for (int r = 0; r < J->k; ++r) { idx[r] = -1; if (val) val[r] = NAN; }
+        return;
+    }
+    double* q = (double*)scratch;
+    double* w = q + (size_t)H * d;
+    double* x = w + H + d;
+    scored_t* items = (scored_t*)(x + d);
+    load_query(J, i, q, w);
+    if (all) for (long s = 0; s < J->c.cap; ++s) all[s] = NAN;
+    for (long s = 0; s <= t; ++s) {
+        key_row(&J->c, b, s, x);
+        items[s].v = indexer_score(q, w, H, d, x);
+        items[s].i = s;
+        if (all) all[s] = items[s].v;
+    }
+    keep_top(items, t + 1, J->k, idx, val);
+}
+
+static int check_cache(const void* keys, const float* scale, int dtype, int batch, int cap, int d) {
+    if (!keys || batch < 1 || cap < 1 || d < 1) return 1;
+    if (dtype != KEY_BF16 && dtype != KEY_E4M3) return 1;
+    if (dtype == KEY_E4M3 && !scale) return 1;
+    return 0;
+}
+
+/* ------------------------------------------------------------- exports */
+
+/* Cache-level pooling: pooled[b, j, :] = mean of keys j*B .. min((j+1)B, len[b]) - 1;
+ * blocks at or past len[b] are left untouched. */
+int hisa_oracle_pool(const void* keys, const float* scale, int dtype, int batch, int cap, int d,
+                     int B, const int32_t* lens, double* pooled) {
+    if (check_cache(keys, scale, dtype, batch, cap, d) || B < 1 || !lens || !pooled) return 1;
+    cache_t c = {keys, scale, dtype, batch, cap, d};
+    long nblk = (cap + B - 1) / B;
+    double* tmp = (double*)malloc(sizeof(double) * (size_t)d);
+    if (!tmp) return 3;
+    for (int b = 0; b < batch; ++b) {
+        long n = lens[b];
+        if (n < 0 || n > cap) { free(tmp); return 1; }
+        for (long j = 0; j * B < n; ++j)
+            pool_block(&c, b, B, j, n, pooled + ((size_t)b * nblk + (size_t)j) * d, tmp);
+    }
+    free(tmp);
+    return 0;
+}
+
+int hisa_oracle_select(const void* keys, const float* scale, int dtype, int batch, int cap, int d,
+                       int B, const int32_t* lens, const uint16_t* Q, const float* w,
+                       const int32_t* q_seq, const int32_t* q_pos, int n_q, int H, int m, int k,
+                       int n_threads, int32_t* idx, double* score, int32_t* blocks,
+                       int32_t* nblocks, double* block_scores, int64_t* counts) {
+    if (check_cache(keys, scale, dtype, batch, cap, d) || B < 1 || !lens || !Q || !w || !q_seq ||
+        n_q < 0 || H < 1 || m < 1 || m > 4096 || k < 1 || !idx)
+        return 1;
+    job_t J;
+    memset(&J, 0, sizeof J);
+    J.c = (cache_t){keys, scale, dtype, batch, cap, d};
+    J.B = B; J.lens = lens; J.Q = Q; J.w = w; J.q_seq = q_seq; J.q_pos = q_pos;
+    J.n_q = n_q; J.H = H; J.m = m; J.k = k; J.nbmax = (cap + B - 1) / B;
+    J.idx = idx; J.score = score; J.blocks = blocks; J.nblocks = nblocks;
+    J.block_scores = block_scores; J.counts = counts;
+    long items = J.nbmax > (long)m * B ? J.nbmax : (long)m * B;
+    int rc = for_rows(hisa_row, &J, n_q, n_threads, row_scratch_bytes(H, d, items));
+    return rc ? rc : (J.bad ? 2 : 0);
+}
+
+int hisa_oracle_refine(const void* keys, const float* scale, int dtype, int batch, int cap, int d,
+                       int B, const int32_t* lens, const uint16_t* Q, const float* w,
+                       const int32_t* q_seq, const int32_t* q_pos, int n_q, int H, int k,
+                       const int32_t* in_blocks, const int32_t* in_nblocks, int mm, int n_threads,
+                       int32_t* idx, double* score, double* cand_scores) {
+    if (check_cache(keys, scale, dtype, batch, cap, d) || B < 1 || !lens || !Q || !w || !q_seq ||
+        n_q < 0 || H < 1 || k < 1 || mm < 1 || !in_blocks || !in_nblocks || !idx)
+        return 1;
+    job_t J;
+    memset(&J, 0, sizeof J);
+    J.c = (cache_t){keys, scale, dtype, batch, cap, d};
+    J.B = B; J.lens = lens; J.Q = Q; J.w = w; J.q_seq = q_seq; J.q_pos = q_pos;
+    J.n_q = n_q; J.H = H; J.k = k; J.in_blocks = in_blocks; J.in_nblocks = in_nblocks;
+    J.mm = mm; J.idx = idx; J.score = score; J.cand_scores = cand_scores;
+    int rc = for_rows(refine_row, &J, n_q, n_threads, row_scratch_bytes(H, d, (long)mm * B));
+    return rc ? rc : (J.bad ? 2 : 0);
+}
+
+int hisa_oracle_flat(const void* keys, const float* scale, int dtype, int batch, int cap, int d,
+                     const int32_t* lens, const uint16_t* Q, const float* w, const int32_t* q_seq,
+                     const int32_t* q_pos, int n_q, int H, int k, int n_threads, int32_t* idx,
+                     double* score, double* all_scores) {
+    if (check_cache(keys, scale, dtype, batch, cap, d) || !lens || !Q || !w || !q_seq || n_q < 0 ||
+        H < 1 || k < 1 || !idx)
+        return 1;
+    job_t J;
+    memset(&J, 0, sizeof J);
+    J.c = (cache_t){keys, scale, dtype, batch, cap, d};
+    J.B = 1; J.lens = lens; J.Q = Q; J.w = w; J.q_seq = q_seq; J.q_pos = q_pos;
+    J.n_q = n_q; J.H = H; J.k = k; J.idx = idx; J.score = score; J.all_scores = all_scores;
+    int rc = for_rows(flat_row, &J, n_q, n_threads, row_scratch_bytes(H, d, cap));
+    return rc ? rc : (J.bad ? 2 : 0);
+}
+
+/* The selection rule alone, on given fp32 values: per row keep the k largest
+ * (ties: lower index), indices ascending, -1 padded.  Both sides decide on
+ * the same fp32 numbers here, so the result is exact. */
+int hisa_oracle_topk_f32(const float* x, int rows, int n, int k, int32_t* idx) {
+    if (!x || rows < 0 || n < 0 || k < 1 || !idx) return 1;
+    scored_t* items = (scored_t*)malloc(sizeof(scored_t) * (size_t)(n > 0 ? n : 1));
+    if (!items) return 3;
+    for (int r = 0; r < rows; ++r) {
+        for (int s = 0; s < n; ++s) {
+            items[s].v = (double)x[(size_t)r * n + s];
+            items[s].i = s;
+        }
+        keep_top(items, n, k, idx + (size_t)r * k, NULL);
+    }
+    free(items);
+    return 0;
+}

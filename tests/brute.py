@@ -1,0 +1,93 @@
+"""Exact brute force for tiny HISA cases (pure Python, rational arithmetic).
+
+Independent of the C oracle: every value is a ``fractions.Fraction``, so the
+pooled means, the indexer scores and every comparison are exact, and top-k
+membership is decided by its definition (an item is kept iff fewer than k
+items beat it) rather than by sorting.  Only for inputs of a few dozen
+tokens.
+
+Method: HISA (gptget.net summary, "Methodology"; Chinese summary, method
+details): mean-pool contiguous blocks of size B, score the representatives
+with the indexer, keep the top-m blocks (own block forced, counted in m),
+score the tokens of the kept blocks, keep the top-k tokens.
+"""
+from __future__ import annotations
+
+from fractions import Fraction
+
+import numpy as np
+
+from hisa_inputs import bf16_to_f32, e4m3_to_f32
+
+
+def key_values(case_keys, key_scale, dtype, b, s):
+    """Exact rational value of key row (b, s) as the indexer sees it."""
+    if dtype == "bf16":
+        return [Fraction(float(v)) for v in bf16_to_f32(case_keys[b, s])]
+    vals = e4m3_to_f32(case_keys[b, s])
+    sc = np.float32(key_scale[b, s])
+    # numpy fp32 multiply: one round-to-nearest of the exact product
+    return [Fraction(float(np.float32(v) * sc)) for v in vals]
+
+
+def query_values(Q, w, i):
+    q = [[Fraction(float(v)) for v in bf16_to_f32(Q[i, h])] for h in range(Q.shape[1])]
+    ww = [Fraction(float(v)) for v in w[i]]
+    return q, ww
+
+
+def score(q, ww, x):
+    tot = Fraction(0)
+    for qh, wh in zip(q, ww):
+        z = sum((a * b for a, b in zip(qh, x)), Fraction(0))
+        if z > 0:
+            tot += wh * z
+    return tot
+
+
+def beats(a, b):
+    """(value, index) a ranks above b: larger value, or equal value and lower index."""
+    return a[0] > b[0] or (a[0] == b[0] and a[1] < b[1])
+
+
+def keep_by_definition(items, k):
+    """items: list of (value, index).  Returns the set of indices kept."""
+    kept = []
+    for it in items:
+        n_above = sum(1 for o in items if o is not it and beats(o, it))
+        if n_above < k:
+            kept.append(it[1])
+    return sorted(kept)
+
+
+def block_mean(keys, key_scale, dtype, b, B, j, n):
+    s0, s1 = j * B, min((j + 1) * B, n)
+    rows = [key_values(keys, key_scale, dtype, b, s) for s in range(s0, s1)]
+    return [sum(col, Fraction(0)) / (s1 - s0) for col in zip(*rows)]
+
+
+def hisa_row(keys, key_scale, dtype, Q, w, b, t, i, B, m, k):
+    q, ww = query_values(Q, w, i)
+    n = t + 1
+    nb = -(-n // B)
+    S = [score(q, ww, block_mean(keys, key_scale, dtype, b, B, j, n)) for j in range(nb)]
+    if nb <= m:
+        chosen = list(range(nb))
+    else:
+        others = [(S[j], j) for j in range(nb - 1)]
+        chosen = keep_by_definition(others, m - 1) + [nb - 1]
+    cand = []
+    for j in chosen:
+        for s in range(j * B, min((j + 1) * B, n)):
+            cand.append((score(q, ww, key_values(keys, key_scale, dtype, b, s)), s))
+    kept = keep_by_definition(cand, k)
+    val = {s: v for v, s in cand}
+    return dict(idx=kept, scores=[val[s] for s in kept], blocks=chosen, block_scores=S)
+
+
+def flat_row(keys, key_scale, dtype, Q, w, b, t, i, k):
+    q, ww = query_values(Q, w, i)
+    cand = [(score(q, ww, key_values(keys, key_scale, dtype, b, s)), s) for s in range(t + 1)]
+    kept = keep_by_definition(cand, k)
+    val = {s: v for v, s in cand}
+    return dict(idx=kept, scores=[val[s] for s in kept])

@@ -1,0 +1,101 @@
+"""The oracle's pins catch plausible mistakes.
+
+Each case copies the oracle source, plants one mistake (a dropped term, a
+wrong sign or index, a reversed tie rule ...), builds the copy on the CPU and
+checks that the exact brute force or a closed form rejects it.  The committed
+oracle is never modified.
+"""
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from hisa_inputs import bf16_bits, make_case
+from tests import brute
+
+MUTANTS = {
+    "relu_dropped": ("acc += w[h] * (z > 0.0 ? z : 0.0);", "acc += w[h] * z;"),
+    "causal_off_by_one": ("if (blk[r] >= 0 && s <= t) {", "if (blk[r] >= 0 && s < t) {"),
+    "ties_to_higher_index": ("return (a->i > b->i) - (a->i < b->i);",
+                             "return (a->i < b->i) - (a->i > b->i);"),
+    "mean_over_B_not_valid_count": ("mu[e] /= (double)(s1 - s0);", "mu[e] /= (double)B;"),
+    "own_block_not_forced": ("chosen[J->m - 1] = (int32_t)(nb - 1);",
+                             "chosen[J->m - 1] = (int32_t)items[J->m - 1].i;"),
+    "first_head_dropped": ("for (int h = 0; h < H; ++h) {\n        double z",
+                           "for (int h = 1; h < H; ++h) {\n        double z"),
+    "query_stride_transposed": ("double z = dot(q + (size_t)h * d, x, d);",
+                                "double z = dot(q + (size_t)h, x, d);"),
+    "e4m3_bias_wrong": ("else v = ldexp(1.0 + m / 8.0, e - 7);",
+                        "else v = ldexp(1.0 + m / 8.0, e - 8);"),
+    "flat_misses_last_token": ("for (long s = 0; s <= t; ++s) {", "for (long s = 0; s < t; ++s) {"),
+}
+
+
+def _cases():
+    out = []
+    for seed, dtype in [(1, "bf16"), (2, "e4m3"), (3, "bf16"), (4, "e4m3")]:
+        rng = np.random.default_rng(seed)
+        B = [4, 8, 4, 2][seed - 1]
+        L = [37, 45, 30, 21][seed - 1]
+        c = make_case(batch=2, L=L, H=3, d=8, B=B, m=2 + seed % 2, k=5 + seed, dtype=dtype,
+                      seed=300 + seed, positions=np.array([L - 1, L // 2, B + 1]))
+        out.append(c)
+    t = make_case(batch=1, L=32, H=3, d=8, B=4, m=3, k=6, seed=305)
+    t.keys[:, 9] = t.keys[:, 2]
+    t.keys[:, 20:24] = t.keys[:, 4:8]
+    t.keys[:, 12:16] = t.keys[:, 4:8]
+    out.append(t)
+    return out
+
+
+def _pool_closed_form_fails(lib) -> bool:
+    L, B, d = 61, 16, 4                       # trailing block holds 13 tokens
+    s = np.arange(L)[:, None]
+    keys = ((s + np.arange(d)[None, :]) / 16.0).astype(np.float32)[None]
+    P = oracle.pool(oracle.Cache(bf16_bits(keys), None, [L], "bf16"), B, lib=lib)
+    for j in range(-(-L // B)):
+        s0, s1 = j * B, min((j + 1) * B, L)
+        if not np.allclose(P[0, j], ((s0 + s1 - 1) / 2.0 + np.arange(d)) / 16.0, rtol=0,
+                           atol=1e-15):
+            return True
+    return False
+
+
+def _detects(lib) -> bool:
+    """True if some pin rejects the library `lib`."""
+    if _pool_closed_form_fails(lib):
+        return True
+    for c in _cases():
+        cache = oracle.Cache.of(c)
+        r = oracle.hisa_select(cache, c.Q, c.w, c.q_seq, c.q_pos, c.B, c.m, c.k, threads=1,
+                               lib=lib)
+        f = oracle.flat_select(cache, c.Q, c.w, c.q_seq, c.q_pos, c.k, threads=1, lib=lib)
+        for i in range(c.n_q):
+            b, t = int(c.q_seq[i]), int(c.q_pos[i])
+            ref = brute.hisa_row(c.keys, c.key_scale, c.dtype, c.Q, c.w, b, t, i, c.B, c.m, c.k)
+            got = [x for x in r["idx"][i] if x >= 0]
+            if got != ref["idx"]:
+                return True
+            if not np.allclose(r["score"][i][:len(got)], [float(v) for v in ref["scores"]],
+                               rtol=1e-12, atol=1e-15):
+                return True
+            fref = brute.flat_row(c.keys, c.key_scale, c.dtype, c.Q, c.w, b, t, i, c.k)
+            if [x for x in f["idx"][i] if x >= 0] != fref["idx"]:
+                return True
+    return False
+
+
+def test_unmutated_oracle_passes():
+    assert not _detects(oracle.load())
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistake_is_caught(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(oracle.SRC).read()
+    assert src.count(old) == 1, f"mutation anchor for {name} not unique"
+    path = tmp_path / "mutant.c"
+    path.write_text(src.replace(old, new))
+    lib = oracle.load(oracle.build(str(path), str(tmp_path / f"lib_{name}.so")))
+    assert _detects(lib), f"planted mistake {name} went unnoticed"

@@ -1,0 +1,268 @@
+"""Pins of the CPU oracle to things other than itself (no GPU needed).
+
+* exact rational brute force on tiny inputs (tests/brute.py), with forced ties;
+* closed-form block means (constant blocks, arithmetic progressions, the
+  trailing partial block) and the B = 1 identity;
+* closed-form indexer scores (one-hot queries and keys, w = 0, all-negative
+  dot products, scaling w);
+* structure: m >= #blocks makes HISA the flat scan; the tokens-scored count
+  ceil(L/B) + min(m, nb) * B of the pages' O(L/B + mB) (golden fixture);
+  causality, ascending output, -1 tail padding, own block always kept.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from hisa_inputs import bf16_bits, bf16_to_f32, e4m3_to_f32, make_case, quantize_e4m3_rows
+from tests import brute
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def tiny(seed, dtype="bf16", L=40, B=4, m=3, k=7, H=3, d=8, batch=2, positions=None):
+    return make_case(batch=batch, L=L, H=H, d=d, B=B, m=m, k=k, dtype=dtype, seed=seed,
+                     positions=positions)
+
+
+def oracle_select(c, m=None, k=None):
+    return oracle.hisa_select(oracle.Cache.of(c), c.Q, c.w, c.q_seq, c.q_pos, c.B,
+                              m or c.m, k or c.k, threads=2)
+
+
+# ----------------------------------------------------------------- pooling
+
+
+def test_pool_constant_block_is_exact():
+    d, B = 8, 16
+    keys = np.zeros((1, 64, d), np.float32)
+    for j in range(4):
+        keys[0, j * B:(j + 1) * B] = 0.375 * (j + 1) - 1.0   # exact in bf16
+    c = oracle.Cache(bf16_bits(keys), None, [64], "bf16")
+    P = oracle.pool(c, B)
+    for j in range(4):
+        assert np.all(P[0, j] == 0.375 * (j + 1) - 1.0)
+
+
+@pytest.mark.parametrize("L,B", [(64, 16), (61, 16), (37, 8), (5, 8)])
+def test_pool_arithmetic_progression_closed_form(L, B):
+    # key[s, e] = (s + e) / 16: exact in bf16 for s + e <= 256.
+    d = 4
+    s = np.arange(L)[:, None]
+    e = np.arange(d)[None, :]
+    keys = ((s + e) / 16.0).astype(np.float32)[None]
+    c = oracle.Cache(bf16_bits(keys), None, [L], "bf16")
+    P = oracle.pool(c, B)
+    for j in range(-(-L // B)):
+        s0, s1 = j * B, min((j + 1) * B, L)          # trailing block: valid tokens only
+        expect = ((s0 + s1 - 1) / 2.0 + np.arange(d)) / 16.0
+        np.testing.assert_allclose(P[0, j], expect, rtol=0, atol=1e-15)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+def test_pool_block_size_one_is_identity(dtype):
+    c = tiny(11, dtype=dtype, L=33, B=1)
+    P = oracle.pool(oracle.Cache.of(c), 1)
+    if dtype == "bf16":
+        expect = bf16_to_f32(c.keys)
+    else:   # fp32 product of the e4m3 value and the token's scale, computed by numpy
+        expect = (e4m3_to_f32(c.keys) * c.key_scale[..., None]).astype(np.float32)
+    assert np.array_equal(P[:, :33], expect[:, :33].astype(np.float64))
+
+
+def test_pool_leaves_blocks_past_len_untouched():
+    c = tiny(3, L=40, B=8)
+    P = oracle.pool(oracle.Cache(c.keys, None, [17, 40], "bf16"), 8)
+    assert np.all(np.isnan(P[0, 3:]))        # blocks 3.. start at >= 24 > 17
+    assert not np.any(np.isnan(P[0, :3]))
+
+
+# ----------------------------------------------------------------- scoring
+
+
+def _onehot_case():
+    d, H, L = 8, 3, 12
+    alpha = np.array([0.5, -0.25, 1.5], np.float32)      # head h looks at coordinate a_h
+    a = np.array([1, 4, 6])
+    Q = np.zeros((1, H, d), np.float32)
+    Q[0, np.arange(H), a] = alpha
+    beta = (np.arange(L) % 5 - 2).astype(np.float32) * 0.125
+    b = np.arange(L) % d
+    keys = np.zeros((1, L, d), np.float32)
+    keys[0, np.arange(L), b] = beta
+    w = np.array([[0.75, 2.0, 0.5]], np.float32)
+    expect = np.zeros(L)
+    for s in range(L):
+        for h in range(H):
+            z = alpha[h] * beta[s] if a[h] == b[s] else 0.0
+            expect[s] += w[0, h] * max(z, 0.0)
+    return keys, Q, w, expect
+
+
+def test_score_one_hot_closed_form():
+    keys, Q, w, expect = _onehot_case()
+    L = keys.shape[1]
+    c = oracle.Cache(bf16_bits(keys), None, [L], "bf16")
+    r = oracle.flat_select(c, bf16_bits(Q), w, [0], [L - 1], k=L, want_all=True)
+    assert np.array_equal(r["all_scores"][0, :L], expect)
+
+
+def test_score_zero_weights_ties_go_to_lowest_index():
+    c = tiny(5, L=30)
+    w0 = np.zeros_like(c.w)
+    r = oracle.flat_select(oracle.Cache.of(c), c.Q, w0, c.q_seq, c.q_pos, k=7)
+    assert np.all(r["score"] == 0.0)
+    assert np.array_equal(r["idx"], np.tile(np.arange(7), (c.n_q, 1)))
+
+
+def test_score_all_negative_dots_give_zero():
+    c = tiny(6, L=20)
+    Qf = np.abs(bf16_to_f32(c.Q))
+    keys = -np.abs(bf16_to_f32(c.keys))
+    cc = oracle.Cache(bf16_bits(keys), None, c.lens, "bf16")
+    r = oracle.flat_select(cc, bf16_bits(Qf), c.w, c.q_seq, c.q_pos, k=5, want_all=True)
+    assert np.all(r["all_scores"][:, :20] == 0.0)
+
+
+def test_score_doubling_weights_doubles_scores():
+    c = tiny(7, L=50, B=8, m=3, k=9)
+    a = oracle_select(c)
+    c2 = tiny(7, L=50, B=8, m=3, k=9)
+    c2.w = (c.w * 2).astype(np.float32)
+    b = oracle_select(c2)
+    assert np.array_equal(a["idx"], b["idx"])
+    assert np.array_equal(a["blocks"], b["blocks"])
+    np.testing.assert_allclose(b["score"], 2 * a["score"], rtol=1e-15)
+
+
+# --------------------------------------------------------- exact brute force
+
+
+def _check_against_brute(c, m, k):
+    r = oracle_select(c, m=m, k=k)
+    f = oracle.flat_select(oracle.Cache.of(c), c.Q, c.w, c.q_seq, c.q_pos, k=k)
+    for i in range(c.n_q):
+        b, t = int(c.q_seq[i]), int(c.q_pos[i])
+        ref = brute.hisa_row(c.keys, c.key_scale, c.dtype, c.Q, c.w, b, t, i, c.B, m, k)
+        got = [x for x in r["idx"][i] if x >= 0]
+        assert got == ref["idx"], (i, got, ref["idx"])
+        assert list(r["idx"][i][len(got):]) == [-1] * (k - len(got))
+        np.testing.assert_allclose(r["score"][i][:len(got)], [float(v) for v in ref["scores"]],
+                                   rtol=1e-12, atol=1e-15)
+        nb = int(r["nblocks"][i])
+        assert list(r["blocks"][i][:nb]) == ref["blocks"]
+        np.testing.assert_allclose(r["block_scores"][i][:len(ref["block_scores"])],
+                                   [float(v) for v in ref["block_scores"]], rtol=1e-12, atol=1e-15)
+        fref = brute.flat_row(c.keys, c.key_scale, c.dtype, c.Q, c.w, b, t, i, k)
+        fgot = [x for x in f["idx"][i] if x >= 0]
+        assert fgot == fref["idx"]
+
+
+@pytest.mark.parametrize("seed", range(6))
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+def test_oracle_matches_exact_bruteforce(seed, dtype):
+    rng = np.random.default_rng(seed)
+    B = int(rng.choice([1, 2, 4, 16]))
+    L = int(rng.integers(5, 48))
+    nb = -(-L // B)
+    m = int(rng.integers(1, nb + 2))
+    k = int(rng.integers(1, L + 6))
+    pos = np.unique(rng.integers(0, L, size=3))
+    c = make_case(batch=2, L=L, H=int(rng.integers(1, 4)), d=int(rng.choice([4, 8])), B=B, m=m,
+                  k=k, dtype=dtype, seed=100 + seed, positions=pos)
+    _check_against_brute(c, m, k)
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_oracle_forced_ties_match_bruteforce(seed):
+    # duplicated key rows and duplicated whole blocks: exact score ties at
+    # token and block level, which must resolve toward the lower index.
+    c = tiny(200 + seed, L=32, B=4, m=3, k=6)
+    c.keys[:, 9] = c.keys[:, 2]
+    c.keys[:, 17] = c.keys[:, 2]
+    c.keys[:, 20:24] = c.keys[:, 4:8]
+    c.keys[:, 12:16] = c.keys[:, 4:8]
+    _check_against_brute(c, 3, 6)
+    _check_against_brute(c, 2, 3)
+
+
+# -------------------------------------------------------------- structure
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+def test_hisa_with_all_blocks_is_the_flat_scan(dtype):
+    c = make_case(batch=2, L=700, H=4, d=16, B=32, m=22, k=50, dtype=dtype, seed=9,
+                  positions=np.array([0, 31, 32, 400, 699]))
+    r = oracle_select(c, m=22)       # 22 blocks cover the whole prefix
+    f = oracle.flat_select(oracle.Cache.of(c), c.Q, c.w, c.q_seq, c.q_pos, k=50)
+    assert np.array_equal(r["idx"], f["idx"])
+    assert np.array_equal(np.nan_to_num(r["score"], nan=-7), np.nan_to_num(f["score"], nan=-7))
+
+
+def test_tokens_scored_count_matches_golden():
+    g = json.load(open(os.path.join(GOLDEN, "complexity_counts.json")))
+    for case in g["cases"]:
+        L, B, m = case["L"], case["B"], case["m"]
+        nb = -(-L // B)
+        assert nb == case["block_scores"]
+        assert min(m, nb) * B == case["token_slots"]
+    # and the oracle's own counters agree on a small case
+    c = make_case(batch=1, L=100, H=2, d=8, B=16, m=64, k=10, seed=4)
+    r = oracle_select(c)
+    assert tuple(r["counts"][0]) == (7, 112)
+    c = make_case(batch=1, L=300, H=2, d=8, B=16, m=5, k=10, seed=4)
+    r = oracle_select(c)
+    assert tuple(r["counts"][0]) == (19, 80)
+
+
+def test_output_format_and_causality():
+    c = make_case(batch=3, L=[200, 150, 97], H=3, d=16, B=16, m=4, k=40, seed=12,
+                  positions=[np.array([0, 5, 16, 199]), np.array([100, 149]), np.array([96])])
+    r = oracle_select(c)
+    for i in range(c.n_q):
+        t = c.q_pos[i]
+        row = r["idx"][i]
+        valid = row[row >= 0]
+        assert np.all(row[len(valid):] == -1)
+        assert np.all(np.diff(valid) > 0)
+        assert np.all(valid <= t)
+        assert len(valid) == min(c.k, t + 1, r["nblocks"][i] * c.B)
+        nb = -(-(t + 1) // c.B)
+        assert (nb - 1) in r["blocks"][i]          # own block kept
+        assert r["nblocks"][i] == min(c.m, nb)
+
+
+def test_refine_on_own_blocks_reproduces_select():
+    c = make_case(batch=2, L=500, H=4, d=16, B=16, m=6, k=33, seed=21,
+                  positions=np.array([77, 499]))
+    r = oracle_select(c)
+    rr = oracle.hisa_refine(oracle.Cache.of(c), c.Q, c.w, c.q_seq, c.q_pos, c.B, c.k,
+                            r["blocks"], r["nblocks"])
+    assert np.array_equal(r["idx"], rr["idx"])
+
+
+def test_topk_f32_rule_by_definition():
+    rng = np.random.default_rng(3)
+    x = rng.integers(-3, 4, size=(20, 37)).astype(np.float32) * 0.5   # many ties
+    x[0] = 0.0
+    x[1, ::2] = -0.0
+    for k in (1, 5, 37, 50):
+        got = oracle.topk_f32(x, k)
+        for r in range(x.shape[0]):
+            items = [(float(v), s) for s, v in enumerate(x[r])]
+            ref = brute.keep_by_definition(items, k)
+            assert [v for v in got[r] if v >= 0] == ref
+
+
+def test_e4m3_dequant_is_fp32_product():
+    rng = np.random.default_rng(1)
+    k32 = rng.standard_normal((1, 24, 8)).astype(np.float32)
+    codes, scale = quantize_e4m3_rows(k32)
+    c = oracle.Cache(codes, scale, [24], "e4m3")
+    P = oracle.pool(c, 1)
+    import torch
+    ref = (torch.from_numpy(codes).view(torch.float8_e4m3fn).float()
+           * torch.from_numpy(scale)[..., None]).numpy()
+    assert np.array_equal(P[0, :24], ref[0].astype(np.float64))
