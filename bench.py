@@ -1,0 +1,461 @@
+"""Benchmark of the HISA indexer on B200: selections/s on the 32K decode workload.
+
+One step = one decode step of a 64-sequence batch at 32K context: append the
+new key of every sequence to the cache (hisa_append: trailing block mean
+recomputed) and run the two-stage selection for every sequence's new last
+position (hisa_select: H_I=64, d_I=128, B=128, m=64, k=2048).  Inputs are
+seeded synthetic block-clustered keys (hisa_inputs) resident in HBM; L2 is
+flushed (256 MiB write) between timed steps, outside the timed events.
+
+The JSON line also carries: the flat-scan comparison (dsa_flat_select on
+the same rows: speedup and mean IoU), the roofline of the dominant kernel
+(stage-2 token scoring, HBM-bound), the pool kernel's bandwidth, an
+end-to-end figure through the public API with host buffers, SM clocks
+sampled during the timed region, and the CPU oracle timed on a bounded
+sample of the same workload.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+Multi-GPU (torchrun): every rank runs its own 64 sequences (weak scaling, no
+data-path collective); time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = dict(cfg=1, name="decode-32k-b64")
+L2_FLUSH_BYTES = 256 << 20
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=p["hbm_gbs"], bf16_tflops=p["bf16_tflops"], source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, source="fallback")
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------ clocks
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed region runs."""
+
+    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.uuid = uuid
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return None
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            if self.uuid and self.uuid not in parts[1]:
+                continue
+            try:
+                sm.append(float(parts[2]))
+                mx.append(float(parts[3]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[6:10]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)),
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# --------------------------------------------------------------- workload
+
+
+def make_workload(steps_total: int, seed_shift: int = 0):
+    from hisa_inputs import make_config
+    spec_cap = 32768 + steps_total
+    case = make_config(WORKLOAD["cfg"], cap=spec_cap, append_steps=steps_total,
+                       seed=20260330 + WORKLOAD["cfg"] + seed_shift)
+    return case
+
+
+def algorithmic_bytes(case):
+    """Bytes the method must move per query row in each kernel (decode, bf16)."""
+    H, d, B, m, k = case.H, case.d, case.B, case.m, case.k
+    nb = -(-case.cap // B)
+    q = H * d * 2 + H * 4
+    token_score = m * B * d * 2 + q + m * 4 + m * B * 4      # keys + Q,w + block ids + score keys
+    block_score = nb * 2 * d * 2 + q + nb * 4                 # hi/lo representatives + Q,w + keys
+    return dict(token_score=token_score, block_score=block_score,
+                step=token_score + block_score + m * B * 4 + k * 4 + nb * 4 + 2 * d + 2 * B * d,
+                flat_row=case.cap * d * 2 + q + case.cap * 4)
+
+
+def traffic_record():
+    """ncu DRAM bytes per launch of the token-scoring kernel, if taken on this source."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    src = os.path.join(ROOT, "hierarchical_top_indexer_b200", "csrc", "score.cu")
+    if not os.path.exists(path):
+        return None
+    rec = json.load(open(path))
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    ent = rec.get("token_score")
+    if not ent or ent.get("score_cu_sha256_16") != sha:
+        return None
+    return ent.get("bytes_per_launch")
+
+
+# --------------------------------------------------------------------- GPU
+
+
+def run_gpu(args, rank, world):
+    import torch
+    import hierarchical_top_indexer_b200 as hisa
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    K, W = args.steps, args.warmup
+    E = args.e2e_steps
+    n_flat = args.flat_steps
+    total_steps = W + K + E + 1
+    case = make_workload(total_steps, seed_shift=rank)
+    kv = hisa.KVCache.from_case(case, device=dev)
+    stream = torch.cuda.current_stream()
+    batch, H, d, m, k = case.batch, case.H, case.d, case.m, case.k
+
+    # pool: the index build (also times the pool kernel)
+    hisa.hisa_profile_enable(True)
+    hisa.hisa_pool_blocks(kv)
+    torch.cuda.synchronize()
+    hisa.hisa_profile_read(reset=True)
+    pool_ms = []
+    for _ in range(3):
+        hisa.hisa_pool_blocks(kv)
+        torch.cuda.synchronize()
+        pool_ms.append(hisa.hisa_profile_read(reset=True)["pool"][0])
+    hisa.hisa_profile_enable(False)
+
+    # device-resident per-step inputs
+    toks = torch.from_numpy(case.append_keys.view(np.int16)).view(torch.bfloat16).to(dev)
+    Qs = torch.from_numpy(case.append_Q.view(np.int16)).view(torch.bfloat16).to(dev)
+    Ws = torch.from_numpy(case.append_w).to(dev)
+    q_seq = torch.arange(batch, dtype=torch.int32, device=dev)
+    ws = hisa.workspace(hisa.hisa_select_workspace_bytes(kv, batch, H, m, k), dev)
+    idx = torch.empty((2, batch, k), dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(s, out):
+        hisa.hisa_append(kv, toks[s])
+        hisa.hisa_select(kv, Qs[s], Ws[s], q_seq, None, m, k, ws=ws, idx=out)
+
+    for s in range(W):
+        step(s, idx[s % 2])
+        flush.fill_(7)
+    torch.cuda.synchronize()
+
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    hisa.hisa_profile_enable(True)
+    hisa.hisa_profile_read(reset=True)
+    with ClockSampler(uuid) as clk:
+        wall0 = time.perf_counter()
+        for i in range(K):
+            s = W + i
+            ev[i][0].record(stream)
+            step(s, idx[s % 2])
+            ev[i][1].record(stream)
+            flush.fill_(7)
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - wall0
+    if world > 1:
+        dist.barrier()
+    phases = hisa.hisa_profile_read(reset=True)
+    hisa.hisa_profile_enable(False)
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = float(sum(step_ms))
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    launches = sum(n for _, n in phases.values())
+
+    # select-only comparison: HISA vs the flat scan on the same rows
+    s_cmp = W + K
+    hisa.hisa_append(kv, toks[s_cmp])
+    fws = hisa.workspace(hisa.dsa_flat_workspace_bytes(kv, batch, H, k), dev)
+    fidx = torch.empty((batch, k), dtype=torch.int32, device=dev)
+    hidx = torch.empty((batch, k), dtype=torch.int32, device=dev)
+
+    def time_calls(fn, n):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n)]
+        for _ in range(2):
+            fn()
+            flush.fill_(7)
+        for a, b in evs:
+            a.record(stream)
+            fn()
+            b.record(stream)
+            flush.fill_(7)
+        torch.cuda.synchronize()
+        return float(np.median([a.elapsed_time(b) for a, b in evs]))
+
+    hisa_sel_ms = time_calls(lambda: hisa.hisa_select(kv, Qs[s_cmp], Ws[s_cmp], q_seq, None, m, k,
+                                                      ws=ws, idx=hidx), n_flat)
+    flat_ms = time_calls(lambda: hisa.dsa_flat_select(kv, Qs[s_cmp], Ws[s_cmp], q_seq, None, k,
+                                                      ws=fws, idx=fidx), n_flat)
+    torch.cuda.synchronize()
+    from tests.parity import iou
+    hi, fi = hidx.cpu().numpy(), fidx.cpu().numpy()
+    mean_iou = float(np.mean([iou(a, b) for a, b in zip(hi, fi)]))
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if E > 0:
+        ptok = torch.from_numpy(case.append_keys.view(np.int16)).view(torch.bfloat16).pin_memory()
+        pQ = torch.from_numpy(case.append_Q.view(np.int16)).view(torch.bfloat16).pin_memory()
+        pW = torch.from_numpy(case.append_w).pin_memory()
+        pidx = torch.empty((batch, k), dtype=torch.int32).pin_memory()
+        dtok = torch.empty_like(toks[0])
+        dQ = torch.empty_like(Qs[0])
+        dW = torch.empty_like(Ws[0])
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(E)]
+        base = W + K + 1
+        for i, (a, b) in enumerate(evs):
+            s = base + i
+            a.record(stream)
+            dtok.copy_(ptok[s], non_blocking=True)
+            dQ.copy_(pQ[s], non_blocking=True)
+            dW.copy_(pW[s], non_blocking=True)
+            hisa.hisa_append(kv, dtok)
+            out = hisa.hisa_select(kv, dQ, dW, q_seq, None, m, k, ws=ws, idx=hidx)
+            pidx.copy_(out, non_blocking=True)
+            b.record(stream)
+            b.synchronize()
+            flush.fill_(7)
+        torch.cuda.synchronize()
+        e2e_ms = float(sum(a.elapsed_time(b) for a, b in evs))
+        e2e = {"value": batch * E / (e2e_ms / 1e3), "unit": "selections/s",
+               "h2d_bytes_per_step": int(dtok.numel() * 2 + dQ.numel() * 2 + dW.numel() * 4),
+               "d2h_bytes_per_step": int(pidx.numel() * 4), "steps": E,
+               "path": "pinned host -> hisa_append + hisa_select (python binding of the C ABI) -> pinned host"}
+    assert kv.status_bits() == 0, f"device status {kv.status_bits():#x}"
+
+    peaks = measured_peaks()
+    ab = algorithmic_bytes(case)
+    tok_ms, tok_n = phases["token_score"]
+    tok_launch_s = tok_ms / max(tok_n, 1) / 1e3
+    tok_bytes = ab["token_score"] * batch
+    achieved = tok_bytes / tok_launch_s / 1e9
+    nb = -(-case.cap // case.B)
+    pool_bytes = batch * 32768 * d * 2 + batch * nb * (d * 4 + 2 * d * 2)
+    pool_gbs = pool_bytes / (float(np.median(pool_ms)) / 1e3) / 1e9
+    kernels = {name: {"ms_per_launch": (ms / n if n else None), "launches": n,
+                      "share": ms / max(sum(x for x, _ in phases.values()), 1e-9)}
+               for name, (ms, n) in phases.items() if n}
+    return dict(
+        total_ms=total_ms, step_ms=step_ms, wall=wall, clocks=clk.summary(), launches=launches,
+        kernels=kernels, tok_bytes=tok_bytes, achieved=achieved, peaks=peaks,
+        pool_gbs=pool_gbs, pool_ms=float(np.median(pool_ms)), hisa_sel_ms=hisa_sel_ms,
+        flat_ms=flat_ms, mean_iou=mean_iou, e2e=e2e, case=case)
+
+
+# ----------------------------------------------------------- CPU baseline
+
+
+def cpu_oracle_rate(case=None, budget_s: float = 12.0, rows_per_call: int = 16):
+    """The oracle as it stands, on all host cores, on a bounded sample of rows."""
+    import oracle
+    if case is None:
+        case = make_workload(1)
+    cache = oracle.Cache.of(case)
+    threads = host_cores()
+    done, t0 = 0, time.perf_counter()
+    r0 = 0
+    while True:
+        rows = np.arange(r0, r0 + rows_per_call) % case.n_q
+        oracle.hisa_select(cache, case.Q[rows], case.w[rows], case.q_seq[rows], case.q_pos[rows],
+                           case.B, case.m, case.k, threads=threads)
+        done += len(rows)
+        r0 += rows_per_call
+        el = time.perf_counter() - t0
+        if el >= budget_s or done >= 4 * case.n_q:
+            break
+    return dict(value=done / el, unit="selections/s", cores=threads, kind="oracle",
+                sample=f"{done} query rows of {WORKLOAD['name']} (HISA oracle, double, pooling "
+                       f"from scratch per row), {el:.1f} s wall")
+
+
+def run_reference(args, rank, world):
+    """--impl reference: the CPU oracle on the same workload (rank 0 only)."""
+    if rank != 0:
+        return None
+    import oracle
+    case = make_workload(1)
+    cache = oracle.Cache.of(case)
+    threads = host_cores()
+    rows_per_step = args.ref_rows
+    for s in range(args.warmup):
+        rows = (np.arange(rows_per_step) + s * rows_per_step) % case.n_q
+        oracle.hisa_select(cache, case.Q[rows], case.w[rows], case.q_seq[rows], case.q_pos[rows],
+                           case.B, case.m, case.k, threads=threads)
+    t0 = time.perf_counter()
+    for s in range(args.steps):
+        rows = (np.arange(rows_per_step) + s * rows_per_step) % case.n_q
+        oracle.hisa_select(cache, case.Q[rows], case.w[rows], case.q_seq[rows], case.q_pos[rows],
+                           case.B, case.m, case.k, threads=threads)
+    el = time.perf_counter() - t0
+    v = rows_per_step * args.steps / el
+    line = {
+        "impl": "reference", "metric": "HISA indexer top-k selections/s (decode, 32K context)",
+        "value": v, "unit": "selections/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD["name"], "batch": case.batch, "L": 32768, "H_I": case.H,
+                   "d_I": case.d, "B": case.B, "m": case.m, "k": case.k,
+                   "step": f"{rows_per_step} query rows (bounded sample of the 64-row batch)"},
+        "cpu_baseline": {"value": v, "unit": "selections/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{rows_per_step} rows per step x {args.steps} steps"},
+        "e2e": {"value": v, "unit": "selections/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    return line
+
+
+# -------------------------------------------------------------------- main
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["hisa", "reference"], default="hisa")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--flat-steps", type=int, default=5)
+    ap.add_argument("--ref-rows", type=int, default=16)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, rank, world)
+            if line is not None:
+                print(json.dumps(line), flush=True)
+            return 0
+
+        r = run_gpu(args, rank, world)
+        if rank != 0:
+            return 0
+        case = r["case"]
+        K = args.steps
+        value = case.batch * K * world / (r["total_ms"] / 1e3)
+        peaks = r["peaks"]
+        cpu = None
+        if not args.no_cpu_baseline and world == 1:
+            cpu = cpu_oracle_rate(case)
+        traffic = traffic_record()
+        line = {
+            "metric": "HISA indexer top-k selections/s (decode, 32K context)",
+            "value": value, "unit": "selections/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": r["total_ms"] / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD["name"], "batch": case.batch, "L": 32768,
+                       "H_I": case.H, "d_I": case.d, "B": case.B, "m": case.m, "k": case.k,
+                       "key_dtype": "bf16", "parallelism": f"replicas x{world}" if world > 1 else "1 gpu",
+                       "step": "hisa_append (64 keys) + hisa_select (64 rows at the new last position)",
+                       "l2": "flushed between timed steps (256 MiB write, outside the timed events)"},
+            "clocks": r["clocks"],
+            "gpu_launches": r["launches"],
+            "roofline": {"kernel": "token_score (stage 2: gather + tcgen05 scoring)",
+                         "bound": "hbm", "achieved": r["achieved"], "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": r["achieved"] / peaks["hbm_gbs"],
+                         "traffic": traffic, "peak_source": peaks["source"],
+                         "algorithmic_bytes_per_launch": r["tok_bytes"]},
+            "kernels": r["kernels"],
+            "pool": {"GB/s": r["pool_gbs"], "frac": r["pool_gbs"] / peaks["hbm_gbs"],
+                     "ms": r["pool_ms"]},
+            "flat_scan": {"ms_per_select": r["flat_ms"], "hisa_ms_per_select": r["hisa_sel_ms"],
+                          "speedup": r["flat_ms"] / r["hisa_sel_ms"],
+                          "flat_selections_per_s": case.batch / (r["flat_ms"] / 1e3),
+                          "mean_iou_hisa_vs_flat": r["mean_iou"]},
+            "e2e": r["e2e"],
+            "cpu_baseline": cpu,
+            "wall_s_timed_region": r["wall"],
+        }
+        print(json.dumps(line), flush=True)
+        return 0
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            if dist.is_initialized():
+                dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,264 @@
+"""HISA hierarchical top-k indexer on B200 — Python binding of libhisa_b200.so.
+
+Argument marshalling only: every step of the indexer runs in the library's
+CUDA kernels (see include/hisa.h for the contract of each call).  PyTorch
+provides device memory and the current CUDA stream.  There is no CPU or
+PyTorch fallback: if the library is missing, importing this package fails.
+
+    import hierarchical_top_indexer_b200 as hisa
+    kv = hisa.KVCache(batch, cap, d=128, B=128, dtype="bf16")
+    kv.load(keys_bf16, lens)             # host or device tensors
+    hisa.hisa_pool_blocks(kv)
+    idx = hisa.hisa_select(kv, Q, w, q_seq, q_pos, m=64, k=2048)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libhisa_b200.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python hierarchical_top_indexer_b200/build.py` "
+        "(there is no fallback implementation)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+HISA_KEY_BF16, HISA_KEY_E4M3 = 0, 1
+HISA_OK, HISA_E_INVAL, HISA_E_UNSUPPORTED, HISA_E_WORKSPACE, HISA_E_CUDA = range(5)
+HISA_DEV_BAD_QUERY, HISA_DEV_CAPACITY, HISA_DEV_BAD_LEN, HISA_DEV_TIMEOUT = 0x1, 0x2, 0x4, 0x8
+
+EXPORTS = ("hisa_pool_blocks", "hisa_append", "hisa_select_workspace_bytes", "hisa_select",
+           "hisa_select_inspect", "dsa_flat_workspace_bytes", "dsa_flat_select", "hisa_topk_f32",
+           "hisa_profile_enable", "hisa_profile_read", "hisa_status_string")
+PHASES = ("block_score", "block_select", "token_score", "token_select", "flat_score",
+          "flat_select", "pool", "append", "topk")
+
+
+class hisa_kv(ctypes.Structure):
+    _fields_ = [("keys", ctypes.c_void_p), ("key_scale", ctypes.c_void_p),
+                ("pooled", ctypes.c_void_p), ("pooled_hl", ctypes.c_void_p),
+                ("len", ctypes.c_void_p), ("status", ctypes.c_void_p),
+                ("batch", ctypes.c_int32), ("cap", ctypes.c_int32), ("d", ctypes.c_int32),
+                ("B", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+
+
+_P, _I, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+_KVP = ctypes.POINTER(hisa_kv)
+_lib.hisa_pool_blocks.argtypes = [_KVP, _P]
+_lib.hisa_append.argtypes = [_KVP, _P, _P, _P]
+_lib.hisa_select_workspace_bytes.argtypes = [_KVP, _I, _I, _I, _I]
+_lib.hisa_select_workspace_bytes.restype = _Z
+_lib.hisa_select.argtypes = [_KVP, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _Z, _P]
+_lib.hisa_select_inspect.argtypes = [_KVP, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P,
+                                     _P, _Z, _P]
+_lib.dsa_flat_workspace_bytes.argtypes = [_KVP, _I, _I, _I]
+_lib.dsa_flat_workspace_bytes.restype = _Z
+_lib.dsa_flat_select.argtypes = [_KVP, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _Z, _P]
+_lib.hisa_topk_f32.argtypes = [_P, _I, _I, _I, _P, _P]
+_lib.hisa_profile_enable.argtypes = [_I]
+_lib.hisa_profile_read.argtypes = [_P, _P, _I]
+_lib.hisa_status_string.argtypes = [_I]
+_lib.hisa_status_string.restype = ctypes.c_char_p
+for _f in ("hisa_pool_blocks", "hisa_append", "hisa_select", "hisa_select_inspect",
+           "dsa_flat_select", "hisa_topk_f32", "hisa_profile_enable", "hisa_profile_read"):
+    getattr(_lib, _f).restype = _I
+
+
+class HisaError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn}: {_lib.hisa_status_string(code).decode()} (code {code})")
+        self.code = code
+
+
+def _check(fn: str, code: int):
+    if code != HISA_OK:
+        raise HisaError(fn, code)
+
+
+def lib():
+    """The loaded ctypes library (for direct C-ABI calls)."""
+    return _lib
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    assert t.is_contiguous(), "tensors passed to the library must be contiguous"
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dev(x, dtype, device):
+    if not isinstance(x, torch.Tensor):
+        x = torch.as_tensor(x)
+    if x.dtype != dtype:
+        x = x.view(dtype) if x.element_size() == torch.empty((), dtype=dtype).element_size() \
+            else x.to(dtype)
+    return x.to(device).contiguous()
+
+
+class KVCache:
+    """Device storage of the indexer keys and the block index (hisa_kv)."""
+
+    def __init__(self, batch: int, cap: int, d: int, B: int, dtype: str = "bf16",
+                 device="cuda"):
+        self.batch, self.cap, self.d, self.B = batch, cap, d, B
+        self.dtype = dtype
+        self.device = torch.device(device)
+        self.nblk = -(-cap // B)
+        kdt = torch.bfloat16 if dtype == "bf16" else torch.uint8
+        self.keys = torch.zeros((batch, cap, d), dtype=kdt, device=self.device)
+        self.key_scale = (torch.ones((batch, cap), dtype=torch.float32, device=self.device)
+                          if dtype == "e4m3" else None)
+        self.pooled = torch.zeros((batch, self.nblk, d), dtype=torch.float32, device=self.device)
+        self.pooled_hl = torch.zeros((batch, self.nblk, 2 * d), dtype=torch.bfloat16,
+                                     device=self.device)
+        self.len = torch.zeros(batch, dtype=torch.int32, device=self.device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=self.device)
+        self._struct = hisa_kv(
+            keys=self.keys.data_ptr(),
+            key_scale=self.key_scale.data_ptr() if self.key_scale is not None else None,
+            pooled=self.pooled.data_ptr(), pooled_hl=self.pooled_hl.data_ptr(),
+            len=self.len.data_ptr(), status=self.status.data_ptr(), batch=batch, cap=cap, d=d,
+            B=B, dtype=HISA_KEY_BF16 if dtype == "bf16" else HISA_KEY_E4M3)
+
+    @property
+    def struct(self):
+        return ctypes.byref(self._struct)
+
+    def load(self, keys, lens, key_scale=None):
+        """Copy keys [batch, <=cap, d] (bf16 bits / e4m3 codes), lens and scales in."""
+        kdt = torch.bfloat16 if self.dtype == "bf16" else torch.uint8
+        k = _dev(keys, kdt, self.device)
+        self.keys[:, :k.shape[1]].copy_(k)
+        self.len.copy_(_dev(lens, torch.int32, self.device))
+        if self.dtype == "e4m3":
+            sc = _dev(key_scale, torch.float32, self.device)
+            self.key_scale[:, :sc.shape[1]].copy_(sc)
+        return self
+
+    @classmethod
+    def from_case(cls, case, device="cuda"):
+        kv = cls(case.batch, case.cap, case.d, case.B, case.dtype, device)
+        return kv.load(torch.from_numpy(case.keys), torch.from_numpy(case.lens),
+                       None if case.key_scale is None else torch.from_numpy(case.key_scale))
+
+    def status_bits(self) -> int:
+        return int(self.status.item()) & 0xFFFFFFFF
+
+    def clear_status(self):
+        self.status.zero_()
+
+
+def hisa_pool_blocks(kv: KVCache, stream=None):
+    _check("hisa_pool_blocks", _lib.hisa_pool_blocks(kv.struct, _stream(stream)))
+
+
+def hisa_append(kv: KVCache, tok: torch.Tensor, tok_scale: Optional[torch.Tensor] = None,
+                stream=None):
+    _check("hisa_append", _lib.hisa_append(kv.struct, _ptr(tok), _ptr(tok_scale), _stream(stream)))
+
+
+def _queries(kv, Q, w, q_seq, q_pos):
+    Q = _dev(Q, torch.bfloat16, kv.device)
+    w = _dev(w, torch.float32, kv.device)
+    q_seq = _dev(q_seq, torch.int32, kv.device)
+    q_pos = None if q_pos is None else _dev(q_pos, torch.int32, kv.device)
+    return Q, w, q_seq, q_pos
+
+
+def hisa_select_workspace_bytes(kv: KVCache, n_q: int, H: int, m: int, k: int) -> int:
+    return int(_lib.hisa_select_workspace_bytes(kv.struct, n_q, H, m, k))
+
+
+def dsa_flat_workspace_bytes(kv: KVCache, n_q: int, H: int, k: int) -> int:
+    return int(_lib.dsa_flat_workspace_bytes(kv.struct, n_q, H, k))
+
+
+def workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """A caller-owned workspace buffer (256-byte aligned by the allocator)."""
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def hisa_select(kv: KVCache, Q, w, q_seq, q_pos, m: int, k: int, want_scores: bool = False,
+                ws: Optional[torch.Tensor] = None, idx: Optional[torch.Tensor] = None,
+                scores: Optional[torch.Tensor] = None, stream=None):
+    """Two-stage HISA selection.  Returns idx [n_q, k] (and scores if asked)."""
+    Q, w, q_seq, q_pos = _queries(kv, Q, w, q_seq, q_pos)
+    n_q, H = Q.shape[0], Q.shape[1]
+    need = hisa_select_workspace_bytes(kv, n_q, H, m, k)
+    ws = workspace(need, kv.device) if ws is None else ws
+    idx = torch.empty((n_q, k), dtype=torch.int32, device=kv.device) if idx is None else idx
+    if want_scores and scores is None:
+        scores = torch.empty((n_q, k), dtype=torch.float32, device=kv.device)
+    _check("hisa_select", _lib.hisa_select(
+        kv.struct, _ptr(Q), _ptr(w), _ptr(q_seq), _ptr(q_pos), n_q, H, m, k, _ptr(idx),
+        _ptr(scores), _ptr(ws), ws.numel(), _stream(stream)))
+    return (idx, scores) if want_scores else idx
+
+
+def hisa_select_inspect(kv: KVCache, Q, w, q_seq, q_pos, m: int, k: int, stream=None):
+    """hisa_select plus kept blocks, their count and the per-row work counters."""
+    Q, w, q_seq, q_pos = _queries(kv, Q, w, q_seq, q_pos)
+    n_q, H = Q.shape[0], Q.shape[1]
+    mm = min(m, kv.nblk)
+    ws = workspace(hisa_select_workspace_bytes(kv, n_q, H, m, k), kv.device)
+    idx = torch.empty((n_q, k), dtype=torch.int32, device=kv.device)
+    scores = torch.empty((n_q, k), dtype=torch.float32, device=kv.device)
+    blocks = torch.empty((n_q, mm), dtype=torch.int32, device=kv.device)
+    nblocks = torch.empty(n_q, dtype=torch.int32, device=kv.device)
+    counts = torch.empty((n_q, 2), dtype=torch.int64, device=kv.device)
+    _check("hisa_select_inspect", _lib.hisa_select_inspect(
+        kv.struct, _ptr(Q), _ptr(w), _ptr(q_seq), _ptr(q_pos), n_q, H, m, k, _ptr(idx),
+        _ptr(scores), _ptr(blocks), _ptr(nblocks), _ptr(counts), _ptr(ws), ws.numel(),
+        _stream(stream)))
+    return dict(idx=idx, scores=scores, blocks=blocks, nblocks=nblocks, counts=counts)
+
+
+def dsa_flat_select(kv: KVCache, Q, w, q_seq, q_pos, k: int, want_scores: bool = False,
+                    ws: Optional[torch.Tensor] = None, idx: Optional[torch.Tensor] = None,
+                    scores: Optional[torch.Tensor] = None, stream=None):
+    """Flat indexer scan over every visible key.  Returns idx [n_q, k] (and scores)."""
+    Q, w, q_seq, q_pos = _queries(kv, Q, w, q_seq, q_pos)
+    n_q, H = Q.shape[0], Q.shape[1]
+    need = dsa_flat_workspace_bytes(kv, n_q, H, k)
+    ws = workspace(need, kv.device) if ws is None else ws
+    idx = torch.empty((n_q, k), dtype=torch.int32, device=kv.device) if idx is None else idx
+    if want_scores and scores is None:
+        scores = torch.empty((n_q, k), dtype=torch.float32, device=kv.device)
+    _check("dsa_flat_select", _lib.dsa_flat_select(
+        kv.struct, _ptr(Q), _ptr(w), _ptr(q_seq), _ptr(q_pos), n_q, H, k, _ptr(idx),
+        _ptr(scores), _ptr(ws), ws.numel(), _stream(stream)))
+    return (idx, scores) if want_scores else idx
+
+
+def hisa_topk_f32(x: torch.Tensor, k: int, stream=None) -> torch.Tensor:
+    """Top-k selection rule on fp32 rows (ties: lower index; ascending output, -1 pad)."""
+    x = x.to(torch.float32).contiguous()
+    rows, n = x.shape
+    idx = torch.empty((rows, k), dtype=torch.int32, device=x.device)
+    _check("hisa_topk_f32", _lib.hisa_topk_f32(_ptr(x), rows, n, k, _ptr(idx), _stream(stream)))
+    return idx
+
+
+def hisa_profile_enable(on: bool = True):
+    """Record CUDA events around every kernel the library launches."""
+    _check("hisa_profile_enable", _lib.hisa_profile_enable(1 if on else 0))
+
+
+def hisa_profile_read(reset: bool = True) -> dict:
+    """{phase: (milliseconds, launches)} accumulated since the last reset."""
+    ms = (ctypes.c_float * len(PHASES))()
+    n = (ctypes.c_int * len(PHASES))()
+    _check("hisa_profile_read", _lib.hisa_profile_read(ms, n, 1 if reset else 0))
+    return {name: (float(ms[i]), int(n[i])) for i, name in enumerate(PHASES)}

@@ -1,0 +1,489 @@
+// C ABI of the HISA indexer (include/hisa.h): argument checks, workspace
+// layout, TMA tensor maps and kernel launches.  No allocation happens here:
+// every buffer, scratch space included, belongs to the caller.
+#include <climits>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "hisa_kernels.cuh"
+
+using namespace hisa;
+
+namespace {
+
+// ------------------------------------------------------------- driver API
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D row-major tensor [rows, cols] with boxes of [box_rows, box_cols].
+bool make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, size_t elem, uint64_t rows,
+              uint64_t cols, uint32_t box_rows, uint32_t box_cols, CUtensorMapSwizzle sw) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * elem};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------- phase profiling
+
+struct PhaseEvents {
+    cudaEvent_t start, stop;
+    int phase;
+};
+
+struct Profiler {
+    std::mutex mu;
+    bool on = false;
+    std::vector<PhaseEvents> pending;   // recorded since the last read
+    std::vector<cudaEvent_t> spare;     // reusable events
+
+    cudaEvent_t take() {
+        if (!spare.empty()) {
+            cudaEvent_t e = spare.back();
+            spare.pop_back();
+            return e;
+        }
+        cudaEvent_t e = nullptr;
+        cudaEventCreate(&e);
+        return e;
+    }
+};
+
+Profiler& profiler() {
+    static Profiler p;
+    return p;
+}
+
+// Records an event pair around one kernel launch while profiling is on.
+struct PhaseScope {
+    int phase;
+    cudaStream_t s;
+    cudaEvent_t stop = nullptr;
+    PhaseScope(int ph, cudaStream_t st) : phase(ph), s(st) {
+        Profiler& P = profiler();
+        std::lock_guard<std::mutex> g(P.mu);
+        if (!P.on) return;
+        cudaEvent_t start = P.take();
+        stop = P.take();
+        if (!start || !stop) {
+            stop = nullptr;
+            return;
+        }
+        cudaEventRecord(start, s);
+        P.pending.push_back({start, stop, phase});
+    }
+    ~PhaseScope() {
+        if (stop) cudaEventRecord(stop, s);
+    }
+};
+
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return n;
+}
+
+// ------------------------------------------------------------- validation
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int check_kv(const hisa_kv* kv, KvView* v) {
+    if (!kv || !kv->keys || !kv->pooled || !kv->pooled_hl || !kv->len) return HISA_E_INVAL;
+    if (kv->batch < 1 || kv->cap < 1 || kv->B < 1) return HISA_E_INVAL;
+    if (kv->dtype != HISA_KEY_BF16 && kv->dtype != HISA_KEY_E4M3) return HISA_E_INVAL;
+    if (kv->d != 64 && kv->d != 128) return HISA_E_UNSUPPORTED;
+    const bool e4m3 = kv->dtype == HISA_KEY_E4M3;
+    if (e4m3 && !kv->key_scale) return HISA_E_INVAL;
+    if (!aligned(kv->keys, 16) || !aligned(kv->pooled, 16) || !aligned(kv->pooled_hl, 16) ||
+        !aligned(kv->len, 4) || (kv->key_scale && !aligned(kv->key_scale, 4)) ||
+        (kv->status && !aligned(kv->status, 4)))
+        return HISA_E_INVAL;
+    if (static_cast<long long>(kv->batch) * kv->cap > INT_MAX) return HISA_E_UNSUPPORTED;
+    v->keys = kv->keys;
+    v->key_scale = kv->key_scale;
+    v->pooled = kv->pooled;
+    v->pooled_hl = kv->pooled_hl;
+    v->len = kv->len;
+    v->status = kv->status;
+    v->batch = kv->batch;
+    v->cap = kv->cap;
+    v->d = kv->d;
+    v->B = kv->B;
+    v->nblk = (kv->cap + kv->B - 1) / kv->B;
+    v->e4m3 = e4m3;
+    return HISA_OK;
+}
+
+bool select_block_size_ok(int B) {
+    if (B == 8 || B == 16 || B == 32 || B == 64) return true;
+    return B >= 128 && B <= 1024 && B % 128 == 0;
+}
+
+int check_queries(const uint16_t* Q, const float* w, const int32_t* q_seq, int n_q, int H, int k,
+                  const int32_t* idx) {
+    if (n_q < 0 || k < 1) return HISA_E_INVAL;
+    if (H < 1 || H > 128) return HISA_E_UNSUPPORTED;
+    if (n_q == 0) return HISA_OK;
+    if (!Q || !w || !q_seq || !idx) return HISA_E_INVAL;
+    if (!aligned(Q, 16) || !aligned(w, 4) || !aligned(q_seq, 4) || !aligned(idx, 4))
+        return HISA_E_INVAL;
+    return HISA_OK;
+}
+
+int npad_of(int H) { return (H + 15) / 16 * 16; }
+
+// Workspace carving: consecutive 256-byte aligned regions.
+struct Carve {
+    size_t off = 0;
+    size_t take(size_t bytes) {
+        const size_t o = off;
+        off = round_up(off + bytes, 256);
+        return o;
+    }
+};
+
+struct HisaWs {
+    size_t bkeys, blocks, nblocks, tkeys, total;
+    int ldb, ldt, mm;
+};
+
+HisaWs hisa_ws(const KvView& v, int n_q, int m) {
+    HisaWs w;
+    w.mm = m < v.nblk ? m : v.nblk;
+    w.ldb = static_cast<int>(round_up(v.nblk, 128));
+    w.ldt = static_cast<int>(round_up(static_cast<size_t>(w.mm) * v.B, 128));
+    Carve c;
+    w.bkeys = c.take(static_cast<size_t>(n_q) * w.ldb * 4);
+    w.blocks = c.take(static_cast<size_t>(n_q) * w.mm * 4);
+    w.nblocks = c.take(static_cast<size_t>(n_q) * 4);
+    w.tkeys = c.take(static_cast<size_t>(n_q) * w.ldt * 4);
+    w.total = c.off;
+    return w;
+}
+
+size_t flat_ld(const KvView& v) { return round_up(v.cap, 128); }
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? HISA_OK : HISA_E_CUDA; }
+
+bool keys_map(CUtensorMap* map, const KvView& v, int box_rows) {
+    const uint64_t rows = static_cast<uint64_t>(v.batch) * v.cap;
+    if (v.e4m3)
+        return make_map(map, v.keys, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows, v.d, box_rows, v.d,
+                        CU_TENSOR_MAP_SWIZZLE_NONE);
+    return make_map(map, v.keys, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, v.d, box_rows, 64,
+                    CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+bool query_map(CUtensorMap* map, const uint16_t* Q, int n_q, int H, int d) {
+    return make_map(map, Q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, static_cast<uint64_t>(n_q) * H, d,
+                    npad_of(H), 64, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+ScoreParams score_params(const KvView& v, const float* w, const int32_t* q_seq, const int32_t* q_pos,
+                         int n_q, int H) {
+    ScoreParams p;
+    std::memset(&p, 0, sizeof p);
+    p.len = v.len;
+    p.key_scale = v.key_scale;
+    p.status = v.status;
+    p.batch = v.batch;
+    p.cap = v.cap;
+    p.nblk = v.nblk;
+    p.B = v.B;
+    p.w = w;
+    p.q_seq = q_seq;
+    p.q_pos = q_pos;
+    p.n_q = n_q;
+    p.H = H;
+    p.npad = npad_of(H);
+    return p;
+}
+
+int run_score(int mode, const KvView& v, const CUtensorMap& amap, const CUtensorMap& qmap,
+              ScoreParams& p, cudaStream_t s) {
+    p.stages = score_stages(mode, mode != kScoreBlocks && v.e4m3, v.d, p.npad);
+    if (p.stages < 2) return HISA_E_UNSUPPORTED;
+    p.total_tiles = static_cast<long long>(p.n_q) * p.tiles_per_row;
+    if (p.total_tiles == 0) return HISA_OK;
+    const int sms = sm_count();
+    if (sms <= 0) return HISA_E_CUDA;
+    const int grid = static_cast<int>(p.total_tiles < sms ? p.total_tiles : sms);
+    const int phase = mode == kScoreBlocks ? HISA_PHASE_BLOCK_SCORE
+                      : mode == kScoreFlat ? HISA_PHASE_FLAT_SCORE
+                                           : HISA_PHASE_TOKEN_SCORE;
+    PhaseScope ps(phase, s);
+    return cuda_status(launch_score(mode, mode != kScoreBlocks && v.e4m3, v.d, amap, qmap, p, grid, s));
+}
+
+int hisa_select_impl(const hisa_kv* kv, const uint16_t* Q, const float* w, const int32_t* q_seq,
+                     const int32_t* q_pos, int n_q, int H, int m, int k, int32_t* idx, float* scores,
+                     int32_t* blocks_out, int32_t* nblocks_out, uint64_t* counts, void* ws,
+                     size_t ws_bytes, cudaStream_t s) {
+    KvView v;
+    int rc = check_kv(kv, &v);
+    if (rc) return rc;
+    if (!select_block_size_ok(v.B)) return HISA_E_UNSUPPORTED;
+    if (m < 1) return HISA_E_INVAL;
+    rc = check_queries(Q, w, q_seq, n_q, H, k, idx);
+    if (rc) return rc;
+    if (n_q == 0) return HISA_OK;
+    const HisaWs L = hisa_ws(v, n_q, m);
+    if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return HISA_E_WORKSPACE;
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    uint32_t* bkeys = reinterpret_cast<uint32_t*>(base + L.bkeys);
+    int32_t* blocks = reinterpret_cast<int32_t*>(base + L.blocks);
+    int32_t* nblocks = reinterpret_cast<int32_t*>(base + L.nblocks);
+    uint32_t* tkeys = reinterpret_cast<uint32_t*>(base + L.tkeys);
+
+    CUtensorMap pmap, kmap, qmap;
+    const int br = v.B < 128 ? v.B : 128;
+    if (!make_map(&pmap, v.pooled_hl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  static_cast<uint64_t>(v.batch) * v.nblk, 2 * v.d, 128, 64,
+                  CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !keys_map(&kmap, v, br) || !query_map(&qmap, Q, n_q, H, v.d))
+        return HISA_E_CUDA;
+
+    if (counts && cudaMemsetAsync(counts, 0, sizeof(uint64_t) * 2 * n_q, s) != cudaSuccess)
+        return HISA_E_CUDA;
+
+    // stage 1: score the block representatives, keep the top-m blocks
+    ScoreParams p = score_params(v, w, q_seq, q_pos, n_q, H);
+    p.out = bkeys;
+    p.ldo = L.ldb;
+    p.tiles_per_row = L.ldb / 128;
+    p.counts = reinterpret_cast<unsigned long long*>(counts);
+    rc = run_score(kScoreBlocks, v, pmap, qmap, p, s);
+    if (rc) return rc;
+
+    SelectParams sp;
+    std::memset(&sp, 0, sizeof sp);
+    sp.mode = kSelBlocks;
+    sp.keys = bkeys;
+    sp.ldk = L.ldb;
+    sp.rows = n_q;
+    sp.k = k;
+    sp.len = v.len;
+    sp.q_seq = q_seq;
+    sp.q_pos = q_pos;
+    sp.status = v.status;
+    sp.batch = v.batch;
+    sp.cap = v.cap;
+    sp.B = v.B;
+    sp.m = m;
+    sp.mm = L.mm;
+    sp.blocks = blocks;
+    sp.nblocks = nblocks;
+    sp.blocks_out = blocks_out;
+    sp.nblocks_out = nblocks_out;
+    {
+        PhaseScope ps(HISA_PHASE_BLOCK_SELECT, s);
+        rc = cuda_status(launch_select(sp, v.nblk, s));
+    }
+    if (rc) return rc;
+
+    // stage 2: score the kept blocks' tokens, keep the top-k tokens
+    p.out = tkeys;
+    p.ldo = L.ldt;
+    p.tiles_per_row = L.ldt / 128;
+    p.blocks = blocks;
+    p.nblocks = nblocks;
+    p.mm = L.mm;
+    rc = run_score(kScoreHisa, v, kmap, qmap, p, s);
+    if (rc) return rc;
+
+    sp.mode = kSelHisaTokens;
+    sp.keys = tkeys;
+    sp.ldk = L.ldt;
+    sp.idx = idx;
+    sp.scores = scores;
+    sp.blocks_out = nullptr;
+    sp.nblocks_out = nullptr;
+    PhaseScope ps(HISA_PHASE_TOKEN_SELECT, s);
+    return cuda_status(launch_select(sp, L.mm * v.B, s));
+}
+
+}  // namespace
+
+extern "C" {
+
+int hisa_pool_blocks(const hisa_kv* kv, hisa_stream_t stream) {
+    KvView v;
+    const int rc = check_kv(kv, &v);
+    if (rc) return rc;
+    PhaseScope ps(HISA_PHASE_POOL, reinterpret_cast<cudaStream_t>(stream));
+    return cuda_status(launch_pool(v, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int hisa_append(const hisa_kv* kv, const void* tok, const float* tok_scale, hisa_stream_t stream) {
+    KvView v;
+    const int rc = check_kv(kv, &v);
+    if (rc) return rc;
+    if (!tok || !aligned(tok, 16)) return HISA_E_INVAL;
+    if (v.e4m3 && (!tok_scale || !aligned(tok_scale, 4))) return HISA_E_INVAL;
+    PhaseScope ps(HISA_PHASE_APPEND, reinterpret_cast<cudaStream_t>(stream));
+    return cuda_status(launch_append(v, tok, tok_scale, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t hisa_select_workspace_bytes(const hisa_kv* kv, int n_q, int H, int m, int k) {
+    (void)H;
+    (void)k;
+    KvView v;
+    if (check_kv(kv, &v) || n_q < 0 || m < 1) return 0;
+    return hisa_ws(v, n_q, m).total;
+}
+
+int hisa_select(const hisa_kv* kv, const uint16_t* Q, const float* w, const int32_t* q_seq,
+                const int32_t* q_pos, int n_q, int H, int m, int k, int32_t* idx, float* scores,
+                void* ws, size_t ws_bytes, hisa_stream_t stream) {
+    return hisa_select_impl(kv, Q, w, q_seq, q_pos, n_q, H, m, k, idx, scores, nullptr, nullptr,
+                            nullptr, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int hisa_select_inspect(const hisa_kv* kv, const uint16_t* Q, const float* w, const int32_t* q_seq,
+                        const int32_t* q_pos, int n_q, int H, int m, int k, int32_t* idx,
+                        float* scores, int32_t* blocks, int32_t* nblocks, uint64_t* counts, void* ws,
+                        size_t ws_bytes, hisa_stream_t stream) {
+    return hisa_select_impl(kv, Q, w, q_seq, q_pos, n_q, H, m, k, idx, scores, blocks, nblocks,
+                            counts, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t dsa_flat_workspace_bytes(const hisa_kv* kv, int n_q, int H, int k) {
+    (void)H;
+    (void)k;
+    KvView v;
+    if (check_kv(kv, &v) || n_q < 0) return 0;
+    Carve c;
+    c.take(static_cast<size_t>(n_q) * flat_ld(v) * 4);
+    return c.off;
+}
+
+int dsa_flat_select(const hisa_kv* kv, const uint16_t* Q, const float* w, const int32_t* q_seq,
+                    const int32_t* q_pos, int n_q, int H, int k, int32_t* idx, float* scores, void* ws,
+                    size_t ws_bytes, hisa_stream_t stream) {
+    KvView v;
+    int rc = check_kv(kv, &v);
+    if (rc) return rc;
+    if (!select_block_size_ok(v.B)) return HISA_E_UNSUPPORTED;
+    rc = check_queries(Q, w, q_seq, n_q, H, k, idx);
+    if (rc) return rc;
+    if (n_q == 0) return HISA_OK;
+    const size_t ld = flat_ld(v);
+    if (!ws || !aligned(ws, 256) || ws_bytes < dsa_flat_workspace_bytes(kv, n_q, H, k))
+        return HISA_E_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    CUtensorMap kmap, qmap;
+    if (!keys_map(&kmap, v, v.B < 128 ? v.B : 128) || !query_map(&qmap, Q, n_q, H, v.d))
+        return HISA_E_CUDA;
+    uint32_t* keys = static_cast<uint32_t*>(ws);
+    ScoreParams p = score_params(v, w, q_seq, q_pos, n_q, H);
+    p.out = keys;
+    p.ldo = static_cast<int>(ld);
+    p.tiles_per_row = static_cast<int>(ld / 128);
+    rc = run_score(kScoreFlat, v, kmap, qmap, p, s);
+    if (rc) return rc;
+    SelectParams sp;
+    std::memset(&sp, 0, sizeof sp);
+    sp.mode = kSelFlatTokens;
+    sp.keys = keys;
+    sp.ldk = static_cast<int>(ld);
+    sp.rows = n_q;
+    sp.k = k;
+    sp.len = v.len;
+    sp.q_seq = q_seq;
+    sp.q_pos = q_pos;
+    sp.status = v.status;
+    sp.batch = v.batch;
+    sp.cap = v.cap;
+    sp.B = v.B;
+    sp.idx = idx;
+    sp.scores = scores;
+    PhaseScope ps(HISA_PHASE_FLAT_SELECT, s);
+    return cuda_status(launch_select(sp, v.cap, s));
+}
+
+int hisa_topk_f32(const float* x, int rows, int n, int k, int32_t* idx, hisa_stream_t stream) {
+    if (rows < 0 || n < 0 || k < 1) return HISA_E_INVAL;
+    if (rows == 0) return HISA_OK;
+    if (!x || !idx || !aligned(x, 4) || !aligned(idx, 4)) return HISA_E_INVAL;
+    SelectParams sp;
+    std::memset(&sp, 0, sizeof sp);
+    sp.mode = kSelF32Rows;
+    sp.x = x;
+    sp.n = n;
+    sp.rows = rows;
+    sp.k = k;
+    sp.idx = idx;
+    PhaseScope ps(HISA_PHASE_TOPK, reinterpret_cast<cudaStream_t>(stream));
+    return cuda_status(launch_select(sp, n, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int hisa_profile_enable(int on) {
+    Profiler& P = profiler();
+    std::lock_guard<std::mutex> g(P.mu);
+    P.on = on != 0;
+    return HISA_OK;
+}
+
+int hisa_profile_read(float* ms, int* launches, int reset) {
+    Profiler& P = profiler();
+    std::lock_guard<std::mutex> g(P.mu);
+    if (ms)
+        for (int i = 0; i < HISA_NUM_PHASES; ++i) ms[i] = 0.f;
+    if (launches)
+        for (int i = 0; i < HISA_NUM_PHASES; ++i) launches[i] = 0;
+    int rc = HISA_OK;
+    for (const PhaseEvents& e : P.pending) {
+        float t = 0.f;
+        if (cudaEventSynchronize(e.stop) != cudaSuccess || cudaEventElapsedTime(&t, e.start, e.stop) != cudaSuccess)
+            rc = HISA_E_CUDA;
+        if (ms) ms[e.phase] += t;
+        if (launches) launches[e.phase] += 1;
+    }
+    if (reset) {
+        for (const PhaseEvents& e : P.pending) {
+            P.spare.push_back(e.start);
+            P.spare.push_back(e.stop);
+        }
+        P.pending.clear();
+    }
+    return rc;
+}
+
+const char* hisa_status_string(int code) {
+    switch (code) {
+        case HISA_OK: return "ok";
+        case HISA_E_INVAL: return "invalid argument";
+        case HISA_E_UNSUPPORTED: return "unsupported size";
+        case HISA_E_WORKSPACE: return "workspace too small or misaligned";
+        case HISA_E_CUDA: return "CUDA error";
+        default: return "unknown status";
+    }
+}
+
+}  // extern "C"

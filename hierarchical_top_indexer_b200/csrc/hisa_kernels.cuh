@@ -1,0 +1,95 @@
+// Internal interface between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include "hisa_device.cuh"
+
+namespace hisa {
+
+// The cache as the kernels see it (validated copy of hisa_kv).
+struct KvView {
+    void* keys;
+    float* key_scale;
+    float* pooled;
+    uint16_t* pooled_hl;
+    int32_t* len;
+    uint32_t* status;
+    int batch, cap, d, B, nblk;
+    bool e4m3;
+};
+
+// What a scoring launch scores.
+enum ScoreMode : int {
+    kScoreBlocks = 0,   // block representatives (pooled_hl), candidates j < nb(t)
+    kScoreFlat = 1,     // every key s <= t
+    kScoreHisa = 2      // the keys of each row's kept blocks
+};
+
+struct ScoreParams {
+    // cache
+    const int32_t* len;
+    const float* key_scale;
+    uint32_t* status;
+    int batch, cap, nblk, B;
+    // query rows
+    const float* w;
+    const int32_t* q_seq;
+    const int32_t* q_pos;
+    int n_q, H, npad;
+    // kept blocks (kScoreHisa): blocks [n_q, mm], nblocks [n_q]
+    const int32_t* blocks;
+    const int32_t* nblocks;
+    int mm;
+    // output: order-preserving score keys [n_q, ldo]; 0 = masked slot
+    uint32_t* out;
+    int ldo;
+    unsigned long long* counts;   // [n_q, 2] or null
+    int tiles_per_row;
+    long long total_tiles;
+    int stages;
+};
+
+enum SelectMode : int {
+    kSelBlocks = 0,      // keep own block + best m-1 others -> blocks list
+    kSelHisaTokens = 1,  // keep top-k of the kept blocks' token slots
+    kSelFlatTokens = 2,  // keep top-k of keys 0..t
+    kSelF32Rows = 3      // keep top-k of n given fp32 values per row
+};
+
+struct SelectParams {
+    int mode;
+    const uint32_t* keys;   // [rows, ldk] score keys (modes 0-2)
+    const float* x;         // [rows, n] fp32 (mode 3)
+    int ldk, n;
+    int rows, k;
+    // query rows (modes 0-2)
+    const int32_t* len;
+    const int32_t* q_seq;
+    const int32_t* q_pos;
+    uint32_t* status;
+    int batch, cap, B, m, mm;
+    // kept blocks: written by mode 0, read by mode 1
+    int32_t* blocks;
+    int32_t* nblocks;
+    // outputs
+    int32_t* idx;       // [rows, k]   (modes 1-3)
+    float* scores;      // [rows, k] or null
+    int32_t* blocks_out;     // [rows, mm] or null (mode 0 copy for inspection)
+    int32_t* nblocks_out;    // [rows] or null
+};
+
+cudaError_t launch_pool(const KvView& kv, cudaStream_t s);
+cudaError_t launch_append(const KvView& kv, const void* tok, const float* tok_scale,
+                          cudaStream_t s);
+
+// Scoring: tensor maps built by the caller.  `keys_map` covers keys
+// ([batch*cap, d], bf16 swizzled 128B boxes, or e4m3 plain boxes) or, for
+// kScoreBlocks, pooled_hl ([batch*nblk, 2d] bf16).
+int score_stages(int mode, bool e4m3, int d, int npad);
+size_t score_smem_bytes(int mode, bool e4m3, int d, int npad, int stages);
+cudaError_t launch_score(int mode, bool e4m3, int d, const CUtensorMap& keys_map,
+                         const CUtensorMap& q_map, const ScoreParams& p, int grid,
+                         cudaStream_t s);
+
+cudaError_t launch_select(const SelectParams& p, int max_n, cudaStream_t s);
+
+}  // namespace hisa

@@ -1,0 +1,231 @@
+/*
+ * hisa.h — C ABI of the HISA hierarchical top-k indexer for B200 (sm_100a).
+ *
+ * HISA (HISA: Efficient Hierarchical Indexing for Fine-Grained Sparse
+ * Attention; gptget.net English summary, "Methodology"; Chinese summary,
+ * "方法详解" method details; arXiv abstract) replaces the flat indexer scan of
+ * token-level sparse attention with two stages:
+ *   1. block-level coarse filter: the key prefix is cut into contiguous
+ *      blocks of B tokens, each block is mean-pooled into a representative,
+ *      the representatives are scored with the same indexer and the top-m
+ *      blocks are kept;
+ *   2. token-level refinement: the m*B tokens of the kept blocks are scored
+ *      with the indexer and the exact top-k token indices are emitted for the
+ *      downstream sparse attention operator.
+ * The flat scan it replaces (blog "Hierarchical Indexing Makes Sparse
+ * Attention Actually Fast", "How Fine-Grained Sparse Attention Works Today")
+ * scores every prefix token and keeps the top-k; it is exported as
+ * dsa_flat_select for comparison.
+ *
+ * Indexer score of key x for query row i (H indexer heads, head dim d):
+ *     score(i, x) = sum_h w[i,h] * max(0, q[i,h,:] . x)
+ * Keys are visible to a query at position t iff their position s <= t.
+ * The block holding t is always kept and counts inside m.  Ties go to the
+ * lower token index (and the lower block id).
+ *
+ * Conventions for every entry point
+ *   - All array arguments are DEVICE pointers to caller-owned memory, unless
+ *     stated otherwise.  The library allocates nothing: scratch space is the
+ *     caller's workspace buffer (size from the *_workspace_bytes queries).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream).  The return value only reports argument checks and
+ *     launch errors.  Conditions found on the device (a query position
+ *     outside its sequence, an append past capacity, a bounded wait that ran
+ *     out) set bits in the cache's device status word; read it after the
+ *     stream has synchronised.
+ *   - Calls that share a cache or workspace must be ordered on one stream.
+ *   - Arrays are row-major and densely packed.  Pointers must be 16-byte
+ *     aligned; the workspace must be 256-byte aligned.
+ */
+#ifndef HISA_H_
+#define HISA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* hisa_stream_t;   /* same handle as cudaStream_t */
+
+/* Key storage formats. */
+enum hisa_key_dtype {
+    HISA_KEY_BF16 = 0,   /* bf16 keys */
+    HISA_KEY_E4M3 = 1    /* OCP e4m3 codes + one fp32 scale (> 0) per token;
+                            the key value is fp32(e4m3 value * scale) */
+};
+
+/* Return codes. */
+enum hisa_status {
+    HISA_OK = 0,
+    HISA_E_INVAL = 1,        /* a NULL, misaligned or out-of-range argument */
+    HISA_E_UNSUPPORTED = 2,  /* a size outside the built kernels (d, B, H) */
+    HISA_E_WORKSPACE = 3,    /* workspace too small or misaligned */
+    HISA_E_CUDA = 4          /* a CUDA call or launch failed */
+};
+
+/* Bits of the device status word (sticky: the library only ORs bits in). */
+#define HISA_DEV_BAD_QUERY 0x1u  /* a query's position is not inside its prefix;
+                                    that row's output is all -1 */
+#define HISA_DEV_CAPACITY  0x2u  /* hisa_append found len == cap; nothing appended
+                                    for that sequence */
+#define HISA_DEV_BAD_LEN   0x4u  /* a len[] entry outside [0, cap] */
+#define HISA_DEV_TIMEOUT   0x8u  /* a bounded in-kernel wait ran out; outputs of
+                                    that launch are undefined */
+
+/*
+ * The indexer key cache and its block index ("hierarchical index").
+ *
+ *   keys       [batch, cap, d]   bf16, or e4m3 bytes (dtype)
+ *   key_scale  [batch, cap]      fp32 > 0, E4M3 only (NULL for BF16)
+ *   pooled     [batch, nblk, d]  fp32 block means, nblk = ceil(cap / B)
+ *   pooled_hl  [batch, nblk, 2*d] bf16: row j holds hi = bf16(pooled[j])
+ *                                 then lo = bf16(pooled[j] - hi), the
+ *                                 tensor-core form of the block means
+ *   len        [batch]           int32 valid prefix length per sequence
+ *   status     [1]               uint32 device status word (see HISA_DEV_*)
+ *
+ * Block representatives are the means of the visible keys of each block
+ * (HISA Methodology: mean pooling generates the block representatives).  The
+ * trailing partial block is the mean of its len - j*B valid keys.
+ *
+ * Sizes: d in {64, 128}.  Pooling and append take any B >= 1; the select
+ * calls need B in {8, 16, 32, 64} or a multiple of 128 up to 1024.
+ */
+typedef struct hisa_kv {
+    void* keys;
+    float* key_scale;
+    float* pooled;
+    uint16_t* pooled_hl;
+    int32_t* len;
+    uint32_t* status;
+    int32_t batch;
+    int32_t cap;
+    int32_t d;
+    int32_t B;
+    int32_t dtype;   /* enum hisa_key_dtype */
+} hisa_kv;
+
+/*
+ * hisa_pool_blocks — build the block index from scratch.
+ * HISA Chinese summary, method details (first step): the length-L prefix is
+ * split into contiguous blocks of size B and each block is mean-pooled.
+ * For every sequence b and block j with j*B < len[b], writes pooled[b, j, :]
+ * (fp32 mean of keys j*B .. min((j+1)*B, len[b]) - 1, summed in fp32) and
+ * pooled_hl[b, j, :].  Rows of blocks at or past len[b] are not written.
+ * One streaming pass over the keys.
+ */
+int hisa_pool_blocks(const hisa_kv* kv, hisa_stream_t stream);
+
+/*
+ * hisa_append — append one key per sequence and keep the index current.
+ * Blog "Hierarchical Indexing Makes Sparse Attention Actually Fast", "HISA's
+ * Approach": the summary structure is maintained incrementally as tokens are
+ * appended.  In the two-stage form only the trailing block changes.
+ *   tok        [batch, d]  the new key rows (bf16 or e4m3, as kv->dtype)
+ *   tok_scale  [batch]     fp32 scales (E4M3) or NULL
+ * For each sequence b with len[b] < cap: writes the key at position len[b],
+ * recomputes the trailing block's mean over its valid keys (O(B*d) work, the
+ * same arithmetic as hisa_pool_blocks, so the result equals a full re-pool
+ * bit for bit), then len[b] += 1.  A full sequence sets HISA_DEV_CAPACITY and
+ * is left unchanged.
+ */
+int hisa_append(const hisa_kv* kv, const void* tok, const float* tok_scale,
+                hisa_stream_t stream);
+
+/*
+ * hisa_select — the two-stage HISA selection for n_q query rows.
+ * HISA arXiv abstract, stages (1) and (2); gptget.net summary, "Methodology"
+ * (top-m blocks by pooled score, then token scoring inside them); Chinese
+ * summary, method details (the final k tokens feed sparse attention).
+ *   Q      [n_q, H, d] bf16  indexer queries
+ *   w      [n_q, H]    fp32  per-row head weights
+ *   q_seq  [n_q]       int32 sequence of each row
+ *   q_pos  [n_q]       int32 position t of each row (keys s <= t visible);
+ *                            NULL = each row's last position len[q_seq] - 1
+ *   m      blocks kept per row (the own block included); m >= #blocks keeps
+ *          every block, which makes the result equal dsa_flat_select
+ *   k      tokens kept per row
+ *   idx    [n_q, k] int32 out: selected positions within the row's sequence,
+ *          ascending, then -1 padding when fewer than k are visible
+ *   scores [n_q, k] fp32 out (or NULL): the indexer score of each idx entry
+ *          (NaN under -1 padding)
+ *   ws     workspace of at least hisa_select_workspace_bytes(...) bytes
+ * H in 1..128.  The pooled index must be current for every row (built by
+ * hisa_pool_blocks / hisa_append); the own block's representative may cover
+ * keys past t — it is kept whatever its score.
+ */
+size_t hisa_select_workspace_bytes(const hisa_kv* kv, int n_q, int H, int m, int k);
+int hisa_select(const hisa_kv* kv, const uint16_t* Q, const float* w, const int32_t* q_seq,
+                const int32_t* q_pos, int n_q, int H, int m, int k, int32_t* idx,
+                float* scores, void* ws, size_t ws_bytes, hisa_stream_t stream);
+
+/*
+ * hisa_select_inspect — hisa_select plus its intermediate results, for
+ * verification of the two stages separately.
+ *   blocks  [n_q, min(m, nblk)] int32 out (or NULL): kept block ids per row,
+ *           ascending, -1 padded
+ *   nblocks [n_q] int32 out (or NULL): number of kept blocks per row
+ *   counts  [n_q, 2] uint64 out (or NULL), zeroed by the call: per row the
+ *           number of block representatives scored and of token slots scored
+ *           (HISA Methodology: O(L/B + mB) indexer work per query)
+ */
+int hisa_select_inspect(const hisa_kv* kv, const uint16_t* Q, const float* w,
+                        const int32_t* q_seq, const int32_t* q_pos, int n_q, int H, int m,
+                        int k, int32_t* idx, float* scores, int32_t* blocks, int32_t* nblocks,
+                        uint64_t* counts, void* ws, size_t ws_bytes, hisa_stream_t stream);
+
+/*
+ * dsa_flat_select — the flat indexer scan HISA replaces: every visible key
+ * s <= t is scored and the top-k kept (blog "How Fine-Grained Sparse
+ * Attention Works Today"; HISA abstract: the indexer scans the entire
+ * prefix).  Arguments as hisa_select without m.  Scores come from the same
+ * scoring kernel as hisa_select, so both paths give the same fp32 score to
+ * the same key.
+ */
+size_t dsa_flat_workspace_bytes(const hisa_kv* kv, int n_q, int H, int k);
+int dsa_flat_select(const hisa_kv* kv, const uint16_t* Q, const float* w, const int32_t* q_seq,
+                    const int32_t* q_pos, int n_q, int H, int k, int32_t* idx, float* scores,
+                    void* ws, size_t ws_bytes, hisa_stream_t stream);
+
+/*
+ * hisa_topk_f32 — the selection rule alone: for each of `rows` rows of n
+ * fp32 values x[r, :], the k largest (ties: lower index), indices ascending
+ * then -1 padding, into idx[rows, k].  NaN inputs are not allowed; -0.0 and
+ * +0.0 are equal.  The same routine selects blocks and tokens inside
+ * hisa_select and dsa_flat_select (HISA Chinese summary, method details:
+ * final k tokens; gptget.net summary: top-m blocks).
+ */
+int hisa_topk_f32(const float* x, int rows, int n, int k, int32_t* idx, hisa_stream_t stream);
+
+/*
+ * Phase timing for measurement tools (no counterpart on the pages).  While
+ * enabled, every call records a CUDA event pair around each kernel it
+ * launches, on the call's stream.  hisa_profile_read waits for the recorded
+ * events, adds up their durations per phase (milliseconds) and launch counts,
+ * and with reset != 0 starts a new accumulation.  Phases:
+ */
+enum hisa_phase {
+    HISA_PHASE_BLOCK_SCORE = 0,   /* stage 1: score block representatives */
+    HISA_PHASE_BLOCK_SELECT = 1,  /* stage 1: keep top-m blocks */
+    HISA_PHASE_TOKEN_SCORE = 2,   /* stage 2: gather + score candidate tokens */
+    HISA_PHASE_TOKEN_SELECT = 3,  /* stage 2: keep top-k tokens */
+    HISA_PHASE_FLAT_SCORE = 4,    /* flat scan: score every visible token */
+    HISA_PHASE_FLAT_SELECT = 5,   /* flat scan: keep top-k */
+    HISA_PHASE_POOL = 6,          /* hisa_pool_blocks */
+    HISA_PHASE_APPEND = 7,        /* hisa_append */
+    HISA_PHASE_TOPK = 8,          /* hisa_topk_f32 */
+    HISA_NUM_PHASES = 9
+};
+int hisa_profile_enable(int on);
+int hisa_profile_read(float* ms, int* launches, int reset);
+
+/* Human-readable name of a return code. */
+const char* hisa_status_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HISA_H_ */

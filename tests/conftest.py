@@ -25,3 +25,15 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+def pytest_sessionstart(session):
+    """Build the CUDA library and the oracle if their sources are newer."""
+    import importlib.util
+    import shutil
+    path = os.path.join(ROOT, "hierarchical_top_indexer_b200", "build.py")
+    spec = importlib.util.spec_from_file_location("hisa_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    if mod.stale() and (os.path.exists(mod.NVCC) or shutil.which(mod.NVCC)):
+        mod.build()

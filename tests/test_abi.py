@@ -1,0 +1,118 @@
+"""The C-ABI library builds, loads and exports what include/hisa.h declares,
+and its host-side argument checks reject bad calls before touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hisa.h")
+
+
+def build_module():
+    """The build script, loaded by path (importing the package needs the library)."""
+    import importlib.util
+    path = os.path.join(ROOT, "hierarchical_top_indexer_b200", "build.py")
+    spec = importlib.util.spec_from_file_location("hisa_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+@pytest.fixture(scope="module")
+def hisa():
+    build = build_module()
+    if build.stale():
+        build.build()
+    import hierarchical_top_indexer_b200 as h
+    return h
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(\w+)\s*\(", text, flags=re.M)
+    return sorted(set(n for n in names if n.startswith(("hisa_", "dsa_"))))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for fn in ("hisa_pool_blocks", "hisa_append", "hisa_select", "dsa_flat_select"):
+        assert fn in names
+
+
+def test_library_exports_every_declared_symbol(hisa):
+    lib = ctypes.CDLL(hisa.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in hisa.h but not exported"
+    assert set(hisa.EXPORTS) <= set(declared_functions())
+
+
+def test_library_has_no_link_time_dependency_on_the_driver(hisa):
+    # The driver API is reached through cudaGetDriverEntryPoint, so the
+    # library loads on machines without libcuda (like this one).
+    import subprocess
+    out = subprocess.run(["ldd", hisa.LIB_PATH], capture_output=True, text=True).stdout
+    assert "libcuda.so" not in out
+
+
+def test_status_strings(hisa):
+    lib = hisa.lib()
+    assert lib.hisa_status_string(0) == b"ok"
+    assert lib.hisa_status_string(3).startswith(b"workspace")
+    assert lib.hisa_status_string(99) == b"unknown status"
+
+
+def _kv(hisa, **over):
+    fields = dict(keys=16, key_scale=None, pooled=32, pooled_hl=48, len=64, status=128,
+                  batch=1, cap=1024, d=128, B=128, dtype=0)
+    fields.update(over)
+    return hisa.hisa_kv(**fields)
+
+
+def test_argument_checks_reject_before_any_launch(hisa):
+    lib = hisa.lib()
+    kv = _kv(hisa)
+    P = ctypes.c_void_p
+    good = dict(Q=P(16), w=P(16), q_seq=P(16), idx=P(16))
+    # NULL cache, bad sizes, missing pointers, unsupported d / B / H
+    assert lib.hisa_pool_blocks(None, None) == hisa.HISA_E_INVAL
+    assert lib.hisa_pool_blocks(ctypes.byref(_kv(hisa, batch=0)), None) == hisa.HISA_E_INVAL
+    assert lib.hisa_pool_blocks(ctypes.byref(_kv(hisa, d=96)), None) == hisa.HISA_E_UNSUPPORTED
+    assert lib.hisa_pool_blocks(ctypes.byref(_kv(hisa, dtype=1)), None) == hisa.HISA_E_INVAL
+    assert lib.hisa_pool_blocks(ctypes.byref(_kv(hisa, keys=8)), None) == hisa.HISA_E_INVAL
+    assert lib.hisa_append(ctypes.byref(kv), None, None, None) == hisa.HISA_E_INVAL
+
+    def sel(kvp, n_q=4, H=64, m=8, k=16, ws=P(256), ws_bytes=1 << 30, **kw):
+        a = dict(good)
+        a.update(kw)
+        return lib.hisa_select(kvp, a["Q"], a["w"], a["q_seq"], None, n_q, H, m, k, a["idx"],
+                               None, ws, ws_bytes, None)
+
+    assert sel(ctypes.byref(kv), k=0) == hisa.HISA_E_INVAL
+    assert sel(ctypes.byref(kv), m=0) == hisa.HISA_E_INVAL
+    assert sel(ctypes.byref(kv), H=129) == hisa.HISA_E_UNSUPPORTED
+    assert sel(ctypes.byref(kv), H=0) == hisa.HISA_E_UNSUPPORTED
+    assert sel(ctypes.byref(kv), n_q=-1) == hisa.HISA_E_INVAL
+    assert sel(ctypes.byref(_kv(hisa, B=100))) == hisa.HISA_E_UNSUPPORTED
+    assert sel(ctypes.byref(kv), Q=None) == hisa.HISA_E_INVAL
+    assert sel(ctypes.byref(kv), Q=P(8)) == hisa.HISA_E_INVAL          # misaligned
+    assert sel(ctypes.byref(kv), ws=None) == hisa.HISA_E_WORKSPACE
+    assert sel(ctypes.byref(kv), ws=P(128)) == hisa.HISA_E_WORKSPACE   # not 256-aligned
+    assert sel(ctypes.byref(kv), ws_bytes=16) == hisa.HISA_E_WORKSPACE
+    assert sel(ctypes.byref(kv), n_q=0) == hisa.HISA_OK                # nothing to do
+    assert lib.dsa_flat_select(ctypes.byref(kv), P(16), P(16), P(16), None, 4, 64, 0, P(16),
+                               None, P(256), 1 << 30, None) == hisa.HISA_E_INVAL
+    assert lib.hisa_topk_f32(None, 3, 10, 2, None, None) == hisa.HISA_E_INVAL
+    assert lib.hisa_topk_f32(P(16), 0, 10, 2, P(16), None) == hisa.HISA_OK
+
+
+def test_workspace_sizes(hisa):
+    lib = hisa.lib()
+    kv = _kv(hisa, cap=32768, B=128)
+    ws = lib.hisa_select_workspace_bytes(ctypes.byref(kv), 64, 64, 64, 2048)
+    # block keys 64x256x4 + blocks 64x64x4 + counts 64x4 + token keys 64x8192x4
+    assert ws == 65536 + 16384 + 256 + 2097152
+    assert lib.dsa_flat_workspace_bytes(ctypes.byref(kv), 64, 64, 2048) == 64 * 32768 * 4
+    assert lib.hisa_select_workspace_bytes(None, 1, 1, 1, 1) == 0
