@@ -24,7 +24,6 @@ import argparse
 import hashlib
 import json
 import os
-import subprocess
 import sys
 import time
 
@@ -57,70 +56,96 @@ def host_cores():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle samples while the timed region runs."""
+    """SM clock and throttle reasons sampled through NVML from a background
+    thread while the timed region runs (about every millisecond)."""
 
-    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, uuid: str | None):
-        self.uuid = uuid
-        self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+    def __init__(self, device_index: int):
+        self.device_index = device_index
+        self.samples = []
+        self.max_mhz = None
+        self.err = None
 
     def __enter__(self):
+        import threading
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+            import pynvml
+            pynvml.nvmlInit()
+            h = self._handle(pynvml)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # NVML missing: report no clocks
+            self.err = repr(e)
+            self.thread = None
+            return self
+        self.stop = threading.Event()
+
+        def loop():
+            while not self.stop.is_set():
+                try:
+                    mhz = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                    rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    self.samples.append((mhz, rs))
+                except Exception as e:
+                    self.err = repr(e)
+                    break
+                self.stop.wait(0.001)
+
+        self.thread = threading.Thread(target=loop, daemon=True)
+        self.thread.start()
         return self
 
-    def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
+    def _handle(self, pynvml):
+        import torch
+        uuid = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.device_index).uuid)
+        except Exception:
+            pass
+        if uuid:
+            u = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
             try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-            self.f.close()
+                return pynvml.nvmlDeviceGetHandleByUUID(u)
+            except Exception:
+                pass
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        idx = int(vis.split(",")[self.device_index]) if vis and vis.split(",")[0].isdigit() \
+            else self.device_index
+        return pynvml.nvmlDeviceGetHandleByIndex(idx)
+
+    def __exit__(self, *exc):
+        if getattr(self, "thread", None) is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
 
     def summary(self):
-        if self.proc is None or not os.path.exists(self.path):
-            return None
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 10:
-                continue
-            if self.uuid and self.uuid not in parts[1]:
-                continue
-            try:
-                sm.append(float(parts[2]))
-                mx.append(float(parts[3]))
-            except ValueError:
-                continue
-            for nm, v in zip(names, parts[6:10]):
-                if v.lower() == "active":
-                    reasons.add(nm)
-        if not sm:
-            return None
-        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)),
-                "samples": len(sm), "reasons": sorted(reasons)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "samples": 0, "reasons": [],
+                    "note": self.err or "no samples"}
+        mhz = [m for m, _ in self.samples]
+        reasons = set()
+        for _, rs in self.samples:
+            for bit, name in self.REASONS.items():
+                if rs & bit:
+                    reasons.add(name)
+        return {"sm_mhz": float(np.median(mhz)), "sm_max_mhz": self.max_mhz,
+                "samples": len(mhz), "reasons": sorted(reasons)}
 
 
 # --------------------------------------------------------------- workload
 
 
+QUERY_SETS = 32
+
+
 def make_workload(steps_total: int, seed_shift: int = 0):
+    """The 32K decode workload with room for `steps_total` appended keys per
+    sequence; decode step s uses query set s % QUERY_SETS."""
     from hisa_inputs import make_config
     spec_cap = 32768 + steps_total
     case = make_config(WORKLOAD["cfg"], cap=spec_cap, append_steps=steps_total,
-                       seed=20260330 + WORKLOAD["cfg"] + seed_shift)
+                       append_query_sets=QUERY_SETS, seed=20260330 + WORKLOAD["cfg"] + seed_shift)
     return case
 
 
@@ -189,20 +214,17 @@ def run_gpu(args, rank, world):
     idx = torch.empty((2, batch, k), dtype=torch.int32, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
+    nsets = Qs.shape[0]
+
     def step(s, out):
         hisa.hisa_append(kv, toks[s])
-        hisa.hisa_select(kv, Qs[s], Ws[s], q_seq, None, m, k, ws=ws, idx=out)
+        hisa.hisa_select(kv, Qs[s % nsets], Ws[s % nsets], q_seq, None, m, k, ws=ws, idx=out)
 
     for s in range(W):
         step(s, idx[s % 2])
         flush.fill_(7)
     torch.cuda.synchronize()
 
-    uuid = None
-    try:
-        uuid = str(torch.cuda.get_device_properties(dev).uuid)
-    except Exception:
-        pass
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(K)]
     if world > 1:
@@ -211,7 +233,7 @@ def run_gpu(args, rank, world):
     torch.cuda.synchronize()
     hisa.hisa_profile_enable(True)
     hisa.hisa_profile_read(reset=True)
-    with ClockSampler(uuid) as clk:
+    with ClockSampler(dev.index) as clk:
         wall0 = time.perf_counter()
         for i in range(K):
             s = W + i
@@ -254,9 +276,10 @@ def run_gpu(args, rank, world):
         torch.cuda.synchronize()
         return float(np.median([a.elapsed_time(b) for a, b in evs]))
 
-    hisa_sel_ms = time_calls(lambda: hisa.hisa_select(kv, Qs[s_cmp], Ws[s_cmp], q_seq, None, m, k,
+    qc, wc = Qs[s_cmp % nsets], Ws[s_cmp % nsets]
+    hisa_sel_ms = time_calls(lambda: hisa.hisa_select(kv, qc, wc, q_seq, None, m, k,
                                                       ws=ws, idx=hidx), n_flat)
-    flat_ms = time_calls(lambda: hisa.dsa_flat_select(kv, Qs[s_cmp], Ws[s_cmp], q_seq, None, k,
+    flat_ms = time_calls(lambda: hisa.dsa_flat_select(kv, qc, wc, q_seq, None, k,
                                                       ws=fws, idx=fidx), n_flat)
     torch.cuda.synchronize()
     from tests.parity import iou
@@ -280,8 +303,8 @@ def run_gpu(args, rank, world):
             s = base + i
             a.record(stream)
             dtok.copy_(ptok[s], non_blocking=True)
-            dQ.copy_(pQ[s], non_blocking=True)
-            dW.copy_(pW[s], non_blocking=True)
+            dQ.copy_(pQ[s % nsets], non_blocking=True)
+            dW.copy_(pW[s % nsets], non_blocking=True)
             hisa.hisa_append(kv, dtok)
             out = hisa.hisa_select(kv, dQ, dW, q_seq, None, m, k, ws=ws, idx=hidx)
             pidx.copy_(out, non_blocking=True)
@@ -383,11 +406,11 @@ def run_reference(args, rank, world):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["hisa", "reference"], default="hisa")
-    ap.add_argument("--e2e-steps", type=int, default=10)
-    ap.add_argument("--flat-steps", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--flat-steps", type=int, default=20)
     ap.add_argument("--ref-rows", type=int, default=16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

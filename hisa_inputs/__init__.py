@@ -127,8 +127,8 @@ class Case:
     q_pos: np.ndarray
     append_keys: Optional[np.ndarray] = None      # [steps, batch, d]
     append_scale: Optional[np.ndarray] = None     # [steps, batch]
-    append_Q: Optional[np.ndarray] = None         # [steps, batch, H, d]
-    append_w: Optional[np.ndarray] = None         # [steps, batch, H]
+    append_Q: Optional[np.ndarray] = None         # [sets, batch, H, d] (step s: set s % sets)
+    append_w: Optional[np.ndarray] = None         # [sets, batch, H]
     meta: dict = field(default_factory=dict)
 
     @property
@@ -152,7 +152,7 @@ def make_case(*, batch: int, L, H: int, d: int, B: int, m: int, k: int,
               positions=None, dtype: str = "bf16", seed: int = SEED_BASE,
               cap: Optional[int] = None, append_steps: int = 0,
               cluster_B: Optional[int] = None, noise: float = 0.5,
-              name: str = "case") -> Case:
+              append_query_sets: Optional[int] = None, name: str = "case") -> Case:
     """Build a case.
 
     L          prefix length, an int or one int per sequence.
@@ -160,6 +160,8 @@ def make_case(*, batch: int, L, H: int, d: int, B: int, m: int, k: int,
                position; an int array -> the same positions in every
                sequence; a list of arrays -> per sequence.
     cluster_B  block size of the synthetic clusters (defaults to B).
+    append_query_sets  number of per-step query sets drawn for the appended
+               steps (default: one per step; step s uses set s % sets).
     """
     rng = np.random.Generator(np.random.PCG64(seed))
     Ls = np.full(batch, L, dtype=np.int64) if np.isscalar(L) else np.asarray(L, dtype=np.int64)
@@ -221,9 +223,10 @@ def make_case(*, batch: int, L, H: int, d: int, B: int, m: int, k: int,
                 asc[:, b] = sc
         case.append_keys = ak
         case.append_scale = asc
+        nsets = append_steps if append_query_sets is None else min(append_query_sets, append_steps)
         case.append_Q = bf16_bits(
-            rng.standard_normal((append_steps, batch, H, d), dtype=np.float32) * inv_sqrt_d)
-        case.append_w = rng.random((append_steps, batch, H), dtype=np.float32)
+            rng.standard_normal((nsets, batch, H, d), dtype=np.float32) * inv_sqrt_d)
+        case.append_w = rng.random((nsets, batch, H), dtype=np.float32)
     return case
 
 
