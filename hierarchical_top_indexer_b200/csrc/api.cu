@@ -169,7 +169,7 @@ struct Carve {
 };
 
 struct HisaWs {
-    size_t bkeys, blocks, nblocks, tkeys, total;
+    size_t bkeys, blocks, nblocks, plan, tkeys, total;
     int ldb, ldt, mm;
 };
 
@@ -182,6 +182,7 @@ HisaWs hisa_ws(const KvView& v, int n_q, int m) {
     w.bkeys = c.take(static_cast<size_t>(n_q) * w.ldb * 4);
     w.blocks = c.take(static_cast<size_t>(n_q) * w.mm * 4);
     w.nblocks = c.take(static_cast<size_t>(n_q) * 4);
+    w.plan = c.take(static_cast<size_t>(n_q) * 16);
     w.tkeys = c.take(static_cast<size_t>(n_q) * w.ldt * 4);
     w.total = c.off;
     return w;
@@ -225,6 +226,8 @@ ScoreParams score_params(const KvView& v, const float* w, const int32_t* q_seq, 
     return p;
 }
 
+// Grid shape: `slices` CTAs per query row (so that few rows still spread over
+// every SM), groups of slices covering the rows, at most one CTA per SM.
 int run_score(int mode, const KvView& v, const CUtensorMap& amap, const CUtensorMap& qmap,
               ScoreParams& p, cudaStream_t s) {
     p.stages = score_stages(mode, mode != kScoreBlocks && v.e4m3, v.d, p.npad);
@@ -233,12 +236,16 @@ int run_score(int mode, const KvView& v, const CUtensorMap& amap, const CUtensor
     if (p.total_tiles == 0) return HISA_OK;
     const int sms = sm_count();
     if (sms <= 0) return HISA_E_CUDA;
-    const int grid = static_cast<int>(p.total_tiles < sms ? p.total_tiles : sms);
+    int slices = 1;
+    while (slices * 2 <= p.tiles_per_row && static_cast<long long>(p.n_q) * slices * 2 <= sms) slices *= 2;
+    const int groups = p.n_q < sms / slices ? p.n_q : sms / slices;
+    p.slices = slices;
     const int phase = mode == kScoreBlocks ? HISA_PHASE_BLOCK_SCORE
                       : mode == kScoreFlat ? HISA_PHASE_FLAT_SCORE
                                            : HISA_PHASE_TOKEN_SCORE;
     PhaseScope ps(phase, s);
-    return cuda_status(launch_score(mode, mode != kScoreBlocks && v.e4m3, v.d, amap, qmap, p, grid, s));
+    return cuda_status(
+        launch_score(mode, mode != kScoreBlocks && v.e4m3, v.d, amap, qmap, p, groups * slices, s));
 }
 
 int hisa_select_impl(const hisa_kv* kv, const uint16_t* Q, const float* w, const int32_t* q_seq,
@@ -259,6 +266,7 @@ int hisa_select_impl(const hisa_kv* kv, const uint16_t* Q, const float* w, const
     uint32_t* bkeys = reinterpret_cast<uint32_t*>(base + L.bkeys);
     int32_t* blocks = reinterpret_cast<int32_t*>(base + L.blocks);
     int32_t* nblocks = reinterpret_cast<int32_t*>(base + L.nblocks);
+    int4* plan = reinterpret_cast<int4*>(base + L.plan);
     uint32_t* tkeys = reinterpret_cast<uint32_t*>(base + L.tkeys);
 
     CUtensorMap pmap, kmap, qmap;
@@ -299,11 +307,12 @@ int hisa_select_impl(const hisa_kv* kv, const uint16_t* Q, const float* w, const
     sp.mm = L.mm;
     sp.blocks = blocks;
     sp.nblocks = nblocks;
+    sp.plan = plan;
     sp.blocks_out = blocks_out;
     sp.nblocks_out = nblocks_out;
     {
         PhaseScope ps(HISA_PHASE_BLOCK_SELECT, s);
-        rc = cuda_status(launch_select(sp, v.nblk, s));
+        rc = cuda_status(launch_select(sp, v.nblk, sm_count(), s));
     }
     if (rc) return rc;
 
@@ -313,6 +322,7 @@ int hisa_select_impl(const hisa_kv* kv, const uint16_t* Q, const float* w, const
     p.tiles_per_row = L.ldt / 128;
     p.blocks = blocks;
     p.nblocks = nblocks;
+    p.plan = plan;
     p.mm = L.mm;
     rc = run_score(kScoreHisa, v, kmap, qmap, p, s);
     if (rc) return rc;
@@ -325,7 +335,7 @@ int hisa_select_impl(const hisa_kv* kv, const uint16_t* Q, const float* w, const
     sp.blocks_out = nullptr;
     sp.nblocks_out = nullptr;
     PhaseScope ps(HISA_PHASE_TOKEN_SELECT, s);
-    return cuda_status(launch_select(sp, L.mm * v.B, s));
+    return cuda_status(launch_select(sp, L.mm * v.B, sm_count(), s));
 }
 
 }  // namespace
@@ -424,7 +434,7 @@ int dsa_flat_select(const hisa_kv* kv, const uint16_t* Q, const float* w, const 
     sp.idx = idx;
     sp.scores = scores;
     PhaseScope ps(HISA_PHASE_FLAT_SELECT, s);
-    return cuda_status(launch_select(sp, v.cap, s));
+    return cuda_status(launch_select(sp, v.cap, sm_count(), s));
 }
 
 int hisa_topk_f32(const float* x, int rows, int n, int k, int32_t* idx, hisa_stream_t stream) {
@@ -440,7 +450,7 @@ int hisa_topk_f32(const float* x, int rows, int n, int k, int32_t* idx, hisa_str
     sp.k = k;
     sp.idx = idx;
     PhaseScope ps(HISA_PHASE_TOPK, reinterpret_cast<cudaStream_t>(stream));
-    return cuda_status(launch_select(sp, n, reinterpret_cast<cudaStream_t>(stream)));
+    return cuda_status(launch_select(sp, n, sm_count(), reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int hisa_profile_enable(int on) {

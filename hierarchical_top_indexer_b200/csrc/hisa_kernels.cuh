@@ -35,17 +35,20 @@ struct ScoreParams {
     const int32_t* q_seq;
     const int32_t* q_pos;
     int n_q, H, npad;
-    // kept blocks (kScoreHisa): blocks [n_q, mm], nblocks [n_q]
+    // kept blocks (kScoreHisa): blocks [n_q, mm], nblocks [n_q], and the
+    // row plan {sequence, position (-1: bad row), kept blocks, 0} [n_q]
     const int32_t* blocks;
     const int32_t* nblocks;
+    const int4* plan;
     int mm;
     // output: order-preserving score keys [n_q, ldo]; 0 = masked slot
     uint32_t* out;
     int ldo;
     unsigned long long* counts;   // [n_q, 2] or null
-    int tiles_per_row;
+    int tiles_per_row;      // upper bound of candidate tiles per row
     long long total_tiles;
     int stages;
+    int slices;             // CTAs sharing one query row
 };
 
 enum SelectMode : int {
@@ -70,6 +73,7 @@ struct SelectParams {
     // kept blocks: written by mode 0, read by mode 1
     int32_t* blocks;
     int32_t* nblocks;
+    int4* plan;              // {sequence, position or -1, kept blocks, 0} per row
     // outputs
     int32_t* idx;       // [rows, k]   (modes 1-3)
     float* scores;      // [rows, k] or null
@@ -90,6 +94,6 @@ cudaError_t launch_score(int mode, bool e4m3, int d, const CUtensorMap& keys_map
                          const CUtensorMap& q_map, const ScoreParams& p, int grid,
                          cudaStream_t s);
 
-cudaError_t launch_select(const SelectParams& p, int max_n, cudaStream_t s);
+cudaError_t launch_select(const SelectParams& p, int max_n, int sms, cudaStream_t s);
 
 }  // namespace hisa

@@ -20,7 +20,12 @@
 // converter warps (exact), and their per-token scale multiplies the score
 // (ReLU(s*x) = s*ReLU(x) for s > 0).
 //
-// Warp roles (persistent, one CTA per SM, contiguous range of tiles):
+// Work split: the CTAs form groups of `slices` CTAs; group g takes query
+// rows g, g + groups, ...; within a row, CTA r of the group scores the r-th
+// contiguous slice of the row's candidate tiles.  Row metadata is read once
+// per row; HISA block ids are prefetched one tile ahead.
+//
+// Warp roles:
 //   warp 0       TMA producer (keys / representatives, query heads)
 //   warp 1       TMEM owner and UMMA issuer
 //   warps 2-5    epilogue (TMEM -> registers -> score key -> global)
@@ -41,10 +46,13 @@ constexpr int kWarpEpi0 = 2;
 constexpr int kWarpConv0 = 6;
 constexpr int kMinSmem = 120 * 1024;          // keeps one CTA (and its TMEM) per SM
 constexpr int kMaxSmem = 232448;
+constexpr int kMaxAcc = 4;
 
 struct Layout {
     uint32_t a, s8, q, w, bars, misc, total;
 };
+
+__host__ __device__ inline int acc_count(int npad) { return 4 * npad <= 512 ? 4 : 2; }
 
 __host__ __device__ inline Layout score_layout(int mode, bool e4m3, int d, int npad, int stages) {
     const int halves = d / 64;
@@ -61,7 +69,7 @@ __host__ __device__ inline Layout score_layout(int mode, bool e4m3, int d, int n
     L.w = off;
     off += 4 * 128 * 4;                      // one 128-float weight slot per epilogue warp
     L.bars = off;
-    off += (4 * stages + 8) * 8;
+    off += (4 * stages + 2 * kMaxAcc + 4) * 8;
     L.misc = off;
     off += 16;
     L.total = off;
@@ -70,44 +78,83 @@ __host__ __device__ inline Layout score_layout(int mode, bool e4m3, int d, int n
 
 __host__ __device__ inline uint32_t tmem_columns(int npad) {
     uint32_t c = 32;
-    while (c < static_cast<uint32_t>(2 * npad)) c <<= 1;
+    while (c < static_cast<uint32_t>(acc_count(npad) * npad)) c <<= 1;
     return c;
 }
 
-struct Tile {
-    int row, ti, b, t, lim;
+// A query row as one CTA of its group sees it.
+struct RowSlice {
+    int b, t, lim;    // sequence, position, candidate slots of the row
+    int t0, t1;       // this CTA's tiles [t0, t1)
 };
 
-// Next tile of [g, g1) that holds at least one candidate.  All roles walk the
-// same sequence, so they agree on tile order without exchanging metadata.
 template <int MODE>
-__device__ __forceinline__ bool next_tile(const ScoreParams& p, long long& g, long long g1,
-                                          Tile& T) {
-    while (g < g1) {
-        const long long cur = g++;
-        const int row = static_cast<int>(cur / p.tiles_per_row);
-        const int ti = static_cast<int>(cur % p.tiles_per_row);
-        int b;
-        const int t = query_position(p.q_seq, p.q_pos, p.len, p.batch, p.cap, row, &b);
-        if (t < 0) continue;
-        int lim;
-        if (MODE == kScoreBlocks) lim = t / p.B + 1;          // visible blocks
-        else if (MODE == kScoreFlat) lim = t + 1;             // visible keys
-        else lim = p.nblocks[row] * p.B;                      // kept token slots
-        if (ti * kTileRows >= lim) continue;
-        T.row = row;
-        T.ti = ti;
-        T.b = b;
-        T.t = t;
-        T.lim = lim;
-        return true;
+__device__ __forceinline__ RowSlice row_slice(const ScoreParams& p, int row, int rank, int slices) {
+    RowSlice R;
+    R.t0 = R.t1 = 0;
+    R.lim = 0;
+    if (MODE == kScoreHisa) {
+        const int4 pl = p.plan[row];        // written by the block selection
+        R.b = pl.x;
+        R.t = pl.y;
+        if (R.t < 0) return R;
+        R.lim = pl.z * p.B;                 // kept token slots
+    } else {
+        R.t = query_position(p.q_seq, p.q_pos, p.len, p.batch, p.cap, row, &R.b);
+        if (R.t < 0) return R;
+        R.lim = MODE == kScoreBlocks ? R.t / p.B + 1   // visible blocks
+                                     : R.t + 1;        // visible keys
     }
-    return false;
+    const int nt = (R.lim + kTileRows - 1) / kTileRows;
+    R.t0 = static_cast<int>(static_cast<long long>(nt) * rank / slices);
+    R.t1 = static_cast<int>(static_cast<long long>(nt) * (rank + 1) / slices);
+    return R;
+}
+
+// sum_h w_h * ReLU(acc_h) over the NP head columns of one TMEM lane: loads
+// of up to 64 columns at a time, one wait per group, four interleaved partial
+// sums (fixed order).
+template <int NP>
+__device__ __forceinline__ float head_sum(uint32_t taddr, const float* wv) {
+    float a[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int g = 0; g < NP; g += 64) {
+        constexpr int kG = NP < 64 ? NP : 64;
+        uint32_t r[kG];
+#pragma unroll
+        for (int c = 0; c < kG; c += 16)
+            if (g + c < NP) tmem_ld16_nowait(taddr + g + c, r + c);
+        tmem_ld_wait();
+#pragma unroll
+        for (int h = 0; h < kG; ++h)
+            if (g + h < NP) a[h & 3] = fmaf(wv[g + h], fmaxf(__uint_as_float(r[h]), 0.f), a[h & 3]);
+    }
+    return (a[0] + a[1]) + (a[2] + a[3]);
+}
+
+__device__ __forceinline__ float head_sum_any(int npad, uint32_t taddr, const float* wv) {
+    switch (npad) {
+        case 16: return head_sum<16>(taddr, wv);
+        case 32: return head_sum<32>(taddr, wv);
+        case 48: return head_sum<48>(taddr, wv);
+        case 64: return head_sum<64>(taddr, wv);
+        case 80: return head_sum<80>(taddr, wv);
+        case 96: return head_sum<96>(taddr, wv);
+        case 112: return head_sum<112>(taddr, wv);
+        default: return head_sum<128>(taddr, wv);
+    }
 }
 
 __device__ __forceinline__ void raise_abort(volatile int* abort_flag, uint32_t* status) {
     *abort_flag = 1;
     set_status(status, HISA_DEV_TIMEOUT);
+}
+
+// Lane 0 waits; the whole warp learns the outcome (keeps the warp converged).
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    bool ok = true;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag);
+    return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -131,6 +178,17 @@ __device__ __forceinline__ uint4 e4m3x8_to_bf16x8(uint2 raw) {
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// First key row of sub-box `sub` of tile `ti` (lanes hold one sub-box each).
+template <int MODE>
+__device__ __forceinline__ int tile_sub_row(const ScoreParams& p, const RowSlice& R, int row, int ti,
+                                            int sub, int BR) {
+    if (MODE == kScoreBlocks) return R.b * p.nblk + ti * kTileRows;
+    if (MODE == kScoreFlat) return R.b * p.cap + ti * kTileRows + sub * BR;
+    const int slot = ti * kTileRows + sub * BR;
+    const int blk = slot < R.lim ? __ldg(p.blocks + static_cast<size_t>(row) * p.mm + slot / p.B) : 0;
+    return R.b * p.cap + blk * p.B + slot % p.B;
+}
+
 template <int MODE, bool E4M3, int D>
 __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
     score_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap qmap,
@@ -145,19 +203,20 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const Layout L = score_layout(MODE, E4M3, D, p.npad, p.stages);
     const int S = p.stages;
+    const int NACC = acc_count(p.npad);
     uint8_t* sA = smem + L.a;
     uint8_t* s8 = smem + L.s8;
     uint8_t* sQ = smem + L.q;
     float* sW = reinterpret_cast<float*>(smem + L.w);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
-    uint64_t* full = bars;             // stage holds bf16 operands (TMA or converters)
-    uint64_t* empty = bars + S;        // stage free again (UMMA done reading)
-    uint64_t* sfull = bars + 2 * S;    // e4m3 staging landed
-    uint64_t* sempty = bars + 3 * S;   // e4m3 staging converted
-    uint64_t* tfull = bars + 4 * S;    // accumulator ready   [2]
-    uint64_t* tempty = tfull + 2;      // accumulator drained [2]
-    uint64_t* qfull = tfull + 4;       // query heads landed  [2]
-    uint64_t* qempty = tfull + 6;      // query heads free    [2]
+    uint64_t* full = bars;                   // stage holds bf16 operands (TMA or converters)
+    uint64_t* empty = bars + S;              // stage free again (UMMA done reading)
+    uint64_t* sfull = bars + 2 * S;          // e4m3 staging landed
+    uint64_t* sempty = bars + 3 * S;         // e4m3 staging converted
+    uint64_t* tfull = bars + 4 * S;          // accumulator ready   [kMaxAcc]
+    uint64_t* tempty = tfull + kMaxAcc;      // accumulator drained [kMaxAcc]
+    uint64_t* qfull = tempty + kMaxAcc;      // query heads landed  [2]
+    uint64_t* qempty = qfull + 2;            // query heads free    [2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.misc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.misc + 4);
 
@@ -166,6 +225,12 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
     const int npad = p.npad;
     const uint32_t ncols = tmem_columns(npad);
     const int q_slot_bytes = kHalves * npad * 128;
+    const int slices = p.slices;
+    const int rank = blockIdx.x % slices;
+    const int group = blockIdx.x / slices;
+    const int groups = gridDim.x / slices;
+    const int BR = (MODE == kScoreBlocks) ? kTileRows : (p.B < kTileRows ? p.B : kTileRows);
+    const int nsub = kTileRows / BR;
 
     if (warp == kWarpProducer && lane == 0) {
         for (int s = 0; s < S; ++s) {
@@ -174,9 +239,11 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
             mbar_init(sfull + s, 1);
             mbar_init(sempty + s, 4);
         }
-        for (int a = 0; a < 2; ++a) {
+        for (int a = 0; a < kMaxAcc; ++a) {
             mbar_init(tfull + a, 1);
             mbar_init(tempty + a, 4);
+        }
+        for (int a = 0; a < 2; ++a) {
             mbar_init(qfull + a, 1);
             mbar_init(qempty + a, 1);
         }
@@ -194,65 +261,72 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-
-    const long long g0 = p.total_tiles * blockIdx.x / gridDim.x;
-    const long long g1 = p.total_tiles * (blockIdx.x + 1) / gridDim.x;
-    const int BR = (MODE == kScoreBlocks) ? kTileRows : (p.B < kTileRows ? p.B : kTileRows);
+    // everything above overlaps the previous kernel; its outputs are read below
+    grid_dependency_wait();
+    grid_launch_dependents();
 
     if (warp == kWarpProducer) {
-        if (lane == 0) {
-            const uint64_t pol = policy_evict_first();
-            long long g = g0;
-            Tile T;
-            int it = 0, qloads = 0, cur_row = -1;
-            bool ok = true;
-            while (next_tile<MODE>(p, g, g1, T)) {
-                if (T.row != cur_row) {
-                    const int qs = qloads & 1;
-                    if (qloads >= 2 && !mbar_wait(qempty + qs, ((qloads - 2) >> 1) & 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    mbar_arrive_expect_tx(qfull + qs, q_slot_bytes);
+        const uint64_t pol = policy_evict_first();
+        int it = 0, qloads = 0;
+        bool ok = true;
+        for (int row = group; row < p.n_q && ok; row += groups) {
+            const RowSlice R = row_slice<MODE>(p, row, rank, slices);
+            if (R.t0 >= R.t1) continue;
+            const int qs = qloads & 1;
+            if (qloads >= 2 && !warp_wait(qempty + qs, ((qloads - 2) >> 1) & 1, abort_flag)) {
+                ok = false;
+                break;
+            }
+            if (lane == 0) {
+                mbar_arrive_expect_tx(qfull + qs, q_slot_bytes);
 #pragma unroll
-                    for (int kh = 0; kh < kHalves; ++kh)
-                        tma_load_2d(sQ + qs * q_slot_bytes + kh * npad * 128, &qmap, qfull + qs,
-                                    kh * 64, T.row * p.H);
-                    ++qloads;
-                    cur_row = T.row;
+                for (int kh = 0; kh < kHalves; ++kh)
+                    tma_load_2d(sQ + qs * q_slot_bytes + kh * npad * 128, &qmap, qfull + qs, kh * 64,
+                                row * p.H);
+            }
+            ++qloads;
+            // Lane j holds the first key row of sub-box 32*w + j of this slice
+            // for the current window w and the next one (prefetched).
+            const int nsub_slice = (R.t1 - R.t0) * nsub;
+            auto window = [&](int w) -> int {
+                const int g = 32 * w + lane;
+                return g < nsub_slice ? tile_sub_row<MODE>(p, R, row, R.t0 + g / nsub, g % nsub, BR) : 0;
+            };
+            int win_cur = window(0);
+            int win_nxt = window(1);
+            int cur_w = 0;
+            for (int ti = R.t0; ti < R.t1; ++ti) {
+                const int g0 = (ti - R.t0) * nsub;
+                if ((g0 >> 5) != cur_w) {
+                    cur_w = g0 >> 5;
+                    win_cur = win_nxt;
+                    win_nxt = window(cur_w + 1);
                 }
                 const int s = it % S;
                 const uint32_t ph = (it / S) & 1;
                 uint64_t* fb = E4M3 ? sfull + s : full + s;
                 uint64_t* eb = E4M3 ? sempty + s : empty + s;
-                if (!mbar_wait(eb, ph ^ 1, abort_flag)) {
+                if (!warp_wait(eb, ph ^ 1, abort_flag)) {
                     ok = false;
                     break;
                 }
                 if (MODE == kScoreBlocks) {
-                    mbar_arrive_expect_tx(fb, kStageBytes);
-                    const int row0 = T.b * p.nblk + T.ti * kTileRows;
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(fb, kStageBytes);
 #pragma unroll
-                    for (int op = 0; op < 2; ++op)
+                        for (int op = 0; op < 2; ++op)
 #pragma unroll
-                        for (int kh = 0; kh < kHalves; ++kh)
-                            tma_load_2d(sA + s * kStageBytes + (op * kHalves + kh) * kHalfBytes, &amap,
-                                        fb, op * D + kh * 64, row0);
+                            for (int kh = 0; kh < kHalves; ++kh)
+                                tma_load_2d(sA + s * kStageBytes + (op * kHalves + kh) * kHalfBytes,
+                                            &amap, fb, op * D + kh * 64, R.b * p.nblk + ti * kTileRows);
+                    }
                 } else {
-                    mbar_arrive_expect_tx(fb, E4M3 ? kStage8Bytes : kStageBytes);
-                    for (int sub = 0; sub < kTileRows / BR; ++sub) {
-                        int srow;
-                        if (MODE == kScoreFlat) {
-                            srow = T.b * p.cap + T.ti * kTileRows + sub * BR;
-                        } else {
-                            const int slot = T.ti * kTileRows + sub * BR;
-                            const int r = slot / p.B, off = slot % p.B;
-                            const int blk = slot < T.lim ? p.blocks[T.row * p.mm + r] : 0;
-                            srow = T.b * p.cap + blk * p.B + off;
-                        }
+                    if (lane == 0) mbar_arrive_expect_tx(fb, E4M3 ? kStage8Bytes : kStageBytes);
+                    for (int sub = 0; sub < nsub; ++sub) {
+                        const int srow = __shfl_sync(0xffffffffu, win_cur, (g0 & 31) + sub);
+                        if (lane != 0) continue;
                         if (E4M3) {
-                            tma_load_2d_hint(s8 + s * kStage8Bytes + sub * BR * D, &amap, fb, 0, srow,
-                                             pol);
+                            tma_load_2d_hint(s8 + s * kStage8Bytes + sub * BR * D, &amap, fb, 0, srow, pol);
                         } else {
 #pragma unroll
                             for (int kh = 0; kh < kHalves; ++kh)
@@ -261,8 +335,11 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
                         }
                     }
                 }
+                __syncwarp();
                 ++it;
             }
+        }
+        if (lane == 0) {
             if (!ok) raise_abort(abort_flag, p.status);
             // Drain: no copy into, and no arrive on, this CTA's shared memory
             // may still be pending when it exits.
@@ -281,153 +358,144 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
     } else if (warp == kWarpMma) {
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16_f32(static_cast<uint32_t>(npad));
-            long long g = g0;
-            Tile T;
-            int it = 0, qloads = 0, cur_row = -1;
+            int it = 0, qloads = 0;
             bool ok = true;
-            while (next_tile<MODE>(p, g, g1, T)) {
-                if (T.row != cur_row) {
-                    if (qloads > 0) umma_commit(qempty + ((qloads - 1) & 1));
-                    if (!mbar_wait(qfull + (qloads & 1), (qloads >> 1) & 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    ++qloads;
-                    cur_row = T.row;
-                }
-                const int s = it % S;
-                const int a = it & 1;
-                if (!mbar_wait(full + s, (it / S) & 1, abort_flag) ||
-                    !mbar_wait(tempty + a, ((it >> 1) & 1) ^ 1, abort_flag)) {
+            for (int row = group; row < p.n_q && ok; row += groups) {
+                const RowSlice R = row_slice<MODE>(p, row, rank, slices);
+                if (R.t0 >= R.t1) continue;
+                if (qloads > 0) umma_commit(qempty + ((qloads - 1) & 1));
+                if (!mbar_wait(qfull + (qloads & 1), (qloads >> 1) & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
-                tc_fence_after();
-                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * npad);
-                const uint32_t a_base = smem_addr(sA + s * kStageBytes);
-                const uint32_t q_base = smem_addr(sQ + ((qloads - 1) & 1) * q_slot_bytes);
+                const uint32_t q_base = smem_addr(sQ + (qloads & 1) * q_slot_bytes);
+                ++qloads;
+                for (int ti = R.t0; ti < R.t1; ++ti) {
+                    const int s = it % S;
+                    const int a = it % NACC;
+                    if (!mbar_wait(full + s, (it / S) & 1, abort_flag) ||
+                        !mbar_wait(tempty + a, ((it / NACC) & 1) ^ 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * npad);
+                    const uint32_t a_base = smem_addr(sA + s * kStageBytes);
 #pragma unroll
-                for (int kh = 0; kh < kHalves; ++kh) {
+                    for (int kh = 0; kh < kHalves; ++kh) {
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint64_t bdesc = sw128_kmajor_desc(q_base + kh * npad * 128 + kk * 32);
-                        const uint64_t adesc = sw128_kmajor_desc(a_base + kh * kHalfBytes + kk * 32);
-                        umma_bf16(d_tmem, adesc, bdesc, idesc, (kh | kk) ? 1u : 0u);
-                        if (MODE == kScoreBlocks) {
-                            const uint64_t ldesc =
-                                sw128_kmajor_desc(a_base + (kHalves + kh) * kHalfBytes + kk * 32);
-                            umma_bf16(d_tmem, ldesc, bdesc, idesc, 1u);
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint64_t bdesc = sw128_kmajor_desc(q_base + kh * npad * 128 + kk * 32);
+                            const uint64_t adesc = sw128_kmajor_desc(a_base + kh * kHalfBytes + kk * 32);
+                            umma_bf16(d_tmem, adesc, bdesc, idesc, (kh | kk) ? 1u : 0u);
+                            if (MODE == kScoreBlocks) {
+                                const uint64_t ldesc =
+                                    sw128_kmajor_desc(a_base + (kHalves + kh) * kHalfBytes + kk * 32);
+                                umma_bf16(d_tmem, ldesc, bdesc, idesc, 1u);
+                            }
                         }
                     }
+                    umma_commit(empty + s);
+                    umma_commit(tfull + a);
+                    ++it;
                 }
-                umma_commit(empty + s);
-                umma_commit(tfull + a);
-                ++it;
             }
             if (!ok) raise_abort(abort_flag, p.status);
             // every UMMA of this CTA has finished before TMEM is released
-            if (it > 0) mbar_wait(tfull + ((it - 1) & 1), ((it - 1) >> 1) & 1, nullptr);
+            if (it > 0) mbar_wait(tfull + ((it - 1) % NACC), ((it - 1) / NACC) & 1, nullptr);
         }
     } else if (warp >= kWarpEpi0 && warp < kWarpEpi0 + 4) {
         const int quad = warp & 3;             // TMEM lanes this warp may read
         const int r = quad * 32 + lane;        // tile row = candidate
         float* wv = sW + (warp - kWarpEpi0) * 128;
-        long long g = g0;
-        Tile T;
-        int it = 0, cur_row = -1;
-        while (next_tile<MODE>(p, g, g1, T)) {
-            if (T.row != cur_row) {
-                __syncwarp();
-                for (int h = lane; h < 128; h += 32) wv[h] = h < p.H ? p.w[T.row * p.H + h] : 0.f;
-                __syncwarp();
-                cur_row = T.row;
-            }
-            const int a = it & 1;
-            if (!mbar_wait(tfull + a, (it >> 1) & 1, abort_flag)) {
-                raise_abort(abort_flag, p.status);
-                break;
-            }
-            tc_fence_after();
-            const uint32_t taddr =
-                tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(a * npad);
-            float acc = 0.f;
-            for (int c = 0; c < npad; c += 16) {
-                float v[16];
-                tmem_ld16(taddr + c, v);
-                tmem_ld_wait();
-#pragma unroll
-                for (int h = 0; h < 16; ++h)
-                    if (c + h < p.H) acc = fmaf(wv[c + h], fmaxf(v[h], 0.f), acc);
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(tempty + a);
-
-            uint32_t* out = p.out + static_cast<size_t>(T.row) * p.ldo;
-            if (MODE == kScoreBlocks) {
-                const int j = T.ti * kTileRows + r;
-                const bool valid = j < T.lim;
-                out[j] = valid ? score_key(acc) : 0u;
-                if (p.counts) {
-                    const int n = __popc(__ballot_sync(0xffffffffu, valid));
-                    if (lane == 0 && n) atomicAdd(p.counts + 2 * T.row, static_cast<unsigned long long>(n));
-                }
-            } else {
-                const int c = T.ti * kTileRows + r;
-                int s;
-                bool valid;
-                if (MODE == kScoreFlat) {
-                    s = c;
-                    valid = s <= T.t;
-                } else {
-                    const bool slot_ok = c < T.lim;
-                    const int blk = slot_ok ? p.blocks[T.row * p.mm + c / p.B] : 0;
-                    s = blk * p.B + c % p.B;
-                    valid = slot_ok && s <= T.t;
-                    if (p.counts) {
-                        const int n = __popc(__ballot_sync(0xffffffffu, slot_ok));
-                        if (lane == 0 && n)
-                            atomicAdd(p.counts + 2 * T.row + 1, static_cast<unsigned long long>(n));
-                    }
-                }
-                if (E4M3 && valid) acc *= p.key_scale[static_cast<size_t>(T.b) * p.cap + s];
-                out[c] = valid ? score_key(acc) : 0u;
-            }
-            ++it;
-        }
-    } else if (E4M3 && warp >= kWarpConv0) {
-        const int cw = warp - kWarpConv0;
-        long long g = g0;
-        Tile T;
         int it = 0;
         bool ok = true;
-        while (next_tile<MODE>(p, g, g1, T)) {
-            const int s = it % S;
-            const uint32_t ph = (it / S) & 1;
-            if (!mbar_wait(sfull + s, ph, abort_flag) || !mbar_wait(empty + s, ph ^ 1, abort_flag)) {
-                ok = false;
-                break;
-            }
-            const uint8_t* src = s8 + s * kStage8Bytes;
-            uint8_t* dst = sA + s * kStageBytes;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int rr = cw * 32 + i * 4 + (lane >> 3);
-                const int cc = lane & 7;
-#pragma unroll
-                for (int kh = 0; kh < kHalves; ++kh) {
-                    const uint2 raw = *reinterpret_cast<const uint2*>(src + rr * D + kh * 64 + cc * 8);
-                    *reinterpret_cast<uint4*>(dst + kh * kHalfBytes + rr * 128 + ((cc ^ (rr & 7)) << 4)) =
-                        e4m3x8_to_bf16x8(raw);
-                }
-            }
-            fence_async_smem();
+        for (int row = group; row < p.n_q && ok; row += groups) {
+            const RowSlice R = row_slice<MODE>(p, row, rank, slices);
+            if (R.t0 >= R.t1) continue;
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(full + s);
-                mbar_arrive(sempty + s);
+            for (int h = lane; h < 128; h += 32) wv[h] = h < p.H ? p.w[row * p.H + h] : 0.f;
+            __syncwarp();
+            uint32_t* out = p.out + static_cast<size_t>(row) * p.ldo;
+            const int own_rank = R.lim / p.B - 1;         // HISA: the own block is listed last
+            const int t_in_own = R.t % p.B;
+            for (int ti = R.t0; ti < R.t1; ++ti) {
+                const int c = ti * kTileRows + r;
+                // validity and (e4m3) scale, fetched before waiting for the MMA
+                bool valid;
+                float scale = 1.f;
+                if (MODE == kScoreBlocks) {
+                    valid = c < R.lim;
+                } else if (MODE == kScoreFlat) {
+                    valid = c <= R.t;
+                    if (E4M3 && valid) scale = __ldg(p.key_scale + static_cast<size_t>(R.b) * p.cap + c);
+                } else {
+                    const int br = c / p.B, o = c % p.B;
+                    valid = c < R.lim && (br < own_rank || o <= t_in_own);
+                    if (E4M3 && valid) {
+                        const int blk = __ldg(p.blocks + static_cast<size_t>(row) * p.mm + br);
+                        scale = __ldg(p.key_scale + static_cast<size_t>(R.b) * p.cap + blk * p.B + o);
+                    }
+                }
+                const int a = it % NACC;
+                if (!mbar_wait(tfull + a, (it / NACC) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
+                                       static_cast<uint32_t>(a * npad);
+                float acc = head_sum_any(npad, taddr, wv);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(tempty + a);
+                if (E4M3) acc *= scale;
+                out[c] = valid ? score_key(acc) : 0u;
+                if (p.counts) {
+                    const bool slot = MODE == kScoreBlocks ? valid : c < R.lim;
+                    const int n = __popc(__ballot_sync(0xffffffffu, slot));
+                    if (lane == 0 && n)
+                        atomicAdd(p.counts + 2 * row + (MODE == kScoreBlocks ? 0 : 1),
+                                  static_cast<unsigned long long>(n));
+                }
+                ++it;
             }
-            ++it;
+        }
+        if (!ok) raise_abort(abort_flag, p.status);
+    } else if (E4M3 && warp >= kWarpConv0) {
+        const int cw = warp - kWarpConv0;
+        int it = 0;
+        bool ok = true;
+        for (int row = group; row < p.n_q && ok; row += groups) {
+            const RowSlice R = row_slice<MODE>(p, row, rank, slices);
+            for (int ti = R.t0; ti < R.t1; ++ti) {
+                const int s = it % S;
+                const uint32_t ph = (it / S) & 1;
+                if (!mbar_wait(sfull + s, ph, abort_flag) || !mbar_wait(empty + s, ph ^ 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const uint8_t* src = s8 + s * kStage8Bytes;
+                uint8_t* dst = sA + s * kStageBytes;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int rr = cw * 32 + i * 4 + (lane >> 3);
+                    const int cc = lane & 7;
+#pragma unroll
+                    for (int kh = 0; kh < kHalves; ++kh) {
+                        const uint2 raw = *reinterpret_cast<const uint2*>(src + rr * D + kh * 64 + cc * 8);
+                        *reinterpret_cast<uint4*>(dst + kh * kHalfBytes + rr * 128 + ((cc ^ (rr & 7)) << 4)) =
+                            e4m3x8_to_bf16x8(raw);
+                    }
+                }
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(full + s);
+                    mbar_arrive(sempty + s);
+                }
+                ++it;
+            }
         }
         if (!ok) raise_abort(abort_flag, p.status);
         if (ok && cw == 0 && lane == 0)
@@ -448,8 +516,18 @@ cudaError_t launch_t(const CUtensorMap& amap, const CUtensorMap& qmap, const Sco
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    fn<<<grid, E4M3 ? 320 : 192, smem, s>>>(amap, qmap, p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(E4M3 ? 320 : 192);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // prologue overlaps
+    attr[0].val.programmaticStreamSerializationAllowed = 1;            // the previous kernel
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, fn, amap, qmap, p);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace

@@ -3,37 +3,59 @@
 // HISA keeps the top-m blocks by representative score and then the top-k
 // tokens of the kept blocks (gptget.net summary, "Methodology"; Chinese
 // summary, method details); the flat scan keeps the top-k of all visible
-// tokens.  All three use this kernel, one CTA per row:
+// tokens.  All of them use this kernel on 32-bit order-preserving score keys
+// (key 0 = empty / masked slot).
 //
-//   1. radix select on the 32-bit order-preserving score keys (four 8-bit
-//      digit passes, per-warp histograms, warp-aggregated increments) finds
-//      the exact k-th largest key T and how many keys equal to T are taken;
-//   2. an ordered compaction (each warp owns a contiguous slot range; ballots
-//      give in-warp ranks, a scan over warps gives offsets) writes the kept
-//      slots in ascending slot order, taking keys == T lowest slot first.
+// One thread-block cluster per row; CTA r of the cluster stages the r-th
+// contiguous chunk of the row's slots in its shared memory, and the CTAs
+// exchange partial results through distributed shared memory:
+//   1. count, min and max of the nonzero keys (reduced on rank 0);
+//   2. a 2048-bin histogram over [min, max] (bins of 2^shift keys, reduced
+//      on rank 0) locates the bin of the k-th largest key; a crowded bin
+//      narrows the range and the histogram repeats;
+//   3. the bin's members are gathered on rank 0 and ranked by counting,
+//      which gives the exact k-th largest key T and how many keys equal to
+//      T belong to the top k;
+//   4. each CTA counts its keys above / equal to T; the counts of lower
+//      ranks give its output offset and its share of the keys == T (lowest
+//      slots first); an ordered compaction (warp-contiguous slot ranges,
+//      ballots for in-warp ranks) writes the kept slots in ascending order.
 // Slots are laid out in ascending token order, so the output is ascending in
-// token index, followed by -1 padding.  Key 0 marks an empty (masked) slot.
+// token index, followed by -1 padding.
+#include <cooperative_groups.h>
+
 #include "hisa_kernels.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace hisa {
 
 namespace {
 
-constexpr int kSelThreads = 512;
+constexpr int kSelThreads = 1024;
 constexpr int kSelWarps = kSelThreads / 32;
-constexpr int kSmemKeys = 16384;   // rows up to this many slots are staged in shared memory
+constexpr int kMaxChunk = 32768;    // slots staged per CTA
+constexpr int kMaxCluster = 8;
+constexpr int kBins = 2048;
+constexpr int kBinBits = 11;
+constexpr int kMembersCap = 1024;   // bin members ranked directly
 
 struct SelShared {
-    uint32_t hist[kSelWarps][256];
-    uint32_t tot[256];
+    uint32_t hist[kBins];                         // local histogram / copy of the reduced one
+    uint32_t hist_red[kBins];                     // rank 0: cluster-wide histogram
+    unsigned long long members[kMembersCap];      // rank 0: gathered bin members
+    unsigned long long mloc[kMembersCap];         // local copy of the members
+    uint32_t stats[kMaxCluster][3];               // rank 0: per-rank count, min, max
+    uint32_t counts[kMaxCluster][2];              // rank 0: per-rank keys above / equal to T
+    uint32_t member_count;                        // rank 0
     uint32_t warp_a[kSelWarps];
     uint32_t warp_b[kSelWarps];
     uint32_t warp_c[kSelWarps];
     uint32_t warp_d[kSelWarps];
-    uint32_t bcast[4];
+    uint32_t bcast[8];
 };
 
-// Where a row's keys come from.
+// Where the CTA's keys come from (slots are CTA-local: 0 .. nl-1).
 struct Keys {
     const uint32_t* smem;   // staged keys (or null)
     const uint32_t* g;      // keys in global memory
@@ -45,90 +67,130 @@ struct Keys {
     }
 };
 
-__device__ __forceinline__ uint32_t block_sum(uint32_t v, SelShared& sh) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+__device__ __forceinline__ uint32_t warp_sum(uint32_t v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (lane == 0) sh.warp_a[warp] = v;
-    __syncthreads();
-    uint32_t t = 0;
-    for (int w = 0; w < kSelWarps; ++w) t += sh.warp_a[w];
-    __syncthreads();
-    return t;
+    return v;
 }
 
-// Exact k-th largest key among the nonzero keys of [0, n) (n_valid > k).
-// Returns T and the number of keys equal to T that belong to the top k.
-__device__ void radix_threshold(const Keys& keys, int n, int k, SelShared& sh, uint32_t& T,
-                                int& take_eq) {
+// Exact k-th largest nonzero key T over the cluster's keys and the number of
+// keys == T inside the top k (requires more than k nonzero keys).
+__device__ void cluster_kth_key(cg::cluster_group& cluster, const Keys& keys, int nl, int slot0, int k,
+                                uint32_t lo, uint32_t hi, SelShared& sh, uint32_t& T, int& take_eq) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    uint32_t prefix = 0, mask = 0;
+    const unsigned rank = cluster.block_rank();
+    uint32_t* red = cluster.map_shared_rank(sh.hist_red, 0);
     int krem = k;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int i = lane; i < 256; i += 32) sh.hist[warp][i] = 0;
-        __syncwarp();
-        for (int base = warp * 32; base < n; base += kSelThreads) {
-            const int c = base + lane;
-            const uint32_t x = c < n ? keys(c) : 0u;
-            const bool act = x != 0u && (x & mask) == prefix;
-            const uint32_t bin = act ? ((x >> shift) & 255u) : 256u;
-            const unsigned peers = __match_any_sync(0xffffffffu, bin);
-            if (act && lane == __ffs(peers) - 1) atomicAdd(&sh.hist[warp][bin], __popc(peers));
+    for (;;) {
+        const uint32_t span = hi - lo;
+        const int shift = span == 0 ? 0 : max(0, 32 - __clz(span) - kBinBits);
+        for (int i = tid; i < kBins; i += kSelThreads) sh.hist[i] = 0;
+        __syncthreads();
+        for (int c = tid; c < nl; c += kSelThreads) {
+            const uint32_t x = keys(c);
+            if (x != 0u && x >= lo && x <= hi) atomicAdd(&sh.hist[(x - lo) >> shift], 1u);
         }
         __syncthreads();
-        if (tid < 256) {
-            uint32_t s = 0;
-            for (int w = 0; w < kSelWarps; ++w) s += sh.hist[w][tid];
-            sh.tot[tid] = s;
+        for (int i = tid; i < kBins; i += kSelThreads)
+            if (sh.hist[i]) atomicAdd(red + i, sh.hist[i]);
+        cluster.sync();
+        for (int i = tid; i < kBins; i += kSelThreads) sh.hist[i] = red[i];
+        __syncthreads();
+        // highest bin whose suffix count reaches krem: each thread owns 2 bins
+        const int b0 = kBins - 1 - 2 * tid;   // thread 0 owns the top bins
+        const uint32_t l0 = sh.hist[b0], l1 = sh.hist[b0 - 1];
+        const uint32_t lsum = l0 + l1;
+        uint32_t incl = lsum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        if (lane == 31) sh.warp_a[warp] = incl;
+        __syncthreads();
+        uint32_t before = 0;
+        for (int w = 0; w < warp; ++w) before += sh.warp_a[w];
+        const uint32_t excl = before + incl - lsum;
+        const uint32_t kr = static_cast<uint32_t>(krem);
+        if (excl < kr && kr <= excl + lsum) {
+            if (excl + l0 >= kr) {
+                sh.bcast[0] = static_cast<uint32_t>(b0);
+                sh.bcast[1] = kr - excl;
+                sh.bcast[2] = l0;
+            } else {
+                sh.bcast[0] = static_cast<uint32_t>(b0 - 1);
+                sh.bcast[1] = kr - excl - l0;
+                sh.bcast[2] = l1;
+            }
         }
         __syncthreads();
-        if (warp == 0) {
-            // lane L owns bins 255-8L .. 248-8L, highest first
-            uint32_t loc[8], lsum = 0;
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                loc[q] = sh.tot[255 - 8 * lane - q];
-                lsum += loc[q];
-            }
-            uint32_t incl = lsum;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += v;
-            }
-            const uint32_t excl = incl - lsum;
-            if (excl < static_cast<uint32_t>(krem) && static_cast<uint32_t>(krem) <= incl) {
-                uint32_t run = excl;
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    if (run + loc[q] >= static_cast<uint32_t>(krem)) {
-                        sh.bcast[0] = 255u - 8u * lane - q;
-                        sh.bcast[1] = static_cast<uint32_t>(krem) - run;
-                        break;
-                    }
-                    run += loc[q];
+        const uint32_t bin = sh.bcast[0];
+        krem = static_cast<int>(sh.bcast[1]);
+        const uint32_t nmem = sh.bcast[2];
+        const uint32_t blo = lo + (bin << shift);
+        const uint32_t bhi = shift == 0 ? blo : blo + ((1u << shift) - 1u);
+        __syncthreads();
+        if (shift == 0) {          // a single key value: it is T
+            T = blo;
+            take_eq = krem;
+            return;
+        }
+        if (nmem <= static_cast<uint32_t>(kMembersCap)) {
+            unsigned long long* rmem = cluster.map_shared_rank(sh.members, 0);
+            uint32_t* rcnt = cluster.map_shared_rank(&sh.member_count, 0);
+            for (int c = tid; c < nl; c += kSelThreads) {
+                const uint32_t x = keys(c);
+                if (x >= blo && x <= bhi && x != 0u) {
+                    const uint32_t at = atomicAdd(rcnt, 1u);
+                    rmem[at] = (static_cast<unsigned long long>(x) << 32) | static_cast<uint32_t>(slot0 + c);
                 }
             }
+            cluster.sync();
+            const int cnt = static_cast<int>(*rcnt);
+            for (int i = tid; i < cnt; i += kSelThreads) sh.mloc[i] = rmem[i];
+            __syncthreads();
+            for (int i = tid; i < cnt; i += kSelThreads) {
+                const uint32_t xi = static_cast<uint32_t>(sh.mloc[i] >> 32);
+                int above = 0, equal = 0;
+                for (int j = 0; j < cnt; ++j) {
+                    const uint32_t xj = static_cast<uint32_t>(sh.mloc[j] >> 32);
+                    above += xj > xi;
+                    equal += xj == xi;
+                }
+                // xi is T iff the krem-th position falls in xi's run of equal keys
+                if (above < krem && krem <= above + equal) {
+                    sh.bcast[4] = xi;
+                    sh.bcast[5] = static_cast<uint32_t>(krem - above);
+                }
+            }
+            __syncthreads();
+            T = sh.bcast[4];
+            take_eq = static_cast<int>(sh.bcast[5]);
+            __syncthreads();
+            return;
         }
-        __syncthreads();
-        prefix |= sh.bcast[0] << shift;
-        mask |= 0xFFu << shift;
-        krem = static_cast<int>(sh.bcast[1]);
-        __syncthreads();
+        // too many keys in the bin: narrow the range and repeat
+        cluster.sync();                 // everyone has read the reduced histogram
+        if (rank == 0)
+            for (int i = tid; i < kBins; i += kSelThreads) sh.hist_red[i] = 0;
+        cluster.sync();
+        lo = blo;
+        hi = bhi;
     }
-    T = prefix;
-    take_eq = krem;
 }
 
-// Ordered compaction.  Keeps keys > T, plus the first `take_eq` keys == T in
-// slot order (with T == 0 every nonzero key is kept).  Calls emit(pos, slot,
-// key) with pos = rank among kept slots in slot order.  Returns the count.
+// Block-wide exclusive scan helper for the per-warp totals in warp_a / warp_b.
+// Ordered compaction of the CTA's keys: keeps keys > T plus keys == T whose
+// cluster-wide rank among equal keys is below take_eq.  eq_base = keys == T
+// in lower ranks, out_base = kept keys in lower ranks.  Calls emit(pos, slot,
+// key).  Returns the number kept by this CTA.
 template <class Emit>
-__device__ int compact(const Keys& keys, int n, uint32_t T, int take_eq, SelShared& sh, Emit emit) {
+__device__ int compact(const Keys& keys, int nl, uint32_t T, int take_eq, uint32_t eq_base,
+                       uint32_t out_base, SelShared& sh, Emit emit) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int per_warp = ((n + kSelWarps - 1) / kSelWarps + 31) & ~31;
+    const int per_warp = ((nl + kSelWarps - 1) / kSelWarps + 31) & ~31;
     const int w0 = warp * per_warp;
-    const int w1 = min(n, w0 + per_warp);
+    const int w1 = min(nl, w0 + per_warp);
     uint32_t gt = 0, eq = 0;
     for (int base = w0; base < w1; base += 32) {
         const int c = base + lane;
@@ -142,7 +204,7 @@ __device__ int compact(const Keys& keys, int n, uint32_t T, int take_eq, SelShar
     }
     __syncthreads();
     if (threadIdx.x == 0) {
-        uint32_t eq_before = 0, off = 0;
+        uint32_t eq_before = eq_base, off = out_base;
         for (int w = 0; w < kSelWarps; ++w) {
             const uint32_t e = sh.warp_b[w];
             const int room = take_eq - static_cast<int>(eq_before);
@@ -152,7 +214,7 @@ __device__ int compact(const Keys& keys, int n, uint32_t T, int take_eq, SelShar
             eq_before += e;
             off += sh.warp_a[w] + take;
         }
-        sh.bcast[2] = off;
+        sh.bcast[6] = off - out_base;
     }
     __syncthreads();
     uint32_t eq_run = sh.warp_c[warp];
@@ -171,137 +233,299 @@ __device__ int compact(const Keys& keys, int n, uint32_t T, int take_eq, SelShar
         eq_run += __popc(eqb);
         pos += __popc(selb);
     }
-    const int total = static_cast<int>(sh.bcast[2]);
+    const int total = static_cast<int>(sh.bcast[6]);
     __syncthreads();
     return total;
 }
 
-template <bool SMEM>
-__global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectParams p) {
+// Keys of the CTA's chunk with T known: counts above / equal to T.
+__device__ void count_vs(const Keys& keys, int nl, uint32_t T, SelShared& sh, uint32_t& gt_out,
+                         uint32_t& eq_out) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint32_t gt = 0, eq = 0;
+    for (int c = threadIdx.x; c < nl; c += kSelThreads) {
+        const uint32_t x = keys(c);
+        gt += x != 0u && x > T;
+        eq += x != 0u && x == T;
+    }
+    gt = warp_sum(gt);
+    eq = warp_sum(eq);
+    if (lane == 0) {
+        sh.warp_c[warp] = gt;
+        sh.warp_d[warp] = eq;
+    }
+    __syncthreads();
+    gt_out = eq_out = 0;
+    for (int w = 0; w < kSelWarps; ++w) {
+        gt_out += sh.warp_c[w];
+        eq_out += sh.warp_d[w];
+    }
+    __syncthreads();
+}
+
+template <bool STAGE>
+__global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectParams p) {
     extern __shared__ uint32_t staged[];
     __shared__ SelShared sh;
-    const int row = blockIdx.x;
+    grid_dependency_wait();
+    grid_launch_dependents();
+    cg::cluster_group cluster = cg::this_cluster();
+    const int csize = static_cast<int>(cluster.num_blocks());
+    const int rank = static_cast<int>(cluster.block_rank());
+    const int row = blockIdx.x / csize;
     const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
 
+    // ---- row geometry (identical on every rank of the cluster)
     int n = 0, kk = p.k, b = 0, t = 0, nb = 0;
-    Keys keys{nullptr, nullptr, nullptr};
+    bool bad = false;
     if (p.mode == kSelF32Rows) {
         n = p.n;
-        keys.x = p.x + static_cast<size_t>(row) * p.n;
+    } else if (p.mode == kSelHisaTokens) {
+        const int4 pl = p.plan[row];
+        b = pl.x;
+        t = pl.y;
+        bad = t < 0;
+        n = pl.z * p.B;
     } else {
         t = query_position(p.q_seq, p.q_pos, p.len, p.batch, p.cap, row, &b);
-        if (t < 0) {
-            if (tid == 0) set_status(p.status, HISA_DEV_BAD_QUERY);
+        bad = t < 0;
+        if (p.mode == kSelBlocks) {
+            nb = t / p.B + 1;
+            n = nb - 1;          // every block but the own one competes
+            kk = p.m - 1;        // for m - 1 places
+        } else {
+            n = t + 1;
+        }
+    }
+
+    if (bad || (p.mode == kSelBlocks && nb <= p.m)) {
+        if (rank == 0) {
             if (p.mode == kSelBlocks) {
+                // bad row: nothing kept; short row: every visible block kept
+                const int keep = bad ? 0 : nb;
                 for (int r = tid; r < p.mm; r += kSelThreads) {
-                    p.blocks[static_cast<size_t>(row) * p.mm + r] = -1;
-                    if (p.blocks_out) p.blocks_out[static_cast<size_t>(row) * p.mm + r] = -1;
+                    const int v = r < keep ? r : -1;
+                    p.blocks[static_cast<size_t>(row) * p.mm + r] = v;
+                    if (p.blocks_out) p.blocks_out[static_cast<size_t>(row) * p.mm + r] = v;
                 }
                 if (tid == 0) {
-                    p.nblocks[row] = 0;
-                    if (p.nblocks_out) p.nblocks_out[row] = 0;
+                    p.nblocks[row] = keep;
+                    if (p.nblocks_out) p.nblocks_out[row] = keep;
+                    p.plan[row] = make_int4(b, bad ? -1 : t, keep, 0);
+                    if (bad) set_status(p.status, HISA_DEV_BAD_QUERY);
                 }
             } else {
                 for (int r = tid; r < p.k; r += kSelThreads) {
                     p.idx[static_cast<size_t>(row) * p.k + r] = -1;
                     if (p.scores) p.scores[static_cast<size_t>(row) * p.k + r] = __int_as_float(0x7fc00000);
                 }
+                if (tid == 0 && p.mode != kSelHisaTokens) set_status(p.status, HISA_DEV_BAD_QUERY);
             }
-            return;
         }
-        keys.g = p.keys + static_cast<size_t>(row) * p.ldk;
-        if (p.mode == kSelBlocks) {
-            nb = t / p.B + 1;
-            n = nb - 1;          // every block but the own one competes
-            kk = p.m - 1;        // for m - 1 places
-        } else if (p.mode == kSelHisaTokens) {
-            n = p.nblocks[row] * p.B;
-        } else {
-            n = t + 1;
-        }
-    }
-
-    if (p.mode == kSelBlocks && nb <= p.m) {
-        // every visible block is kept
-        int32_t* out = p.blocks + static_cast<size_t>(row) * p.mm;
-        for (int r = tid; r < p.mm; r += kSelThreads) {
-            const int v = r < nb ? r : -1;
-            out[r] = v;
-            if (p.blocks_out) p.blocks_out[static_cast<size_t>(row) * p.mm + r] = v;
-        }
-        if (tid == 0) {
-            p.nblocks[row] = nb;
-            if (p.nblocks_out) p.nblocks_out[row] = nb;
-        }
+        cluster.sync();
         return;
     }
 
-    if (SMEM) {
-        for (int c = tid; c < n; c += kSelThreads) staged[c] = keys(c);
-        __syncthreads();
-        keys.smem = staged;
+    // ---- this rank's chunk of slots
+    const int chunk = ((n + csize - 1) / csize + 127) & ~127;
+    const int s0 = min(n, rank * chunk);
+    const int nl = min(n, s0 + chunk) - s0;
+    Keys keys{nullptr, nullptr, nullptr};
+    if (p.mode == kSelF32Rows) keys.x = p.x + static_cast<size_t>(row) * p.n + s0;
+    else keys.g = p.keys + static_cast<size_t>(row) * p.ldk + s0;
+
+    if (rank == 0) {
+        for (int i = tid; i < kBins; i += kSelThreads) sh.hist_red[i] = 0;
+        if (tid == 0) sh.member_count = 0;
     }
 
+    // ---- pass 1: stage, count, min, max
+    uint32_t cnt = 0, mn = 0xFFFFFFFFu, mx = 0u;
+    if (keys.g) {
+        const uint4* g4 = reinterpret_cast<const uint4*>(keys.g);   // s0, ldk: multiples of 128
+        const int n4 = (nl + 3) >> 2;
+#pragma unroll 4
+        for (int c4 = tid; c4 < n4; c4 += kSelThreads) {
+            const uint4 v = __ldcg(g4 + c4);
+            const uint32_t xs[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int c = 4 * c4 + j;
+                const uint32_t x = c < nl ? xs[j] : 0u;
+                if (STAGE && c < nl) staged[c] = x;
+                if (x != 0u) {
+                    ++cnt;
+                    mn = min(mn, x);
+                    mx = max(mx, x);
+                }
+            }
+        }
+    } else {
+        for (int c = tid; c < nl; c += kSelThreads) {
+            const uint32_t x = keys(c);
+            if (STAGE) staged[c] = x;
+            if (x != 0u) {
+                ++cnt;
+                mn = min(mn, x);
+                mx = max(mx, x);
+            }
+        }
+    }
+    cnt = warp_sum(cnt);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    if (lane == 0) {
+        sh.warp_a[warp] = cnt;
+        sh.warp_b[warp] = mn;
+        sh.warp_c[warp] = mx;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        uint32_t c0 = 0, m0 = 0xFFFFFFFFu, m1 = 0u;
+        for (int w = 0; w < kSelWarps; ++w) {
+            c0 += sh.warp_a[w];
+            m0 = min(m0, sh.warp_b[w]);
+            m1 = max(m1, sh.warp_c[w]);
+        }
+        uint32_t* rs = cluster.map_shared_rank(&sh.stats[rank][0], 0);
+        rs[0] = c0;
+        rs[1] = m0;
+        rs[2] = m1;
+    }
+    if (STAGE) keys.smem = staged;
+    cluster.sync();
+    uint32_t nvalid = 0;
+    mn = 0xFFFFFFFFu;
+    mx = 0u;
+    {
+        const uint32_t* rs = cluster.map_shared_rank(&sh.stats[0][0], 0);
+        for (int r = 0; r < csize; ++r) {
+            nvalid += rs[3 * r];
+            mn = min(mn, rs[3 * r + 1]);
+            mx = max(mx, rs[3 * r + 2]);
+        }
+    }
+
+    // ---- threshold
     uint32_t T = 0;
     int take_eq = 0;
+    if (kk > 0 && nvalid > static_cast<uint32_t>(kk))
+        cluster_kth_key(cluster, keys, nl, s0, kk, mn, mx, sh, T, take_eq);
+
+    // ---- offsets from the lower ranks
+    uint32_t eq_base = 0, out_base = 0, kept_total = 0;
     if (kk > 0) {
-        uint32_t nvalid = 0;
-        for (int c = tid; c < n; c += kSelThreads) nvalid += keys(c) != 0u;
-        nvalid = block_sum(nvalid, sh);
-        if (nvalid > static_cast<uint32_t>(kk)) radix_threshold(keys, n, kk, sh, T, take_eq);
+        uint32_t gt_l, eq_l;
+        count_vs(keys, nl, T, sh, gt_l, eq_l);
+        if (tid == 0) {
+            uint32_t* rc = cluster.map_shared_rank(&sh.counts[rank][0], 0);
+            rc[0] = gt_l;
+            rc[1] = eq_l;
+        }
+        cluster.sync();
+        const uint32_t* rc = cluster.map_shared_rank(&sh.counts[0][0], 0);
+        uint32_t eqb = 0, outb = 0;
+        for (int r = 0; r < csize; ++r) {
+            const uint32_t g = rc[2 * r], e = rc[2 * r + 1];
+            const int room = take_eq - static_cast<int>(eqb);
+            const uint32_t take = room <= 0 ? 0u : (static_cast<uint32_t>(room) < e ? room : e);
+            if (r == rank) {
+                eq_base = eqb;
+                out_base = outb;
+            }
+            eqb += e;
+            outb += g + take;
+        }
+        kept_total = outb;
     }
 
+    // ---- outputs
     if (p.mode == kSelBlocks) {
         int32_t* out = p.blocks + static_cast<size_t>(row) * p.mm;
         int32_t* dbg = p.blocks_out ? p.blocks_out + static_cast<size_t>(row) * p.mm : nullptr;
-        int kept = 0;
         if (kk > 0)
-            kept = compact(keys, n, T, take_eq, sh, [&](int pos, int c, uint32_t) {
-                out[pos] = c;
-                if (dbg) dbg[pos] = c;
+            compact(keys, nl, T, take_eq, eq_base, out_base, sh, [&](int pos, int c, uint32_t) {
+                out[pos] = s0 + c;
+                if (dbg) dbg[pos] = s0 + c;
             });
-        __syncthreads();
-        for (int r = kept + tid; r < p.mm; r += kSelThreads) {
-            const int v = r == kept ? nb - 1 : -1;   // own block last (largest id)
-            out[r] = v;
-            if (dbg) dbg[r] = v;
+        if (rank == 0) {
+            for (int r = static_cast<int>(kept_total) + tid; r < p.mm; r += kSelThreads) {
+                const int v = r == static_cast<int>(kept_total) ? nb - 1 : -1;   // own block last
+                out[r] = v;
+                if (dbg) dbg[r] = v;
+            }
+            if (tid == 0) {
+                const int keep = static_cast<int>(kept_total) + 1;
+                p.nblocks[row] = keep;
+                if (p.nblocks_out) p.nblocks_out[row] = keep;
+                p.plan[row] = make_int4(b, t, keep, 0);
+            }
         }
-        if (tid == 0) {
-            p.nblocks[row] = kept + 1;
-            if (p.nblocks_out) p.nblocks_out[row] = kept + 1;
-        }
-        return;
+    } else {
+        int32_t* idx = p.idx + static_cast<size_t>(row) * p.k;
+        float* sc = p.scores ? p.scores + static_cast<size_t>(row) * p.k : nullptr;
+        const int32_t* blk =
+            p.mode == kSelHisaTokens ? p.blocks + static_cast<size_t>(row) * p.mm : nullptr;
+        const int Bsz = p.B;
+        compact(keys, nl, T, take_eq, eq_base, out_base, sh, [&](int pos, int c, uint32_t x) {
+            const int slot = s0 + c;
+            idx[pos] = blk ? blk[slot / Bsz] * Bsz + slot % Bsz : slot;
+            if (sc) sc[pos] = key_score(x);
+        });
+        if (rank == 0)
+            for (int r = static_cast<int>(kept_total) + tid; r < p.k; r += kSelThreads) {
+                idx[r] = -1;
+                if (sc) sc[r] = __int_as_float(0x7fc00000);
+            }
     }
+    cluster.sync();   // no CTA leaves while another may still read its shared memory
+}
 
-    int32_t* idx = p.idx + static_cast<size_t>(row) * p.k;
-    float* sc = p.scores ? p.scores + static_cast<size_t>(row) * p.k : nullptr;
-    const int32_t* blk = p.mode == kSelHisaTokens ? p.blocks + static_cast<size_t>(row) * p.mm : nullptr;
-    const int Bsz = p.B;
-    const int kept = compact(keys, n, T, take_eq, sh, [&](int pos, int c, uint32_t x) {
-        idx[pos] = blk ? blk[c / Bsz] * Bsz + c % Bsz : c;
-        if (sc) sc[pos] = key_score(x);
-    });
-    for (int r = kept + tid; r < p.k; r += kSelThreads) {
-        idx[r] = -1;
-        if (sc) sc[r] = __int_as_float(0x7fc00000);
-    }
+template <bool STAGE>
+cudaError_t launch_t(const SelectParams& p, int csize, int chunk, cudaStream_t s) {
+    const size_t smem = STAGE ? static_cast<size_t>(chunk) * sizeof(uint32_t) : 0;
+    auto* fn = select_kernel<STAGE>;
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(p.rows * csize));
+    cfg.blockDim = dim3(kSelThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(csize);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, fn, p);
 }
 
 }  // namespace
 
-cudaError_t launch_select(const SelectParams& p, int max_n, cudaStream_t s) {
+cudaError_t launch_select(const SelectParams& p, int max_n, int sms, cudaStream_t s) {
     if (p.rows <= 0) return cudaSuccess;
-    if (max_n <= kSmemKeys) {
-        const size_t smem = static_cast<size_t>(max_n > 0 ? max_n : 1) * sizeof(uint32_t);
-        cudaError_t e = cudaFuncSetAttribute(select_kernel<true>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(smem));
-        if (e != cudaSuccess) return e;
-        select_kernel<true><<<p.rows, kSelThreads, smem, s>>>(p);
-    } else {
-        select_kernel<false><<<p.rows, kSelThreads, 0, s>>>(p);
-    }
-    return cudaGetLastError();
+    // cluster size: enough CTAs to stage the longest row, and more while
+    // there are SMs to spare; chunks stay at least 1024 slots
+    int csize = 1;
+    while (csize < kMaxCluster && static_cast<long long>(csize) * kMaxChunk < max_n) csize *= 2;
+    while (csize < kMaxCluster && static_cast<long long>(p.rows) * csize * 2 <= sms &&
+           max_n / (csize * 2) >= 1024)
+        csize *= 2;
+    const int chunk = ((max_n + csize - 1) / csize + 127) & ~127;
+    cudaError_t e;
+    if (chunk <= kMaxChunk) e = launch_t<true>(p, csize, chunk > 0 ? chunk : 128, s);
+    else e = launch_t<false>(p, csize, 0, s);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    return e;
 }
 
 }  // namespace hisa

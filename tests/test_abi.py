@@ -112,7 +112,7 @@ def test_workspace_sizes(hisa):
     lib = hisa.lib()
     kv = _kv(hisa, cap=32768, B=128)
     ws = lib.hisa_select_workspace_bytes(ctypes.byref(kv), 64, 64, 64, 2048)
-    # block keys 64x256x4 + blocks 64x64x4 + counts 64x4 + token keys 64x8192x4
-    assert ws == 65536 + 16384 + 256 + 2097152
+    # block keys 64x256x4 + blocks 64x64x4 + counts 64x4 + plan 64x16 + token keys 64x8192x4
+    assert ws == 65536 + 16384 + 256 + 1024 + 2097152
     assert lib.dsa_flat_workspace_bytes(ctypes.byref(kv), 64, 64, 2048) == 64 * 32768 * 4
     assert lib.hisa_select_workspace_bytes(None, 1, 1, 1, 1) == 0
