@@ -187,7 +187,8 @@ def run_gpu(args, rank, world):
     K, W = args.steps, args.warmup
     E = args.e2e_steps
     n_flat = args.flat_steps
-    total_steps = W + K + E + 1
+    n_prof = min(K, 50)
+    total_steps = W + K + n_prof + 1 + E
     case = make_workload(total_steps, seed_shift=rank)
     kv = hisa.KVCache.from_case(case, device=dev)
     stream = torch.cuda.current_stream()
@@ -231,8 +232,6 @@ def run_gpu(args, rank, world):
         import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize()
-    hisa.hisa_profile_enable(True)
-    hisa.hisa_profile_read(reset=True)
     with ClockSampler(dev.index) as clk:
         wall0 = time.perf_counter()
         for i in range(K):
@@ -245,18 +244,28 @@ def run_gpu(args, rank, world):
         wall = time.perf_counter() - wall0
     if world > 1:
         dist.barrier()
-    phases = hisa.hisa_profile_read(reset=True)
-    hisa.hisa_profile_enable(False)
     step_ms = [a.elapsed_time(b) for a, b in ev]
     total_ms = float(sum(step_ms))
     if world > 1:
         t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         total_ms = float(t.item())
-    launches = sum(n for _, n in phases.values())
+    # Per-kernel durations: the same steps again with an event pair around
+    # every launch (separate pass: those events stop the launches from
+    # overlapping, so the timed steps above run without them).
+    hisa.hisa_profile_enable(True)
+    hisa.hisa_profile_read(reset=True)
+    for i in range(n_prof):
+        s = W + K + i
+        step(s, idx[s % 2])
+        flush.fill_(7)
+    torch.cuda.synchronize()
+    phases = hisa.hisa_profile_read(reset=True)
+    hisa.hisa_profile_enable(False)
+    launches = sum(n for _, n in phases.values()) * K // n_prof
 
     # select-only comparison: HISA vs the flat scan on the same rows
-    s_cmp = W + K
+    s_cmp = W + K + n_prof
     hisa.hisa_append(kv, toks[s_cmp])
     fws = hisa.workspace(hisa.dsa_flat_workspace_bytes(kv, batch, H, k), dev)
     fidx = torch.empty((batch, k), dtype=torch.int32, device=dev)
@@ -298,7 +307,7 @@ def run_gpu(args, rank, world):
         dW = torch.empty_like(Ws[0])
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(E)]
-        base = W + K + 1
+        base = W + K + n_prof + 1
         for i, (a, b) in enumerate(evs):
             s = base + i
             a.record(stream)
@@ -328,7 +337,7 @@ def run_gpu(args, rank, world):
     nb = -(-case.cap // case.B)
     pool_bytes = batch * 32768 * d * 2 + batch * nb * (d * 4 + 2 * d * 2)
     pool_gbs = pool_bytes / (float(np.median(pool_ms)) / 1e3) / 1e9
-    kernels = {name: {"ms_per_launch": (ms / n if n else None), "launches": n,
+    kernels = {name: {"ms_per_launch": (ms / n if n else None), "launches_profiled": n,
                       "share": ms / max(sum(x for x, _ in phases.values()), 1e-9)}
                for name, (ms, n) in phases.items() if n}
     return dict(
@@ -461,6 +470,8 @@ def main(argv=None):
                          "traffic": traffic, "peak_source": peaks["source"],
                          "algorithmic_bytes_per_launch": r["tok_bytes"]},
             "kernels": r["kernels"],
+            "kernels_note": "per-launch times from a separate pass of the same steps with an event "
+                            "pair around every launch",
             "pool": {"GB/s": r["pool_gbs"], "frac": r["pool_gbs"] / peaks["hbm_gbs"],
                      "ms": r["pool_ms"]},
             "flat_scan": {"ms_per_select": r["flat_ms"], "hisa_ms_per_select": r["hisa_sel_ms"],

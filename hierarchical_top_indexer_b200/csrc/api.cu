@@ -226,26 +226,23 @@ ScoreParams score_params(const KvView& v, const float* w, const int32_t* q_seq, 
     return p;
 }
 
-// Grid shape: `slices` CTAs per query row (so that few rows still spread over
-// every SM), groups of slices covering the rows, at most one CTA per SM.
+// Grid: one CTA per SM at most, each taking an equal contiguous range of the
+// row-major (row, tile) slots.
 int run_score(int mode, const KvView& v, const CUtensorMap& amap, const CUtensorMap& qmap,
               ScoreParams& p, cudaStream_t s) {
-    p.stages = score_stages(mode, mode != kScoreBlocks && v.e4m3, v.d, p.npad);
+    const bool e4m3 = mode != kScoreBlocks && v.e4m3;
+    score_stages(mode, e4m3, v.d, p.npad, &p.stages, &p.stages8);
     if (p.stages < 2) return HISA_E_UNSUPPORTED;
     p.total_tiles = static_cast<long long>(p.n_q) * p.tiles_per_row;
     if (p.total_tiles == 0) return HISA_OK;
     const int sms = sm_count();
     if (sms <= 0) return HISA_E_CUDA;
-    int slices = 1;
-    while (slices * 2 <= p.tiles_per_row && static_cast<long long>(p.n_q) * slices * 2 <= sms) slices *= 2;
-    const int groups = p.n_q < sms / slices ? p.n_q : sms / slices;
-    p.slices = slices;
+    const int grid = static_cast<int>(p.total_tiles < sms ? p.total_tiles : sms);
     const int phase = mode == kScoreBlocks ? HISA_PHASE_BLOCK_SCORE
                       : mode == kScoreFlat ? HISA_PHASE_FLAT_SCORE
                                            : HISA_PHASE_TOKEN_SCORE;
     PhaseScope ps(phase, s);
-    return cuda_status(
-        launch_score(mode, mode != kScoreBlocks && v.e4m3, v.d, amap, qmap, p, groups * slices, s));
+    return cuda_status(launch_score(mode, e4m3, v.d, amap, qmap, p, grid, s));
 }
 
 int hisa_select_impl(const hisa_kv* kv, const uint16_t* Q, const float* w, const int32_t* q_seq,
@@ -279,8 +276,9 @@ int hisa_select_impl(const hisa_kv* kv, const uint16_t* Q, const float* w, const
 
     if (counts && cudaMemsetAsync(counts, 0, sizeof(uint64_t) * 2 * n_q, s) != cudaSuccess)
         return HISA_E_CUDA;
+    const int sms = sm_count();
 
-    // stage 1: score the block representatives, keep the top-m blocks
+    // stage 1: score the block representatives, keep the own block + best m-1
     ScoreParams p = score_params(v, w, q_seq, q_pos, n_q, H);
     p.out = bkeys;
     p.ldo = L.ldb;
@@ -312,7 +310,7 @@ int hisa_select_impl(const hisa_kv* kv, const uint16_t* Q, const float* w, const
     sp.nblocks_out = nblocks_out;
     {
         PhaseScope ps(HISA_PHASE_BLOCK_SELECT, s);
-        rc = cuda_status(launch_select(sp, v.nblk, sm_count(), s));
+        rc = cuda_status(launch_select(sp, v.nblk, sms, s));
     }
     if (rc) return rc;
 
@@ -321,8 +319,7 @@ int hisa_select_impl(const hisa_kv* kv, const uint16_t* Q, const float* w, const
     p.ldo = L.ldt;
     p.tiles_per_row = L.ldt / 128;
     p.blocks = blocks;
-    p.nblocks = nblocks;
-    p.plan = plan;
+    p.plan_in = plan;
     p.mm = L.mm;
     rc = run_score(kScoreHisa, v, kmap, qmap, p, s);
     if (rc) return rc;
@@ -335,7 +332,7 @@ int hisa_select_impl(const hisa_kv* kv, const uint16_t* Q, const float* w, const
     sp.blocks_out = nullptr;
     sp.nblocks_out = nullptr;
     PhaseScope ps(HISA_PHASE_TOKEN_SELECT, s);
-    return cuda_status(launch_select(sp, L.mm * v.B, sm_count(), s));
+    return cuda_status(launch_select(sp, L.mm * v.B, sms, s));
 }
 
 }  // namespace

@@ -35,20 +35,19 @@ struct ScoreParams {
     const int32_t* q_seq;
     const int32_t* q_pos;
     int n_q, H, npad;
-    // kept blocks (kScoreHisa): blocks [n_q, mm], nblocks [n_q], and the
-    // row plan {sequence, position (-1: bad row), kept blocks, 0} [n_q]
+    // kept blocks (kScoreHisa input): blocks [n_q, mm], and the row plan
+    // {sequence, position (-1: invalid row), kept blocks, 0} [n_q]
     const int32_t* blocks;
-    const int32_t* nblocks;
-    const int4* plan;
+    const int4* plan_in;
     int mm;
-    // output: order-preserving score keys [n_q, ldo]; 0 = masked slot
+    // score keys [n_q, ldo] (order-preserving; 0 = masked slot)
     uint32_t* out;
     int ldo;
-    unsigned long long* counts;   // [n_q, 2] or null
-    int tiles_per_row;      // upper bound of candidate tiles per row
-    long long total_tiles;
-    int stages;
-    int slices;             // CTAs sharing one query row
+    unsigned long long* counts;   // [n_q, 2] or null: representatives / token slots scored
+    int tiles_per_row;            // tile slots per row (upper bound)
+    long long total_tiles;        // n_q * tiles_per_row
+    int stages;                   // bf16 operand stages
+    int stages8;                  // e4m3 staging stages
 };
 
 enum SelectMode : int {
@@ -88,8 +87,8 @@ cudaError_t launch_append(const KvView& kv, const void* tok, const float* tok_sc
 // Scoring: tensor maps built by the caller.  `keys_map` covers keys
 // ([batch*cap, d], bf16 swizzled 128B boxes, or e4m3 plain boxes) or, for
 // kScoreBlocks, pooled_hl ([batch*nblk, 2d] bf16).
-int score_stages(int mode, bool e4m3, int d, int npad);
-size_t score_smem_bytes(int mode, bool e4m3, int d, int npad, int stages);
+void score_stages(int mode, bool e4m3, int d, int npad, int* stages, int* stages8);
+size_t score_smem_bytes(int mode, bool e4m3, int d, int npad, int stages, int stages8);
 cudaError_t launch_score(int mode, bool e4m3, int d, const CUtensorMap& keys_map,
                          const CUtensorMap& q_map, const ScoreParams& p, int grid,
                          cudaStream_t s);

@@ -20,10 +20,10 @@
 // converter warps (exact), and their per-token scale multiplies the score
 // (ReLU(s*x) = s*ReLU(x) for s > 0).
 //
-// Work split: the CTAs form groups of `slices` CTAs; group g takes query
-// rows g, g + groups, ...; within a row, CTA r of the group scores the r-th
-// contiguous slice of the row's candidate tiles.  Row metadata is read once
-// per row; HISA block ids are prefetched one tile ahead.
+// Work split: the (row, tile) pairs are laid out row-major with a fixed
+// number of tile slots per row; CTA c takes the c-th contiguous range, so all
+// SMs get equal shares whatever the number of rows.  Score keys go to a
+// global row buffer that the selection kernel reads.
 //
 // Warp roles:
 //   warp 0       TMA producer (keys / representatives, query heads)
@@ -47,6 +47,7 @@ constexpr int kWarpConv0 = 6;
 constexpr int kMinSmem = 120 * 1024;          // keeps one CTA (and its TMEM) per SM
 constexpr int kMaxSmem = 232448;
 constexpr int kMaxAcc = 4;
+constexpr int kMaxStages = 8;
 
 struct Layout {
     uint32_t a, s8, q, w, bars, misc, total;
@@ -54,22 +55,21 @@ struct Layout {
 
 __host__ __device__ inline int acc_count(int npad) { return 4 * npad <= 512 ? 4 : 2; }
 
-__host__ __device__ inline Layout score_layout(int mode, bool e4m3, int d, int npad, int stages) {
+__host__ __device__ inline Layout score_layout(int mode, bool e4m3, int d, int npad, int sa, int s8) {
     const int halves = d / 64;
     const int stage = (mode == kScoreBlocks ? 2 : 1) * halves * kHalfBytes;
-    const int stage8 = e4m3 ? kTileRows * d : 0;
     Layout L;
     uint32_t off = 0;
     L.a = off;
-    off += stages * stage;
+    off += sa * stage;
     L.s8 = off;
-    off += stages * stage8;
+    off += e4m3 ? s8 * kTileRows * d : 0;
     L.q = off;
     off += 2 * halves * npad * 128;
     L.w = off;
     off += 4 * 128 * 4;                      // one 128-float weight slot per epilogue warp
     L.bars = off;
-    off += (4 * stages + 2 * kMaxAcc + 4) * 8;
+    off += (4 * kMaxStages + 2 * kMaxAcc + 4) * 8;
     L.misc = off;
     off += 16;
     L.total = off;
@@ -82,19 +82,19 @@ __host__ __device__ inline uint32_t tmem_columns(int npad) {
     return c;
 }
 
-// A query row as one CTA of its group sees it.
-struct RowSlice {
-    int b, t, lim;    // sequence, position, candidate slots of the row
-    int t0, t1;       // this CTA's tiles [t0, t1)
+// A query row: sequence, position, candidate slots, candidate tiles (0 if
+// the row is invalid).
+struct RowInfo {
+    int b, t, lim, nt;
 };
 
 template <int MODE>
-__device__ __forceinline__ RowSlice row_slice(const ScoreParams& p, int row, int rank, int slices) {
-    RowSlice R;
-    R.t0 = R.t1 = 0;
+__device__ __forceinline__ RowInfo load_row(const ScoreParams& p, int row) {
+    RowInfo R;
     R.lim = 0;
+    R.nt = 0;
     if (MODE == kScoreHisa) {
-        const int4 pl = p.plan[row];        // written by the block selection
+        const int4 pl = p.plan_in[row];     // written by the block selection
         R.b = pl.x;
         R.t = pl.y;
         if (R.t < 0) return R;
@@ -105,44 +105,8 @@ __device__ __forceinline__ RowSlice row_slice(const ScoreParams& p, int row, int
         R.lim = MODE == kScoreBlocks ? R.t / p.B + 1   // visible blocks
                                      : R.t + 1;        // visible keys
     }
-    const int nt = (R.lim + kTileRows - 1) / kTileRows;
-    R.t0 = static_cast<int>(static_cast<long long>(nt) * rank / slices);
-    R.t1 = static_cast<int>(static_cast<long long>(nt) * (rank + 1) / slices);
+    R.nt = (R.lim + kTileRows - 1) / kTileRows;
     return R;
-}
-
-// sum_h w_h * ReLU(acc_h) over the NP head columns of one TMEM lane: loads
-// of up to 64 columns at a time, one wait per group, four interleaved partial
-// sums (fixed order).
-template <int NP>
-__device__ __forceinline__ float head_sum(uint32_t taddr, const float* wv) {
-    float a[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int g = 0; g < NP; g += 64) {
-        constexpr int kG = NP < 64 ? NP : 64;
-        uint32_t r[kG];
-#pragma unroll
-        for (int c = 0; c < kG; c += 16)
-            if (g + c < NP) tmem_ld16_nowait(taddr + g + c, r + c);
-        tmem_ld_wait();
-#pragma unroll
-        for (int h = 0; h < kG; ++h)
-            if (g + h < NP) a[h & 3] = fmaf(wv[g + h], fmaxf(__uint_as_float(r[h]), 0.f), a[h & 3]);
-    }
-    return (a[0] + a[1]) + (a[2] + a[3]);
-}
-
-__device__ __forceinline__ float head_sum_any(int npad, uint32_t taddr, const float* wv) {
-    switch (npad) {
-        case 16: return head_sum<16>(taddr, wv);
-        case 32: return head_sum<32>(taddr, wv);
-        case 48: return head_sum<48>(taddr, wv);
-        case 64: return head_sum<64>(taddr, wv);
-        case 80: return head_sum<80>(taddr, wv);
-        case 96: return head_sum<96>(taddr, wv);
-        case 112: return head_sum<112>(taddr, wv);
-        default: return head_sum<128>(taddr, wv);
-    }
 }
 
 __device__ __forceinline__ void raise_abort(volatile int* abort_flag, uint32_t* status) {
@@ -178,15 +142,57 @@ __device__ __forceinline__ uint4 e4m3x8_to_bf16x8(uint2 raw) {
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// First key row of sub-box `sub` of tile `ti` (lanes hold one sub-box each).
+// First key row of sub-box `sub` of tile `ti`.
 template <int MODE>
-__device__ __forceinline__ int tile_sub_row(const ScoreParams& p, const RowSlice& R, int row, int ti,
+__device__ __forceinline__ int tile_sub_row(const ScoreParams& p, const RowInfo& R, int row, int ti,
                                             int sub, int BR) {
     if (MODE == kScoreBlocks) return R.b * p.nblk + ti * kTileRows;
     if (MODE == kScoreFlat) return R.b * p.cap + ti * kTileRows + sub * BR;
     const int slot = ti * kTileRows + sub * BR;
     const int blk = slot < R.lim ? __ldg(p.blocks + static_cast<size_t>(row) * p.mm + slot / p.B) : 0;
     return R.b * p.cap + blk * p.B + slot % p.B;
+}
+
+// Shared-memory load the compiler keeps in place (the head weights are read
+// per tile instead of being held in registers across the tile loop).
+__device__ __forceinline__ float lds_f32(const float* p) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(smem_addr(p)));
+    return v;
+}
+
+// sum_h w_h * ReLU(acc_h) over the NP head columns of one TMEM lane: loads
+// of up to 64 columns at a time, one wait per group, four interleaved partial
+// sums (fixed order).
+template <int NP>
+__device__ __forceinline__ float head_sum(uint32_t taddr, const float* wv) {
+    float a[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int g = 0; g < NP; g += 64) {
+        constexpr int kG = NP < 64 ? NP : 64;
+        uint32_t r[kG];
+#pragma unroll
+        for (int c = 0; c < kG; c += 16)
+            if (g + c < NP) tmem_ld16_nowait(taddr + g + c, r + c);
+        tmem_ld_wait();
+#pragma unroll
+        for (int h = 0; h < kG; ++h)
+            if (g + h < NP) a[h & 3] = fmaf(lds_f32(wv + g + h), fmaxf(__uint_as_float(r[h]), 0.f), a[h & 3]);
+    }
+    return (a[0] + a[1]) + (a[2] + a[3]);
+}
+
+__device__ __forceinline__ float head_sum_any(int npad, uint32_t taddr, const float* wv) {
+    switch (npad) {
+        case 16: return head_sum<16>(taddr, wv);
+        case 32: return head_sum<32>(taddr, wv);
+        case 48: return head_sum<48>(taddr, wv);
+        case 64: return head_sum<64>(taddr, wv);
+        case 80: return head_sum<80>(taddr, wv);
+        case 96: return head_sum<96>(taddr, wv);
+        case 112: return head_sum<112>(taddr, wv);
+        default: return head_sum<128>(taddr, wv);
+    }
 }
 
 template <int MODE, bool E4M3, int D>
@@ -201,22 +207,23 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    const Layout L = score_layout(MODE, E4M3, D, p.npad, p.stages);
-    const int S = p.stages;
+    const int SA = p.stages;                    // bf16 operand stages
+    const int S8 = E4M3 ? p.stages8 : 1;        // e4m3 staging stages
+    const Layout L = score_layout(MODE, E4M3, D, p.npad, SA, S8);
     const int NACC = acc_count(p.npad);
     uint8_t* sA = smem + L.a;
     uint8_t* s8 = smem + L.s8;
     uint8_t* sQ = smem + L.q;
     float* sW = reinterpret_cast<float*>(smem + L.w);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
-    uint64_t* full = bars;                   // stage holds bf16 operands (TMA or converters)
-    uint64_t* empty = bars + S;              // stage free again (UMMA done reading)
-    uint64_t* sfull = bars + 2 * S;          // e4m3 staging landed
-    uint64_t* sempty = bars + 3 * S;         // e4m3 staging converted
-    uint64_t* tfull = bars + 4 * S;          // accumulator ready   [kMaxAcc]
-    uint64_t* tempty = tfull + kMaxAcc;      // accumulator drained [kMaxAcc]
-    uint64_t* qfull = tempty + kMaxAcc;      // query heads landed  [2]
-    uint64_t* qempty = qfull + 2;            // query heads free    [2]
+    uint64_t* full = bars;                         // operand stage ready   [SA]
+    uint64_t* empty = bars + kMaxStages;           // operand stage free    [SA]
+    uint64_t* sfull = bars + 2 * kMaxStages;       // e4m3 staging landed   [S8]
+    uint64_t* sempty = bars + 3 * kMaxStages;      // e4m3 staging consumed [S8]
+    uint64_t* tfull = bars + 4 * kMaxStages;       // accumulator ready   [kMaxAcc]
+    uint64_t* tempty = tfull + kMaxAcc;            // accumulator drained [kMaxAcc]
+    uint64_t* qfull = tempty + kMaxAcc;            // query heads landed  [2]
+    uint64_t* qempty = qfull + 2;                  // query heads free    [2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.misc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.misc + 4);
 
@@ -225,17 +232,18 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
     const int npad = p.npad;
     const uint32_t ncols = tmem_columns(npad);
     const int q_slot_bytes = kHalves * npad * 128;
-    const int slices = p.slices;
-    const int rank = blockIdx.x % slices;
-    const int group = blockIdx.x / slices;
-    const int groups = gridDim.x / slices;
+    const int tpr = p.tiles_per_row;
     const int BR = (MODE == kScoreBlocks) ? kTileRows : (p.B < kTileRows ? p.B : kTileRows);
     const int nsub = kTileRows / BR;
+    const long long g0 = p.total_tiles * blockIdx.x / gridDim.x;
+    const long long g1 = p.total_tiles * (blockIdx.x + 1) / gridDim.x;
 
     if (warp == kWarpProducer && lane == 0) {
-        for (int s = 0; s < S; ++s) {
+        for (int s = 0; s < SA; ++s) {
             mbar_init(full + s, E4M3 ? 4 : 1);
             mbar_init(empty + s, 1);
+        }
+        for (int s = 0; s < S8; ++s) {
             mbar_init(sfull + s, 1);
             mbar_init(sempty + s, 4);
         }
@@ -267,85 +275,102 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
 
     if (warp == kWarpProducer) {
         const uint64_t pol = policy_evict_first();
-        int it = 0, qloads = 0;
+        int it = 0, qloads = 0, cur_row = -1, tb = 0;
+        RowInfo R;
+        R.nt = 0;
+        int win_cur = 0, win_nxt = 0, cur_w = 0;
         bool ok = true;
-        for (int row = group; row < p.n_q && ok; row += groups) {
-            const RowSlice R = row_slice<MODE>(p, row, rank, slices);
-            if (R.t0 >= R.t1) continue;
-            const int qs = qloads & 1;
-            if (qloads >= 2 && !warp_wait(qempty + qs, ((qloads - 2) >> 1) & 1, abort_flag)) {
+        for (long long g = g0; g < g1 && ok;) {
+            const int row = static_cast<int>(g / tpr);
+            const int ti = static_cast<int>(g % tpr);
+            if (row != cur_row) {
+                cur_row = row;
+                R = load_row<MODE>(p, row);
+                if (ti < R.nt) {
+                    // new row with work here: its query heads and block-id windows
+                    const int qs = qloads & 1;
+                    if (qloads >= 2 && !warp_wait(qempty + qs, ((qloads - 2) >> 1) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(qfull + qs, q_slot_bytes);
+#pragma unroll
+                        for (int kh = 0; kh < kHalves; ++kh)
+                            tma_load_2d(sQ + qs * q_slot_bytes + kh * npad * 128, &qmap, qfull + qs,
+                                        kh * 64, row * p.H);
+                    }
+                    ++qloads;
+                    tb = ti;
+                    const int nsub_row = (R.nt - tb) * nsub;
+                    const int gsub0 = lane, gsub1 = 32 + lane;
+                    win_cur = gsub0 < nsub_row
+                                  ? tile_sub_row<MODE>(p, R, row, tb + gsub0 / nsub, gsub0 % nsub, BR)
+                                  : 0;
+                    win_nxt = gsub1 < nsub_row
+                                  ? tile_sub_row<MODE>(p, R, row, tb + gsub1 / nsub, gsub1 % nsub, BR)
+                                  : 0;
+                    cur_w = 0;
+                }
+            }
+            if (ti >= R.nt) {
+                g = static_cast<long long>(row + 1) * tpr;
+                continue;
+            }
+            const int gs = (ti - tb) * nsub;
+            if ((gs >> 5) != cur_w) {
+                cur_w = gs >> 5;
+                win_cur = win_nxt;
+                const int gn = 32 * (cur_w + 1) + lane;
+                win_nxt = gn < (R.nt - tb) * nsub
+                              ? tile_sub_row<MODE>(p, R, row, tb + gn / nsub, gn % nsub, BR)
+                              : 0;
+            }
+            const int ss = E4M3 ? it % S8 : it % SA;
+            const uint32_t ph = (E4M3 ? it / S8 : it / SA) & 1;
+            uint64_t* fb = E4M3 ? sfull + ss : full + ss;
+            uint64_t* eb = E4M3 ? sempty + ss : empty + ss;
+            if (!warp_wait(eb, ph ^ 1, abort_flag)) {
                 ok = false;
                 break;
             }
-            if (lane == 0) {
-                mbar_arrive_expect_tx(qfull + qs, q_slot_bytes);
+            if (MODE == kScoreBlocks) {
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(fb, kStageBytes);
 #pragma unroll
-                for (int kh = 0; kh < kHalves; ++kh)
-                    tma_load_2d(sQ + qs * q_slot_bytes + kh * npad * 128, &qmap, qfull + qs, kh * 64,
-                                row * p.H);
-            }
-            ++qloads;
-            // Lane j holds the first key row of sub-box 32*w + j of this slice
-            // for the current window w and the next one (prefetched).
-            const int nsub_slice = (R.t1 - R.t0) * nsub;
-            auto window = [&](int w) -> int {
-                const int g = 32 * w + lane;
-                return g < nsub_slice ? tile_sub_row<MODE>(p, R, row, R.t0 + g / nsub, g % nsub, BR) : 0;
-            };
-            int win_cur = window(0);
-            int win_nxt = window(1);
-            int cur_w = 0;
-            for (int ti = R.t0; ti < R.t1; ++ti) {
-                const int g0 = (ti - R.t0) * nsub;
-                if ((g0 >> 5) != cur_w) {
-                    cur_w = g0 >> 5;
-                    win_cur = win_nxt;
-                    win_nxt = window(cur_w + 1);
+                    for (int op = 0; op < 2; ++op)
+#pragma unroll
+                        for (int kh = 0; kh < kHalves; ++kh)
+                            tma_load_2d(sA + ss * kStageBytes + (op * kHalves + kh) * kHalfBytes, &amap, fb,
+                                        op * D + kh * 64, R.b * p.nblk + ti * kTileRows);
                 }
-                const int s = it % S;
-                const uint32_t ph = (it / S) & 1;
-                uint64_t* fb = E4M3 ? sfull + s : full + s;
-                uint64_t* eb = E4M3 ? sempty + s : empty + s;
-                if (!warp_wait(eb, ph ^ 1, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                if (MODE == kScoreBlocks) {
-                    if (lane == 0) {
-                        mbar_arrive_expect_tx(fb, kStageBytes);
+            } else {
+                if (lane == 0) mbar_arrive_expect_tx(fb, E4M3 ? kStage8Bytes : kStageBytes);
+                for (int sub = 0; sub < nsub; ++sub) {
+                    const int srow = __shfl_sync(0xffffffffu, win_cur, (gs & 31) + sub);
+                    if (lane != 0) continue;
+                    if (E4M3) {
+                        tma_load_2d_hint(s8 + ss * kStage8Bytes + sub * BR * D, &amap, fb, 0, srow, pol);
+                    } else {
 #pragma unroll
-                        for (int op = 0; op < 2; ++op)
-#pragma unroll
-                            for (int kh = 0; kh < kHalves; ++kh)
-                                tma_load_2d(sA + s * kStageBytes + (op * kHalves + kh) * kHalfBytes,
-                                            &amap, fb, op * D + kh * 64, R.b * p.nblk + ti * kTileRows);
-                    }
-                } else {
-                    if (lane == 0) mbar_arrive_expect_tx(fb, E4M3 ? kStage8Bytes : kStageBytes);
-                    for (int sub = 0; sub < nsub; ++sub) {
-                        const int srow = __shfl_sync(0xffffffffu, win_cur, (g0 & 31) + sub);
-                        if (lane != 0) continue;
-                        if (E4M3) {
-                            tma_load_2d_hint(s8 + s * kStage8Bytes + sub * BR * D, &amap, fb, 0, srow, pol);
-                        } else {
-#pragma unroll
-                            for (int kh = 0; kh < kHalves; ++kh)
-                                tma_load_2d_hint(sA + s * kStageBytes + kh * kHalfBytes + sub * BR * 128,
-                                                 &amap, fb, kh * 64, srow, pol);
-                        }
+                        for (int kh = 0; kh < kHalves; ++kh)
+                            tma_load_2d_hint(sA + ss * kStageBytes + kh * kHalfBytes + sub * BR * 128, &amap,
+                                             fb, kh * 64, srow, pol);
                     }
                 }
-                __syncwarp();
-                ++it;
             }
+            __syncwarp();
+            ++it;
+            ++g;
         }
         if (lane == 0) {
             if (!ok) raise_abort(abort_flag, p.status);
             // Drain: no copy into, and no arrive on, this CTA's shared memory
             // may still be pending when it exits.
-            for (int n = it > S ? it - S : 0; n < it; ++n) {
-                const int s = n % S;
-                const uint32_t ph = (n / S) & 1;
+            const int NS = E4M3 ? S8 : SA;
+            for (int n = it > NS ? it - NS : 0; n < it; ++n) {
+                const int s = n % NS;
+                const uint32_t ph = (n / NS) & 1;
                 if (ok) mbar_wait(E4M3 ? sempty + s : empty + s, ph, nullptr);
                 else mbar_wait(E4M3 ? sfull + s : full + s, ph, nullptr);
             }
@@ -358,148 +383,180 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
     } else if (warp == kWarpMma) {
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16_f32(static_cast<uint32_t>(npad));
-            int it = 0, qloads = 0;
+            int it = 0, qloads = 0, cur_row = -1;
+            uint32_t q_base = 0;
+            RowInfo R;
+            R.nt = 0;
             bool ok = true;
-            for (int row = group; row < p.n_q && ok; row += groups) {
-                const RowSlice R = row_slice<MODE>(p, row, rank, slices);
-                if (R.t0 >= R.t1) continue;
-                if (qloads > 0) umma_commit(qempty + ((qloads - 1) & 1));
-                if (!mbar_wait(qfull + (qloads & 1), (qloads >> 1) & 1, abort_flag)) {
+            for (long long g = g0; g < g1 && ok;) {
+                const int row = static_cast<int>(g / tpr);
+                const int ti = static_cast<int>(g % tpr);
+                if (row != cur_row) {
+                    cur_row = row;
+                    R = load_row<MODE>(p, row);
+                    if (ti < R.nt) {
+                        if (qloads > 0) umma_commit(qempty + ((qloads - 1) & 1));
+                        if (!mbar_wait(qfull + (qloads & 1), (qloads >> 1) & 1, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        q_base = smem_addr(sQ + (qloads & 1) * q_slot_bytes);
+                        ++qloads;
+                    }
+                }
+                if (ti >= R.nt) {
+                    g = static_cast<long long>(row + 1) * tpr;
+                    continue;
+                }
+                const int s = it % SA;
+                const int a = it % NACC;
+                if (!mbar_wait(full + s, (it / SA) & 1, abort_flag) ||
+                    !mbar_wait(tempty + a, ((it / NACC) & 1) ^ 1, abort_flag)) {
                     ok = false;
                     break;
                 }
-                const uint32_t q_base = smem_addr(sQ + (qloads & 1) * q_slot_bytes);
-                ++qloads;
-                for (int ti = R.t0; ti < R.t1; ++ti) {
-                    const int s = it % S;
-                    const int a = it % NACC;
-                    if (!mbar_wait(full + s, (it / S) & 1, abort_flag) ||
-                        !mbar_wait(tempty + a, ((it / NACC) & 1) ^ 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * npad);
-                    const uint32_t a_base = smem_addr(sA + s * kStageBytes);
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * npad);
+                const uint32_t a_base = smem_addr(sA + s * kStageBytes);
 #pragma unroll
-                    for (int kh = 0; kh < kHalves; ++kh) {
+                for (int kh = 0; kh < kHalves; ++kh) {
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            const uint64_t bdesc = sw128_kmajor_desc(q_base + kh * npad * 128 + kk * 32);
-                            const uint64_t adesc = sw128_kmajor_desc(a_base + kh * kHalfBytes + kk * 32);
-                            umma_bf16(d_tmem, adesc, bdesc, idesc, (kh | kk) ? 1u : 0u);
-                            if (MODE == kScoreBlocks) {
-                                const uint64_t ldesc =
-                                    sw128_kmajor_desc(a_base + (kHalves + kh) * kHalfBytes + kk * 32);
-                                umma_bf16(d_tmem, ldesc, bdesc, idesc, 1u);
-                            }
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t bdesc = sw128_kmajor_desc(q_base + kh * npad * 128 + kk * 32);
+                        const uint64_t adesc = sw128_kmajor_desc(a_base + kh * kHalfBytes + kk * 32);
+                        umma_bf16(d_tmem, adesc, bdesc, idesc, (kh | kk) ? 1u : 0u);
+                        if (MODE == kScoreBlocks) {
+                            const uint64_t ldesc =
+                                sw128_kmajor_desc(a_base + (kHalves + kh) * kHalfBytes + kk * 32);
+                            umma_bf16(d_tmem, ldesc, bdesc, idesc, 1u);
                         }
                     }
-                    umma_commit(empty + s);
-                    umma_commit(tfull + a);
-                    ++it;
                 }
+                umma_commit(empty + s);
+                umma_commit(tfull + a);
+                ++it;
+                ++g;
             }
             if (!ok) raise_abort(abort_flag, p.status);
             // every UMMA of this CTA has finished before TMEM is released
             if (it > 0) mbar_wait(tfull + ((it - 1) % NACC), ((it - 1) / NACC) & 1, nullptr);
         }
     } else if (warp >= kWarpEpi0 && warp < kWarpEpi0 + 4) {
-        const int quad = warp & 3;             // TMEM lanes this warp may read
-        const int r = quad * 32 + lane;        // tile row = candidate
+        const int quad = warp & 3;                    // TMEM lanes this warp may read
+        const int r = quad * 32 + lane;               // tile row = candidate
         float* wv = sW + (warp - kWarpEpi0) * 128;
-        int it = 0;
+        int it = 0, cur_row = -1;
+        RowInfo R;
+        R.nt = 0;
         bool ok = true;
-        for (int row = group; row < p.n_q && ok; row += groups) {
-            const RowSlice R = row_slice<MODE>(p, row, rank, slices);
-            if (R.t0 >= R.t1) continue;
-            __syncwarp();
-            for (int h = lane; h < 128; h += 32) wv[h] = h < p.H ? p.w[row * p.H + h] : 0.f;
-            __syncwarp();
-            uint32_t* out = p.out + static_cast<size_t>(row) * p.ldo;
-            const int own_rank = R.lim / p.B - 1;         // HISA: the own block is listed last
-            const int t_in_own = R.t % p.B;
-            for (int ti = R.t0; ti < R.t1; ++ti) {
-                const int c = ti * kTileRows + r;
-                // validity and (e4m3) scale, fetched before waiting for the MMA
-                bool valid;
-                float scale = 1.f;
-                if (MODE == kScoreBlocks) {
-                    valid = c < R.lim;
-                } else if (MODE == kScoreFlat) {
-                    valid = c <= R.t;
-                    if (E4M3 && valid) scale = __ldg(p.key_scale + static_cast<size_t>(R.b) * p.cap + c);
-                } else {
-                    const int br = c / p.B, o = c % p.B;
-                    valid = c < R.lim && (br < own_rank || o <= t_in_own);
-                    if (E4M3 && valid) {
-                        const int blk = __ldg(p.blocks + static_cast<size_t>(row) * p.mm + br);
-                        scale = __ldg(p.key_scale + static_cast<size_t>(R.b) * p.cap + blk * p.B + o);
-                    }
+        for (long long g = g0; g < g1;) {
+            const int row = static_cast<int>(g / tpr);
+            const int ti = static_cast<int>(g % tpr);
+            if (row != cur_row) {
+                cur_row = row;
+                R = load_row<MODE>(p, row);
+                if (ti < R.nt) {
+                    __syncwarp();
+                    for (int h = lane; h < 128; h += 32) wv[h] = h < p.H ? p.w[row * p.H + h] : 0.f;
+                    __syncwarp();
                 }
-                const int a = it % NACC;
-                if (!mbar_wait(tfull + a, (it / NACC) & 1, abort_flag)) {
-                    ok = false;
-                    break;
+            }
+            if (ti >= R.nt) {
+                g = static_cast<long long>(row + 1) * tpr;
+                continue;
+            }
+            const int c = ti * kTileRows + r;
+            bool valid;
+            float scale = 1.f;
+            if (MODE == kScoreBlocks) {
+                valid = c < R.lim;
+            } else if (MODE == kScoreFlat) {
+                valid = c <= R.t;
+                if (E4M3 && valid) scale = __ldg(p.key_scale + static_cast<size_t>(R.b) * p.cap + c);
+            } else {
+                const int br = c / p.B, o = c % p.B;
+                const int own_rank = R.lim / p.B - 1;    // the own block is listed last
+                valid = c < R.lim && (br < own_rank || o <= R.t % p.B);
+                if (E4M3 && valid) {
+                    const int blk = __ldg(p.blocks + static_cast<size_t>(row) * p.mm + br);
+                    scale = __ldg(p.key_scale + static_cast<size_t>(R.b) * p.cap + blk * p.B + o);
                 }
+            }
+            const int a = it % NACC;
+            float acc = 0.f;
+            if (ok && mbar_wait(tfull + a, (it / NACC) & 1, abort_flag)) {
                 tc_fence_after();
                 const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                                        static_cast<uint32_t>(a * npad);
-                float acc = head_sum_any(npad, taddr, wv);
+                acc = head_sum_any(npad, taddr, wv);
                 tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(tempty + a);
-                if (E4M3) acc *= scale;
-                out[c] = valid ? score_key(acc) : 0u;
-                if (p.counts) {
-                    const bool slot = MODE == kScoreBlocks ? valid : c < R.lim;
-                    const int n = __popc(__ballot_sync(0xffffffffu, slot));
-                    if (lane == 0 && n)
-                        atomicAdd(p.counts + 2 * row + (MODE == kScoreBlocks ? 0 : 1),
-                                  static_cast<unsigned long long>(n));
-                }
-                ++it;
+            } else if (ok) {
+                ok = false;
+                raise_abort(abort_flag, p.status);
             }
+            __syncwarp();
+            if (lane == 0 && ok) mbar_arrive(tempty + a);
+            if (E4M3) acc *= scale;
+            p.out[static_cast<size_t>(row) * p.ldo + c] = valid ? score_key(acc) : 0u;
+            if (p.counts) {
+                const bool slot = MODE == kScoreBlocks ? valid : c < R.lim;
+                const int n = __popc(__ballot_sync(0xffffffffu, slot));
+                if (lane == 0 && n)
+                    atomicAdd(p.counts + 2 * row + (MODE == kScoreBlocks ? 0 : 1),
+                              static_cast<unsigned long long>(n));
+            }
+            ++it;
+            ++g;
         }
-        if (!ok) raise_abort(abort_flag, p.status);
     } else if (E4M3 && warp >= kWarpConv0) {
         const int cw = warp - kWarpConv0;
-        int it = 0;
+        int it = 0, cur_row = -1;
+        RowInfo R;
+        R.nt = 0;
         bool ok = true;
-        for (int row = group; row < p.n_q && ok; row += groups) {
-            const RowSlice R = row_slice<MODE>(p, row, rank, slices);
-            for (int ti = R.t0; ti < R.t1; ++ti) {
-                const int s = it % S;
-                const uint32_t ph = (it / S) & 1;
-                if (!mbar_wait(sfull + s, ph, abort_flag) || !mbar_wait(empty + s, ph ^ 1, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                const uint8_t* src = s8 + s * kStage8Bytes;
-                uint8_t* dst = sA + s * kStageBytes;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int rr = cw * 32 + i * 4 + (lane >> 3);
-                    const int cc = lane & 7;
-#pragma unroll
-                    for (int kh = 0; kh < kHalves; ++kh) {
-                        const uint2 raw = *reinterpret_cast<const uint2*>(src + rr * D + kh * 64 + cc * 8);
-                        *reinterpret_cast<uint4*>(dst + kh * kHalfBytes + rr * 128 + ((cc ^ (rr & 7)) << 4)) =
-                            e4m3x8_to_bf16x8(raw);
-                    }
-                }
-                fence_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(full + s);
-                    mbar_arrive(sempty + s);
-                }
-                ++it;
+        for (long long g = g0; g < g1 && ok;) {
+            const int row = static_cast<int>(g / tpr);
+            const int ti = static_cast<int>(g % tpr);
+            if (row != cur_row) {
+                cur_row = row;
+                R = load_row<MODE>(p, row);
             }
+            if (ti >= R.nt) {
+                g = static_cast<long long>(row + 1) * tpr;
+                continue;
+            }
+            const int s8i = it % S8;
+            const int sa = it % SA;
+            if (!mbar_wait(sfull + s8i, (it / S8) & 1, abort_flag) ||
+                !mbar_wait(empty + sa, ((it / SA) & 1) ^ 1, abort_flag)) {
+                ok = false;
+                break;
+            }
+            const uint8_t* src = s8 + s8i * kStage8Bytes;
+            uint8_t* dst = sA + sa * kStageBytes;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int rr = cw * 32 + i * 4 + (lane >> 3);
+                const int cc = lane & 7;
+#pragma unroll
+                for (int kh = 0; kh < kHalves; ++kh) {
+                    const uint2 raw = *reinterpret_cast<const uint2*>(src + rr * D + kh * 64 + cc * 8);
+                    *reinterpret_cast<uint4*>(dst + kh * kHalfBytes + rr * 128 + ((cc ^ (rr & 7)) << 4)) =
+                        e4m3x8_to_bf16x8(raw);
+                }
+            }
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(full + sa);
+                mbar_arrive(sempty + s8i);
+            }
+            ++it;
+            ++g;
         }
         if (!ok) raise_abort(abort_flag, p.status);
         if (ok && cw == 0 && lane == 0)
-            for (int n = it > S ? it - S : 0; n < it; ++n) mbar_wait(empty + n % S, (n / S) & 1, nullptr);
+            for (int n = it > SA ? it - SA : 0; n < it; ++n) mbar_wait(empty + n % SA, (n / SA) & 1, nullptr);
     }
 
     tc_fence_before();
@@ -511,7 +568,7 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
 template <int MODE, bool E4M3, int D>
 cudaError_t launch_t(const CUtensorMap& amap, const CUtensorMap& qmap, const ScoreParams& p, int grid,
                      cudaStream_t s) {
-    const size_t smem = score_smem_bytes(MODE, E4M3, D, p.npad, p.stages);
+    const size_t smem = score_smem_bytes(MODE, E4M3, D, p.npad, p.stages, p.stages8);
     auto* fn = score_kernel<MODE, E4M3, D>;
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
@@ -532,16 +589,27 @@ cudaError_t launch_t(const CUtensorMap& amap, const CUtensorMap& qmap, const Sco
 
 }  // namespace
 
-size_t score_smem_bytes(int mode, bool e4m3, int d, int npad, int stages) {
-    const size_t need = score_layout(mode, e4m3, d, npad, stages).total + 1024;
+size_t score_smem_bytes(int mode, bool e4m3, int d, int npad, int stages, int stages8) {
+    const size_t need = score_layout(mode, e4m3, d, npad, stages, stages8).total + 1024;
     return need < static_cast<size_t>(kMinSmem) ? static_cast<size_t>(kMinSmem) : need;
 }
 
-int score_stages(int mode, bool e4m3, int d, int npad) {
-    int best = 0;
-    for (int s = 2; s <= 8; ++s)
-        if (score_layout(mode, e4m3, d, npad, s).total + 1024 <= static_cast<uint32_t>(kMaxSmem)) best = s;
-    return best;
+// Operand stages (and e4m3 staging stages): as many as fit; the e4m3 path
+// keeps two bf16 operand stages and spends the rest on staging.
+void score_stages(int mode, bool e4m3, int d, int npad, int* stages, int* stages8) {
+    *stages = 0;
+    *stages8 = 0;
+    if (!e4m3) {
+        for (int s = 2; s <= kMaxStages; ++s)
+            if (score_layout(mode, false, d, npad, s, 0).total + 1024 <= static_cast<uint32_t>(kMaxSmem))
+                *stages = s;
+        return;
+    }
+    for (int s8 = 2; s8 <= kMaxStages; ++s8)
+        if (score_layout(mode, true, d, npad, 2, s8).total + 1024 <= static_cast<uint32_t>(kMaxSmem)) {
+            *stages = 2;
+            *stages8 = s8;
+        }
 }
 
 cudaError_t launch_score(int mode, bool e4m3, int d, const CUtensorMap& amap, const CUtensorMap& qmap,

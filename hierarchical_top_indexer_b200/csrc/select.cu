@@ -485,6 +485,338 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectPara
     cluster.sync();   // no CTA leaves while another may still read its shared memory
 }
 
+// ------------------------------------------------ single-CTA rows
+//
+// Rows of up to kRowKeys slots: one CTA of kRowThreads, keys staged in shared
+// memory, the same four steps without any cross-CTA exchange.
+
+constexpr int kRowThreads = 512;
+constexpr int kRowWarps = kRowThreads / 32;
+constexpr int kRowKeys = 24576;
+
+struct RowShared {
+    uint32_t hist[kBins];
+    unsigned long long members[kMembersCap];
+    uint32_t wa[kRowWarps];
+    uint32_t wb[kRowWarps];
+    uint32_t wc[kRowWarps];
+    uint32_t wd[kRowWarps];
+    uint32_t bc[8];
+};
+
+// Exclusive block scan of one value per thread (512 threads).
+__device__ __forceinline__ uint32_t row_scan(uint32_t v, uint32_t* wtot, uint32_t* total) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint32_t incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += x;
+    }
+    if (lane == 31) wtot[warp] = incl;
+    __syncthreads();
+    uint32_t before = 0, tot = 0;
+#pragma unroll
+    for (int w = 0; w < kRowWarps; ++w) {
+        const uint32_t x = wtot[w];
+        before += w < warp ? x : 0u;
+        tot += x;
+    }
+    *total = tot;
+    return before + incl - v;
+}
+
+__global__ void __launch_bounds__(kRowThreads) select_row_kernel(const SelectParams p) {
+    extern __shared__ uint32_t ks[];
+    __shared__ RowShared sh;
+    grid_dependency_wait();
+    grid_launch_dependents();
+    const int row = blockIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    int n = 0, kk = p.k, b = 0, t = 0, nb = 0;
+    bool bad = false;
+    if (p.mode == kSelF32Rows) {
+        n = p.n;
+    } else if (p.mode == kSelHisaTokens) {
+        const int4 pl = p.plan[row];
+        b = pl.x;
+        t = pl.y;
+        bad = t < 0;
+        n = pl.z * p.B;
+    } else {
+        t = query_position(p.q_seq, p.q_pos, p.len, p.batch, p.cap, row, &b);
+        bad = t < 0;
+        if (p.mode == kSelBlocks) {
+            nb = t / p.B + 1;
+            n = nb - 1;
+            kk = p.m - 1;
+        } else {
+            n = t + 1;
+        }
+    }
+    if (bad || (p.mode == kSelBlocks && nb <= p.m)) {
+        if (p.mode == kSelBlocks) {
+            const int keep = bad ? 0 : nb;
+            for (int r = tid; r < p.mm; r += kRowThreads) {
+                const int v = r < keep ? r : -1;
+                p.blocks[static_cast<size_t>(row) * p.mm + r] = v;
+                if (p.blocks_out) p.blocks_out[static_cast<size_t>(row) * p.mm + r] = v;
+            }
+            if (tid == 0) {
+                p.nblocks[row] = keep;
+                if (p.nblocks_out) p.nblocks_out[row] = keep;
+                p.plan[row] = make_int4(b, bad ? -1 : t, keep, 0);
+                if (bad) set_status(p.status, HISA_DEV_BAD_QUERY);
+            }
+        } else {
+            for (int r = tid; r < p.k; r += kRowThreads) {
+                p.idx[static_cast<size_t>(row) * p.k + r] = -1;
+                if (p.scores) p.scores[static_cast<size_t>(row) * p.k + r] = __int_as_float(0x7fc00000);
+            }
+            if (tid == 0 && bad && p.mode != kSelHisaTokens) set_status(p.status, HISA_DEV_BAD_QUERY);
+        }
+        return;
+    }
+
+    // 1. stage the keys; count, min, max of the nonzero ones
+    uint32_t cnt = 0, mn = 0xFFFFFFFFu, mx = 0u;
+    if (p.mode == kSelF32Rows) {
+        const float* x = p.x + static_cast<size_t>(row) * p.n;
+        for (int c = tid; c < n; c += kRowThreads) {
+            const uint32_t v = score_key(x[c]);
+            ks[c] = v;
+            cnt += v != 0u;
+            mn = min(mn, v);
+            mx = max(mx, v);
+        }
+    } else {
+        const uint4* g4 = reinterpret_cast<const uint4*>(p.keys + static_cast<size_t>(row) * p.ldk);
+        const int n4 = (n + 3) >> 2;
+#pragma unroll 4
+        for (int c4 = tid; c4 < n4; c4 += kRowThreads) {
+            const uint4 v = __ldcg(g4 + c4);
+            const uint32_t xs[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int c = 4 * c4 + j;
+                const uint32_t x = c < n ? xs[j] : 0u;
+                if (c < n) ks[c] = x;
+                if (x != 0u) {
+                    ++cnt;
+                    mn = min(mn, x);
+                    mx = max(mx, x);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+        mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    if (lane == 0) {
+        sh.wa[warp] = cnt;
+        sh.wb[warp] = mn;
+        sh.wc[warp] = mx;
+    }
+    __syncthreads();
+    uint32_t nvalid = 0;
+    mn = 0xFFFFFFFFu;
+    mx = 0u;
+#pragma unroll
+    for (int w = 0; w < kRowWarps; ++w) {
+        nvalid += sh.wa[w];
+        mn = min(mn, sh.wb[w]);
+        mx = max(mx, sh.wc[w]);
+    }
+
+    // 2-3. the k-th largest key T and how many keys == T are kept
+    uint32_t T = 0;
+    int take_eq = 0;
+    if (kk > 0 && nvalid > static_cast<uint32_t>(kk)) {
+        uint32_t lo = mn, hi = mx;
+        int krem = kk;
+        for (;;) {
+            const uint32_t span = hi - lo;
+            const int shift = span == 0 ? 0 : max(0, 32 - __clz(span) - kBinBits);
+            for (int i = tid; i < kBins; i += kRowThreads) sh.hist[i] = 0;
+            __syncthreads();
+            for (int c = tid; c < n; c += kRowThreads) {
+                const uint32_t x = ks[c];
+                if (x != 0u && x >= lo && x <= hi) atomicAdd(&sh.hist[(x - lo) >> shift], 1u);
+            }
+            __syncthreads();
+            // thread t owns bins 2047-4t .. 2044-4t (highest first)
+            const int b0 = kBins - 1 - 4 * tid;
+            const uint32_t h0 = sh.hist[b0], h1 = sh.hist[b0 - 1], h2 = sh.hist[b0 - 2], h3 = sh.hist[b0 - 3];
+            const uint32_t loc = h0 + h1 + h2 + h3;
+            uint32_t tot;
+            const uint32_t excl = row_scan(loc, sh.wd, &tot);
+            const uint32_t kr = static_cast<uint32_t>(krem);
+            if (excl < kr && kr <= excl + loc) {
+                const uint32_t hs[4] = {h0, h1, h2, h3};
+                uint32_t run = excl;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    if (run < kr && kr <= run + hs[q]) {
+                        sh.bc[0] = static_cast<uint32_t>(b0 - q);
+                        sh.bc[1] = kr - run;
+                        sh.bc[2] = hs[q];
+                    }
+                    run += hs[q];
+                }
+            }
+            if (tid == 0) sh.bc[3] = 0;
+            __syncthreads();
+            const uint32_t bin = sh.bc[0];
+            krem = static_cast<int>(sh.bc[1]);
+            const uint32_t nmem = sh.bc[2];
+            const uint32_t blo = lo + (bin << shift);
+            const uint32_t bhi = shift == 0 ? blo : blo + ((1u << shift) - 1u);
+            if (shift == 0) {
+                T = blo;
+                take_eq = krem;
+                break;
+            }
+            if (nmem <= static_cast<uint32_t>(kMembersCap)) {
+                for (int c = tid; c < n; c += kRowThreads) {
+                    const uint32_t x = ks[c];
+                    if (x != 0u && x >= blo && x <= bhi) {
+                        const uint32_t at = atomicAdd(&sh.bc[3], 1u);
+                        sh.members[at] = (static_cast<unsigned long long>(x) << 32) | static_cast<uint32_t>(c);
+                    }
+                }
+                __syncthreads();
+                const int m = static_cast<int>(sh.bc[3]);
+                for (int i = tid; i < m; i += kRowThreads) {
+                    const uint32_t xi = static_cast<uint32_t>(sh.members[i] >> 32);
+                    int above = 0, equal = 0;
+                    for (int j = 0; j < m; ++j) {
+                        const uint32_t xj = static_cast<uint32_t>(sh.members[j] >> 32);
+                        above += xj > xi;
+                        equal += xj == xi;
+                    }
+                    if (above < krem && krem <= above + equal) {
+                        sh.bc[4] = xi;
+                        sh.bc[5] = static_cast<uint32_t>(krem - above);
+                    }
+                }
+                __syncthreads();
+                T = sh.bc[4];
+                take_eq = static_cast<int>(sh.bc[5]);
+                break;
+            }
+            lo = blo;   // crowded bin: narrow the range and repeat
+            hi = bhi;
+            __syncthreads();
+        }
+    }
+
+    // 4. ordered compaction: warp w owns a contiguous slot range
+    const int per_warp = ((n + kRowWarps - 1) / kRowWarps + 31) & ~31;
+    const int w0 = warp * per_warp;
+    const int w1 = min(n, w0 + per_warp);
+    uint32_t gt = 0, eq = 0;
+    if (kk > 0) {
+        for (int base = w0; base < w1; base += 32) {
+            const int c = base + lane;
+            const uint32_t x = c < w1 ? ks[c] : 0u;
+            gt += __popc(__ballot_sync(0xffffffffu, x != 0u && x > T));
+            eq += __popc(__ballot_sync(0xffffffffu, x != 0u && x == T));
+        }
+    }
+    __syncthreads();   // bc / wa reuse below
+    if (lane == 0) {
+        sh.wa[warp] = gt;
+        sh.wb[warp] = eq;
+    }
+    __syncthreads();
+    uint32_t eq_run = 0, pos = 0, kept = 0;
+    {
+        uint32_t eqb = 0, off = 0;
+        for (int w = 0; w < kRowWarps; ++w) {
+            const uint32_t e = sh.wb[w];
+            const int room = take_eq - static_cast<int>(eqb);
+            const uint32_t take = room <= 0 ? 0u : (static_cast<uint32_t>(room) < e ? room : e);
+            if (w == warp) {
+                eq_run = eqb;
+                pos = off;
+            }
+            eqb += e;
+            off += sh.wa[w] + take;
+        }
+        kept = off;
+    }
+    const unsigned lt = (1u << lane) - 1u;
+    int32_t* blist = p.mode == kSelBlocks ? p.blocks + static_cast<size_t>(row) * p.mm : nullptr;
+    int32_t* bdbg = p.mode == kSelBlocks && p.blocks_out ? p.blocks_out + static_cast<size_t>(row) * p.mm : nullptr;
+    int32_t* idx = p.mode != kSelBlocks ? p.idx + static_cast<size_t>(row) * p.k : nullptr;
+    float* sc = p.mode != kSelBlocks && p.scores ? p.scores + static_cast<size_t>(row) * p.k : nullptr;
+    const int32_t* blk = p.mode == kSelHisaTokens ? p.blocks + static_cast<size_t>(row) * p.mm : nullptr;
+    if (kk > 0) {
+        for (int base = w0; base < w1; base += 32) {
+            const int c = base + lane;
+            const uint32_t x = c < w1 ? ks[c] : 0u;
+            const bool is_gt = x != 0u && x > T;
+            const bool is_eq = x != 0u && x == T;
+            const unsigned eqm = __ballot_sync(0xffffffffu, is_eq);
+            const uint32_t eq_rank = eq_run + __popc(eqm & lt);
+            const bool sel = is_gt || (is_eq && eq_rank < static_cast<uint32_t>(take_eq));
+            const unsigned selm = __ballot_sync(0xffffffffu, sel);
+            if (sel) {
+                const int at = static_cast<int>(pos + __popc(selm & lt));
+                if (blist) {
+                    blist[at] = c;
+                    if (bdbg) bdbg[at] = c;
+                } else {
+                    idx[at] = blk ? blk[c / p.B] * p.B + c % p.B : c;
+                    if (sc) sc[at] = key_score(x);
+                }
+            }
+            eq_run += __popc(eqm);
+            pos += __popc(selm);
+        }
+    }
+    if (p.mode == kSelBlocks) {
+        for (int r = static_cast<int>(kept) + tid; r < p.mm; r += kRowThreads) {
+            const int v = r == static_cast<int>(kept) ? nb - 1 : -1;   // own block last
+            blist[r] = v;
+            if (bdbg) bdbg[r] = v;
+        }
+        if (tid == 0) {
+            const int keep = static_cast<int>(kept) + 1;
+            p.nblocks[row] = keep;
+            if (p.nblocks_out) p.nblocks_out[row] = keep;
+            p.plan[row] = make_int4(b, t, keep, 0);
+        }
+    } else {
+        for (int r = static_cast<int>(kept) + tid; r < p.k; r += kRowThreads) {
+            idx[r] = -1;
+            if (sc) sc[r] = __int_as_float(0x7fc00000);
+        }
+    }
+}
+
+cudaError_t launch_row(const SelectParams& p, int max_n, cudaStream_t s) {
+    const size_t smem = static_cast<size_t>(max_n > 4 ? max_n : 4) * sizeof(uint32_t);
+    cudaError_t e = cudaFuncSetAttribute(select_row_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(p.rows));
+    cfg.blockDim = dim3(kRowThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, select_row_kernel, p);
+}
+
 template <bool STAGE>
 cudaError_t launch_t(const SelectParams& p, int csize, int chunk, cudaStream_t s) {
     const size_t smem = STAGE ? static_cast<size_t>(chunk) * sizeof(uint32_t) : 0;
@@ -513,6 +845,10 @@ cudaError_t launch_t(const SelectParams& p, int csize, int chunk, cudaStream_t s
 
 cudaError_t launch_select(const SelectParams& p, int max_n, int sms, cudaStream_t s) {
     if (p.rows <= 0) return cudaSuccess;
+    if (max_n <= kRowKeys) {
+        const cudaError_t e = launch_row(p, max_n, s);
+        return e == cudaSuccess ? cudaGetLastError() : e;
+    }
     // cluster size: enough CTAs to stage the longest row, and more while
     // there are SMs to spare; chunks stay at least 1024 slots
     int csize = 1;
