@@ -494,7 +494,10 @@ constexpr int kRowThreads = 512;
 constexpr int kRowWarps = kRowThreads / 32;
 constexpr int kRowKeys = 24576;
 
+constexpr int kRowBlocks = 2048;   // kept-block ids staged in shared memory
+
 struct RowShared {
+    int32_t blk[kRowBlocks];
     uint32_t hist[kBins];
     unsigned long long members[kMembersCap];
     uint32_t wa[kRowWarps];
@@ -578,6 +581,11 @@ __global__ void __launch_bounds__(kRowThreads) select_row_kernel(const SelectPar
         }
         return;
     }
+
+    // kept-block ids of a HISA row (slot c belongs to block blk[c / B])
+    const bool blk_smem = p.mode == kSelHisaTokens && p.mm <= kRowBlocks;
+    if (blk_smem)
+        for (int r = tid; r < p.mm; r += kRowThreads) sh.blk[r] = p.blocks[static_cast<size_t>(row) * p.mm + r];
 
     // 1. stage the keys; count, min, max of the nonzero ones
     uint32_t cnt = 0, mn = 0xFFFFFFFFu, mx = 0u;
@@ -754,7 +762,12 @@ __global__ void __launch_bounds__(kRowThreads) select_row_kernel(const SelectPar
     int32_t* bdbg = p.mode == kSelBlocks && p.blocks_out ? p.blocks_out + static_cast<size_t>(row) * p.mm : nullptr;
     int32_t* idx = p.mode != kSelBlocks ? p.idx + static_cast<size_t>(row) * p.k : nullptr;
     float* sc = p.mode != kSelBlocks && p.scores ? p.scores + static_cast<size_t>(row) * p.k : nullptr;
-    const int32_t* blk = p.mode == kSelHisaTokens ? p.blocks + static_cast<size_t>(row) * p.mm : nullptr;
+    const int32_t* blk = p.mode != kSelHisaTokens ? nullptr
+                         : blk_smem ? sh.blk
+                                    : p.blocks + static_cast<size_t>(row) * p.mm;
+    const int Bsz = p.B;
+    const bool pow2 = (Bsz & (Bsz - 1)) == 0;
+    const int lgB = __ffs(Bsz) - 1;
     if (kk > 0) {
         for (int base = w0; base < w1; base += 32) {
             const int c = base + lane;
@@ -771,7 +784,12 @@ __global__ void __launch_bounds__(kRowThreads) select_row_kernel(const SelectPar
                     blist[at] = c;
                     if (bdbg) bdbg[at] = c;
                 } else {
-                    idx[at] = blk ? blk[c / p.B] * p.B + c % p.B : c;
+                    if (blk) {
+                        const int bi = pow2 ? c >> lgB : c / Bsz;
+                        idx[at] = blk[bi] * Bsz + (c - bi * Bsz);
+                    } else {
+                        idx[at] = c;
+                    }
                     if (sc) sc[at] = key_score(x);
                 }
             }
