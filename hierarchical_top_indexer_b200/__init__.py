@@ -31,10 +31,12 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 HISA_KEY_BF16, HISA_KEY_E4M3 = 0, 1
 HISA_OK, HISA_E_INVAL, HISA_E_UNSUPPORTED, HISA_E_WORKSPACE, HISA_E_CUDA = range(5)
+HISA_E_SCRATCH_LIMIT = 5
+HISA_STATIC_SCRATCH_BYTES = 8 << 20
 HISA_DEV_BAD_QUERY, HISA_DEV_CAPACITY, HISA_DEV_BAD_LEN, HISA_DEV_TIMEOUT = 0x1, 0x2, 0x4, 0x8
 
 EXPORTS = ("hisa_pool_blocks", "hisa_append", "hisa_select_workspace_bytes", "hisa_select",
-           "hisa_select_inspect", "dsa_flat_workspace_bytes", "dsa_flat_select", "hisa_topk_f32",
+           "hisa_select_inspect", "hisa_select_static", "dsa_flat_workspace_bytes", "dsa_flat_select", "hisa_topk_f32",
            "hisa_profile_enable", "hisa_profile_read", "hisa_status_string")
 PHASES = ("block_score", "block_select", "token_score", "token_select", "flat_score",
           "flat_select", "pool", "append", "topk")
@@ -57,6 +59,7 @@ _lib.hisa_select_workspace_bytes.restype = _Z
 _lib.hisa_select.argtypes = [_KVP, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _Z, _P]
 _lib.hisa_select_inspect.argtypes = [_KVP, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P,
                                      _P, _Z, _P]
+_lib.hisa_select_static.argtypes = [_KVP, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P]
 _lib.dsa_flat_workspace_bytes.argtypes = [_KVP, _I, _I, _I]
 _lib.dsa_flat_workspace_bytes.restype = _Z
 _lib.dsa_flat_select.argtypes = [_KVP, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _Z, _P]
@@ -65,7 +68,7 @@ _lib.hisa_profile_enable.argtypes = [_I]
 _lib.hisa_profile_read.argtypes = [_P, _P, _I]
 _lib.hisa_status_string.argtypes = [_I]
 _lib.hisa_status_string.restype = ctypes.c_char_p
-for _f in ("hisa_pool_blocks", "hisa_append", "hisa_select", "hisa_select_inspect",
+for _f in ("hisa_pool_blocks", "hisa_append", "hisa_select", "hisa_select_inspect", "hisa_select_static",
            "dsa_flat_select", "hisa_topk_f32", "hisa_profile_enable", "hisa_profile_read"):
     getattr(_lib, _f).restype = _I
 
@@ -223,6 +226,29 @@ def hisa_select_inspect(kv: KVCache, Q, w, q_seq, q_pos, m: int, k: int, stream=
         _ptr(scores), _ptr(blocks), _ptr(nblocks), _ptr(counts), _ptr(ws), ws.numel(),
         _stream(stream)))
     return dict(idx=idx, scores=scores, blocks=blocks, nblocks=nblocks, counts=counts)
+
+
+def hisa_select_static(kv: KVCache, Q: torch.Tensor, w: torch.Tensor, q_seq: torch.Tensor,
+                       q_pos: Optional[torch.Tensor], m: int, k: int, idx: torch.Tensor,
+                       scores: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """hisa_select with the library's fixed scratch array instead of a workspace.
+
+    Every tensor must already be on the cache's device with its final dtype and
+    layout (Q bf16 [n_q, H, d], w fp32 [n_q, H], q_seq / q_pos / idx int32,
+    scores fp32 or None): this wrapper converts and allocates nothing, and
+    neither does the library call.  Calls on one device share the scratch, so
+    they must be ordered on one stream."""
+    for t, dt in ((Q, torch.bfloat16), (w, torch.float32), (q_seq, torch.int32),
+                  (q_pos, torch.int32), (idx, torch.int32), (scores, torch.float32)):
+        if t is not None and (t.dtype != dt or t.device.type != kv.device.type
+                              or not t.is_contiguous()):
+            raise ValueError("hisa_select_static takes contiguous tensors of the final dtype "
+                             "on the cache's device")
+    n_q, H = Q.shape[0], Q.shape[1]
+    _check("hisa_select_static", _lib.hisa_select_static(
+        kv.struct, _ptr(Q), _ptr(w), _ptr(q_seq), _ptr(q_pos), n_q, H, m, k, _ptr(idx),
+        _ptr(scores), _stream(stream)))
+    return idx
 
 
 def dsa_flat_select(kv: KVCache, Q, w, q_seq, q_pos, k: int, want_scores: bool = False,

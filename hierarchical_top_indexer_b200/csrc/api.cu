@@ -1,6 +1,8 @@
 // C ABI of the HISA indexer (include/hisa.h): argument checks, workspace
 // layout, TMA tensor maps and kernel launches.  No allocation happens here:
-// every buffer, scratch space included, belongs to the caller.
+// every buffer belongs to the caller, and so does the scratch space, except
+// for hisa_select_static, whose scratch is one fixed device array below.
+#include <atomic>
 #include <climits>
 #include <cstring>
 #include <mutex>
@@ -335,6 +337,32 @@ int hisa_select_impl(const hisa_kv* kv, const uint16_t* Q, const float* w, const
     return cuda_status(launch_select(sp, L.mm * v.B, sms, s));
 }
 
+// Scratch of hisa_select_static: a file-scope device array, one per device
+// (the runtime gives every device its own copy when it loads this module).
+// Its address is looked up once per device and cached.
+static __device__ __align__(256) uint8_t g_static_scratch[HISA_STATIC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::atomic<void*> g_static_scratch_ptr[kMaxDevices];
+std::mutex g_static_scratch_mu;
+
+// Device address of the current device's copy of g_static_scratch.
+int static_scratch(void** out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HISA_E_CUDA;
+    void* p = g_static_scratch_ptr[dev].load(std::memory_order_acquire);
+    if (!p) {
+        std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+        p = g_static_scratch_ptr[dev].load(std::memory_order_relaxed);
+        if (!p) {
+            if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return HISA_E_CUDA;
+            g_static_scratch_ptr[dev].store(p, std::memory_order_release);
+        }
+    }
+    *out = p;
+    return HISA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -378,6 +406,26 @@ int hisa_select_inspect(const hisa_kv* kv, const uint16_t* Q, const float* w, co
                         size_t ws_bytes, hisa_stream_t stream) {
     return hisa_select_impl(kv, Q, w, q_seq, q_pos, n_q, H, m, k, idx, scores, blocks, nblocks,
                             counts, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int hisa_select_static(const hisa_kv* kv, const uint16_t* Q, const float* w, const int32_t* q_seq,
+                       const int32_t* q_pos, int n_q, int H, int m, int k, int32_t* idx,
+                       float* scores, hisa_stream_t stream) {
+    KvView v;
+    int rc = check_kv(kv, &v);
+    if (rc) return rc;
+    if (!select_block_size_ok(v.B)) return HISA_E_UNSUPPORTED;
+    if (m < 1) return HISA_E_INVAL;
+    rc = check_queries(Q, w, q_seq, n_q, H, k, idx);
+    if (rc) return rc;
+    const size_t need = hisa_ws(v, n_q, m).total;
+    if (need > HISA_STATIC_SCRATCH_BYTES) return HISA_E_SCRATCH_LIMIT;
+    void* ws = nullptr;
+    rc = static_scratch(&ws);
+    if (rc) return rc;
+    return hisa_select_impl(kv, Q, w, q_seq, q_pos, n_q, H, m, k, idx, scores, nullptr, nullptr,
+                            nullptr, ws, HISA_STATIC_SCRATCH_BYTES,
+                            reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t dsa_flat_workspace_bytes(const hisa_kv* kv, int n_q, int H, int k) {
@@ -489,6 +537,7 @@ const char* hisa_status_string(int code) {
         case HISA_E_UNSUPPORTED: return "unsupported size";
         case HISA_E_WORKSPACE: return "workspace too small or misaligned";
         case HISA_E_CUDA: return "CUDA error";
+        case HISA_E_SCRATCH_LIMIT: return "call needs more than HISA_STATIC_SCRATCH_BYTES of scratch";
         default: return "unknown status";
     }
 }

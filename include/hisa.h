@@ -62,7 +62,9 @@ enum hisa_status {
     HISA_E_INVAL = 1,        /* a NULL, misaligned or out-of-range argument */
     HISA_E_UNSUPPORTED = 2,  /* a size outside the built kernels (d, B, H) */
     HISA_E_WORKSPACE = 3,    /* workspace too small or misaligned */
-    HISA_E_CUDA = 4          /* a CUDA call or launch failed */
+    HISA_E_CUDA = 4,         /* a CUDA call or launch failed */
+    HISA_E_SCRATCH_LIMIT = 5 /* hisa_select_static: the call needs more than
+                                HISA_STATIC_SCRATCH_BYTES of scratch */
 };
 
 /* Bits of the device status word (sticky: the library only ORs bits in). */
@@ -175,6 +177,38 @@ int hisa_select_inspect(const hisa_kv* kv, const uint16_t* Q, const float* w,
                         const int32_t* q_seq, const int32_t* q_pos, int n_q, int H, int m,
                         int k, int32_t* idx, float* scores, int32_t* blocks, int32_t* nblocks,
                         uint64_t* counts, void* ws, size_t ws_bytes, hisa_stream_t stream);
+
+/*
+ * hisa_select_static — hisa_select without a caller workspace.  The pages
+ * have no counterpart: this is a deployment convenience of this library.
+ * The scratch hisa_select keeps in `ws` lives instead in one fixed device
+ * array inside the library, HISA_STATIC_SCRATCH_BYTES (8 MiB) per device, so
+ * the call allocates no device or host memory at all.  It is meant for
+ * callers that cannot allocate on their selection path: an engine whose
+ * device memory is fully reserved up front (KV cache pages fill what is
+ * left), or a C caller with no allocator of its own that should not own a
+ * workspace's lifetime.
+ *   Arguments, outputs and results are those of hisa_select (same kernels,
+ *   same arithmetic: results are identical to hisa_select's).
+ *   Limit: hisa_select_workspace_bytes(kv, n_q, H, m, k) must be at most
+ *   HISA_STATIC_SCRATCH_BYTES, else HISA_E_SCRATCH_LIMIT and nothing is
+ *   launched (64 decode rows over 32K keys with B = 128, m = 64 need about
+ *   2.2 MB; a 4096-row prefill chunk does not fit — use hisa_select).
+ *   Setup: the first call on a device, with that device current, looks up
+ *   the array's device address (cudaGetSymbolAddress, which loads the
+ *   library's device code if it is not loaded yet); later calls on that
+ *   device reuse it.  Make that first call before any stream capture.
+ *   Contents: nothing in the array needs to start at zero; every byte a call
+ *   reads was written earlier in the same call.
+ *   Races: all calls on one device share the one array.  Two calls whose
+ *   kernels may overlap (different streams, or host threads without
+ *   ordering) race on it and give undefined results; order them on one
+ *   stream.
+ */
+#define HISA_STATIC_SCRATCH_BYTES ((size_t)8 << 20)
+int hisa_select_static(const hisa_kv* kv, const uint16_t* Q, const float* w,
+                       const int32_t* q_seq, const int32_t* q_pos, int n_q, int H, int m,
+                       int k, int32_t* idx, float* scores, hisa_stream_t stream);
 
 /*
  * dsa_flat_select — the flat indexer scan HISA replaces: every visible key

@@ -116,3 +116,27 @@ def test_workspace_sizes(hisa):
     assert ws == 65536 + 16384 + 256 + 1024 + 2097152
     assert lib.dsa_flat_workspace_bytes(ctypes.byref(kv), 64, 64, 2048) == 64 * 32768 * 4
     assert lib.hisa_select_workspace_bytes(None, 1, 1, 1, 1) == 0
+
+
+def test_static_scratch_entry_checks_before_setup(hisa):
+    """hisa_select_static validates its arguments and its scratch limit on the
+    host: bad calls return an error code without any CUDA call (none is
+    possible on this machine)."""
+    lib = hisa.lib()
+    P = ctypes.c_void_p
+    kv = _kv(hisa, cap=32768, B=128)
+
+    def sel(n_q=64, m=64, k=2048, Q=P(16)):
+        return lib.hisa_select_static(ctypes.byref(kv), Q, P(16), P(16), None, n_q, 64, m, k,
+                                      P(16), None, None)
+
+    assert sel(Q=None) == hisa.HISA_E_INVAL
+    assert sel(m=0) == hisa.HISA_E_INVAL
+    assert sel(k=0) == hisa.HISA_E_INVAL
+    assert lib.hisa_select_static(None, P(16), P(16), P(16), None, 1, 64, 8, 16, P(16), None,
+                                  None) == hisa.HISA_E_INVAL
+    # 256 rows over 32K keys with B = 128, m = 64 need 8.65 MB > 8 MiB
+    assert lib.hisa_select_workspace_bytes(ctypes.byref(kv), 256, 64, 64, 2048) > \
+        hisa.HISA_STATIC_SCRATCH_BYTES
+    assert sel(n_q=256) == hisa.HISA_E_SCRATCH_LIMIT
+    assert lib.hisa_status_string(hisa.HISA_E_SCRATCH_LIMIT).startswith(b"call needs more")
