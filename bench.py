@@ -189,7 +189,7 @@ def run_gpu(args, rank, world):
     n_flat = args.flat_steps
     n_prof = min(K, 50)
     total_steps = W + K + n_prof + 1 + E
-    case = make_workload(total_steps, seed_shift=rank)
+    case = make_workload(total_steps, seed_shift=rank_seed_shift(rank))
     kv = hisa.KVCache.from_case(case, device=dev)
     stream = torch.cuda.current_stream()
     batch, H, d, m, k = case.batch, case.H, case.d, case.m, case.k
@@ -246,10 +246,7 @@ def run_gpu(args, rank, world):
         dist.barrier()
     step_ms = [a.elapsed_time(b) for a, b in ev]
     total_ms = float(sum(step_ms))
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world, dev)
     # Per-kernel durations: the same steps again with an event pair around
     # every launch (separate pass: those events stop the launches from
     # overlapping, so the timed steps above run without them).
@@ -366,7 +363,7 @@ def cpu_oracle_rate(case=None, budget_s: float = 12.0, rows_per_call: int = 16):
         done += len(rows)
         r0 += rows_per_call
         el = time.perf_counter() - t0
-        if el >= budget_s or done >= 4 * case.n_q:
+        if el >= budget_s:
             break
     return dict(value=done / el, unit="selections/s", cores=threads, kind="oracle",
                 sample=f"{done} query rows of {WORKLOAD['name']} (HISA oracle, double, pooling "
@@ -409,10 +406,49 @@ def run_reference(args, rank, world):
     return line
 
 
+# ------------------------------------------------------------------ ranks
+
+
+def init_ranks(backend: str = "nccl"):
+    """(rank, world) from the torchrun environment; joins the process group
+    when there is more than one rank.  One process per GPU."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        if backend == "nccl":
+            torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world
+
+
+def rank_seed_shift(rank: int) -> int:
+    """Every rank draws its own sequences (weak scaling over disjoint batches)."""
+    return 1000 * rank
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The slowest rank's value: the job's time."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(rows_per_rank: int, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job selections/s: the rows every rank finished over the slowest rank's time."""
+    return rows_per_rank * steps * world / (max_ms / 1e3)
+
+
 # -------------------------------------------------------------------- main
 
 
-def main(argv=None):
+def main(argv=None, backend: str = "nccl"):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
@@ -425,14 +461,7 @@ def main(argv=None):
     args = ap.parse_args(argv)
     assert args.warmup >= 3, "at least 3 warm-up steps"
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    if world > 1:
-        import datetime
-        import torch
-        import torch.distributed as dist
-        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    rank, world = init_ranks(backend)
 
     try:
         if args.impl == "reference":
@@ -446,7 +475,7 @@ def main(argv=None):
             return 0
         case = r["case"]
         K = args.steps
-        value = case.batch * K * world / (r["total_ms"] / 1e3)
+        value = job_rate(case.batch, K, world, r["total_ms"])
         peaks = r["peaks"]
         cpu = None
         if not args.no_cpu_baseline and world == 1:
