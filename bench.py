@@ -344,6 +344,160 @@ def run_gpu(args, rank, world):
         flat_ms=flat_ms, mean_iou=mean_iou, e2e=e2e, case=case)
 
 
+# ------------------------------------------------------ other workloads
+
+
+def _median_ms(fn, n, flush, stream, warm=2):
+    """Median device time of fn() over n calls, L2 flushed between calls."""
+    import torch
+    for _ in range(warm):
+        fn()
+        flush.fill_(7)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n)]
+    for a, b in evs:
+        a.record(stream)
+        fn()
+        b.record(stream)
+        flush.fill_(7)
+    torch.cuda.synchronize()
+    return float(np.median([a.elapsed_time(b) for a, b in evs]))
+
+
+def _phase_ms(hisa, fn, phase, n):
+    """Mean per-launch time of one library phase over n calls (events around every launch)."""
+    import torch
+    hisa.hisa_profile_enable(True)
+    hisa.hisa_profile_read(reset=True)
+    for _ in range(n):
+        fn()
+    torch.cuda.synchronize()
+    ph = hisa.hisa_profile_read(reset=True)
+    hisa.hisa_profile_enable(False)
+    ms, cnt = ph[phase]
+    return ms / max(cnt, 1)
+
+
+def run_workloads(args, dev, peaks):
+    """Select-only timings on the other workloads: HISA against the flat scan
+    (speedup, mean IoU) at 64K prefill and 128K e4m3 decode, and the streaming
+    append + select step at 128K.  Parity on these sizes is in the GPU tests."""
+    import torch
+    import hierarchical_top_indexer_b200 as hisa
+    from hisa_inputs import make_config
+    from tests.parity import iou
+
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    n = args.workload_steps
+    out = {}
+
+    def one(cfg):
+        case = make_config(cfg)
+        kv = hisa.KVCache.from_case(case, device=dev)
+        hisa.hisa_pool_blocks(kv)
+        Q = torch.from_numpy(case.Q.view(np.int16)).view(torch.bfloat16).to(dev)
+        w = torch.from_numpy(case.w).to(dev)
+        qs = torch.from_numpy(case.q_seq).to(dev)
+        qp = torch.from_numpy(case.q_pos).to(dev)
+        n_q, H, m, k = case.n_q, case.H, case.m, case.k
+        ws = hisa.workspace(hisa.hisa_select_workspace_bytes(kv, n_q, H, m, k), dev)
+        fws = hisa.workspace(hisa.dsa_flat_workspace_bytes(kv, n_q, H, k), dev)
+        hidx = torch.empty((n_q, k), dtype=torch.int32, device=dev)
+        fidx = torch.empty((n_q, k), dtype=torch.int32, device=dev)
+        sel = lambda: hisa.hisa_select(kv, Q, w, qs, qp, m, k, ws=ws, idx=hidx)
+        flat = lambda: hisa.dsa_flat_select(kv, Q, w, qs, qp, k, ws=fws, idx=fidx)
+        h_ms = _median_ms(sel, n, flush, stream)
+        f_ms = _median_ms(flat, max(3, n // 4), flush, stream)
+        tok_ms = _phase_ms(hisa, sel, "token_score", 3)
+        pool_ms = _phase_ms(hisa, lambda: hisa.hisa_pool_blocks(kv), "pool", 3)
+        mi = float(np.mean([iou(a, b) for a, b in zip(hidx.cpu().numpy(), fidx.cpu().numpy())]))
+        assert kv.status_bits() == 0, f"device status {kv.status_bits():#x}"
+        kbytes = case.d * (1 if case.dtype == "e4m3" else 2) + (4 if case.dtype == "e4m3" else 0)
+        mm = min(m, -(-case.cap // case.B))
+        tok_bytes = n_q * (mm * case.B * (kbytes + 4) + H * case.d * 2 + H * 4 + mm * 4)
+        tok_flops = n_q * mm * case.B * 2 * H * case.d
+        pool_bytes = int(case.lens.sum()) * kbytes + case.batch * kv.nblk * case.d * 8
+        r = {"rows": n_q, "hisa_ms_per_select": h_ms, "flat_ms_per_select": f_ms,
+             "hisa_selections_per_s": n_q / (h_ms / 1e3),
+             "flat_selections_per_s": n_q / (f_ms / 1e3), "speedup": f_ms / h_ms,
+             "mean_iou_hisa_vs_flat": mi,
+             "token_score": {"ms_per_launch": tok_ms,
+                             "GB/s": tok_bytes / (tok_ms / 1e3) / 1e9,
+                             "hbm_frac": tok_bytes / (tok_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                             "TFLOP/s": tok_flops / (tok_ms / 1e3) / 1e12,
+                             "tensor_frac": tok_flops / (tok_ms / 1e3) / 1e12 / peaks["bf16_tflops"]},
+             "pool": {"ms": pool_ms, "GB/s": pool_bytes / (pool_ms / 1e3) / 1e9}}
+        del kv, ws, fws
+        torch.cuda.empty_cache()
+        return case, r
+
+    case, r = one(2)
+    r["l2"] = "64K x bf16 keys (16 MiB) stay L2-resident across query rows"
+    out[case.name] = r
+    case, r = one(3)
+    r["l2"] = "flushed between calls (cache 528 MiB)"
+    out[case.name] = r
+
+    # streaming append + select for the new last position, one row per step
+    case = make_config(4)
+    kv = hisa.KVCache.from_case(case, device=dev)
+    hisa.hisa_pool_blocks(kv)
+    steps = case.append_keys.shape[0]
+    toks = torch.from_numpy(case.append_keys.view(np.int16)).view(torch.bfloat16).to(dev)
+    AQ = torch.from_numpy(case.append_Q.view(np.int16)).view(torch.bfloat16).to(dev)
+    AW = torch.from_numpy(case.append_w).to(dev)
+    qs = torch.zeros(1, dtype=torch.int32, device=dev)
+    ws = hisa.workspace(hisa.hisa_select_workspace_bytes(kv, 1, case.H, case.m, case.k), dev)
+    idx = torch.empty((1, case.k), dtype=torch.int32, device=dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for s, (a, b) in enumerate(evs):
+        a.record(stream)
+        hisa.hisa_append(kv, toks[s])
+        hisa.hisa_select(kv, AQ[s], AW[s], qs, None, case.m, case.k, ws=ws, idx=idx)
+        b.record(stream)
+    torch.cuda.synchronize()
+    assert kv.status_bits() == 0, f"device status {kv.status_bits():#x}"
+    st = [a.elapsed_time(b) for a, b in evs]
+    out[case.name] = {"steps": steps, "us_per_step_mean": 1e3 * float(np.mean(st)),
+                      "us_per_step_median": 1e3 * float(np.median(st)),
+                      "steps_per_s": steps / (sum(st) / 1e3),
+                      "l2": "cache (32 MiB) L2-resident; no flush: each step follows the last"}
+    return out
+
+
+def run_select_only(args):
+    """--select-only NAME: hisa_select (or --flat: dsa_flat_select) on one
+    workload, `warmup` untimed then `steps` timed calls; for profiling one
+    kernel of one workload."""
+    import torch
+    import hierarchical_top_indexer_b200 as hisa
+    from hisa_inputs import CONFIGS, make_config
+    cfg = next(i for i, c in CONFIGS.items() if c["name"] == args.select_only)
+    dev = torch.device("cuda", 0)
+    case = make_config(cfg)
+    kv = hisa.KVCache.from_case(case, device=dev)
+    hisa.hisa_pool_blocks(kv)
+    Q = torch.from_numpy(case.Q.view(np.int16)).view(torch.bfloat16).to(dev)
+    w = torch.from_numpy(case.w).to(dev)
+    qs = torch.from_numpy(case.q_seq).to(dev)
+    qp = torch.from_numpy(case.q_pos).to(dev)
+    n_q, H, m, k = case.n_q, case.H, case.m, case.k
+    idx = torch.empty((n_q, k), dtype=torch.int32, device=dev)
+    if args.flat:
+        ws = hisa.workspace(hisa.dsa_flat_workspace_bytes(kv, n_q, H, k), dev)
+        fn = lambda: hisa.dsa_flat_select(kv, Q, w, qs, qp, k, ws=ws, idx=idx)
+    else:
+        ws = hisa.workspace(hisa.hisa_select_workspace_bytes(kv, n_q, H, m, k), dev)
+        fn = lambda: hisa.hisa_select(kv, Q, w, qs, qp, m, k, ws=ws, idx=idx)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    ms = _median_ms(fn, args.steps, flush, torch.cuda.current_stream(), warm=args.warmup)
+    assert kv.status_bits() == 0, f"device status {kv.status_bits():#x}"
+    return {"select_only": case.name, "flat": bool(args.flat), "rows": n_q,
+            "ms_per_select": ms, "selections_per_s": n_q / (ms / 1e3)}
+
+
 # ----------------------------------------------------------- CPU baseline
 
 
@@ -458,6 +612,11 @@ def main(argv=None, backend: str = "nccl"):
     ap.add_argument("--flat-steps", type=int, default=20)
     ap.add_argument("--ref-rows", type=int, default=16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--select-only", default=None,
+                    help="time only hisa_select on this workload (a name from hisa_inputs)")
+    ap.add_argument("--flat", action="store_true", help="with --select-only: dsa_flat_select")
+    ap.add_argument("--workload-steps", type=int, default=20,
+                    help="timed selects per extra workload (0: skip them)")
     args = ap.parse_args(argv)
     assert args.warmup >= 3, "at least 3 warm-up steps"
 
@@ -468,6 +627,11 @@ def main(argv=None, backend: str = "nccl"):
             line = run_reference(args, rank, world)
             if line is not None:
                 print(json.dumps(line), flush=True)
+            return 0
+
+        if args.select_only:
+            if rank == 0:
+                print(json.dumps(run_select_only(args)), flush=True)
             return 0
 
         r = run_gpu(args, rank, world)
@@ -481,6 +645,10 @@ def main(argv=None, backend: str = "nccl"):
         if not args.no_cpu_baseline and world == 1:
             cpu = cpu_oracle_rate(case)
         traffic = traffic_record()
+        extra = None
+        if world == 1 and args.workload_steps > 0:
+            import torch
+            extra = run_workloads(args, torch.device("cuda", 0), peaks)
         line = {
             "metric": "HISA indexer top-k selections/s (decode, 32K context)",
             "value": value, "unit": "selections/s", "n_gpus": world, "steps": K,
@@ -508,6 +676,7 @@ def main(argv=None, backend: str = "nccl"):
                           "flat_selections_per_s": case.batch / (r["flat_ms"] / 1e3),
                           "mean_iou_hisa_vs_flat": r["mean_iou"]},
             "e2e": r["e2e"],
+            "workloads": extra,
             "cpu_baseline": cpu,
             "wall_s_timed_region": r["wall"],
         }

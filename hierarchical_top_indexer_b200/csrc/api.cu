@@ -225,6 +225,9 @@ ScoreParams score_params(const KvView& v, const float* w, const int32_t* q_seq, 
     p.n_q = n_q;
     p.H = H;
     p.npad = npad_of(H);
+    // More rows than sequences: rows share keys (a prefill chunk), which then
+    // stay in L2; otherwise every row streams its own keys from HBM.
+    p.keep_keys = n_q > v.batch ? 1 : 0;
     return p;
 }
 

@@ -48,6 +48,7 @@ struct ScoreParams {
     long long total_tiles;        // n_q * tiles_per_row
     int stages;                   // bf16 operand stages
     int stages8;                  // e4m3 staging stages
+    int keep_keys;                // rows share keys: keep them in L2 (else stream them)
 };
 
 enum SelectMode : int {

@@ -48,9 +48,10 @@ constexpr int kMinSmem = 120 * 1024;          // keeps one CTA (and its TMEM) pe
 constexpr int kMaxSmem = 232448;
 constexpr int kMaxAcc = 4;
 constexpr int kMaxStages = 8;
+constexpr int kScaleRing = 16;                // e4m3 per-token scale slots (one tile each)
 
 struct Layout {
-    uint32_t a, s8, q, w, bars, misc, total;
+    uint32_t a, s8, sc, q, w, bars, misc, total;
 };
 
 __host__ __device__ inline int acc_count(int npad) { return 4 * npad <= 512 ? 4 : 2; }
@@ -64,12 +65,14 @@ __host__ __device__ inline Layout score_layout(int mode, bool e4m3, int d, int n
     off += sa * stage;
     L.s8 = off;
     off += e4m3 ? s8 * kTileRows * d : 0;
+    L.sc = off;
+    off += (e4m3 && mode != kScoreBlocks) ? kScaleRing * kTileRows * 4 : 0;
     L.q = off;
     off += 2 * halves * npad * 128;
     L.w = off;
     off += 4 * 128 * 4;                      // one 128-float weight slot per epilogue warp
     L.bars = off;
-    off += (4 * kMaxStages + 2 * kMaxAcc + 4) * 8;
+    off += (4 * kMaxStages + 2 * kMaxAcc + 4 + 2 * kScaleRing) * 8;
     L.misc = off;
     off += 16;
     L.total = off;
@@ -108,6 +111,40 @@ __device__ __forceinline__ RowInfo load_row(const ScoreParams& p, int row) {
     R.nt = (R.lim + kTileRows - 1) / kTileRows;
     return R;
 }
+
+// Walks the row-major (row, tile) slots g0, g0 + 1, ... of a CTA's range
+// without a 64-bit division per step.
+struct TileCursor {
+    long long g;
+    int row, ti, tpr;
+    __device__ __forceinline__ TileCursor(long long g0, int tiles_per_row)
+        : g(g0), row(static_cast<int>(g0 / tiles_per_row)), ti(static_cast<int>(g0 % tiles_per_row)),
+          tpr(tiles_per_row) {}
+    __device__ __forceinline__ void next() {
+        ++g;
+        if (++ti == tpr) {
+            ti = 0;
+            ++row;
+        }
+    }
+    __device__ __forceinline__ void next_row() {
+        g += tpr - ti;
+        ti = 0;
+        ++row;
+    }
+};
+
+// Position in a ring of n slots: slot and phase parity.
+struct Ring {
+    int slot = 0;
+    uint32_t phase = 0;
+    __device__ __forceinline__ void next(int n) {
+        if (++slot == n) {
+            slot = 0;
+            phase ^= 1u;
+        }
+    }
+};
 
 __device__ __forceinline__ void raise_abort(volatile int* abort_flag, uint32_t* status) {
     *abort_flag = 1;
@@ -161,6 +198,14 @@ __device__ __forceinline__ float lds_f32(const float* p) {
     return v;
 }
 
+__device__ __forceinline__ float4 lds_f32x4(const float* p) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(smem_addr(p)));
+    return v;
+}
+
 // sum_h w_h * ReLU(acc_h) over the NP head columns of one TMEM lane: loads
 // of up to 64 columns at a time, one wait per group, four interleaved partial
 // sums (fixed order).
@@ -176,8 +221,14 @@ __device__ __forceinline__ float head_sum(uint32_t taddr, const float* wv) {
             if (g + c < NP) tmem_ld16_nowait(taddr + g + c, r + c);
         tmem_ld_wait();
 #pragma unroll
-        for (int h = 0; h < kG; ++h)
-            if (g + h < NP) a[h & 3] = fmaf(lds_f32(wv + g + h), fmaxf(__uint_as_float(r[h]), 0.f), a[h & 3]);
+        for (int h = 0; h < kG; h += 4)
+            if (g + h < NP) {
+                const float4 w4 = lds_f32x4(wv + g + h);
+                a[0] = fmaf(w4.x, fmaxf(__uint_as_float(r[h]), 0.f), a[0]);
+                a[1] = fmaf(w4.y, fmaxf(__uint_as_float(r[h + 1]), 0.f), a[1]);
+                a[2] = fmaf(w4.z, fmaxf(__uint_as_float(r[h + 2]), 0.f), a[2]);
+                a[3] = fmaf(w4.w, fmaxf(__uint_as_float(r[h + 3]), 0.f), a[3]);
+            }
     }
     return (a[0] + a[1]) + (a[2] + a[3]);
 }
@@ -214,6 +265,7 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
     uint8_t* sA = smem + L.a;
     uint8_t* s8 = smem + L.s8;
     uint8_t* sQ = smem + L.q;
+    float* sS = reinterpret_cast<float*>(smem + L.sc);   // e4m3 scales [kScaleRing][128]
     float* sW = reinterpret_cast<float*>(smem + L.w);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
     uint64_t* full = bars;                         // operand stage ready   [SA]
@@ -224,6 +276,8 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
     uint64_t* tempty = tfull + kMaxAcc;            // accumulator drained [kMaxAcc]
     uint64_t* qfull = tempty + kMaxAcc;            // query heads landed  [2]
     uint64_t* qempty = qfull + 2;                  // query heads free    [2]
+    uint64_t* scfull = qempty + 2;                 // tile scales landed  [kScaleRing]
+    uint64_t* scempty = scfull + kScaleRing;       // tile scales read    [kScaleRing]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.misc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.misc + 4);
 
@@ -255,6 +309,10 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
             mbar_init(qfull + a, 1);
             mbar_init(qempty + a, 1);
         }
+        for (int r = 0; r < kScaleRing; ++r) {
+            mbar_init(scfull + r, 32);     // one cp.async arrival per producer lane
+            mbar_init(scempty + r, 4);     // one per epilogue warp
+        }
         *abort_flag = 0;
         fence_barrier_init();
         fence_async_smem();
@@ -274,15 +332,20 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
     grid_launch_dependents();
 
     if (warp == kWarpProducer) {
-        const uint64_t pol = policy_evict_first();
+        // keys read by one row only stream through L2; keys that several rows
+        // read (a prefill chunk) stay
+        const uint64_t pol = p.keep_keys ? policy_evict_last() : policy_evict_first();
+        const long long key_rows = static_cast<long long>(p.batch) * p.cap;
         int it = 0, qloads = 0, cur_row = -1, tb = 0;
         RowInfo R;
         R.nt = 0;
         int win_cur = 0, win_nxt = 0, cur_w = 0;
         bool ok = true;
-        for (long long g = g0; g < g1 && ok;) {
-            const int row = static_cast<int>(g / tpr);
-            const int ti = static_cast<int>(g % tpr);
+        const int NS = E4M3 ? S8 : SA;
+        Ring ring;
+        for (TileCursor cur(g0, tpr); cur.g < g1 && ok;) {
+            const int row = cur.row;
+            const int ti = cur.ti;
             if (row != cur_row) {
                 cur_row = row;
                 R = load_row<MODE>(p, row);
@@ -314,7 +377,7 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
                 }
             }
             if (ti >= R.nt) {
-                g = static_cast<long long>(row + 1) * tpr;
+                cur.next_row();
                 continue;
             }
             const int gs = (ti - tb) * nsub;
@@ -326,8 +389,8 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
                               ? tile_sub_row<MODE>(p, R, row, tb + gn / nsub, gn % nsub, BR)
                               : 0;
             }
-            const int ss = E4M3 ? it % S8 : it % SA;
-            const uint32_t ph = (E4M3 ? it / S8 : it / SA) & 1;
+            const int ss = ring.slot;
+            const uint32_t ph = ring.phase;
             uint64_t* fb = E4M3 ? sfull + ss : full + ss;
             uint64_t* eb = E4M3 ? sempty + ss : empty + ss;
             if (!warp_wait(eb, ph ^ 1, abort_flag)) {
@@ -359,15 +422,33 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
                     }
                 }
             }
+            if (E4M3) {
+                // the tile's per-token scales, one 4-byte copy per key row
+                const int sc = it & (kScaleRing - 1);
+                if (!warp_wait(scempty + sc, ((it / kScaleRing) & 1) ^ 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+#pragma unroll
+                for (int q = 0; q < kTileRows / 32; ++q) {
+                    const int r = q * 32 + lane;
+                    const int sub = r / BR;
+                    int srow = __shfl_sync(0xffffffffu, win_cur, (gs & 31) + (sub < nsub ? sub : 0));
+                    srow = MODE == kScoreFlat ? R.b * p.cap + ti * kTileRows + r : srow + (r - sub * BR);
+                    if (srow < key_rows) cp_async_4(sS + sc * kTileRows + r, p.key_scale + srow);
+                }
+                cp_async_arrive_noinc(scfull + sc);
+            }
             __syncwarp();
             ++it;
-            ++g;
+            ring.next(NS);
+            cur.next();
         }
+        if (E4M3) cp_async_wait_all();   // no scale copy still landing at exit
         if (lane == 0) {
             if (!ok) raise_abort(abort_flag, p.status);
             // Drain: no copy into, and no arrive on, this CTA's shared memory
             // may still be pending when it exits.
-            const int NS = E4M3 ? S8 : SA;
             for (int n = it > NS ? it - NS : 0; n < it; ++n) {
                 const int s = n % NS;
                 const uint32_t ph = (n / NS) & 1;
@@ -388,9 +469,10 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
             RowInfo R;
             R.nt = 0;
             bool ok = true;
-            for (long long g = g0; g < g1 && ok;) {
-                const int row = static_cast<int>(g / tpr);
-                const int ti = static_cast<int>(g % tpr);
+            Ring rs, ra;   // operand stage, accumulator
+            for (TileCursor cur(g0, tpr); cur.g < g1 && ok;) {
+                const int row = cur.row;
+                const int ti = cur.ti;
                 if (row != cur_row) {
                     cur_row = row;
                     R = load_row<MODE>(p, row);
@@ -405,13 +487,13 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
                     }
                 }
                 if (ti >= R.nt) {
-                    g = static_cast<long long>(row + 1) * tpr;
+                    cur.next_row();
                     continue;
                 }
-                const int s = it % SA;
-                const int a = it % NACC;
-                if (!mbar_wait(full + s, (it / SA) & 1, abort_flag) ||
-                    !mbar_wait(tempty + a, ((it / NACC) & 1) ^ 1, abort_flag)) {
+                const int s = rs.slot;
+                const int a = ra.slot;
+                if (!mbar_wait(full + s, rs.phase, abort_flag) ||
+                    !mbar_wait(tempty + a, ra.phase ^ 1u, abort_flag)) {
                     ok = false;
                     break;
                 }
@@ -435,7 +517,9 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
                 umma_commit(empty + s);
                 umma_commit(tfull + a);
                 ++it;
-                ++g;
+                rs.next(SA);
+                ra.next(NACC);
+                cur.next();
             }
             if (!ok) raise_abort(abort_flag, p.status);
             // every UMMA of this CTA has finished before TMEM is released
@@ -448,13 +532,19 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
         int it = 0, cur_row = -1;
         RowInfo R;
         R.nt = 0;
+        int own0 = 0, own_t = 0;     // first slot of the own block (listed last), t within it
         bool ok = true;
-        for (long long g = g0; g < g1;) {
-            const int row = static_cast<int>(g / tpr);
-            const int ti = static_cast<int>(g % tpr);
+        Ring ra;
+        for (TileCursor cur(g0, tpr); cur.g < g1;) {
+            const int row = cur.row;
+            const int ti = cur.ti;
             if (row != cur_row) {
                 cur_row = row;
                 R = load_row<MODE>(p, row);
+                if (MODE == kScoreHisa && R.nt > 0) {
+                    own0 = R.lim - p.B;
+                    own_t = R.t % p.B;
+                }
                 if (ti < R.nt) {
                     __syncwarp();
                     for (int h = lane; h < 128; h += 32) wv[h] = h < p.H ? p.w[row * p.H + h] : 0.f;
@@ -462,29 +552,21 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
                 }
             }
             if (ti >= R.nt) {
-                g = static_cast<long long>(row + 1) * tpr;
+                cur.next_row();
                 continue;
             }
             const int c = ti * kTileRows + r;
             bool valid;
-            float scale = 1.f;
             if (MODE == kScoreBlocks) {
                 valid = c < R.lim;
             } else if (MODE == kScoreFlat) {
                 valid = c <= R.t;
-                if (E4M3 && valid) scale = __ldg(p.key_scale + static_cast<size_t>(R.b) * p.cap + c);
             } else {
-                const int br = c / p.B, o = c % p.B;
-                const int own_rank = R.lim / p.B - 1;    // the own block is listed last
-                valid = c < R.lim && (br < own_rank || o <= R.t % p.B);
-                if (E4M3 && valid) {
-                    const int blk = __ldg(p.blocks + static_cast<size_t>(row) * p.mm + br);
-                    scale = __ldg(p.key_scale + static_cast<size_t>(R.b) * p.cap + blk * p.B + o);
-                }
+                valid = c < own0 || (c < R.lim && c - own0 <= own_t);
             }
-            const int a = it % NACC;
+            const int a = ra.slot;
             float acc = 0.f;
-            if (ok && mbar_wait(tfull + a, (it / NACC) & 1, abort_flag)) {
+            if (ok && mbar_wait(tfull + a, ra.phase, abort_flag)) {
                 tc_fence_after();
                 const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                                        static_cast<uint32_t>(a * npad);
@@ -496,7 +578,19 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
             }
             __syncwarp();
             if (lane == 0 && ok) mbar_arrive(tempty + a);
-            if (E4M3) acc *= scale;
+            if (E4M3) {
+                const int sc = it & (kScaleRing - 1);
+                float scale = 1.f;
+                if (ok && mbar_wait(scfull + sc, (it / kScaleRing) & 1, abort_flag)) {
+                    scale = sS[sc * kTileRows + r];
+                } else if (ok) {
+                    ok = false;
+                    raise_abort(abort_flag, p.status);
+                }
+                __syncwarp();
+                if (lane == 0 && ok) mbar_arrive(scempty + sc);
+                acc *= scale;
+            }
             p.out[static_cast<size_t>(row) * p.ldo + c] = valid ? score_key(acc) : 0u;
             if (p.counts) {
                 const bool slot = MODE == kScoreBlocks ? valid : c < R.lim;
@@ -506,7 +600,8 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
                               static_cast<unsigned long long>(n));
             }
             ++it;
-            ++g;
+            ra.next(NACC);
+            cur.next();
         }
     } else if (E4M3 && warp >= kWarpConv0) {
         const int cw = warp - kWarpConv0;
@@ -514,21 +609,22 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
         RowInfo R;
         R.nt = 0;
         bool ok = true;
-        for (long long g = g0; g < g1 && ok;) {
-            const int row = static_cast<int>(g / tpr);
-            const int ti = static_cast<int>(g % tpr);
+        Ring r8, rs;   // staging slot, operand stage
+        for (TileCursor cur(g0, tpr); cur.g < g1 && ok;) {
+            const int row = cur.row;
+            const int ti = cur.ti;
             if (row != cur_row) {
                 cur_row = row;
                 R = load_row<MODE>(p, row);
             }
             if (ti >= R.nt) {
-                g = static_cast<long long>(row + 1) * tpr;
+                cur.next_row();
                 continue;
             }
-            const int s8i = it % S8;
-            const int sa = it % SA;
-            if (!mbar_wait(sfull + s8i, (it / S8) & 1, abort_flag) ||
-                !mbar_wait(empty + sa, ((it / SA) & 1) ^ 1, abort_flag)) {
+            const int s8i = r8.slot;
+            const int sa = rs.slot;
+            if (!mbar_wait(sfull + s8i, r8.phase, abort_flag) ||
+                !mbar_wait(empty + sa, rs.phase ^ 1u, abort_flag)) {
                 ok = false;
                 break;
             }
@@ -552,7 +648,9 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
                 mbar_arrive(sempty + s8i);
             }
             ++it;
-            ++g;
+            r8.next(S8);
+            rs.next(SA);
+            cur.next();
         }
         if (!ok) raise_abort(abort_flag, p.status);
         if (ok && cw == 0 && lane == 0)
