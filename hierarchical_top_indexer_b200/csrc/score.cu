@@ -49,9 +49,10 @@ constexpr int kMaxSmem = 232448;
 constexpr int kMaxAcc = 4;
 constexpr int kMaxStages = 8;
 constexpr int kScaleRing = 16;                // e4m3 per-token scale slots (one tile each)
+constexpr int kTabSubs = 256;                 // first key row of each sub-box, per row window
 
 struct Layout {
-    uint32_t a, s8, sc, q, w, bars, misc, total;
+    uint32_t a, s8, sc, tab, q, w, bars, misc, total;
 };
 
 __host__ __device__ inline int acc_count(int npad) { return 4 * npad <= 512 ? 4 : 2; }
@@ -67,6 +68,8 @@ __host__ __device__ inline Layout score_layout(int mode, bool e4m3, int d, int n
     off += e4m3 ? s8 * kTileRows * d : 0;
     L.sc = off;
     off += (e4m3 && mode != kScoreBlocks) ? kScaleRing * kTileRows * 4 : 0;
+    L.tab = off;
+    off += kTabSubs * 4;
     L.q = off;
     off += 2 * halves * npad * 128;
     L.w = off;
@@ -151,11 +154,15 @@ __device__ __forceinline__ void raise_abort(volatile int* abort_flag, uint32_t* 
     set_status(status, HISA_DEV_TIMEOUT);
 }
 
-// Lane 0 waits; the whole warp learns the outcome (keeps the warp converged).
+// Lane 0 waits; the whole warp learns the outcome and is ordered after the
+// wait (one waiting thread per warp keeps the barrier traffic off the shared
+// memory pipe that the copies and the other roles need).
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
     bool ok = true;
     if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag);
-    return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    __syncwarp();
+    return ok;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -192,12 +199,6 @@ __device__ __forceinline__ int tile_sub_row(const ScoreParams& p, const RowInfo&
 
 // Shared-memory load the compiler keeps in place (the head weights are read
 // per tile instead of being held in registers across the tile loop).
-__device__ __forceinline__ float lds_f32(const float* p) {
-    float v;
-    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(smem_addr(p)));
-    return v;
-}
-
 __device__ __forceinline__ float4 lds_f32x4(const float* p) {
     float4 v;
     asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
@@ -343,6 +344,83 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
         bool ok = true;
         const int NS = E4M3 ? S8 : SA;
         Ring ring;
+        if constexpr (!E4M3) {
+            // bf16 keys: per row, the warp stages the sub-boxes' first key rows
+            // in shared memory; lane 0 alone then issues the row's tiles, one
+            // barrier wait and one transaction count per tile
+            int* sTab = reinterpret_cast<int*>(smem + L.tab);
+            TileCursor cur(g0, tpr);
+            while (cur.g < g1 && ok) {
+                const int row = cur.row;
+                R = load_row<MODE>(p, row);
+                const long long left = g1 - cur.g;
+                const int t_end = static_cast<int>(R.nt < cur.ti + left ? R.nt : cur.ti + left);
+                if (cur.ti >= t_end) {
+                    cur.next_row();
+                    continue;
+                }
+                const int qs = qloads & 1;
+                if (qloads >= 2 && !warp_wait(qempty + qs, ((qloads - 2) >> 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(qfull + qs, q_slot_bytes);
+#pragma unroll
+                    for (int kh = 0; kh < kHalves; ++kh)
+                        tma_load_2d(sQ + qs * q_slot_bytes + kh * npad * 128, &qmap, qfull + qs, kh * 64,
+                                    row * p.H);
+                }
+                ++qloads;
+                for (int t = cur.ti; t < t_end && ok;) {
+                    const int nwin = min(t_end - t, kTabSubs / nsub);
+                    if (MODE == kScoreHisa) {
+                        for (int j = lane; j < nwin * nsub; j += 32)
+                            sTab[j] = tile_sub_row<MODE>(p, R, row, t + j / nsub, j % nsub, BR);
+                        __syncwarp();
+                    }
+                    if (lane == 0) {
+                        for (int k = 0; k < nwin; ++k) {
+                            if (!mbar_wait(empty + ring.slot, ring.phase ^ 1u, abort_flag)) {
+                                ok = false;
+                                break;
+                            }
+                            uint64_t* fb = full + ring.slot;
+                            uint8_t* dst = sA + ring.slot * kStageBytes;
+                            mbar_arrive_expect_tx(fb, kStageBytes);
+                            if (MODE == kScoreBlocks) {
+#pragma unroll
+                                for (int op = 0; op < 2; ++op)
+#pragma unroll
+                                    for (int kh = 0; kh < kHalves; ++kh)
+                                        tma_load_2d(dst + (op * kHalves + kh) * kHalfBytes, &amap, fb,
+                                                    op * D + kh * 64, R.b * p.nblk + (t + k) * kTileRows);
+                            } else {
+                                for (int sub = 0; sub < nsub; ++sub) {
+                                    const int srow = MODE == kScoreHisa
+                                                         ? sTab[k * nsub + sub]
+                                                         : R.b * p.cap + (t + k) * kTileRows + sub * BR;
+#pragma unroll
+                                    for (int kh = 0; kh < kHalves; ++kh)
+                                        tma_load_2d_hint(dst + kh * kHalfBytes + sub * BR * 128, &amap, fb,
+                                                         kh * 64, srow, pol);
+                                }
+                            }
+                            ++it;
+                            ring.next(SA);
+                        }
+                    }
+                    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                    it = __shfl_sync(0xffffffffu, it, 0);
+                    ring.slot = __shfl_sync(0xffffffffu, ring.slot, 0);
+                    ring.phase = __shfl_sync(0xffffffffu, ring.phase, 0);
+                    __syncwarp();
+                    t += nwin;
+                }
+                if (t_end < R.nt) break;   // the range ends inside this row
+                cur.next_row();
+            }
+        } else
         for (TileCursor cur(g0, tpr); cur.g < g1 && ok;) {
             const int row = cur.row;
             const int ti = cur.ti;
@@ -566,7 +644,7 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
             }
             const int a = ra.slot;
             float acc = 0.f;
-            if (ok && mbar_wait(tfull + a, ra.phase, abort_flag)) {
+            if (ok && warp_wait(tfull + a, ra.phase, abort_flag)) {
                 tc_fence_after();
                 const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                                        static_cast<uint32_t>(a * npad);
@@ -581,7 +659,7 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
             if (E4M3) {
                 const int sc = it & (kScaleRing - 1);
                 float scale = 1.f;
-                if (ok && mbar_wait(scfull + sc, (it / kScaleRing) & 1, abort_flag)) {
+                if (ok && warp_wait(scfull + sc, (it / kScaleRing) & 1, abort_flag)) {
                     scale = sS[sc * kTileRows + r];
                 } else if (ok) {
                     ok = false;
@@ -623,8 +701,8 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
             }
             const int s8i = r8.slot;
             const int sa = rs.slot;
-            if (!mbar_wait(sfull + s8i, r8.phase, abort_flag) ||
-                !mbar_wait(empty + sa, rs.phase ^ 1u, abort_flag)) {
+            if (!warp_wait(sfull + s8i, r8.phase, abort_flag) ||
+                !warp_wait(empty + sa, rs.phase ^ 1u, abort_flag)) {
                 ok = false;
                 break;
             }
