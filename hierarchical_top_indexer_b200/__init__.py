@@ -37,7 +37,7 @@ HISA_DEV_BAD_QUERY, HISA_DEV_CAPACITY, HISA_DEV_BAD_LEN, HISA_DEV_TIMEOUT = 0x1,
 
 EXPORTS = ("hisa_pool_blocks", "hisa_append", "hisa_select_workspace_bytes", "hisa_select",
            "hisa_select_inspect", "hisa_select_static", "dsa_flat_workspace_bytes", "dsa_flat_select", "hisa_topk_f32",
-           "hisa_profile_enable", "hisa_profile_read", "hisa_status_string")
+           "hisa_profile_enable", "hisa_profile_read", "hisa_status_string", "hisa_last_cuda_error")
 PHASES = ("block_score", "block_select", "token_score", "token_select", "flat_score",
           "flat_select", "pool", "append", "topk")
 
@@ -68,6 +68,8 @@ _lib.hisa_profile_enable.argtypes = [_I]
 _lib.hisa_profile_read.argtypes = [_P, _P, _I]
 _lib.hisa_status_string.argtypes = [_I]
 _lib.hisa_status_string.restype = ctypes.c_char_p
+_lib.hisa_last_cuda_error.argtypes = []
+_lib.hisa_last_cuda_error.restype = ctypes.c_char_p
 for _f in ("hisa_pool_blocks", "hisa_append", "hisa_select", "hisa_select_inspect", "hisa_select_static",
            "dsa_flat_select", "hisa_topk_f32", "hisa_profile_enable", "hisa_profile_read"):
     getattr(_lib, _f).restype = _I
@@ -75,7 +77,10 @@ for _f in ("hisa_pool_blocks", "hisa_append", "hisa_select", "hisa_select_inspec
 
 class HisaError(RuntimeError):
     def __init__(self, fn: str, code: int):
-        super().__init__(f"{fn}: {_lib.hisa_status_string(code).decode()} (code {code})")
+        msg = f"{fn}: {_lib.hisa_status_string(code).decode()} (code {code})"
+        if code == HISA_E_CUDA:
+            msg += f": {_lib.hisa_last_cuda_error().decode()}"
+        super().__init__(msg)
         self.code = code
 
 

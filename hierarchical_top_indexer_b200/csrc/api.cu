@@ -192,7 +192,14 @@ HisaWs hisa_ws(const KvView& v, int n_q, int m) {
 
 size_t flat_ld(const KvView& v) { return round_up(v.cap, 128); }
 
-int cuda_status(cudaError_t e) { return e == cudaSuccess ? HISA_OK : HISA_E_CUDA; }
+// The CUDA error behind the calling thread's last HISA_E_CUDA.
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+int cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return HISA_OK;
+    g_last_cuda_error = e;
+    return HISA_E_CUDA;
+}
 
 bool keys_map(CUtensorMap* map, const KvView& v, int box_rows) {
     const uint64_t rows = static_cast<uint64_t>(v.batch) * v.cap;
@@ -242,7 +249,9 @@ int run_score(int mode, const KvView& v, const CUtensorMap& amap, const CUtensor
     if (p.total_tiles == 0) return HISA_OK;
     const int sms = sm_count();
     if (sms <= 0) return HISA_E_CUDA;
-    const int grid = static_cast<int>(p.total_tiles < sms ? p.total_tiles : sms);
+    // one CTA per SM at most; with the block selection fused in, whole rows per CTA
+    const long long units = p.fuse ? p.n_q : p.total_tiles;
+    const int grid = static_cast<int>(units < sms ? units : sms);
     const int phase = mode == kScoreBlocks ? HISA_PHASE_BLOCK_SCORE
                       : mode == kScoreFlat ? HISA_PHASE_FLAT_SCORE
                                            : HISA_PHASE_TOKEN_SCORE;
@@ -289,8 +298,24 @@ int hisa_select_impl(const hisa_kv* kv, const uint16_t* Q, const float* w, const
     p.ldo = L.ldb;
     p.tiles_per_row = L.ldb / 128;
     p.counts = reinterpret_cast<unsigned long long*>(counts);
+    // Short rows (up to kFuseMaxBlocks = 4 tiles of blocks) and at most two rows per SM: the
+    // scoring kernel keeps the blocks itself, one CTA per row, which saves the
+    // selection launch.  Longer rows score faster spread over every SM, and
+    // many rows select faster in the selection kernel's one-CTA-per-row grid.
+    const bool fuse = L.ldb <= kFuseMaxBlocks && n_q <= 2 * sms;
+    if (fuse) {
+        p.fuse = 1;
+        p.m = m;
+        p.mm = L.mm;
+        p.sel_blocks = blocks;
+        p.sel_nblocks = nblocks;
+        p.sel_plan = plan;
+        p.sel_blocks_out = blocks_out;
+        p.sel_nblocks_out = nblocks_out;
+    }
     rc = run_score(kScoreBlocks, v, pmap, qmap, p, s);
     if (rc) return rc;
+    p.fuse = 0;
 
     SelectParams sp;
     std::memset(&sp, 0, sizeof sp);
@@ -313,7 +338,7 @@ int hisa_select_impl(const hisa_kv* kv, const uint16_t* Q, const float* w, const
     sp.plan = plan;
     sp.blocks_out = blocks_out;
     sp.nblocks_out = nblocks_out;
-    {
+    if (!fuse) {
         PhaseScope ps(HISA_PHASE_BLOCK_SELECT, s);
         rc = cuda_status(launch_select(sp, v.nblk, sms, s));
     }
@@ -532,6 +557,8 @@ int hisa_profile_read(float* ms, int* launches, int reset) {
     }
     return rc;
 }
+
+const char* hisa_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda_error); }
 
 const char* hisa_status_string(int code) {
     switch (code) {

@@ -49,7 +49,18 @@ struct ScoreParams {
     int stages;                   // bf16 operand stages
     int stages8;                  // e4m3 staging stages
     int keep_keys;                // rows share keys: keep them in L2 (else stream them)
+    // kScoreBlocks with fuse = 1: each CTA scores whole rows and keeps the own
+    // block plus the best m - 1 others itself (rows of at most kFuseMaxBlocks
+    // blocks); outputs as the block selection's
+    int fuse, m;
+    int32_t* sel_blocks;          // [n_q, mm]
+    int32_t* sel_nblocks;         // [n_q]
+    int4* sel_plan;               // [n_q]
+    int32_t* sel_blocks_out;      // [n_q, mm] or null
+    int32_t* sel_nblocks_out;     // [n_q] or null
 };
+
+constexpr int kFuseMaxBlocks = 512;
 
 enum SelectMode : int {
     kSelBlocks = 0,      // keep own block + best m-1 others -> blocks list

@@ -52,8 +52,12 @@ constexpr int kScaleRing = 16;                // e4m3 per-token scale slots (one
 constexpr int kTabSubs = 256;                 // first key row of each sub-box, per row window
 
 struct Layout {
-    uint32_t a, s8, sc, tab, q, w, bars, misc, total;
+    uint32_t a, s8, sc, tab, sel, q, w, bars, misc, total;
 };
+
+// Fused block selection scratch: the row's block score keys, a 256-bin
+// histogram, scan / result words.
+constexpr int kSelScratch = kFuseMaxBlocks * 4 + 256 * 4 + 16 * 4;
 
 __host__ __device__ inline int acc_count(int npad) { return 4 * npad <= 512 ? 4 : 2; }
 
@@ -61,7 +65,7 @@ __host__ __device__ inline Layout score_layout(int mode, bool e4m3, int d, int n
     const int halves = d / 64;
     const int stage = (mode == kScoreBlocks ? 2 : 1) * halves * kHalfBytes;
     Layout L;
-    uint32_t off = 0;
+    uint32_t off = 0;                        // from a 1024-byte aligned base
     L.a = off;
     off += sa * stage;
     L.s8 = off;
@@ -70,6 +74,9 @@ __host__ __device__ inline Layout score_layout(int mode, bool e4m3, int d, int n
     off += (e4m3 && mode != kScoreBlocks) ? kScaleRing * kTileRows * 4 : 0;
     L.tab = off;
     off += kTabSubs * 4;
+    L.sel = off;
+    off += mode == kScoreBlocks ? kSelScratch : 0;
+    off = (off + 1023u) & ~1023u;            // 128-byte-swizzled TMA boxes need 1024-byte alignment
     L.q = off;
     off += 2 * halves * npad * 128;
     L.w = off;
@@ -247,6 +254,121 @@ __device__ __forceinline__ float head_sum_any(int npad, uint32_t taddr, const fl
     }
 }
 
+// ---------------------------------------------- fused block selection
+// Run by the four epilogue warps (thread e = 0..127) on one row's block score
+// keys in shared memory; the same rule as the selection kernel: the top kk
+// keys, ties to the lower slot, kept slots in ascending order.
+
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// Exclusive scan of one value per epilogue thread (in thread order).
+__device__ __forceinline__ uint32_t epi_scan(uint32_t v, int e, uint32_t* misc) {
+    const int w = e >> 5, l = e & 31;
+    uint32_t incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
+        if (l >= o) incl += x;
+    }
+    if (l == 31) misc[w] = incl;
+    epi_bar();
+    uint32_t before = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) before += i < w ? misc[i] : 0u;
+    epi_bar();
+    return before + incl - v;
+}
+
+// The kk-th largest of the keys s[0..n) (0 < kk < n, every key nonzero):
+// four 8-bit radix rounds from the top.  Returns T; *take_eq = how many keys
+// equal to T are among the top kk.
+__device__ uint32_t epi_threshold(const uint32_t* s, int n, int kk, uint32_t* hist, uint32_t* misc, int e,
+                                  int* take_eq) {
+    uint32_t prefix = 0, mask = 0;
+    uint32_t krem = static_cast<uint32_t>(kk);
+    for (int shift = 24; shift >= 0; shift -= 8) {
+        hist[e] = 0;
+        hist[e + 128] = 0;
+        epi_bar();
+        for (int c = e; c < n; c += 128) {
+            const uint32_t x = s[c];
+            if ((x & mask) == prefix) atomicAdd(&hist[(x >> shift) & 255u], 1u);
+        }
+        epi_bar();
+        // thread e owns bins 255 - 2e and 254 - 2e (highest first)
+        const uint32_t h0 = hist[255 - 2 * e], h1 = hist[254 - 2 * e];
+        const uint32_t excl = epi_scan(h0 + h1, e, misc);
+        if (excl < krem && krem <= excl + h0 + h1) {
+            const bool first = krem <= excl + h0;
+            misc[4] = static_cast<uint32_t>(first ? 255 - 2 * e : 254 - 2 * e);
+            misc[5] = first ? krem - excl : krem - excl - h0;
+        }
+        epi_bar();
+        prefix |= misc[4] << shift;
+        mask |= 255u << shift;
+        krem = misc[5];
+        epi_bar();
+    }
+    *take_eq = static_cast<int>(krem);
+    return prefix;
+}
+
+// Writes the slots of the top kk keys of s[0..n) in ascending order to out
+// (and dbg) given T and take_eq from epi_threshold.
+__device__ void epi_emit(const uint32_t* s, int n, uint32_t T, int take_eq, int32_t* out, int32_t* dbg,
+                         uint32_t* misc, int e) {
+    const int w = e >> 5, l = e & 31;
+    const int per = ((n + 3) / 4 + 31) & ~31;
+    const int w0 = w * per;
+    const int w1 = min(n, w0 + per);
+    uint32_t gt = 0, eq = 0;
+    for (int base = w0; base < w1; base += 32) {
+        const int c = base + l;
+        const uint32_t x = c < w1 ? s[c] : 0u;
+        gt += __popc(__ballot_sync(0xffffffffu, c < w1 && x > T));
+        eq += __popc(__ballot_sync(0xffffffffu, c < w1 && x == T));
+    }
+    if (l == 0) {
+        misc[8 + w] = gt;
+        misc[12 + w] = eq;
+    }
+    epi_bar();
+    uint32_t eq_run = 0, pos = 0;
+    {
+        uint32_t eqb = 0, off = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t ei = misc[12 + i];
+            const int room = take_eq - static_cast<int>(eqb);
+            const uint32_t take = room <= 0 ? 0u : (static_cast<uint32_t>(room) < ei ? room : ei);
+            if (i == w) {
+                eq_run = eqb;
+                pos = off;
+            }
+            eqb += ei;
+            off += misc[8 + i] + take;
+        }
+    }
+    const unsigned lt = (1u << l) - 1u;
+    for (int base = w0; base < w1; base += 32) {
+        const int c = base + l;
+        const uint32_t x = c < w1 ? s[c] : 0u;
+        const bool is_gt = c < w1 && x > T;
+        const bool is_eq = c < w1 && x == T;
+        const unsigned eqm = __ballot_sync(0xffffffffu, is_eq);
+        const uint32_t eq_rank = eq_run + __popc(eqm & lt);
+        const bool sel = is_gt || (is_eq && eq_rank < static_cast<uint32_t>(take_eq));
+        const unsigned selm = __ballot_sync(0xffffffffu, sel);
+        if (sel) {
+            const int at = static_cast<int>(pos + __popc(selm & lt));
+            out[at] = c;
+            if (dbg) dbg[at] = c;
+        }
+        eq_run += __popc(eqm);
+        pos += __popc(selm);
+    }
+}
+
 template <int MODE, bool E4M3, int D>
 __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
     score_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap qmap,
@@ -290,8 +412,13 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
     const int tpr = p.tiles_per_row;
     const int BR = (MODE == kScoreBlocks) ? kTileRows : (p.B < kTileRows ? p.B : kTileRows);
     const int nsub = kTileRows / BR;
-    const long long g0 = p.total_tiles * blockIdx.x / gridDim.x;
-    const long long g1 = p.total_tiles * (blockIdx.x + 1) / gridDim.x;
+    // contiguous ranges of (row, tile) slots; whole rows when the block
+    // selection is fused in
+    const bool fuse = MODE == kScoreBlocks && p.fuse && tpr * kTileRows <= kFuseMaxBlocks;
+    const long long g0 = fuse ? static_cast<long long>(p.n_q) * blockIdx.x / gridDim.x * tpr
+                              : p.total_tiles * blockIdx.x / gridDim.x;
+    const long long g1 = fuse ? static_cast<long long>(p.n_q) * (blockIdx.x + 1) / gridDim.x * tpr
+                              : p.total_tiles * (blockIdx.x + 1) / gridDim.x;
 
     if (warp == kWarpProducer && lane == 0) {
         for (int s = 0; s < SA; ++s) {
@@ -607,6 +734,10 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
         const int quad = warp & 3;                    // TMEM lanes this warp may read
         const int r = quad * 32 + lane;               // tile row = candidate
         float* wv = sW + (warp - kWarpEpi0) * 128;
+        const int e = (warp - kWarpEpi0) * 32 + lane;                 // 0..127
+        uint32_t* sKeys = reinterpret_cast<uint32_t*>(smem + L.sel);  // fused selection
+        uint32_t* sHist = sKeys + kFuseMaxBlocks;
+        uint32_t* sMisc = sHist + 256;
         int it = 0, cur_row = -1;
         RowInfo R;
         R.nt = 0;
@@ -622,6 +753,21 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
                 if (MODE == kScoreHisa && R.nt > 0) {
                     own0 = R.lim - p.B;
                     own_t = R.t % p.B;
+                }
+                if (fuse && R.nt == 0) {
+                    // query position outside its sequence: no blocks
+                    int32_t* bl = p.sel_blocks + static_cast<size_t>(row) * p.mm;
+                    int32_t* bd = p.sel_blocks_out ? p.sel_blocks_out + static_cast<size_t>(row) * p.mm : nullptr;
+                    for (int i = e; i < p.mm; i += 128) {
+                        bl[i] = -1;
+                        if (bd) bd[i] = -1;
+                    }
+                    if (e == 0) {
+                        p.sel_nblocks[row] = 0;
+                        if (p.sel_nblocks_out) p.sel_nblocks_out[row] = 0;
+                        p.sel_plan[row] = make_int4(R.b, -1, 0, 0);
+                        set_status(p.status, HISA_DEV_BAD_QUERY);
+                    }
                 }
                 if (ti < R.nt) {
                     __syncwarp();
@@ -669,13 +815,46 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
                 if (lane == 0 && ok) mbar_arrive(scempty + sc);
                 acc *= scale;
             }
-            p.out[static_cast<size_t>(row) * p.ldo + c] = valid ? score_key(acc) : 0u;
+            if (fuse) sKeys[c] = valid ? score_key(acc) : 0u;
+            else p.out[static_cast<size_t>(row) * p.ldo + c] = valid ? score_key(acc) : 0u;
             if (p.counts) {
                 const bool slot = MODE == kScoreBlocks ? valid : c < R.lim;
                 const int n = __popc(__ballot_sync(0xffffffffu, slot));
                 if (lane == 0 && n)
                     atomicAdd(p.counts + 2 * row + (MODE == kScoreBlocks ? 0 : 1),
                               static_cast<unsigned long long>(n));
+            }
+            if (fuse && ti == R.nt - 1) {
+                // the row is scored: keep its own block and the best m - 1 others
+                epi_bar();
+                const int nb = R.lim;                  // visible blocks; the own block is nb - 1
+                int32_t* bl = p.sel_blocks + static_cast<size_t>(row) * p.mm;
+                int32_t* bd = p.sel_blocks_out ? p.sel_blocks_out + static_cast<size_t>(row) * p.mm : nullptr;
+                const int keep = nb <= p.m ? nb : p.m;
+                if (nb <= p.m) {
+                    for (int i = e; i < p.mm; i += 128) {
+                        const int v = i < nb ? i : -1;
+                        bl[i] = v;
+                        if (bd) bd[i] = v;
+                    }
+                } else {
+                    if (p.m > 1) {
+                        int take_eq;
+                        const uint32_t T = epi_threshold(sKeys, nb - 1, p.m - 1, sHist, sMisc, e, &take_eq);
+                        epi_emit(sKeys, nb - 1, T, take_eq, bl, bd, sMisc, e);
+                    }
+                    for (int i = p.m - 1 + e; i < p.mm; i += 128) {
+                        const int v = i == p.m - 1 ? nb - 1 : -1;   // own block last
+                        bl[i] = v;
+                        if (bd) bd[i] = v;
+                    }
+                }
+                if (e == 0) {
+                    p.sel_nblocks[row] = keep;
+                    if (p.sel_nblocks_out) p.sel_nblocks_out[row] = keep;
+                    p.sel_plan[row] = make_int4(R.b, R.t, keep, 0);
+                }
+                epi_bar();
             }
             ++it;
             ra.next(NACC);
@@ -745,6 +924,9 @@ template <int MODE, bool E4M3, int D>
 cudaError_t launch_t(const CUtensorMap& amap, const CUtensorMap& qmap, const ScoreParams& p, int grid,
                      cudaStream_t s) {
     const size_t smem = score_smem_bytes(MODE, E4M3, D, p.npad, p.stages, p.stages8);
+    // the swizzled TMA destinations (operand stages, query heads) start on 1024-byte boundaries
+    const Layout L = score_layout(MODE, E4M3, D, p.npad, p.stages, p.stages8);
+    if ((L.a | L.q) & 1023u) return cudaErrorInvalidValue;
     auto* fn = score_kernel<MODE, E4M3, D>;
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));

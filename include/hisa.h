@@ -258,6 +258,10 @@ int hisa_profile_read(float* ms, int* launches, int reset);
 /* Human-readable name of a return code. */
 const char* hisa_status_string(int code);
 
+/* The CUDA runtime's description of the error behind the calling thread's
+ * last HISA_E_CUDA from a launch ("no error" if there was none). */
+const char* hisa_last_cuda_error(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -66,6 +66,20 @@ def test_hisa_matches_oracle(dtype, d, H, B, m, k):
     assert kv.status_bits() == 0
 
 
+def test_hisa_rows_longer_than_the_fused_block_selection():
+    """More than 2048 blocks per row (more than the selection kernel stages in
+    one CTA's shared memory, and more than the block scoring kernel keeps
+    itself)."""
+    case = make_case(batch=1, L=20000, H=16, d=64, B=8, m=40, k=200, dtype="bf16", seed=77,
+                     positions=np.array([0, 7, 8, 12345, 19999]))
+    kv = device_case(case)
+    assert kv.nblk > 2048
+    gpu = run_hisa(case, kv)
+    _, swaps = check_hisa(case, gpu)
+    assert sum(s for s, _ in swaps) <= 2
+    assert kv.status_bits() == 0
+
+
 def test_hisa_with_every_block_is_the_flat_scan_bit_exact():
     """m >= #blocks: the same candidates in the same tile order through the
     same scoring kernel, so scores and indices agree exactly."""
