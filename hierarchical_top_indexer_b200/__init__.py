@@ -39,7 +39,7 @@ EXPORTS = ("hisa_pool_blocks", "hisa_append", "hisa_select_workspace_bytes", "hi
            "hisa_select_inspect", "hisa_select_static", "dsa_flat_workspace_bytes", "dsa_flat_select", "hisa_topk_f32",
            "hisa_profile_enable", "hisa_profile_read", "hisa_status_string", "hisa_last_cuda_error")
 PHASES = ("block_score", "block_select", "token_score", "token_select", "flat_score",
-          "flat_select", "pool", "append", "topk")
+          "flat_select", "pool", "append", "topk", "qsplit")
 
 
 class hisa_kv(ctypes.Structure):

@@ -171,11 +171,22 @@ struct Carve {
 };
 
 struct HisaWs {
-    size_t bkeys, blocks, nblocks, plan, tkeys, total;
+    size_t bkeys, blocks, nblocks, plan, tkeys, q8, w8, total;
     int ldb, ldt, mm;
 };
 
-HisaWs hisa_ws(const KvView& v, int n_q, int m) {
+// e4m3 keys with d = 128 are scored on the fp8 tensor cores against split
+// query heads (launch_qsplit), which the workspace holds.
+bool f8_keys(const KvView& v) { return v.e4m3 && v.d == 128; }
+
+void take_q8(Carve& c, const KvView& v, int n_q, int H, size_t* q8, size_t* w8) {
+    *q8 = *w8 = 0;
+    if (!f8_keys(v)) return;
+    *q8 = c.take(static_cast<size_t>(n_q) * 2 * npad_of(H) * 128);
+    *w8 = c.take(static_cast<size_t>(n_q) * npad_of(H) * 4);
+}
+
+HisaWs hisa_ws(const KvView& v, int n_q, int H, int m) {
     HisaWs w;
     w.mm = m < v.nblk ? m : v.nblk;
     w.ldb = static_cast<int>(round_up(v.nblk, 128));
@@ -186,6 +197,7 @@ HisaWs hisa_ws(const KvView& v, int n_q, int m) {
     w.nblocks = c.take(static_cast<size_t>(n_q) * 4);
     w.plan = c.take(static_cast<size_t>(n_q) * 16);
     w.tkeys = c.take(static_cast<size_t>(n_q) * w.ldt * 4);
+    take_q8(c, v, n_q, H, &w.q8, &w.w8);
     w.total = c.off;
     return w;
 }
@@ -203,6 +215,9 @@ int cuda_status(cudaError_t e) {
 
 bool keys_map(CUtensorMap* map, const KvView& v, int box_rows) {
     const uint64_t rows = static_cast<uint64_t>(v.batch) * v.cap;
+    if (f8_keys(v))   // one 128-byte row per key: the fp8 operand layout as loaded
+        return make_map(map, v.keys, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows, 128, box_rows, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B);
     if (v.e4m3)
         return make_map(map, v.keys, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows, v.d, box_rows, v.d,
                         CU_TENSOR_MAP_SWIZZLE_NONE);
@@ -259,6 +274,25 @@ int run_score(int mode, const KvView& v, const CUtensorMap& amap, const CUtensor
     return cuda_status(launch_score(mode, e4m3, v.d, amap, qmap, p, grid, s));
 }
 
+// fp8 scoring of e4m3 keys (d = 128): split the query heads into the
+// workspace and aim the query tensor map and the weights at them.
+int prep_f8(const KvView& v, const uint16_t* Q, const float* w, int n_q, int H, uint8_t* q8, float* w8,
+            CUtensorMap* qmap, ScoreParams& p, cudaStream_t s) {
+    if (!f8_keys(v)) return HISA_OK;
+    const int npad = npad_of(H);
+    {
+        PhaseScope ps(HISA_PHASE_QSPLIT, s);
+        const int rc = cuda_status(launch_qsplit(Q, w, n_q, H, npad, q8, w8, s));
+        if (rc) return rc;
+    }
+    if (!make_map(qmap, q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(n_q) * 2 * npad, 128,
+                  2 * npad, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+        return HISA_E_CUDA;
+    p.w8 = w8;
+    p.scale_bulk = v.cap % 4 == 0 && aligned(v.key_scale, 16) ? 1 : 0;
+    return HISA_OK;
+}
+
 int hisa_select_impl(const hisa_kv* kv, const uint16_t* Q, const float* w, const int32_t* q_seq,
                      const int32_t* q_pos, int n_q, int H, int m, int k, int32_t* idx, float* scores,
                      int32_t* blocks_out, int32_t* nblocks_out, uint64_t* counts, void* ws,
@@ -271,7 +305,7 @@ int hisa_select_impl(const hisa_kv* kv, const uint16_t* Q, const float* w, const
     rc = check_queries(Q, w, q_seq, n_q, H, k, idx);
     if (rc) return rc;
     if (n_q == 0) return HISA_OK;
-    const HisaWs L = hisa_ws(v, n_q, m);
+    const HisaWs L = hisa_ws(v, n_q, H, m);
     if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return HISA_E_WORKSPACE;
     uint8_t* base = static_cast<uint8_t*>(ws);
     uint32_t* bkeys = reinterpret_cast<uint32_t*>(base + L.bkeys);
@@ -345,6 +379,8 @@ int hisa_select_impl(const hisa_kv* kv, const uint16_t* Q, const float* w, const
     if (rc) return rc;
 
     // stage 2: score the kept blocks' tokens, keep the top-k tokens
+    rc = prep_f8(v, Q, w, n_q, H, base + L.q8, reinterpret_cast<float*>(base + L.w8), &qmap, p, s);
+    if (rc) return rc;
     p.out = tkeys;
     p.ldo = L.ldt;
     p.tiles_per_row = L.ldt / 128;
@@ -414,11 +450,10 @@ int hisa_append(const hisa_kv* kv, const void* tok, const float* tok_scale, hisa
 }
 
 size_t hisa_select_workspace_bytes(const hisa_kv* kv, int n_q, int H, int m, int k) {
-    (void)H;
     (void)k;
     KvView v;
-    if (check_kv(kv, &v) || n_q < 0 || m < 1) return 0;
-    return hisa_ws(v, n_q, m).total;
+    if (check_kv(kv, &v) || n_q < 0 || m < 1 || H < 1 || H > 128) return 0;
+    return hisa_ws(v, n_q, H, m).total;
 }
 
 int hisa_select(const hisa_kv* kv, const uint16_t* Q, const float* w, const int32_t* q_seq,
@@ -446,7 +481,7 @@ int hisa_select_static(const hisa_kv* kv, const uint16_t* Q, const float* w, con
     if (m < 1) return HISA_E_INVAL;
     rc = check_queries(Q, w, q_seq, n_q, H, k, idx);
     if (rc) return rc;
-    const size_t need = hisa_ws(v, n_q, m).total;
+    const size_t need = hisa_ws(v, n_q, H, m).total;
     if (need > HISA_STATIC_SCRATCH_BYTES) return HISA_E_SCRATCH_LIMIT;
     void* ws = nullptr;
     rc = static_scratch(&ws);
@@ -456,14 +491,26 @@ int hisa_select_static(const hisa_kv* kv, const uint16_t* Q, const float* w, con
                             reinterpret_cast<cudaStream_t>(stream));
 }
 
+// Flat scan workspace: score keys [n_q, round_up(cap, 128)], then (fp8
+// scoring) the split query heads.
+struct FlatWs {
+    size_t keys, q8, w8, total;
+};
+
+FlatWs flat_ws(const KvView& v, int n_q, int H) {
+    FlatWs f;
+    Carve c;
+    f.keys = c.take(static_cast<size_t>(n_q) * flat_ld(v) * 4);
+    take_q8(c, v, n_q, H, &f.q8, &f.w8);
+    f.total = c.off;
+    return f;
+}
+
 size_t dsa_flat_workspace_bytes(const hisa_kv* kv, int n_q, int H, int k) {
-    (void)H;
     (void)k;
     KvView v;
-    if (check_kv(kv, &v) || n_q < 0) return 0;
-    Carve c;
-    c.take(static_cast<size_t>(n_q) * flat_ld(v) * 4);
-    return c.off;
+    if (check_kv(kv, &v) || n_q < 0 || H < 1 || H > 128) return 0;
+    return flat_ws(v, n_q, H).total;
 }
 
 int dsa_flat_select(const hisa_kv* kv, const uint16_t* Q, const float* w, const int32_t* q_seq,
@@ -477,14 +524,17 @@ int dsa_flat_select(const hisa_kv* kv, const uint16_t* Q, const float* w, const 
     if (rc) return rc;
     if (n_q == 0) return HISA_OK;
     const size_t ld = flat_ld(v);
-    if (!ws || !aligned(ws, 256) || ws_bytes < dsa_flat_workspace_bytes(kv, n_q, H, k))
-        return HISA_E_WORKSPACE;
+    const FlatWs F = flat_ws(v, n_q, H);
+    if (!ws || !aligned(ws, 256) || ws_bytes < F.total) return HISA_E_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     CUtensorMap kmap, qmap;
     if (!keys_map(&kmap, v, v.B < 128 ? v.B : 128) || !query_map(&qmap, Q, n_q, H, v.d))
         return HISA_E_CUDA;
-    uint32_t* keys = static_cast<uint32_t*>(ws);
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    uint32_t* keys = reinterpret_cast<uint32_t*>(base + F.keys);
     ScoreParams p = score_params(v, w, q_seq, q_pos, n_q, H);
+    rc = prep_f8(v, Q, w, n_q, H, base + F.q8, reinterpret_cast<float*>(base + F.w8), &qmap, p, s);
+    if (rc) return rc;
     p.out = keys;
     p.ldo = static_cast<int>(ld);
     p.tiles_per_row = static_cast<int>(ld / 128);

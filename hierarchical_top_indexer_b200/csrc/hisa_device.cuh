@@ -173,6 +173,17 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint
         : "memory");
 }
 
+// D[tmem] (+)= A[smem] * B[smem]^T, e4m3 inputs, fp32 accumulate (K = 32 per op).
+__device__ __forceinline__ void umma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Arrive once on `bar` when every tcgen05 op issued so far by this thread is done.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
     asm volatile(
@@ -228,6 +239,26 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t n) {
            | (1u << 10)              // B format: bf16
            | ((n >> 3) << 17)        // N / 8
            | ((128u >> 4) << 24);    // M / 16
+}
+
+// Instruction descriptor: e4m3 x e4m3 -> fp32, both operands K-major,
+// M = 128, N = n (multiple of 16, 16..256).
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(uint32_t n) {
+    return (1u << 4)                 // D format: f32
+           | (0u << 7)               // A format: e4m3
+           | (0u << 10)              // B format: e4m3
+           | ((n >> 3) << 17)        // N / 8
+           | ((128u >> 4) << 24);    // M / 16
+}
+
+// 1-D bulk copy global -> shared (16-byte aligned addresses, size a multiple
+// of 16), completion counted in bytes on `bar`.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_addr(dst)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
 }
 
 // ------------------------------------------------- programmatic launch

@@ -49,6 +49,11 @@ struct ScoreParams {
     int stages;                   // bf16 operand stages
     int stages8;                  // e4m3 staging stages
     int keep_keys;                // rows share keys: keep them in L2 (else stream them)
+    // e4m3 keys with d = 128 (scored on the fp8 tensor cores): per-row head
+    // weights with each head's query scale folded in [n_q, npad], and whether
+    // every tile's per-token scales start on a 16-byte boundary (cap % 4 == 0)
+    const float* w8;
+    int scale_bulk;
     // kScoreBlocks with fuse = 1: each CTA scores whole rows and keeps the own
     // block plus the best m - 1 others itself (rows of at most kFuseMaxBlocks
     // blocks); outputs as the block selection's
@@ -106,5 +111,12 @@ cudaError_t launch_score(int mode, bool e4m3, int d, const CUtensorMap& keys_map
                          cudaStream_t s);
 
 cudaError_t launch_select(const SelectParams& p, int max_n, int sms, cudaStream_t s);
+
+// Query heads for scoring e4m3 keys (d = 128) on the fp8 tensor cores: every
+// head of Q [n_q, H, 128] bf16 is scaled by a power of two 2^e and split into
+// two e4m3 pieces, q * 2^e = q1 + q2; q8 [n_q, 2 * npad, 128] holds the q1
+// rows then the q2 rows (zero rows pad H to npad); w8 [n_q, npad] = w * 2^-e.
+cudaError_t launch_qsplit(const uint16_t* Q, const float* w, int n_q, int H, int npad, uint8_t* q8,
+                          float* w8, cudaStream_t s);
 
 }  // namespace hisa

@@ -59,17 +59,34 @@ struct Layout {
 // histogram, scan / result words.
 constexpr int kSelScratch = kFuseMaxBlocks * 4 + 256 * 4 + 16 * 4;
 
-__host__ __device__ inline int acc_count(int npad) { return 4 * npad <= 512 ? 4 : 2; }
+// Accumulators that fit TMEM's 512 columns for accumulators of n columns.
+__host__ __device__ inline int acc_count(int n) { return 4 * n <= 512 ? 4 : 2; }
+
+// e4m3 keys with d = 128 are scored on the fp8 tensor cores directly (the
+// 128-byte key rows are one swizzle row); d = 64 keys are widened to bf16.
+__host__ __device__ constexpr bool uses_f8(int mode, bool e4m3, int d) {
+    return e4m3 && d == 128 && mode != kScoreBlocks;
+}
+
+// Columns of one accumulator: the H heads, or for fp8 the two query pieces.
+__host__ __device__ inline int acc_width(int mode, bool e4m3, int d, int npad) {
+    return uses_f8(mode, e4m3, d) ? 2 * npad : npad;
+}
+
+__host__ __device__ constexpr int score_threads(int mode, bool e4m3, int d) {
+    return e4m3 && !uses_f8(mode, e4m3, d) ? 320 : 192;
+}
 
 __host__ __device__ inline Layout score_layout(int mode, bool e4m3, int d, int npad, int sa, int s8) {
     const int halves = d / 64;
-    const int stage = (mode == kScoreBlocks ? 2 : 1) * halves * kHalfBytes;
+    const bool f8 = uses_f8(mode, e4m3, d);
+    const int stage = f8 ? kTileRows * d : (mode == kScoreBlocks ? 2 : 1) * halves * kHalfBytes;
     Layout L;
     uint32_t off = 0;                        // from a 1024-byte aligned base
     L.a = off;
     off += sa * stage;
     L.s8 = off;
-    off += e4m3 ? s8 * kTileRows * d : 0;
+    off += e4m3 && !f8 ? s8 * kTileRows * d : 0;
     L.sc = off;
     off += (e4m3 && mode != kScoreBlocks) ? kScaleRing * kTileRows * 4 : 0;
     L.tab = off;
@@ -241,6 +258,48 @@ __device__ __forceinline__ float head_sum(uint32_t taddr, const float* wv) {
     return (a[0] + a[1]) + (a[2] + a[3]);
 }
 
+// fp8 accumulators: columns [0, NP) hold q1 . x and [NP, 2 NP) hold q2 . x per
+// head; sum_h w'_h * ReLU(q1 . x + q2 . x), w' carrying the query scale 2^-e.
+template <int NP>
+__device__ __forceinline__ float head_sum2(uint32_t taddr, const float* wv) {
+    float a[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int g = 0; g < NP; g += 32) {
+        constexpr int kG = NP < 32 ? NP : 32;
+        uint32_t r1[kG], r2[kG];
+#pragma unroll
+        for (int c = 0; c < kG; c += 16)
+            if (g + c < NP) {
+                tmem_ld16_nowait(taddr + g + c, r1 + c);
+                tmem_ld16_nowait(taddr + NP + g + c, r2 + c);
+            }
+        tmem_ld_wait();
+#pragma unroll
+        for (int h = 0; h < kG; h += 4) {
+            if (g + h >= NP) break;
+            const float4 w4 = lds_f32x4(wv + g + h);
+            a[0] = fmaf(w4.x, fmaxf(__uint_as_float(r1[h]) + __uint_as_float(r2[h]), 0.f), a[0]);
+            a[1] = fmaf(w4.y, fmaxf(__uint_as_float(r1[h + 1]) + __uint_as_float(r2[h + 1]), 0.f), a[1]);
+            a[2] = fmaf(w4.z, fmaxf(__uint_as_float(r1[h + 2]) + __uint_as_float(r2[h + 2]), 0.f), a[2]);
+            a[3] = fmaf(w4.w, fmaxf(__uint_as_float(r1[h + 3]) + __uint_as_float(r2[h + 3]), 0.f), a[3]);
+        }
+    }
+    return (a[0] + a[1]) + (a[2] + a[3]);
+}
+
+__device__ __forceinline__ float head_sum2_any(int npad, uint32_t taddr, const float* wv) {
+    switch (npad) {
+        case 16: return head_sum2<16>(taddr, wv);
+        case 32: return head_sum2<32>(taddr, wv);
+        case 48: return head_sum2<48>(taddr, wv);
+        case 64: return head_sum2<64>(taddr, wv);
+        case 80: return head_sum2<80>(taddr, wv);
+        case 96: return head_sum2<96>(taddr, wv);
+        case 112: return head_sum2<112>(taddr, wv);
+        default: return head_sum2<128>(taddr, wv);
+    }
+}
+
 __device__ __forceinline__ float head_sum_any(int npad, uint32_t taddr, const float* wv) {
     switch (npad) {
         case 16: return head_sum<16>(taddr, wv);
@@ -370,21 +429,24 @@ __device__ void epi_emit(const uint32_t* s, int n, uint32_t T, int take_eq, int3
 }
 
 template <int MODE, bool E4M3, int D>
-__global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
+__global__ void __launch_bounds__(score_threads(MODE, E4M3, D), 1)
     score_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap qmap,
                  const ScoreParams p) {
     constexpr int kHalves = D / 64;
     constexpr int kOps = (MODE == kScoreBlocks) ? 2 : 1;
-    constexpr int kStageBytes = kOps * kHalves * kHalfBytes;
+    constexpr bool kF8 = uses_f8(MODE, E4M3, D);          // fp8 operands straight from TMA
+    constexpr bool kConv = E4M3 && !kF8;                  // e4m3 widened to bf16 by converter warps
+    constexpr int kStageBytes = kF8 ? kTileRows * D : kOps * kHalves * kHalfBytes;
     constexpr int kStage8Bytes = kTileRows * D;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const int SA = p.stages;                    // bf16 operand stages
-    const int S8 = E4M3 ? p.stages8 : 1;        // e4m3 staging stages
+    const int S8 = kConv ? p.stages8 : 1;       // e4m3 staging stages
     const Layout L = score_layout(MODE, E4M3, D, p.npad, SA, S8);
-    const int NACC = acc_count(p.npad);
+    const int NW = acc_width(MODE, E4M3, D, p.npad);   // accumulator columns
+    const int NACC = acc_count(NW);
     uint8_t* sA = smem + L.a;
     uint8_t* s8 = smem + L.s8;
     uint8_t* sQ = smem + L.q;
@@ -407,7 +469,7 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int npad = p.npad;
-    const uint32_t ncols = tmem_columns(npad);
+    const uint32_t ncols = tmem_columns(NW);
     const int q_slot_bytes = kHalves * npad * 128;
     const int tpr = p.tiles_per_row;
     const int BR = (MODE == kScoreBlocks) ? kTileRows : (p.B < kTileRows ? p.B : kTileRows);
@@ -422,7 +484,7 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
 
     if (warp == kWarpProducer && lane == 0) {
         for (int s = 0; s < SA; ++s) {
-            mbar_init(full + s, E4M3 ? 4 : 1);
+            mbar_init(full + s, kConv ? 4 : 1);
             mbar_init(empty + s, 1);
         }
         for (int s = 0; s < S8; ++s) {
@@ -438,7 +500,7 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
             mbar_init(qempty + a, 1);
         }
         for (int r = 0; r < kScaleRing; ++r) {
-            mbar_init(scfull + r, 32);     // one cp.async arrival per producer lane
+            mbar_init(scfull + r, kConv ? 32 : 1);   // per producer lane (converter path) or lane 0
             mbar_init(scempty + r, 4);     // one per epilogue warp
         }
         *abort_flag = 0;
@@ -469,12 +531,12 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
         R.nt = 0;
         int win_cur = 0, win_nxt = 0, cur_w = 0;
         bool ok = true;
-        const int NS = E4M3 ? S8 : SA;
+        const int NS = kConv ? S8 : SA;
         Ring ring;
-        if constexpr (!E4M3) {
-            // bf16 keys: per row, the warp stages the sub-boxes' first key rows
-            // in shared memory; lane 0 alone then issues the row's tiles, one
-            // barrier wait and one transaction count per tile
+        if constexpr (!kConv) {
+            // bf16 and fp8 keys: per row, the warp stages the sub-boxes' first
+            // key rows in shared memory; lane 0 alone then issues the row's
+            // tiles, one barrier wait and one transaction count per tile
             int* sTab = reinterpret_cast<int*>(smem + L.tab);
             TileCursor cur(g0, tpr);
             while (cur.g < g1 && ok) {
@@ -493,10 +555,15 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
                 }
                 if (lane == 0) {
                     mbar_arrive_expect_tx(qfull + qs, q_slot_bytes);
+                    if (kF8) {
+                        // the row's split heads: one [2 npad x 128 B] box
+                        tma_load_2d(sQ + qs * q_slot_bytes, &qmap, qfull + qs, 0, row * 2 * npad);
+                    } else {
 #pragma unroll
-                    for (int kh = 0; kh < kHalves; ++kh)
-                        tma_load_2d(sQ + qs * q_slot_bytes + kh * npad * 128, &qmap, qfull + qs, kh * 64,
-                                    row * p.H);
+                        for (int kh = 0; kh < kHalves; ++kh)
+                            tma_load_2d(sQ + qs * q_slot_bytes + kh * npad * 128, &qmap, qfull + qs, kh * 64,
+                                        row * p.H);
+                    }
                 }
                 ++qloads;
                 for (int t = cur.ti; t < t_end && ok;) {
@@ -508,7 +575,9 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
                     }
                     if (lane == 0) {
                         for (int k = 0; k < nwin; ++k) {
-                            if (!mbar_wait(empty + ring.slot, ring.phase ^ 1u, abort_flag)) {
+                            if (!mbar_wait(empty + ring.slot, ring.phase ^ 1u, abort_flag) ||
+                                (kF8 && !mbar_wait(scempty + (it & (kScaleRing - 1)),
+                                                   ((it / kScaleRing) & 1) ^ 1, abort_flag))) {
                                 ok = false;
                                 break;
                             }
@@ -527,10 +596,49 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
                                     const int srow = MODE == kScoreHisa
                                                          ? sTab[k * nsub + sub]
                                                          : R.b * p.cap + (t + k) * kTileRows + sub * BR;
+                                    if (kF8) {
+                                        tma_load_2d_hint(dst + sub * BR * D, &amap, fb, 0, srow, pol);
+                                    } else {
 #pragma unroll
-                                    for (int kh = 0; kh < kHalves; ++kh)
-                                        tma_load_2d_hint(dst + kh * kHalfBytes + sub * BR * 128, &amap, fb,
-                                                         kh * 64, srow, pol);
+                                        for (int kh = 0; kh < kHalves; ++kh)
+                                            tma_load_2d_hint(dst + kh * kHalfBytes + sub * BR * 128, &amap, fb,
+                                                             kh * 64, srow, pol);
+                                    }
+                                }
+                            }
+                            if (kF8) {
+                                // the tile's per-token scales into the scale ring
+                                const int sc = it & (kScaleRing - 1);   // free: waited above
+                                float* sdst = sS + sc * kTileRows;
+                                if (p.scale_bulk) {
+                                    uint32_t bytes = 0;
+                                    for (int sub = 0; sub < nsub; ++sub) {
+                                        const long long srow = MODE == kScoreHisa
+                                                                   ? sTab[k * nsub + sub]
+                                                                   : R.b * p.cap + (t + k) * kTileRows + sub * BR;
+                                        const long long nv = key_rows - srow < BR ? key_rows - srow : BR;
+                                        bytes += nv > 0 ? static_cast<uint32_t>(nv) * 4u : 0u;
+                                    }
+                                    mbar_arrive_expect_tx(scfull + sc, bytes);
+                                    for (int sub = 0; sub < nsub; ++sub) {
+                                        const long long srow = MODE == kScoreHisa
+                                                                   ? sTab[k * nsub + sub]
+                                                                   : R.b * p.cap + (t + k) * kTileRows + sub * BR;
+                                        const long long nv = key_rows - srow < BR ? key_rows - srow : BR;
+                                        if (nv > 0)
+                                            bulk_load(sdst + sub * BR, p.key_scale + srow,
+                                                      static_cast<uint32_t>(nv) * 4u, scfull + sc);
+                                    }
+                                } else {
+                                    for (int r = 0; r < kTileRows; ++r) {
+                                        const int sub = r / BR;
+                                        const long long srow =
+                                            (MODE == kScoreHisa ? sTab[k * nsub + sub]
+                                                                : R.b * p.cap + (t + k) * kTileRows + sub * BR) +
+                                            (r - sub * BR);
+                                        if (srow < key_rows) cp_async_4(sdst + r, p.key_scale + srow);
+                                    }
+                                    cp_async_arrive_noinc(scfull + sc);
                                 }
                             }
                             ++it;
@@ -652,13 +760,16 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
         if (E4M3) cp_async_wait_all();   // no scale copy still landing at exit
         if (lane == 0) {
             if (!ok) raise_abort(abort_flag, p.status);
+            if (kF8 && !ok)
+                for (int n = it > kScaleRing ? it - kScaleRing : 0; n < it; ++n)
+                    mbar_wait(scfull + (n & (kScaleRing - 1)), (n / kScaleRing) & 1, nullptr);
             // Drain: no copy into, and no arrive on, this CTA's shared memory
             // may still be pending when it exits.
             for (int n = it > NS ? it - NS : 0; n < it; ++n) {
                 const int s = n % NS;
                 const uint32_t ph = (n / NS) & 1;
-                if (ok) mbar_wait(E4M3 ? sempty + s : empty + s, ph, nullptr);
-                else mbar_wait(E4M3 ? sfull + s : full + s, ph, nullptr);
+                if (ok) mbar_wait(kConv ? sempty + s : empty + s, ph, nullptr);
+                else mbar_wait(kConv ? sfull + s : full + s, ph, nullptr);
             }
             if (qloads >= 1) {
                 if (ok && qloads >= 2)
@@ -668,7 +779,8 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
         }
     } else if (warp == kWarpMma) {
         if (lane == 0) {
-            const uint32_t idesc = idesc_bf16_f32(static_cast<uint32_t>(npad));
+            const uint32_t idesc = kF8 ? idesc_e4m3_f32(static_cast<uint32_t>(NW))
+                                       : idesc_bf16_f32(static_cast<uint32_t>(npad));
             int it = 0, qloads = 0, cur_row = -1;
             uint32_t q_base = 0;
             RowInfo R;
@@ -703,8 +815,15 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * npad);
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * NW);
                 const uint32_t a_base = smem_addr(sA + s * kStageBytes);
+                if (kF8) {
+                    // 128 candidates x (q1 | q2 pieces of the heads) x 128 bytes: four K = 32 steps
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_e4m3(d_tmem, sw128_kmajor_desc(a_base + kk * 32), sw128_kmajor_desc(q_base + kk * 32),
+                                  idesc, kk ? 1u : 0u);
+                } else {
 #pragma unroll
                 for (int kh = 0; kh < kHalves; ++kh) {
 #pragma unroll
@@ -718,6 +837,7 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
                             umma_bf16(d_tmem, ldesc, bdesc, idesc, 1u);
                         }
                     }
+                }
                 }
                 umma_commit(empty + s);
                 umma_commit(tfull + a);
@@ -771,7 +891,9 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
                 }
                 if (ti < R.nt) {
                     __syncwarp();
-                    for (int h = lane; h < 128; h += 32) wv[h] = h < p.H ? p.w[row * p.H + h] : 0.f;
+                    for (int h = lane; h < 128; h += 32)
+                        wv[h] = kF8 ? (h < npad ? p.w8[static_cast<size_t>(row) * npad + h] : 0.f)
+                                    : (h < p.H ? p.w[row * p.H + h] : 0.f);
                     __syncwarp();
                 }
             }
@@ -793,8 +915,8 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
             if (ok && warp_wait(tfull + a, ra.phase, abort_flag)) {
                 tc_fence_after();
                 const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
-                                       static_cast<uint32_t>(a * npad);
-                acc = head_sum_any(npad, taddr, wv);
+                                       static_cast<uint32_t>(a * NW);
+                acc = kF8 ? head_sum2_any(npad, taddr, wv) : head_sum_any(npad, taddr, wv);
                 tc_fence_before();
             } else if (ok) {
                 ok = false;
@@ -860,7 +982,7 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
             ra.next(NACC);
             cur.next();
         }
-    } else if (E4M3 && warp >= kWarpConv0) {
+    } else if (kConv && warp >= kWarpConv0) {
         const int cw = warp - kWarpConv0;
         int it = 0, cur_row = -1;
         RowInfo R;
@@ -920,6 +1042,59 @@ __global__ void __launch_bounds__(E4M3 ? 320 : 192, 1)
     if (warp == kWarpMma) tmem_dealloc(tmem_base, ncols);
 }
 
+// Query heads for fp8 scoring (see launch_qsplit).  One CTA per query row,
+// one warp per head, four elements per lane.  The power of two puts the
+// head's largest |q| in (224, 448] (e4m3's largest finite value is 448), so
+// q1 = e4m3(q * 2^e) and q2 = e4m3(q * 2^e - q1) hold the bf16 value exactly
+// unless part of it falls below e4m3's smallest step (2^-9).
+__global__ void __launch_bounds__(128) qsplit_kernel(const uint16_t* __restrict__ Q, const float* __restrict__ w,
+                                                     int H, int npad, uint8_t* __restrict__ q8,
+                                                     float* __restrict__ w8) {
+    const int row = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    grid_dependency_wait();
+    grid_launch_dependents();
+    for (int h = warp; h < npad; h += 4) {
+        uint32_t* o1 = reinterpret_cast<uint32_t*>(q8 + (static_cast<size_t>(row) * 2 * npad + h) * 128);
+        uint32_t* o2 = reinterpret_cast<uint32_t*>(q8 + (static_cast<size_t>(row) * 2 * npad + npad + h) * 128);
+        if (h >= H) {
+            o1[lane] = 0u;
+            o2[lane] = 0u;
+            if (lane == 0) w8[static_cast<size_t>(row) * npad + h] = 0.f;
+            continue;
+        }
+        const uint2 raw = *reinterpret_cast<const uint2*>(Q + (static_cast<size_t>(row) * H + h) * 128 + lane * 4);
+        float v[4] = {__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xFFFF0000u),
+                      __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xFFFF0000u)};
+        float mx = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        int e = 0;
+        if (mx > 0.f) {
+            const int E = static_cast<int>((__float_as_uint(mx) >> 23) & 255u) - 127;   // floor(log2 mx)
+            e = 8 - E;                                        // mx * 2^e in [256, 512)
+            e = e > 126 ? 126 : (e < -126 ? -126 : e);
+            if (mx * __uint_as_float(static_cast<uint32_t>(127 + e) << 23) > 448.f) --e;
+        }
+        const float up = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);     // 2^e, exact
+        uint32_t p1 = 0, p2 = 0;
+#pragma unroll
+        for (int i = 0; i < 4; i += 2) {
+            const float2 a = make_float2(v[i] * up, v[i + 1] * up);
+            const __nv_fp8x2_storage_t c1 = __nv_cvt_float2_to_fp8x2(a, __NV_SATFINITE, __NV_E4M3);
+            const float2 f1 = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(c1, __NV_E4M3)));
+            const float2 r = make_float2(a.x - f1.x, a.y - f1.y);              // exact
+            const __nv_fp8x2_storage_t c2 = __nv_cvt_float2_to_fp8x2(r, __NV_SATFINITE, __NV_E4M3);
+            p1 |= static_cast<uint32_t>(c1) << (8 * i);
+            p2 |= static_cast<uint32_t>(c2) << (8 * i);
+        }
+        o1[lane] = p1;
+        o2[lane] = p2;
+        if (lane == 0)
+            w8[static_cast<size_t>(row) * npad + h] =
+                w[static_cast<size_t>(row) * H + h] * __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+    }
+}
+
 template <int MODE, bool E4M3, int D>
 cudaError_t launch_t(const CUtensorMap& amap, const CUtensorMap& qmap, const ScoreParams& p, int grid,
                      cudaStream_t s) {
@@ -933,7 +1108,7 @@ cudaError_t launch_t(const CUtensorMap& amap, const CUtensorMap& qmap, const Sco
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
-    cfg.blockDim = dim3(E4M3 ? 320 : 192);
+    cfg.blockDim = dim3(score_threads(MODE, E4M3, D));
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
@@ -947,6 +1122,21 @@ cudaError_t launch_t(const CUtensorMap& amap, const CUtensorMap& qmap, const Sco
 
 }  // namespace
 
+cudaError_t launch_qsplit(const uint16_t* Q, const float* w, int n_q, int H, int npad, uint8_t* q8,
+                          float* w8, cudaStream_t s) {
+    if (n_q == 0) return cudaSuccess;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(n_q));
+    cfg.blockDim = dim3(128);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, qsplit_kernel, Q, w, H, npad, q8, w8);
+}
+
 size_t score_smem_bytes(int mode, bool e4m3, int d, int npad, int stages, int stages8) {
     const size_t need = score_layout(mode, e4m3, d, npad, stages, stages8).total + 1024;
     return need < static_cast<size_t>(kMinSmem) ? static_cast<size_t>(kMinSmem) : need;
@@ -957,9 +1147,9 @@ size_t score_smem_bytes(int mode, bool e4m3, int d, int npad, int stages, int st
 void score_stages(int mode, bool e4m3, int d, int npad, int* stages, int* stages8) {
     *stages = 0;
     *stages8 = 0;
-    if (!e4m3) {
+    if (!e4m3 || uses_f8(mode, e4m3, d)) {
         for (int s = 2; s <= kMaxStages; ++s)
-            if (score_layout(mode, false, d, npad, s, 0).total + 1024 <= static_cast<uint32_t>(kMaxSmem))
+            if (score_layout(mode, e4m3, d, npad, s, 0).total + 1024 <= static_cast<uint32_t>(kMaxSmem))
                 *stages = s;
         return;
     }

@@ -157,6 +157,10 @@ int hisa_append(const hisa_kv* kv, const void* tok, const float* tok_scale,
  * H in 1..128.  The pooled index must be current for every row (built by
  * hisa_pool_blocks / hisa_append); the own block's representative may cover
  * keys past t — it is kept whatever its score.
+ * e4m3 keys with d = 128 are scored on the fp8 tensor cores: every query head
+ * is scaled by a power of two and split into two e4m3 parts whose sum is the
+ * bf16 value, except for the parts of an element below e4m3's smallest step
+ * after scaling (under 2^-17 of the head's largest |q|), which are dropped.
  */
 size_t hisa_select_workspace_bytes(const hisa_kv* kv, int n_q, int H, int m, int k);
 int hisa_select(const hisa_kv* kv, const uint16_t* Q, const float* w, const int32_t* q_seq,
@@ -250,7 +254,8 @@ enum hisa_phase {
     HISA_PHASE_POOL = 6,          /* hisa_pool_blocks */
     HISA_PHASE_APPEND = 7,        /* hisa_append */
     HISA_PHASE_TOPK = 8,          /* hisa_topk_f32 */
-    HISA_NUM_PHASES = 9
+    HISA_PHASE_QSPLIT = 9,        /* query heads split for fp8 scoring (e4m3 keys, d = 128) */
+    HISA_NUM_PHASES = 10
 };
 int hisa_profile_enable(int on);
 int hisa_profile_read(float* ms, int* launches, int reset);

@@ -80,6 +80,21 @@ def test_hisa_rows_longer_than_the_fused_block_selection():
     assert kv.status_bits() == 0
 
 
+def test_e4m3_caches_whose_scale_rows_are_not_16_byte_aligned():
+    """cap % 4 != 0: the per-token scales of a tile do not start on a 16-byte
+    boundary, so they are copied one by one instead of in bulk."""
+    case = make_case(batch=3, L=[1001, 999, 517], H=64, d=128, B=64, m=6, k=200, dtype="e4m3",
+                     seed=91, positions=[np.array([1000, 640, 0]), np.array([998, 63]),
+                                         np.array([516, 64])])
+    assert case.cap % 4 != 0
+    kv = device_case(case)
+    _, swaps = check_hisa(case, run_hisa(case, kv))
+    assert sum(s for s, _ in swaps) <= 2
+    _, fswaps = check_flat(case, run_flat(case, kv))
+    assert sum(fswaps) <= 2
+    assert kv.status_bits() == 0
+
+
 def test_hisa_with_every_block_is_the_flat_scan_bit_exact():
     """m >= #blocks: the same candidates in the same tile order through the
     same scoring kernel, so scores and indices agree exactly."""
