@@ -253,20 +253,21 @@ ScoreParams score_params(const KvView& v, const float* w, const int32_t* q_seq, 
     return p;
 }
 
-// Grid: one CTA per SM at most, each taking an equal contiguous range of the
-// row-major (row, tile) slots.
+// Grid: one (or two) CTAs per SM at most, each taking an equal contiguous
+// range of the row-major (row, tile) slots.
 int run_score(int mode, const KvView& v, const CUtensorMap& amap, const CUtensorMap& qmap,
               ScoreParams& p, cudaStream_t s) {
     const bool e4m3 = mode != kScoreBlocks && v.e4m3;
-    score_stages(mode, e4m3, v.d, p.npad, &p.stages, &p.stages8);
-    if (p.stages < 2) return HISA_E_UNSUPPORTED;
+    const int per_sm = score_config(mode, e4m3, v.d, p.npad, &p.stages, &p.stages8, &p.nacc);
+    if (p.stages < 2 || p.nacc < 1) return HISA_E_UNSUPPORTED;
     p.total_tiles = static_cast<long long>(p.n_q) * p.tiles_per_row;
     if (p.total_tiles == 0) return HISA_OK;
     const int sms = sm_count();
     if (sms <= 0) return HISA_E_CUDA;
-    // one CTA per SM at most; with the block selection fused in, whole rows per CTA
+    // with the block selection fused in, whole rows per CTA
     const long long units = p.fuse ? p.n_q : p.total_tiles;
-    const int grid = static_cast<int>(units < sms ? units : sms);
+    const long long slots = static_cast<long long>(per_sm) * sms;
+    const int grid = static_cast<int>(units < slots ? units : slots);
     const int phase = mode == kScoreBlocks ? HISA_PHASE_BLOCK_SCORE
                       : mode == kScoreFlat ? HISA_PHASE_FLAT_SCORE
                                            : HISA_PHASE_TOKEN_SCORE;

@@ -48,6 +48,7 @@ struct ScoreParams {
     long long total_tiles;        // n_q * tiles_per_row
     int stages;                   // bf16 operand stages
     int stages8;                  // e4m3 staging stages
+    int nacc;                     // TMEM accumulators
     int keep_keys;                // rows share keys: keep them in L2 (else stream them)
     // e4m3 keys with d = 128 (scored on the fp8 tensor cores): per-row head
     // weights with each head's query scale folded in [n_q, npad], and whether
@@ -104,7 +105,7 @@ cudaError_t launch_append(const KvView& kv, const void* tok, const float* tok_sc
 // Scoring: tensor maps built by the caller.  `keys_map` covers keys
 // ([batch*cap, d], bf16 swizzled 128B boxes, or e4m3 plain boxes) or, for
 // kScoreBlocks, pooled_hl ([batch*nblk, 2d] bf16).
-void score_stages(int mode, bool e4m3, int d, int npad, int* stages, int* stages8);
+int score_config(int mode, bool e4m3, int d, int npad, int* stages, int* stages8, int* nacc);
 size_t score_smem_bytes(int mode, bool e4m3, int d, int npad, int stages, int stages8);
 cudaError_t launch_score(int mode, bool e4m3, int d, const CUtensorMap& keys_map,
                          const CUtensorMap& q_map, const ScoreParams& p, int grid,

@@ -46,6 +46,8 @@ constexpr int kWarpEpi0 = 2;
 constexpr int kWarpConv0 = 6;
 constexpr int kMinSmem = 120 * 1024;          // keeps one CTA (and its TMEM) per SM
 constexpr int kMaxSmem = 232448;
+constexpr int kSmem2 = 113 * 1024;            // per CTA when two share an SM
+constexpr int kMinSmem2 = 80 * 1024;          // keeps it at two
 constexpr int kMaxAcc = 4;
 constexpr int kMaxStages = 8;
 constexpr int kScaleRing = 16;                // e4m3 per-token scale slots (one tile each)
@@ -59,8 +61,11 @@ struct Layout {
 // histogram, scan / result words.
 constexpr int kSelScratch = kFuseMaxBlocks * 4 + 256 * 4 + 16 * 4;
 
-// Accumulators that fit TMEM's 512 columns for accumulators of n columns.
-__host__ __device__ inline int acc_count(int n) { return 4 * n <= 512 ? 4 : 2; }
+// Accumulators of n columns that fit a CTA's share of TMEM's 512 columns (up to four).
+__host__ __device__ inline int acc_count(int n, int per_sm) {
+    const int c = 512 / per_sm / n;
+    return c > 4 ? 4 : c;
+}
 
 // e4m3 keys with d = 128 are scored on the fp8 tensor cores directly (the
 // 128-byte key rows are one swizzle row); d = 64 keys are widened to bf16.
@@ -75,6 +80,17 @@ __host__ __device__ inline int acc_width(int mode, bool e4m3, int d, int npad) {
 
 __host__ __device__ constexpr int score_threads(int mode, bool e4m3, int d) {
     return e4m3 && !uses_f8(mode, e4m3, d) ? 320 : 192;
+}
+
+// Token and flat scoring of bf16 or fp8 keys run two CTAs per SM (half the
+// shared memory and TMEM each) when the accumulators are at most 128 columns:
+// two independent pipelines per SM hide each other's issue and drain gaps.
+__host__ __device__ constexpr bool two_per_sm_kind(int mode, bool e4m3, int d) {
+    return mode != kScoreBlocks && !(e4m3 && !uses_f8(mode, e4m3, d));
+}
+
+__host__ __device__ inline int ctas_per_sm(int mode, bool e4m3, int d, int npad) {
+    return two_per_sm_kind(mode, e4m3, d) && acc_width(mode, e4m3, d, npad) <= 128 ? 2 : 1;
 }
 
 __host__ __device__ inline Layout score_layout(int mode, bool e4m3, int d, int npad, int sa, int s8) {
@@ -106,9 +122,10 @@ __host__ __device__ inline Layout score_layout(int mode, bool e4m3, int d, int n
     return L;
 }
 
-__host__ __device__ inline uint32_t tmem_columns(int npad) {
+// TMEM allocation for `cols` accumulator columns: a power of two, at least 32.
+__host__ __device__ inline uint32_t tmem_columns(int cols) {
     uint32_t c = 32;
-    while (c < static_cast<uint32_t>(acc_count(npad) * npad)) c <<= 1;
+    while (c < static_cast<uint32_t>(cols)) c <<= 1;
     return c;
 }
 
@@ -429,7 +446,7 @@ __device__ void epi_emit(const uint32_t* s, int n, uint32_t T, int take_eq, int3
 }
 
 template <int MODE, bool E4M3, int D>
-__global__ void __launch_bounds__(score_threads(MODE, E4M3, D), 1)
+__global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(MODE, E4M3, D) ? 2 : 1)
     score_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap qmap,
                  const ScoreParams p) {
     constexpr int kHalves = D / 64;
@@ -446,7 +463,7 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), 1)
     const int S8 = kConv ? p.stages8 : 1;       // e4m3 staging stages
     const Layout L = score_layout(MODE, E4M3, D, p.npad, SA, S8);
     const int NW = acc_width(MODE, E4M3, D, p.npad);   // accumulator columns
-    const int NACC = acc_count(NW);
+    const int NACC = p.nacc;
     uint8_t* sA = smem + L.a;
     uint8_t* s8 = smem + L.s8;
     uint8_t* sQ = smem + L.q;
@@ -469,7 +486,7 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int npad = p.npad;
-    const uint32_t ncols = tmem_columns(NW);
+    const uint32_t ncols = tmem_columns(NACC * NW);
     const int q_slot_bytes = kHalves * npad * 128;
     const int tpr = p.tiles_per_row;
     const int BR = (MODE == kScoreBlocks) ? kTileRows : (p.B < kTileRows ? p.B : kTileRows);
@@ -1139,25 +1156,31 @@ cudaError_t launch_qsplit(const uint16_t* Q, const float* w, int n_q, int H, int
 
 size_t score_smem_bytes(int mode, bool e4m3, int d, int npad, int stages, int stages8) {
     const size_t need = score_layout(mode, e4m3, d, npad, stages, stages8).total + 1024;
-    return need < static_cast<size_t>(kMinSmem) ? static_cast<size_t>(kMinSmem) : need;
+    const size_t lo = ctas_per_sm(mode, e4m3, d, npad) == 2 ? kMinSmem2 : kMinSmem;
+    return need < lo ? lo : need;
 }
 
-// Operand stages (and e4m3 staging stages): as many as fit; the e4m3 path
-// keeps two bf16 operand stages and spends the rest on staging.
-void score_stages(int mode, bool e4m3, int d, int npad, int* stages, int* stages8) {
+// Operand stages (and e4m3 staging stages) as many as fit the CTA's share of
+// shared memory (the e4m3 converter path keeps two bf16 operand stages and
+// spends the rest on staging), and the accumulators that fit its TMEM share.
+// Returns the CTAs per SM.
+int score_config(int mode, bool e4m3, int d, int npad, int* stages, int* stages8, int* nacc) {
+    const int per_sm = ctas_per_sm(mode, e4m3, d, npad);
+    const uint32_t budget = static_cast<uint32_t>(per_sm == 2 ? kSmem2 : kMaxSmem);
     *stages = 0;
     *stages8 = 0;
+    *nacc = acc_count(acc_width(mode, e4m3, d, npad), per_sm);
     if (!e4m3 || uses_f8(mode, e4m3, d)) {
         for (int s = 2; s <= kMaxStages; ++s)
-            if (score_layout(mode, e4m3, d, npad, s, 0).total + 1024 <= static_cast<uint32_t>(kMaxSmem))
-                *stages = s;
-        return;
+            if (score_layout(mode, e4m3, d, npad, s, 0).total + 1024 <= budget) *stages = s;
+        return per_sm;
     }
     for (int s8 = 2; s8 <= kMaxStages; ++s8)
-        if (score_layout(mode, true, d, npad, 2, s8).total + 1024 <= static_cast<uint32_t>(kMaxSmem)) {
+        if (score_layout(mode, true, d, npad, 2, s8).total + 1024 <= budget) {
             *stages = 2;
             *stages8 = s8;
         }
+    return per_sm;
 }
 
 cudaError_t launch_score(int mode, bool e4m3, int d, const CUtensorMap& amap, const CUtensorMap& qmap,
