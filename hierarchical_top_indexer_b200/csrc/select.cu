@@ -651,18 +651,9 @@ __global__ void __launch_bounds__(kRowThreads) select_row_kernel(const SelectPar
             const int shift = span == 0 ? 0 : max(0, 32 - __clz(span) - kBinBits);
             for (int i = tid; i < kBins; i += kRowThreads) sh.hist[i] = 0;
             __syncthreads();
-            {
-                // lane l of warp w takes the contiguous chunk l * 16 + w, so that
-                // the lanes of a warp hold keys from far-apart slots (neighbouring
-                // slots share a block and often a bin); the skew keeps the reads
-                // spread over the banks
-                const int S = (n + kRowThreads - 1) / kRowThreads;
-                const int c0 = (lane * kRowWarps + warp) * S;
-                for (int j = 0; j < S; ++j) {
-                    const int c = c0 + (j + lane) % S;
-                    const uint32_t x = c < n ? ks[c] : 0u;
-                    if (x != 0u && x >= lo && x <= hi) atomicAdd(&sh.hist[(x - lo) >> shift], 1u);
-                }
+            for (int c = tid; c < n; c += kRowThreads) {
+                const uint32_t x = ks[c];
+                if (x != 0u && x >= lo && x <= hi) atomicAdd(&sh.hist[(x - lo) >> shift], 1u);
             }
             __syncthreads();
             // thread t owns bins 2047-4t .. 2044-4t (highest first)
