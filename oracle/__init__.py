@@ -50,8 +50,8 @@ def load(path: Optional[str] = None):
 def _bind(lib):
     P = ctypes.c_void_p
     I = ctypes.c_int
-    lib.hisa_oracle_pool.argtypes = [P, P, I, I, I, I, I, P, P]
-    lib.hisa_oracle_select.argtypes = [P, P, I, I, I, I, I, P, P, P, P, P, I, I, I, I, I,
+    lib.hisa_oracle_pool.argtypes = [P, P, I, I, I, I, I, I, P, P]
+    lib.hisa_oracle_select.argtypes = [P, P, I, I, I, I, I, I, P, P, P, P, P, I, I, I, I, I,
                                        P, P, P, P, P, P]
     lib.hisa_oracle_refine.argtypes = [P, P, I, I, I, I, I, P, P, P, P, P, I, I, I, P, P, I, I,
                                        P, P, P]
@@ -97,12 +97,16 @@ class Cache:
         return (_p(self.keys), _p(self.scale), self.dtype, self.batch, self.cap, self.d)
 
 
-def pool(cache: Cache, B: int, lib=None) -> np.ndarray:
-    """Cache-level block means [batch, ceil(cap/B), d] (double; NaN where unpooled)."""
+POOL_MODES = {"mean": 0, "max": 1}
+
+
+def pool(cache: Cache, B: int, lib=None, mode: str = "mean") -> np.ndarray:
+    """Cache-level block representatives [batch, ceil(cap/B), d]: means, or
+    elementwise maxima with mode="max" (double; NaN where unpooled)."""
     lib = lib or load()
     nblk = -(-cache.cap // B)
     out = np.full((cache.batch, nblk, cache.d), np.nan)
-    rc = lib.hisa_oracle_pool(*cache.args(), B, _p(cache.lens), _p(out))
+    rc = lib.hisa_oracle_pool(*cache.args(), B, POOL_MODES[mode], _p(cache.lens), _p(out))
     if rc:
         raise ValueError(f"hisa_oracle_pool rc={rc}")
     return out
@@ -118,8 +122,9 @@ def _queries(Q, w, q_seq, q_pos):
 
 
 def hisa_select(cache: Cache, Q, w, q_seq, q_pos, B: int, m: int, k: int,
-                threads: Optional[int] = None, lib=None) -> dict:
-    """The two-stage HISA selection, step by step, for every query row."""
+                threads: Optional[int] = None, lib=None, pool: str = "mean") -> dict:
+    """The two-stage HISA selection, step by step, for every query row
+    (block representatives by mean or, with pool="max", elementwise max)."""
     lib = lib or load()
     Q, w, q_seq, q_pos, n_q, H = _queries(Q, w, q_seq, q_pos)
     nbmax = -(-cache.cap // B)
@@ -129,7 +134,8 @@ def hisa_select(cache: Cache, Q, w, q_seq, q_pos, B: int, m: int, k: int,
     nblocks = np.empty(n_q, np.int32)
     bscores = np.empty((n_q, nbmax))
     counts = np.empty((n_q, 2), np.int64)
-    rc = lib.hisa_oracle_select(*cache.args(), B, _p(cache.lens), _p(Q), _p(w), _p(q_seq),
+    rc = lib.hisa_oracle_select(*cache.args(), B, POOL_MODES[pool], _p(cache.lens), _p(Q), _p(w),
+                                _p(q_seq),
                                 _p(q_pos), n_q, H, m, k, threads or default_threads(),
                                 _p(idx), _p(score), _p(blocks), _p(nblocks), _p(bscores),
                                 _p(counts))

@@ -117,10 +117,22 @@ static double indexer_score(const double* q, const double* w, int H, int d, cons
     return acc;
 }
 
+enum { POOL_MEAN = 0, POOL_MAX = 1 };
+
 /* Step 1: block representative = mean of the block's visible keys
- * (tokens j*B .. min((j+1)*B, n) - 1). */
-static void pool_block(const cache_t* c, int b, int B, long j, long n, double* mu, double* tmp) {
+ * (tokens j*B .. min((j+1)*B, n) - 1), or, with POOL_MAX, their elementwise
+ * maximum (blog "Hierarchical Indexing Makes Sparse Attention Actually Fast",
+ * "HISA's Approach": summary nodes pool their token group by mean or by max). */
+static void pool_block(const cache_t* c, int b, int B, long j, long n, double* mu, double* tmp,
+                       int mode) {
     long s0 = j * (long)B, s1 = s0 + B < n ? s0 + B : n;
+    if (mode == POOL_MAX) {
+        for (long s = s0; s < s1; ++s) {
+            key_row(c, b, s, tmp);
+            for (int e = 0; e < c->d; ++e) mu[e] = (s == s0 || tmp[e] > mu[e]) ? tmp[e] : mu[e];
+        }
+        return;
+    }
     for (int e = 0; e < c->d; ++e) mu[e] = 0.0;
     for (long s = s0; s < s1; ++s) {
         key_row(c, b, s, tmp);
@@ -223,6 +235,7 @@ typedef struct {
     /* flat output */
     double* all_scores;
     int bad;
+    int pool_mode;
 } job_t;
 
 static long row_position(const job_t* J, int i, int* b_out) {
@@ -292,7 +305,7 @@ static void hisa_row(void* ctx, int i, void* scratch) {
     double* S = J->block_scores ? J->block_scores + (size_t)i * J->nbmax : NULL;
     if (S) for (int j = 0; j < J->nbmax; ++j) S[j] = NAN;
     for (long j = 0; j < nb; ++j) {
-        pool_block(&J->c, b, B, j, n_t, mu, x);
+        pool_block(&J->c, b, B, j, n_t, mu, x, J->pool_mode);
         double sj = indexer_score(q, w, H, d, mu);
         if (S) S[j] = sj;
         items[j].v = sj;
@@ -384,11 +397,13 @@ static int check_cache(const void* keys, const float* scale, int dtype, int batc
 
 /* ------------------------------------------------------------- exports */
 
-/* Cache-level pooling: pooled[b, j, :] = mean of keys j*B .. min((j+1)B, len[b]) - 1;
+/* Cache-level pooling: pooled[b, j, :] = mean (or max) of keys j*B .. min((j+1)B, len[b]) - 1;
  * blocks at or past len[b] are left untouched. */
 int hisa_oracle_pool(const void* keys, const float* scale, int dtype, int batch, int cap, int d,
-                     int B, const int32_t* lens, double* pooled) {
-    if (check_cache(keys, scale, dtype, batch, cap, d) || B < 1 || !lens || !pooled) return 1;
+                     int B, int pool_mode, const int32_t* lens, double* pooled) {
+    if (check_cache(keys, scale, dtype, batch, cap, d) || B < 1 || !lens || !pooled ||
+        (pool_mode != POOL_MEAN && pool_mode != POOL_MAX))
+        return 1;
     cache_t c = {keys, scale, dtype, batch, cap, d};
     long nblk = (cap + B - 1) / B;
     double* tmp = (double*)malloc(sizeof(double) * (size_t)d);
@@ -397,23 +412,25 @@ int hisa_oracle_pool(const void* keys, const float* scale, int dtype, int batch,
         long n = lens[b];
         if (n < 0 || n > cap) { free(tmp); return 1; }
         for (long j = 0; j * B < n; ++j)
-            pool_block(&c, b, B, j, n, pooled + ((size_t)b * nblk + (size_t)j) * d, tmp);
+            pool_block(&c, b, B, j, n, pooled + ((size_t)b * nblk + (size_t)j) * d, tmp, pool_mode);
     }
     free(tmp);
     return 0;
 }
 
 int hisa_oracle_select(const void* keys, const float* scale, int dtype, int batch, int cap, int d,
-                       int B, const int32_t* lens, const uint16_t* Q, const float* w,
+                       int B, int pool_mode, const int32_t* lens, const uint16_t* Q, const float* w,
                        const int32_t* q_seq, const int32_t* q_pos, int n_q, int H, int m, int k,
                        int n_threads, int32_t* idx, double* score, int32_t* blocks,
                        int32_t* nblocks, double* block_scores, int64_t* counts) {
     if (check_cache(keys, scale, dtype, batch, cap, d) || B < 1 || !lens || !Q || !w || !q_seq ||
-        n_q < 0 || H < 1 || m < 1 || m > 4096 || k < 1 || !idx)
+        n_q < 0 || H < 1 || m < 1 || m > 4096 || k < 1 || !idx ||
+        (pool_mode != POOL_MEAN && pool_mode != POOL_MAX))
         return 1;
     job_t J;
     memset(&J, 0, sizeof J);
     J.c = (cache_t){keys, scale, dtype, batch, cap, d};
+    J.pool_mode = pool_mode;
     J.B = B; J.lens = lens; J.Q = Q; J.w = w; J.q_seq = q_seq; J.q_pos = q_pos;
     J.n_q = n_q; J.H = H; J.m = m; J.k = k; J.nbmax = (cap + B - 1) / B;
     J.idx = idx; J.score = score; J.blocks = blocks; J.nblocks = nblocks;

@@ -7,7 +7,7 @@ items beat it) rather than by sorting.  Only for inputs of a few dozen
 tokens.
 
 Method: HISA (gptget.net summary, "Methodology"; Chinese summary, method
-details): mean-pool contiguous blocks of size B, score the representatives
+details): mean-pool (or max-pool) contiguous blocks of size B, score the representatives
 with the indexer, keep the top-m blocks (own block forced, counted in m),
 score the tokens of the kept blocks, keep the top-k tokens.
 """
@@ -66,11 +66,18 @@ def block_mean(keys, key_scale, dtype, b, B, j, n):
     return [sum(col, Fraction(0)) / (s1 - s0) for col in zip(*rows)]
 
 
-def hisa_row(keys, key_scale, dtype, Q, w, b, t, i, B, m, k):
+def block_max(keys, key_scale, dtype, b, B, j, n):
+    s0, s1 = j * B, min((j + 1) * B, n)
+    rows = [key_values(keys, key_scale, dtype, b, s) for s in range(s0, s1)]
+    return [max(col) for col in zip(*rows)]
+
+
+def hisa_row(keys, key_scale, dtype, Q, w, b, t, i, B, m, k, pool="mean"):
     q, ww = query_values(Q, w, i)
     n = t + 1
     nb = -(-n // B)
-    S = [score(q, ww, block_mean(keys, key_scale, dtype, b, B, j, n)) for j in range(nb)]
+    rep = block_max if pool == "max" else block_mean
+    S = [score(q, ww, rep(keys, key_scale, dtype, b, B, j, n)) for j in range(nb)]
     if nb <= m:
         chosen = list(range(nb))
     else:

@@ -29,6 +29,7 @@ MUTANTS = {
     "e4m3_bias_wrong": ("else v = ldexp(1.0 + m / 8.0, e - 7);",
                         "else v = ldexp(1.0 + m / 8.0, e - 8);"),
     "flat_misses_last_token": ("for (long s = 0; s <= t; ++s) {", "for (long s = 0; s < t; ++s) {"),
+    "max_pool_takes_min": ("(s == s0 || tmp[e] > mu[e])", "(s == s0 || tmp[e] < mu[e])"),
 }
 
 
@@ -83,6 +84,17 @@ def _detects(lib) -> bool:
             fref = brute.flat_row(c.keys, c.key_scale, c.dtype, c.Q, c.w, b, t, i, c.k)
             if [x for x in f["idx"][i] if x >= 0] != fref["idx"]:
                 return True
+    # max-pooled representatives against the exact brute force
+    c = make_case(batch=1, L=24, H=2, d=4, B=4, m=2, k=5, seed=311, positions=np.array([23, 13]))
+    cache = oracle.Cache.of(c)
+    r = oracle.hisa_select(cache, c.Q, c.w, c.q_seq, c.q_pos, c.B, c.m, c.k, threads=1, lib=lib,
+                           pool="max")
+    for i in range(c.n_q):
+        ref = brute.hisa_row(c.keys, c.key_scale, c.dtype, c.Q, c.w, int(c.q_seq[i]),
+                             int(c.q_pos[i]), i, c.B, c.m, c.k, pool="max")
+        if [float(x) for x in r["block_scores"][i][:len(ref["block_scores"])]] != \
+                [float(v) for v in ref["block_scores"]]:
+            return True
     return False
 
 

@@ -2,7 +2,7 @@
 
 * exact rational brute force on tiny inputs (tests/brute.py), with forced ties;
 * closed-form block means (constant blocks, arithmetic progressions, the
-  trailing partial block) and the B = 1 identity;
+  trailing partial block) and the B = 1 identity; the same for max pooling;
 * closed-form indexer scores (one-hot queries and keys, w = 0, all-negative
   dot products, scaling w);
 * structure: m >= #blocks makes HISA the flat scan; the tokens-scored count
@@ -27,9 +27,9 @@ def tiny(seed, dtype="bf16", L=40, B=4, m=3, k=7, H=3, d=8, batch=2, positions=N
                      positions=positions)
 
 
-def oracle_select(c, m=None, k=None):
+def oracle_select(c, m=None, k=None, pool="mean"):
     return oracle.hisa_select(oracle.Cache.of(c), c.Q, c.w, c.q_seq, c.q_pos, c.B,
-                              m or c.m, k or c.k, threads=2)
+                              m or c.m, k or c.k, threads=2, pool=pool)
 
 
 # ----------------------------------------------------------------- pooling
@@ -70,6 +70,41 @@ def test_pool_block_size_one_is_identity(dtype):
     else:   # fp32 product of the e4m3 value and the token's scale, computed by numpy
         expect = (e4m3_to_f32(c.keys) * c.key_scale[..., None]).astype(np.float32)
     assert np.array_equal(P[:, :33], expect[:, :33].astype(np.float64))
+
+
+@pytest.mark.parametrize("L,B", [(64, 16), (61, 16), (37, 8), (5, 8)])
+def test_pool_max_of_a_progression_is_its_last_valid_key(L, B):
+    # key[s, e] = (s + e) / 16 rises with s, except column 0 falls: its max is
+    # the block's first key.  The trailing block stops at its last valid key.
+    d = 4
+    s = np.arange(L)[:, None]
+    e = np.arange(d)[None, :]
+    keys = ((s + e) / 16.0).astype(np.float32)
+    keys[:, 0] = -keys[:, 0]
+    c = oracle.Cache(bf16_bits(keys[None]), None, [L], "bf16")
+    P = oracle.pool(c, B, mode="max")
+    for j in range(-(-L // B)):
+        s0, s1 = j * B, min((j + 1) * B, L)
+        expect = ((s1 - 1) + np.arange(d)) / 16.0
+        expect[0] = -s0 / 16.0
+        np.testing.assert_array_equal(P[0, j], expect)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+def test_pool_max_block_size_one_is_identity(dtype):
+    c = tiny(12, dtype=dtype, L=33, B=1)
+    P = oracle.pool(oracle.Cache.of(c), 1, mode="max")
+    assert np.array_equal(P[:, :33], oracle.pool(oracle.Cache.of(c), 1)[:, :33])
+
+
+def test_pool_max_constant_block_and_sign():
+    d, B = 8, 4
+    keys = np.full((1, 8, d), -0.75, np.float32)
+    keys[0, 5, 3] = 0.5
+    c = oracle.Cache(bf16_bits(keys), None, [8], "bf16")
+    P = oracle.pool(c, B, mode="max")
+    assert np.all(P[0, 0] == -0.75)
+    assert P[0, 1, 3] == 0.5 and np.all(np.delete(P[0, 1], 3) == -0.75)
 
 
 def test_pool_leaves_blocks_past_len_untouched():
@@ -140,12 +175,12 @@ def test_score_doubling_weights_doubles_scores():
 # --------------------------------------------------------- exact brute force
 
 
-def _check_against_brute(c, m, k):
-    r = oracle_select(c, m=m, k=k)
+def _check_against_brute(c, m, k, pool="mean"):
+    r = oracle_select(c, m=m, k=k, pool=pool)
     f = oracle.flat_select(oracle.Cache.of(c), c.Q, c.w, c.q_seq, c.q_pos, k=k)
     for i in range(c.n_q):
         b, t = int(c.q_seq[i]), int(c.q_pos[i])
-        ref = brute.hisa_row(c.keys, c.key_scale, c.dtype, c.Q, c.w, b, t, i, c.B, m, k)
+        ref = brute.hisa_row(c.keys, c.key_scale, c.dtype, c.Q, c.w, b, t, i, c.B, m, k, pool=pool)
         got = [x for x in r["idx"][i] if x >= 0]
         assert got == ref["idx"], (i, got, ref["idx"])
         assert list(r["idx"][i][len(got):]) == [-1] * (k - len(got))
@@ -173,6 +208,21 @@ def test_oracle_matches_exact_bruteforce(seed, dtype):
     c = make_case(batch=2, L=L, H=int(rng.integers(1, 4)), d=int(rng.choice([4, 8])), B=B, m=m,
                   k=k, dtype=dtype, seed=100 + seed, positions=pos)
     _check_against_brute(c, m, k)
+
+
+@pytest.mark.parametrize("seed", range(4))
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+def test_oracle_max_pooling_matches_exact_bruteforce(seed, dtype):
+    rng = np.random.default_rng(50 + seed)
+    B = int(rng.choice([2, 4, 16]))
+    L = int(rng.integers(9, 48))
+    nb = -(-L // B)
+    m = int(rng.integers(1, nb + 1))
+    k = int(rng.integers(1, L + 6))
+    pos = np.unique(rng.integers(0, L, size=3))
+    c = make_case(batch=2, L=L, H=int(rng.integers(1, 4)), d=int(rng.choice([4, 8])), B=B, m=m,
+                  k=k, dtype=dtype, seed=150 + seed, positions=pos)
+    _check_against_brute(c, m, k, pool="max")
 
 
 @pytest.mark.parametrize("seed", range(3))
