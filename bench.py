@@ -439,6 +439,35 @@ def run_workloads(args, dev, peaks):
     r["l2"] = "flushed between calls (cache 528 MiB)"
     out[case.name] = r
 
+    # block size / kept-block count / pooling sweep at a fixed candidate
+    # budget m * B = 8192 on the 32K decode workload: quality (IoU with the
+    # flat scan) against select time
+    case = make_config(1)
+    Q = torch.from_numpy(case.Q.view(np.int16)).view(torch.bfloat16).to(dev)
+    w = torch.from_numpy(case.w).to(dev)
+    qs = torch.from_numpy(case.q_seq).to(dev)
+    fidx = None
+    sweep = []
+    for pool in ("mean", "max"):
+        for B, m in ((64, 128), (128, 64), (256, 32)):
+            kv = hisa.KVCache.from_case(case, device=dev, pool=pool, B=B)
+            hisa.hisa_pool_blocks(kv)
+            if fidx is None:
+                fws = hisa.workspace(hisa.dsa_flat_workspace_bytes(kv, case.n_q, case.H, case.k), dev)
+                fidx = hisa.dsa_flat_select(kv, Q, w, qs, None, case.k, ws=fws).cpu().numpy()
+                del fws
+            ws = hisa.workspace(hisa.hisa_select_workspace_bytes(kv, case.n_q, case.H, m, case.k), dev)
+            hidx = torch.empty((case.n_q, case.k), dtype=torch.int32, device=dev)
+            ms = _median_ms(lambda: hisa.hisa_select(kv, Q, w, qs, None, m, case.k, ws=ws, idx=hidx),
+                            n, flush, stream)
+            mi = float(np.mean([iou(a, b) for a, b in zip(hidx.cpu().numpy(), fidx)]))
+            assert kv.status_bits() == 0, f"device status {kv.status_bits():#x}"
+            sweep.append({"pool": pool, "B": B, "m": m, "hisa_ms_per_select": ms,
+                          "selections_per_s": case.n_q / (ms / 1e3), "mean_iou_hisa_vs_flat": mi})
+            del kv, ws
+            torch.cuda.empty_cache()
+    out["pool_sweep_decode-32k-b64"] = sweep
+
     # streaming append + select for the new last position, one row per step
     case = make_config(4)
     kv = hisa.KVCache.from_case(case, device=dev)

@@ -30,6 +30,7 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 HISA_KEY_BF16, HISA_KEY_E4M3 = 0, 1
+HISA_POOL_MEAN, HISA_POOL_MAX = 0, 1
 HISA_OK, HISA_E_INVAL, HISA_E_UNSUPPORTED, HISA_E_WORKSPACE, HISA_E_CUDA = range(5)
 HISA_E_SCRATCH_LIMIT = 5
 HISA_STATIC_SCRATCH_BYTES = 8 << 20
@@ -47,7 +48,7 @@ class hisa_kv(ctypes.Structure):
                 ("pooled", ctypes.c_void_p), ("pooled_hl", ctypes.c_void_p),
                 ("len", ctypes.c_void_p), ("status", ctypes.c_void_p),
                 ("batch", ctypes.c_int32), ("cap", ctypes.c_int32), ("d", ctypes.c_int32),
-                ("B", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+                ("B", ctypes.c_int32), ("dtype", ctypes.c_int32), ("pool", ctypes.c_int32)]
 
 
 _P, _I, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
@@ -116,12 +117,16 @@ def _dev(x, dtype, device):
 
 
 class KVCache:
-    """Device storage of the indexer keys and the block index (hisa_kv)."""
+    """Device storage of the indexer keys and the block index (hisa_kv).
+    pool="mean" or "max": how block representatives pool their keys."""
 
     def __init__(self, batch: int, cap: int, d: int, B: int, dtype: str = "bf16",
-                 device="cuda"):
+                 device="cuda", pool: str = "mean"):
+        if pool not in ("mean", "max"):
+            raise ValueError("pool must be 'mean' or 'max'")
         self.batch, self.cap, self.d, self.B = batch, cap, d, B
         self.dtype = dtype
+        self.pool = pool
         self.device = torch.device(device)
         self.nblk = -(-cap // B)
         kdt = torch.bfloat16 if dtype == "bf16" else torch.uint8
@@ -138,7 +143,8 @@ class KVCache:
             key_scale=self.key_scale.data_ptr() if self.key_scale is not None else None,
             pooled=self.pooled.data_ptr(), pooled_hl=self.pooled_hl.data_ptr(),
             len=self.len.data_ptr(), status=self.status.data_ptr(), batch=batch, cap=cap, d=d,
-            B=B, dtype=HISA_KEY_BF16 if dtype == "bf16" else HISA_KEY_E4M3)
+            B=B, dtype=HISA_KEY_BF16 if dtype == "bf16" else HISA_KEY_E4M3,
+            pool=HISA_POOL_MAX if pool == "max" else HISA_POOL_MEAN)
 
     @property
     def struct(self):
@@ -156,8 +162,9 @@ class KVCache:
         return self
 
     @classmethod
-    def from_case(cls, case, device="cuda"):
-        kv = cls(case.batch, case.cap, case.d, case.B, case.dtype, device)
+    def from_case(cls, case, device="cuda", pool: str = "mean", B: Optional[int] = None):
+        """A cache holding a seeded case's keys (block size B overrides the case's)."""
+        kv = cls(case.batch, case.cap, case.d, B or case.B, case.dtype, device, pool)
         return kv.load(torch.from_numpy(case.keys), torch.from_numpy(case.lens),
                        None if case.key_scale is None else torch.from_numpy(case.key_scale))
 

@@ -120,6 +120,7 @@ int check_kv(const hisa_kv* kv, KvView* v) {
     if (kv->batch < 1 || kv->cap < 1 || kv->B < 1) return HISA_E_INVAL;
     if (kv->dtype != HISA_KEY_BF16 && kv->dtype != HISA_KEY_E4M3) return HISA_E_INVAL;
     if (kv->d != 64 && kv->d != 128) return HISA_E_UNSUPPORTED;
+    if (kv->pool != HISA_POOL_MEAN && kv->pool != HISA_POOL_MAX) return HISA_E_INVAL;
     const bool e4m3 = kv->dtype == HISA_KEY_E4M3;
     if (e4m3 && !kv->key_scale) return HISA_E_INVAL;
     if (!aligned(kv->keys, 16) || !aligned(kv->pooled, 16) || !aligned(kv->pooled_hl, 16) ||
@@ -139,6 +140,7 @@ int check_kv(const hisa_kv* kv, KvView* v) {
     v->B = kv->B;
     v->nblk = (kv->cap + kv->B - 1) / kv->B;
     v->e4m3 = e4m3;
+    v->pool_max = kv->pool == HISA_POOL_MAX;
     return HISA_OK;
 }
 

@@ -15,6 +15,7 @@ struct KvView {
     uint32_t* status;
     int batch, cap, d, B, nblk;
     bool e4m3;
+    bool pool_max;   // elementwise-max representatives (else means)
 };
 
 // What a scoring launch scores.

@@ -49,10 +49,11 @@ __device__ __forceinline__ void bf16x8(const uint4 raw, float (&v)[8]) {
     }
 }
 
-// Mean of keys [s0, s0 + cnt) of sequence b -> pooled row and its hi/lo split.
-// fp32 sums: each thread adds its rows in order, then the per-group partial
-// sums are added in group order.
-template <int D, bool E4M3>
+// Mean (or, MAX, elementwise maximum) of keys [s0, s0 + cnt) of sequence b ->
+// pooled row and its hi/lo split.  fp32 sums: each thread adds its rows in
+// order, then the per-group partial sums are added in group order.  The
+// maximum is exact whatever the order.
+template <int D, bool E4M3, bool MAX>
 __device__ void block_mean(const KvView& kv, int b, int j, int s0, int cnt, float* partial) {
     using S = PoolShape<D, E4M3>;
     constexpr int V = S::kVec;
@@ -61,7 +62,7 @@ __device__ void block_mean(const KvView& kv, int b, int j, int s0, int cnt, floa
     const int grp = tid / S::kLanes;
     float acc[V];
 #pragma unroll
-    for (int e = 0; e < V; ++e) acc[e] = 0.f;
+    for (int e = 0; e < V; ++e) acc[e] = MAX ? -INFINITY : 0.f;
 
     const size_t row0 = static_cast<size_t>(b) * kv.cap + s0;
     if constexpr (E4M3) {
@@ -72,7 +73,7 @@ __device__ void block_mean(const KvView& kv, int b, int j, int s0, int cnt, floa
             float v[16];
             dequant16(raw, sc, v);
 #pragma unroll
-            for (int e = 0; e < V; ++e) acc[e] += v[e];
+            for (int e = 0; e < V; ++e) acc[e] = MAX ? fmaxf(acc[e], v[e]) : acc[e] + v[e];
         }
     } else {
         const uint16_t* base = static_cast<const uint16_t*>(kv.keys);
@@ -81,16 +82,17 @@ __device__ void block_mean(const KvView& kv, int b, int j, int s0, int cnt, floa
             float v[8];
             bf16x8(raw, v);
 #pragma unroll
-            for (int e = 0; e < V; ++e) acc[e] += v[e];
+            for (int e = 0; e < V; ++e) acc[e] = MAX ? fmaxf(acc[e], v[e]) : acc[e] + v[e];
         }
     }
 #pragma unroll
     for (int e = 0; e < V; ++e) partial[grp * D + lane * V + e] = acc[e];
     __syncthreads();
     if (tid < D) {
-        float sum = 0.f;
-        for (int g = 0; g < S::kGroups; ++g) sum += partial[g * D + tid];
-        const float mean = sum / static_cast<float>(cnt);
+        float sum = MAX ? -INFINITY : 0.f;
+        for (int g = 0; g < S::kGroups; ++g)
+            sum = MAX ? fmaxf(sum, partial[g * D + tid]) : sum + partial[g * D + tid];
+        const float mean = MAX ? sum : sum / static_cast<float>(cnt);
         const size_t prow = static_cast<size_t>(b) * kv.nblk + j;
         kv.pooled[prow * D + tid] = mean;
         const __nv_bfloat16 hi = __float2bfloat16_rn(mean);
@@ -101,7 +103,7 @@ __device__ void block_mean(const KvView& kv, int b, int j, int s0, int cnt, floa
     }
 }
 
-template <int D, bool E4M3>
+template <int D, bool E4M3, bool MAX>
 __global__ void __launch_bounds__(kPoolThreads) pool_kernel(KvView kv) {
     __shared__ __align__(16) float partial[PoolShape<D, E4M3>::kGroups * D];
     const int j = blockIdx.x;
@@ -114,10 +116,10 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(KvView kv) {
     const int s0 = j * kv.B;
     if (s0 >= n) return;
     const int cnt = min(kv.B, n - s0);
-    block_mean<D, E4M3>(kv, b, j, s0, cnt, partial);
+    block_mean<D, E4M3, MAX>(kv, b, j, s0, cnt, partial);
 }
 
-template <int D, bool E4M3>
+template <int D, bool E4M3, bool MAX>
 __global__ void __launch_bounds__(kPoolThreads) append_kernel(KvView kv, const void* tok,
                                                               const float* tok_scale) {
     __shared__ __align__(16) float partial[PoolShape<D, E4M3>::kGroups * D];
@@ -142,7 +144,7 @@ __global__ void __launch_bounds__(kPoolThreads) append_kernel(KvView kv, const v
     // 2. recompute the trailing block over its valid keys
     const int j = pos / kv.B;
     const int s0 = j * kv.B;
-    block_mean<D, E4M3>(kv, b, j, s0, pos - s0 + 1, partial);
+    block_mean<D, E4M3, MAX>(kv, b, j, s0, pos - s0 + 1, partial);
     __syncthreads();
     // 3. publish the new length
     if (threadIdx.x == 0) kv.len[b] = pos + 1;
@@ -151,14 +153,16 @@ __global__ void __launch_bounds__(kPoolThreads) append_kernel(KvView kv, const v
 template <int D, bool E4M3>
 cudaError_t launch_pool_t(const KvView& kv, cudaStream_t s) {
     dim3 grid(kv.nblk, kv.batch);
-    pool_kernel<D, E4M3><<<grid, kPoolThreads, 0, s>>>(kv);
+    if (kv.pool_max) pool_kernel<D, E4M3, true><<<grid, kPoolThreads, 0, s>>>(kv);
+    else pool_kernel<D, E4M3, false><<<grid, kPoolThreads, 0, s>>>(kv);
     return cudaGetLastError();
 }
 
 template <int D, bool E4M3>
 cudaError_t launch_append_t(const KvView& kv, const void* tok, const float* tok_scale,
                             cudaStream_t s) {
-    append_kernel<D, E4M3><<<kv.batch, kPoolThreads, 0, s>>>(kv, tok, tok_scale);
+    if (kv.pool_max) append_kernel<D, E4M3, true><<<kv.batch, kPoolThreads, 0, s>>>(kv, tok, tok_scale);
+    else append_kernel<D, E4M3, false><<<kv.batch, kPoolThreads, 0, s>>>(kv, tok, tok_scale);
     return cudaGetLastError();
 }
 

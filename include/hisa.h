@@ -56,6 +56,15 @@ enum hisa_key_dtype {
                             the key value is fp32(e4m3 value * scale) */
 };
 
+/* Block representatives.  MEAN: the mean of the block's valid keys (HISA
+ * Methodology: mean pooling).  MAX: their elementwise maximum (blog
+ * "Hierarchical Indexing Makes Sparse Attention Actually Fast", "HISA's
+ * Approach": summary nodes pool a token group by mean or by max). */
+enum hisa_pool_mode {
+    HISA_POOL_MEAN = 0,
+    HISA_POOL_MAX = 1
+};
+
 /* Return codes. */
 enum hisa_status {
     HISA_OK = 0,
@@ -88,9 +97,10 @@ enum hisa_status {
  *   len        [batch]           int32 valid prefix length per sequence
  *   status     [1]               uint32 device status word (see HISA_DEV_*)
  *
- * Block representatives are the means of the visible keys of each block
- * (HISA Methodology: mean pooling generates the block representatives).  The
- * trailing partial block is the mean of its len - j*B valid keys.
+ * Block representatives are the means (or, with pool = HISA_POOL_MAX, the
+ * elementwise maxima) of the visible keys of each block (HISA Methodology:
+ * mean pooling generates the block representatives).  The trailing partial
+ * block is pooled over its len - j*B valid keys.
  *
  * Sizes: d in {64, 128}.  Pooling and append take any B >= 1; the select
  * calls need B in {8, 16, 32, 64} or a multiple of 128 up to 1024.
@@ -107,6 +117,7 @@ typedef struct hisa_kv {
     int32_t d;
     int32_t B;
     int32_t dtype;   /* enum hisa_key_dtype */
+    int32_t pool;    /* enum hisa_pool_mode */
 } hisa_kv;
 
 /*

@@ -13,9 +13,9 @@ def lib():
     return h
 
 
-def device_case(case):
+def device_case(case, pool="mean"):
     h = lib()
-    kv = h.KVCache.from_case(case)
+    kv = h.KVCache.from_case(case, pool=pool)
     h.hisa_pool_blocks(kv)
     return kv
 
@@ -48,7 +48,7 @@ def oracle_rows(case, rows):
     return (case.Q[rows], case.w[rows], case.q_seq[rows], case.q_pos[rows])
 
 
-def check_hisa(case, gpu, rows=None, threads=None, m=None, k=None):
+def check_hisa(case, gpu, rows=None, threads=None, m=None, k=None, pool="mean"):
     """Apply the two-level parity rule to the GPU result on the given rows."""
     from tests.parity import hisa_row_check
     m = m or case.m
@@ -56,7 +56,7 @@ def check_hisa(case, gpu, rows=None, threads=None, m=None, k=None):
     rows = np.arange(case.n_q) if rows is None else np.asarray(rows)
     cache = oracle.Cache.of(case)
     Q, w, qs, qp = oracle_rows(case, rows)
-    ora = oracle.hisa_select(cache, Q, w, qs, qp, case.B, m, k, threads=threads)
+    ora = oracle.hisa_select(cache, Q, w, qs, qp, case.B, m, k, threads=threads, pool=pool)
     mm = gpu["blocks"].shape[1]
     ref = oracle.hisa_refine(cache, Q, w, qs, qp, case.B, k, gpu["blocks"][rows],
                              gpu["nblocks"][rows], threads=threads)

@@ -140,3 +140,9 @@ def test_static_scratch_entry_checks_before_setup(hisa):
         hisa.HISA_STATIC_SCRATCH_BYTES
     assert sel(n_q=256) == hisa.HISA_E_SCRATCH_LIMIT
     assert lib.hisa_status_string(hisa.HISA_E_SCRATCH_LIMIT).startswith(b"call needs more")
+
+
+def test_pool_mode_is_checked(hisa):
+    lib = hisa.lib()
+    assert lib.hisa_pool_blocks(ctypes.byref(_kv(hisa, pool=2)), None) == hisa.HISA_E_INVAL
+    assert lib.hisa_pool_blocks(ctypes.byref(_kv(hisa, pool=-1)), None) == hisa.HISA_E_INVAL

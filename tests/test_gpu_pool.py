@@ -1,4 +1,4 @@
-"""GPU parity of the block index: mean-pooling and append (sm_100a kernels)."""
+"""GPU parity of the block index: mean- and max-pooling and append (sm_100a kernels)."""
 import numpy as np
 import pytest
 import torch
@@ -125,3 +125,53 @@ def test_append_past_capacity_sets_status():
     torch.cuda.synchronize()
     assert kv.len.item() == 64
     assert kv.status_bits() & h.HISA_DEV_CAPACITY
+
+
+# ------------------------------------------------------------- max pooling
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("B", [1, 16, 100, 128])
+def test_pool_max_matches_oracle_bit_exact(dtype, d, B):
+    """The elementwise max of fp32 key values is exact on both sides."""
+    h = lib()
+    case = make_case(batch=3, L=[1000, 777, 129], H=2, d=d, B=B, m=4, k=8, dtype=dtype,
+                     seed=60 + B + d)
+    kv = h.KVCache.from_case(case, pool="max")
+    h.hisa_pool_blocks(kv)
+    torch.cuda.synchronize()
+    got = kv.pooled.cpu().numpy().astype(np.float64)
+    ora = oracle.pool(oracle.Cache.of(case), B, mode="max")
+    for b in range(case.batch):
+        nbv = -(-int(case.lens[b]) // B)
+        assert np.array_equal(got[b, :nbv], ora[b, :nbv])
+    hl = kv.pooled_hl.view(torch.int16).cpu().numpy().view(np.uint16)
+    g32 = kv.pooled.cpu().numpy()
+    for b in range(case.batch):
+        nbv = -(-int(case.lens[b]) // B)
+        assert np.array_equal(bf16_bits(g32[b, :nbv]), hl[b, :nbv, :d])
+    assert kv.status_bits() == 0
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+def test_append_equals_repool_max_pooling(dtype):
+    h = lib()
+    steps, B = 200, 64
+    case = make_case(batch=2, L=[1000, 640], H=2, d=128, B=B, m=4, k=8, dtype=dtype, seed=17,
+                     append_steps=steps, cap=1300)
+    kv = h.KVCache.from_case(case, pool="max")
+    h.hisa_pool_blocks(kv)
+    for s in range(steps):
+        tok = torch.from_numpy(case.append_keys[s].view(np.int16 if dtype == "bf16" else np.uint8)).cuda()
+        sc = None if dtype == "bf16" else torch.from_numpy(case.append_scale[s]).cuda()
+        h.hisa_append(kv, tok, sc)
+    torch.cuda.synchronize()
+    inc = kv.pooled.clone()
+    inc_hl = kv.pooled_hl.clone()
+    h.hisa_pool_blocks(kv)
+    torch.cuda.synchronize()
+    for b, n in enumerate([1200, 840]):
+        nb = -(-n // B)
+        assert torch.equal(inc[b, :nb], kv.pooled[b, :nb])
+        assert torch.equal(inc_hl[b, :nb], kv.pooled_hl[b, :nb])

@@ -95,6 +95,18 @@ def test_e4m3_caches_whose_scale_rows_are_not_16_byte_aligned():
     assert kv.status_bits() == 0
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+@pytest.mark.parametrize("d,H,B,m,k", [(128, 64, 128, 8, 512), (64, 16, 16, 40, 200)])
+def test_hisa_max_pooling_matches_oracle(dtype, d, H, B, m, k):
+    case = make_case(batch=2, L=[4000, 1500], H=H, d=d, B=B, m=m, k=k, dtype=dtype, seed=21 + B,
+                     positions=[np.array([0, B, 3999, 2048]), np.array([1499, 700])])
+    kv = device_case(case, pool="max")
+    gpu = run_hisa(case, kv)
+    _, swaps = check_hisa(case, gpu, pool="max")
+    assert sum(s for s, _ in swaps) <= 2
+    assert kv.status_bits() == 0
+
+
 def test_hisa_with_every_block_is_the_flat_scan_bit_exact():
     """m >= #blocks: the same candidates in the same tile order through the
     same scoring kernel, so scores and indices agree exactly."""
