@@ -57,8 +57,10 @@ def _bind(lib):
                                        P, P, P]
     lib.hisa_oracle_flat.argtypes = [P, P, I, I, I, I, P, P, P, P, P, I, I, I, I, P, P, P]
     lib.hisa_oracle_topk_f32.argtypes = [P, I, I, I, P]
+    lib.hisa_oracle_tree_select.argtypes = [P, P, I, I, I, I, I, I, I, P, P, P, P, P, I, I, I, I,
+                                            I, I, P, P, P, P, P, P, P]
     for f in ("hisa_oracle_pool", "hisa_oracle_select", "hisa_oracle_refine",
-              "hisa_oracle_flat", "hisa_oracle_topk_f32"):
+              "hisa_oracle_flat", "hisa_oracle_topk_f32", "hisa_oracle_tree_select"):
         getattr(lib, f).restype = I
     return lib
 
@@ -143,6 +145,29 @@ def hisa_select(cache: Cache, Q, w, q_seq, q_pos, B: int, m: int, k: int,
         raise ValueError(f"hisa_oracle_select rc={rc}")
     return dict(idx=idx, score=score, blocks=blocks, nblocks=nblocks, block_scores=bscores,
                 counts=counts)
+
+
+def tree_select(cache: Cache, Q, w, q_seq, q_pos, B: int, bf: int, W: int, m: int, k: int,
+                threads: Optional[int] = None, lib=None, pool: str = "mean") -> dict:
+    """Three-level search: superblocks of bf blocks (own + best W - 1), then the
+    blocks under them (own + best m - 1), then their tokens (top k)."""
+    lib = lib or load()
+    Q, w, q_seq, q_pos, n_q, H = _queries(Q, w, q_seq, q_pos)
+    idx = np.empty((n_q, k), np.int32)
+    score = np.empty((n_q, k))
+    sblocks = np.empty((n_q, W), np.int32)
+    nsblocks = np.empty(n_q, np.int32)
+    blocks = np.empty((n_q, m), np.int32)
+    nblocks = np.empty(n_q, np.int32)
+    counts = np.empty((n_q, 3), np.int64)
+    rc = lib.hisa_oracle_tree_select(*cache.args(), B, bf, POOL_MODES[pool], _p(cache.lens), _p(Q),
+                                     _p(w), _p(q_seq), _p(q_pos), n_q, H, W, m, k,
+                                     threads or default_threads(), _p(idx), _p(score), _p(sblocks),
+                                     _p(nsblocks), _p(blocks), _p(nblocks), _p(counts))
+    if rc:
+        raise ValueError(f"hisa_oracle_tree_select rc={rc}")
+    return dict(idx=idx, score=score, sblocks=sblocks, nsblocks=nsblocks, blocks=blocks,
+                nblocks=nblocks, counts=counts)
 
 
 def hisa_refine(cache: Cache, Q, w, q_seq, q_pos, B: int, k: int, blocks, nblocks,

@@ -236,6 +236,9 @@ typedef struct {
     double* all_scores;
     int bad;
     int pool_mode;
+    /* tree: branching factor, superblocks kept, outputs */
+    int bf, W;
+    int32_t* sblocks; int32_t* nsblocks;
 } job_t;
 
 static long row_position(const job_t* J, int i, int* b_out) {
@@ -338,6 +341,95 @@ static void hisa_row(void* ctx, int i, void* scratch) {
     refine_blocks(J, i, b, t, q, w, chosen, n_chosen, items, x, idx, val, NULL);
 }
 
+/* Three-level search (blog "Hierarchical Indexing Makes Sparse Attention
+ * Actually Fast", "HISA's Approach": a multi-level summary searched top down,
+ * keeping the best branches at each level).  Superblocks of bf blocks
+ * (bf * B tokens) are pooled and scored; the own superblock plus the best
+ * W - 1 others are kept; the visible blocks under them are pooled and scored;
+ * the own block plus the best m - 1 of those are kept; their tokens are
+ * refined as in the two-stage search. */
+static void tree_row(void* ctx, int i, void* scratch) {
+    job_t* J = (job_t*)ctx;
+    int H = J->H, d = J->c.d, B = J->B, bf = J->bf, b;
+    long B2 = (long)B * bf;
+    long t = row_position(J, i, &b);
+    int32_t* idx = J->idx + (size_t)i * J->k;
+    double* val = J->score ? J->score + (size_t)i * J->k : NULL;
+    int32_t* sblocks = J->sblocks ? J->sblocks + (size_t)i * J->W : NULL;
+    int32_t* blocks = J->blocks ? J->blocks + (size_t)i * J->m : NULL;
+    if (t < 0) {
+        J->bad = 1;
+        for (int r = 0; r < J->k; ++r) { idx[r] = -1; if (val) val[r] = NAN; }
+        return;
+    }
+    double* q = (double*)scratch;
+    double* w = q + (size_t)H * d;
+    double* mu = w + H;
+    double* x = mu + d;
+    scored_t* items = (scored_t*)(x + d);
+    load_query(J, i, q, w);
+    long n_t = t + 1;
+    long nb = (n_t + B - 1) / B;
+    long ns = (n_t + B2 - 1) / B2;
+
+    /* level 2: superblocks */
+    for (long j = 0; j < ns; ++j) {
+        pool_block(&J->c, b, (int)B2, j, n_t, mu, x, J->pool_mode);
+        items[j].v = indexer_score(q, w, H, d, mu);
+        items[j].i = j;
+    }
+    int32_t skept[4096];
+    int n_s;
+    if (ns <= J->W) {
+        n_s = (int)ns;
+        for (int j = 0; j < n_s; ++j) skept[j] = j;
+    } else {
+        qsort(items, (size_t)(ns - 1), sizeof(scored_t), by_value_then_index);
+        n_s = J->W;
+        for (int r = 0; r < J->W - 1; ++r) skept[r] = (int32_t)items[r].i;
+        skept[J->W - 1] = (int32_t)(ns - 1);
+        for (int a = 1; a < n_s; ++a)
+            for (int c2 = a; c2 > 0 && skept[c2 - 1] > skept[c2]; --c2) {
+                int32_t tmp = skept[c2]; skept[c2] = skept[c2 - 1]; skept[c2 - 1] = tmp;
+            }
+    }
+    if (sblocks) for (int r = 0; r < J->W; ++r) sblocks[r] = r < n_s ? skept[r] : -1;
+    if (J->nsblocks) J->nsblocks[i] = n_s;
+
+    /* level 1: the visible blocks under the kept superblocks, own block apart */
+    long nc = 0;
+    for (int r = 0; r < n_s; ++r)
+        for (long j = (long)skept[r] * bf; j < (long)(skept[r] + 1) * bf && j < nb - 1; ++j) {
+            pool_block(&J->c, b, B, j, n_t, mu, x, J->pool_mode);
+            items[nc].v = indexer_score(q, w, H, d, mu);
+            items[nc].i = j;
+            ++nc;
+        }
+    int32_t chosen[4096];
+    int n_chosen;
+    if (nc + 1 <= J->m) {
+        n_chosen = (int)nc + 1;
+        for (long r = 0; r < nc; ++r) chosen[r] = (int32_t)items[r].i;
+    } else {
+        qsort(items, (size_t)nc, sizeof(scored_t), by_value_then_index);
+        n_chosen = J->m;
+        for (int r = 0; r < J->m - 1; ++r) chosen[r] = (int32_t)items[r].i;
+    }
+    chosen[n_chosen - 1] = (int32_t)(nb - 1);
+    for (int a = 1; a < n_chosen; ++a)
+        for (int c2 = a; c2 > 0 && chosen[c2 - 1] > chosen[c2]; --c2) {
+            int32_t tmp = chosen[c2]; chosen[c2] = chosen[c2 - 1]; chosen[c2 - 1] = tmp;
+        }
+    if (blocks) for (int r = 0; r < J->m; ++r) blocks[r] = r < n_chosen ? chosen[r] : -1;
+    if (J->nblocks) J->nblocks[i] = n_chosen;
+    if (J->counts) {
+        J->counts[3 * (size_t)i] = ns;                              /* superblock scores */
+        J->counts[3 * (size_t)i + 1] = nc + 1;                      /* block scores */
+        J->counts[3 * (size_t)i + 2] = (int64_t)n_chosen * B;       /* token slots */
+    }
+    refine_blocks(J, i, b, t, q, w, chosen, n_chosen, items, x, idx, val, NULL);
+}
+
 static void refine_row(void* ctx, int i, void* scratch) {
     job_t* J = (job_t*)ctx;
     int H = J->H, d = J->c.d, b;
@@ -437,6 +529,29 @@ int hisa_oracle_select(const void* keys, const float* scale, int dtype, int batc
     J.block_scores = block_scores; J.counts = counts;
     long items = J.nbmax > (long)m * B ? J.nbmax : (long)m * B;
     int rc = for_rows(hisa_row, &J, n_q, n_threads, row_scratch_bytes(H, d, items));
+    return rc ? rc : (J.bad ? 2 : 0);
+}
+
+int hisa_oracle_tree_select(const void* keys, const float* scale, int dtype, int batch, int cap,
+                            int d, int B, int bf, int pool_mode, const int32_t* lens,
+                            const uint16_t* Q, const float* w, const int32_t* q_seq,
+                            const int32_t* q_pos, int n_q, int H, int W, int m, int k,
+                            int n_threads, int32_t* idx, double* score, int32_t* sblocks,
+                            int32_t* nsblocks, int32_t* blocks, int32_t* nblocks, int64_t* counts) {
+    if (check_cache(keys, scale, dtype, batch, cap, d) || B < 1 || bf < 1 || !lens || !Q || !w ||
+        !q_seq || n_q < 0 || H < 1 || W < 1 || W > 4096 || m < 1 || m > 4096 || k < 1 || !idx ||
+        (pool_mode != POOL_MEAN && pool_mode != POOL_MAX))
+        return 1;
+    job_t J;
+    memset(&J, 0, sizeof J);
+    J.c = (cache_t){keys, scale, dtype, batch, cap, d};
+    J.pool_mode = pool_mode;
+    J.B = B; J.bf = bf; J.W = W; J.lens = lens; J.Q = Q; J.w = w; J.q_seq = q_seq; J.q_pos = q_pos;
+    J.n_q = n_q; J.H = H; J.m = m; J.k = k; J.nbmax = (cap + B - 1) / B;
+    J.idx = idx; J.score = score; J.sblocks = sblocks; J.nsblocks = nsblocks;
+    J.blocks = blocks; J.nblocks = nblocks; J.counts = counts;
+    long items = J.nbmax > (long)m * B ? J.nbmax : (long)m * B;
+    int rc = for_rows(tree_row, &J, n_q, n_threads, row_scratch_bytes(H, d, items));
     return rc ? rc : (J.bad ? 2 : 0);
 }
 

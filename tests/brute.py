@@ -98,3 +98,33 @@ def flat_row(keys, key_scale, dtype, Q, w, b, t, i, k):
     kept = keep_by_definition(cand, k)
     val = {s: v for v, s in cand}
     return dict(idx=kept, scores=[val[s] for s in kept])
+
+
+def tree_row(keys, key_scale, dtype, Q, w, b, t, i, B, bf, W, m, k, pool="mean"):
+    """Three-level search by definition: superblocks of bf blocks (own + best
+    W - 1), the visible blocks under them (own + best m - 1), their tokens."""
+    q, ww = query_values(Q, w, i)
+    n = t + 1
+    nb = -(-n // B)
+    B2 = B * bf
+    ns = -(-n // B2)
+    rep = block_max if pool == "max" else block_mean
+    S2 = [score(q, ww, rep(keys, key_scale, dtype, b, B2, j, n)) for j in range(ns)]
+    if ns <= W:
+        skept = list(range(ns))
+    else:
+        skept = keep_by_definition([(S2[j], j) for j in range(ns - 1)], W - 1) + [ns - 1]
+    cand = [j for s in skept for j in range(s * bf, min((s + 1) * bf, nb - 1))]
+    S1 = {j: score(q, ww, rep(keys, key_scale, dtype, b, B, j, n)) for j in cand}
+    if len(cand) + 1 <= m:
+        chosen = sorted(cand) + [nb - 1]
+    else:
+        chosen = keep_by_definition([(S1[j], j) for j in cand], m - 1) + [nb - 1]
+    toks = []
+    for j in chosen:
+        for s in range(j * B, min((j + 1) * B, n)):
+            toks.append((score(q, ww, key_values(keys, key_scale, dtype, b, s)), s))
+    kept = keep_by_definition(toks, k)
+    val = {s: v for v, s in toks}
+    return dict(idx=kept, scores=[val[s] for s in kept], sblocks=skept, blocks=sorted(chosen),
+                counts=(ns, len(cand) + 1, len(chosen) * B))

@@ -30,6 +30,10 @@ MUTANTS = {
                         "else v = ldexp(1.0 + m / 8.0, e - 8);"),
     "flat_misses_last_token": ("for (long s = 0; s <= t; ++s) {", "for (long s = 0; s < t; ++s) {"),
     "max_pool_takes_min": ("(s == s0 || tmp[e] > mu[e])", "(s == s0 || tmp[e] < mu[e])"),
+    "tree_own_superblock_not_forced": ("skept[J->W - 1] = (int32_t)(ns - 1);",
+                                       "skept[J->W - 1] = (int32_t)items[J->W - 1].i;"),
+    "tree_children_skip_last": ("j < (long)(skept[r] + 1) * bf && j < nb - 1; ++j",
+                                "j < (long)(skept[r] + 1) * bf - 1 && j < nb - 1; ++j"),
 }
 
 
@@ -94,6 +98,16 @@ def _detects(lib) -> bool:
                              int(c.q_pos[i]), i, c.B, c.m, c.k, pool="max")
         if [float(x) for x in r["block_scores"][i][:len(ref["block_scores"])]] != \
                 [float(v) for v in ref["block_scores"]]:
+            return True
+    # the three-level search against its brute force
+    c = make_case(batch=1, L=45, H=2, d=4, B=2, m=4, k=6, seed=312, positions=np.array([44, 30, 9]))
+    cache = oracle.Cache.of(c)
+    r = oracle.tree_select(cache, c.Q, c.w, c.q_seq, c.q_pos, 2, 3, 2, 4, 6, threads=1, lib=lib)
+    for i in range(c.n_q):
+        ref = brute.tree_row(c.keys, c.key_scale, c.dtype, c.Q, c.w, int(c.q_seq[i]),
+                             int(c.q_pos[i]), i, 2, 3, 2, 4, 6)
+        if list(r["blocks"][i][:r["nblocks"][i]]) != ref["blocks"] or \
+                [x for x in r["idx"][i] if x >= 0] != ref["idx"]:
             return True
     return False
 
