@@ -37,7 +37,8 @@ HISA_STATIC_SCRATCH_BYTES = 8 << 20
 HISA_DEV_BAD_QUERY, HISA_DEV_CAPACITY, HISA_DEV_BAD_LEN, HISA_DEV_TIMEOUT = 0x1, 0x2, 0x4, 0x8
 
 EXPORTS = ("hisa_pool_blocks", "hisa_append", "hisa_select_workspace_bytes", "hisa_select",
-           "hisa_select_inspect", "hisa_select_static", "dsa_flat_workspace_bytes", "dsa_flat_select", "hisa_topk_f32",
+           "hisa_select_inspect", "hisa_select_static", "hisa_tree_workspace_bytes",
+           "hisa_tree_select", "hisa_pool_tail", "dsa_flat_workspace_bytes", "dsa_flat_select", "hisa_topk_f32",
            "hisa_profile_enable", "hisa_profile_read", "hisa_status_string", "hisa_last_cuda_error")
 PHASES = ("block_score", "block_select", "token_score", "token_select", "flat_score",
           "flat_select", "pool", "append", "topk", "qsplit")
@@ -61,6 +62,11 @@ _lib.hisa_select.argtypes = [_KVP, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _
 _lib.hisa_select_inspect.argtypes = [_KVP, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P,
                                      _P, _Z, _P]
 _lib.hisa_select_static.argtypes = [_KVP, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P]
+_lib.hisa_tree_workspace_bytes.argtypes = [_KVP, _KVP, _I, _I, _I, _I, _I]
+_lib.hisa_tree_workspace_bytes.restype = _Z
+_lib.hisa_tree_select.argtypes = [_KVP, _KVP, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P,
+                                  _P, _P, _P, _Z, _P]
+_lib.hisa_pool_tail.argtypes = [_KVP, _P]
 _lib.dsa_flat_workspace_bytes.argtypes = [_KVP, _I, _I, _I]
 _lib.dsa_flat_workspace_bytes.restype = _Z
 _lib.dsa_flat_select.argtypes = [_KVP, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _Z, _P]
@@ -72,6 +78,7 @@ _lib.hisa_status_string.restype = ctypes.c_char_p
 _lib.hisa_last_cuda_error.argtypes = []
 _lib.hisa_last_cuda_error.restype = ctypes.c_char_p
 for _f in ("hisa_pool_blocks", "hisa_append", "hisa_select", "hisa_select_inspect", "hisa_select_static",
+           "hisa_tree_select", "hisa_pool_tail",
            "dsa_flat_select", "hisa_topk_f32", "hisa_profile_enable", "hisa_profile_read"):
     getattr(_lib, _f).restype = _I
 
@@ -260,6 +267,61 @@ def hisa_select_static(kv: KVCache, Q: torch.Tensor, w: torch.Tensor, q_seq: tor
     _check("hisa_select_static", _lib.hisa_select_static(
         kv.struct, _ptr(Q), _ptr(w), _ptr(q_seq), _ptr(q_pos), n_q, H, m, k, _ptr(idx),
         _ptr(scores), _stream(stream)))
+    return idx
+
+
+def superblock_index(kv: KVCache, bf: int) -> KVCache:
+    """A second index over kv's keys with superblocks of bf blocks (for
+    hisa_tree_select); shares kv's keys, scales and lengths."""
+    kv2 = KVCache.__new__(KVCache)
+    kv2.batch, kv2.cap, kv2.d, kv2.B = kv.batch, kv.cap, kv.d, kv.B * bf
+    kv2.dtype, kv2.device, kv2.pool = kv.dtype, kv.device, kv.pool
+    kv2.nblk = -(-kv.cap // kv2.B)
+    kv2.keys, kv2.key_scale, kv2.len, kv2.status = kv.keys, kv.key_scale, kv.len, kv.status
+    kv2.pooled = torch.zeros((kv.batch, kv2.nblk, kv.d), dtype=torch.float32, device=kv.device)
+    kv2.pooled_hl = torch.zeros((kv.batch, kv2.nblk, 2 * kv.d), dtype=torch.bfloat16, device=kv.device)
+    kv2._struct = hisa_kv(keys=kv._struct.keys, key_scale=kv._struct.key_scale,
+                          pooled=kv2.pooled.data_ptr(), pooled_hl=kv2.pooled_hl.data_ptr(),
+                          len=kv._struct.len, status=kv._struct.status, batch=kv.batch, cap=kv.cap,
+                          d=kv.d, B=kv2.B, dtype=kv._struct.dtype, pool=kv._struct.pool)
+    return kv2
+
+
+def hisa_pool_tail(kv: KVCache, stream=None):
+    _check("hisa_pool_tail", _lib.hisa_pool_tail(kv.struct, _stream(stream)))
+
+
+def hisa_tree_workspace_bytes(kv: KVCache, kv2: KVCache, n_q: int, H: int, W: int, m: int,
+                              k: int) -> int:
+    return int(_lib.hisa_tree_workspace_bytes(kv.struct, kv2.struct, n_q, H, W, m, k))
+
+
+def hisa_tree_select(kv: KVCache, kv2: KVCache, Q, w, q_seq, q_pos, W: int, m: int, k: int,
+                     inspect: bool = False, ws: Optional[torch.Tensor] = None, stream=None):
+    """Three-level search (superblocks of kv2, blocks of kv, tokens).  Returns
+    idx [n_q, k], or with inspect=True a dict with scores, kept superblocks and
+    blocks and the per-row work counters."""
+    Q, w, q_seq, q_pos = _queries(kv, Q, w, q_seq, q_pos)
+    n_q, H = Q.shape[0], Q.shape[1]
+    dev = kv.device
+    ws = workspace(hisa_tree_workspace_bytes(kv, kv2, n_q, H, W, m, k), dev) if ws is None else ws
+    idx = torch.empty((n_q, k), dtype=torch.int32, device=dev)
+    out = {}
+    if inspect:
+        out = dict(scores=torch.empty((n_q, k), dtype=torch.float32, device=dev),
+                   sblocks=torch.empty((n_q, min(W, kv2.nblk)), dtype=torch.int32, device=dev),
+                   nsblocks=torch.empty(n_q, dtype=torch.int32, device=dev),
+                   blocks=torch.empty((n_q, min(m, kv.nblk)), dtype=torch.int32, device=dev),
+                   nblocks=torch.empty(n_q, dtype=torch.int32, device=dev),
+                   counts=torch.empty((n_q, 3), dtype=torch.int64, device=dev))
+    g = lambda name: _ptr(out.get(name))
+    _check("hisa_tree_select", _lib.hisa_tree_select(
+        kv.struct, kv2.struct, _ptr(Q), _ptr(w), _ptr(q_seq), _ptr(q_pos), n_q, H, W, m, k,
+        _ptr(idx), g("scores"), g("sblocks"), g("nsblocks"), g("blocks"), g("nblocks"),
+        g("counts"), _ptr(ws), ws.numel(), _stream(stream)))
+    if inspect:
+        out["idx"] = idx
+        return out
     return idx
 
 

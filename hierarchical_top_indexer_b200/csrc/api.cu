@@ -249,6 +249,7 @@ ScoreParams score_params(const KvView& v, const float* w, const int32_t* q_seq, 
     p.n_q = n_q;
     p.H = H;
     p.npad = npad_of(H);
+    p.counts_ld = 2;
     // More rows than sequences: rows share keys (a prefill chunk), which then
     // stay in L2; otherwise every row streams its own keys from HBM.
     p.keep_keys = n_q > v.batch ? 1 : 0;
@@ -296,6 +297,134 @@ int prep_f8(const KvView& v, const uint16_t* Q, const float* w, int n_q, int H, 
     return HISA_OK;
 }
 
+// One block level: score the level's representatives (under the kept parent
+// superblocks, if any) and keep each row's own block plus the best m - 1
+// others into blocks [n_q, mm] / nblocks / plan.
+struct BlockLevel {
+    const KvView* v;
+    int m, mm, ldb;
+    uint32_t* bkeys;
+    int32_t* blocks;
+    int32_t* nblocks;
+    int4* plan;
+    int32_t* blocks_out;
+    int32_t* nblocks_out;
+    const int32_t* parent;   // kept superblocks [n_q, parent_ld] or null
+    int parent_ld, bf;
+    int counts_col;
+};
+
+int block_stage(const BlockLevel& lv, const uint16_t* Q, const float* w, const int32_t* q_seq,
+                const int32_t* q_pos, int n_q, int H, int k, uint64_t* counts, int counts_ld,
+                cudaStream_t s) {
+    const KvView& v = *lv.v;
+    CUtensorMap pmap, qmap;
+    if (!make_map(&pmap, v.pooled_hl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  static_cast<uint64_t>(v.batch) * v.nblk, 2 * v.d, 128, 64,
+                  CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !query_map(&qmap, Q, n_q, H, v.d))
+        return HISA_E_CUDA;
+    const int sms = sm_count();
+    ScoreParams p = score_params(v, w, q_seq, q_pos, n_q, H);
+    p.out = lv.bkeys;
+    p.ldo = lv.ldb;
+    p.tiles_per_row = lv.ldb / 128;
+    p.counts = reinterpret_cast<unsigned long long*>(counts);
+    p.counts_ld = counts_ld;
+    p.counts_col = lv.counts_col;
+    p.parent = lv.parent;
+    p.parent_ld = lv.parent_ld;
+    p.bf = lv.bf;
+    // Short rows (up to kFuseMaxBlocks = 4 tiles of blocks) and at most two rows per SM: the
+    // scoring kernel keeps the blocks itself, one CTA per row, which saves the
+    // selection launch.  Longer rows score faster spread over every SM, and
+    // many rows select faster in the selection kernel's one-CTA-per-row grid.
+    const bool fuse = lv.ldb <= kFuseMaxBlocks && n_q <= 2 * sms;
+    if (fuse) {
+        p.fuse = 1;
+        p.m = lv.m;
+        p.mm = lv.mm;
+        p.sel_blocks = lv.blocks;
+        p.sel_nblocks = lv.nblocks;
+        p.sel_plan = lv.plan;
+        p.sel_blocks_out = lv.blocks_out;
+        p.sel_nblocks_out = lv.nblocks_out;
+    }
+    int rc = run_score(kScoreBlocks, v, pmap, qmap, p, s);
+    if (rc || fuse) return rc;
+    SelectParams sp;
+    std::memset(&sp, 0, sizeof sp);
+    sp.mode = kSelBlocks;
+    sp.keys = lv.bkeys;
+    sp.ldk = lv.ldb;
+    sp.rows = n_q;
+    sp.k = k;
+    sp.len = v.len;
+    sp.q_seq = q_seq;
+    sp.q_pos = q_pos;
+    sp.status = v.status;
+    sp.batch = v.batch;
+    sp.cap = v.cap;
+    sp.B = v.B;
+    sp.m = lv.m;
+    sp.mm = lv.mm;
+    sp.blocks = lv.blocks;
+    sp.nblocks = lv.nblocks;
+    sp.plan = lv.plan;
+    sp.blocks_out = lv.blocks_out;
+    sp.nblocks_out = lv.nblocks_out;
+    sp.tree = lv.parent ? 1 : 0;
+    PhaseScope ps(HISA_PHASE_BLOCK_SELECT, s);
+    return cuda_status(launch_select(sp, v.nblk, sms, s));
+}
+
+// Token level: score the kept blocks' tokens, keep the top k.
+int token_stage(const KvView& v, const HisaWs& L, uint8_t* base, const uint16_t* Q, const float* w,
+                const int32_t* q_seq, const int32_t* q_pos, int n_q, int H, int k, int32_t* idx,
+                float* scores, uint64_t* counts, int counts_ld, int counts_col, cudaStream_t s) {
+    int32_t* blocks = reinterpret_cast<int32_t*>(base + L.blocks);
+    int4* plan = reinterpret_cast<int4*>(base + L.plan);
+    uint32_t* tkeys = reinterpret_cast<uint32_t*>(base + L.tkeys);
+    CUtensorMap kmap, qmap;
+    const int br = v.B < 128 ? v.B : 128;
+    if (!keys_map(&kmap, v, br) || !query_map(&qmap, Q, n_q, H, v.d)) return HISA_E_CUDA;
+    ScoreParams p = score_params(v, w, q_seq, q_pos, n_q, H);
+    p.counts = reinterpret_cast<unsigned long long*>(counts);
+    p.counts_ld = counts_ld;
+    p.counts_col = counts_col;
+    int rc = prep_f8(v, Q, w, n_q, H, base + L.q8, reinterpret_cast<float*>(base + L.w8), &qmap, p, s);
+    if (rc) return rc;
+    p.out = tkeys;
+    p.ldo = L.ldt;
+    p.tiles_per_row = L.ldt / 128;
+    p.blocks = blocks;
+    p.plan_in = plan;
+    p.mm = L.mm;
+    rc = run_score(kScoreHisa, v, kmap, qmap, p, s);
+    if (rc) return rc;
+    SelectParams sp;
+    std::memset(&sp, 0, sizeof sp);
+    sp.mode = kSelHisaTokens;
+    sp.keys = tkeys;
+    sp.ldk = L.ldt;
+    sp.rows = n_q;
+    sp.k = k;
+    sp.len = v.len;
+    sp.q_seq = q_seq;
+    sp.q_pos = q_pos;
+    sp.status = v.status;
+    sp.batch = v.batch;
+    sp.cap = v.cap;
+    sp.B = v.B;
+    sp.mm = L.mm;
+    sp.blocks = blocks;
+    sp.plan = plan;
+    sp.idx = idx;
+    sp.scores = scores;
+    PhaseScope ps(HISA_PHASE_TOKEN_SELECT, s);
+    return cuda_status(launch_select(sp, L.mm * v.B, sm_count(), s));
+}
+
 int hisa_select_impl(const hisa_kv* kv, const uint16_t* Q, const float* w, const int32_t* q_seq,
                      const int32_t* q_pos, int n_q, int H, int m, int k, int32_t* idx, float* scores,
                      int32_t* blocks_out, int32_t* nblocks_out, uint64_t* counts, void* ws,
@@ -311,97 +440,60 @@ int hisa_select_impl(const hisa_kv* kv, const uint16_t* Q, const float* w, const
     const HisaWs L = hisa_ws(v, n_q, H, m);
     if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return HISA_E_WORKSPACE;
     uint8_t* base = static_cast<uint8_t*>(ws);
-    uint32_t* bkeys = reinterpret_cast<uint32_t*>(base + L.bkeys);
-    int32_t* blocks = reinterpret_cast<int32_t*>(base + L.blocks);
-    int32_t* nblocks = reinterpret_cast<int32_t*>(base + L.nblocks);
-    int4* plan = reinterpret_cast<int4*>(base + L.plan);
-    uint32_t* tkeys = reinterpret_cast<uint32_t*>(base + L.tkeys);
-
-    CUtensorMap pmap, kmap, qmap;
-    const int br = v.B < 128 ? v.B : 128;
-    if (!make_map(&pmap, v.pooled_hl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-                  static_cast<uint64_t>(v.batch) * v.nblk, 2 * v.d, 128, 64,
-                  CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !keys_map(&kmap, v, br) || !query_map(&qmap, Q, n_q, H, v.d))
-        return HISA_E_CUDA;
-
     if (counts && cudaMemsetAsync(counts, 0, sizeof(uint64_t) * 2 * n_q, s) != cudaSuccess)
         return HISA_E_CUDA;
-    const int sms = sm_count();
-
-    // stage 1: score the block representatives, keep the own block + best m-1
-    ScoreParams p = score_params(v, w, q_seq, q_pos, n_q, H);
-    p.out = bkeys;
-    p.ldo = L.ldb;
-    p.tiles_per_row = L.ldb / 128;
-    p.counts = reinterpret_cast<unsigned long long*>(counts);
-    // Short rows (up to kFuseMaxBlocks = 4 tiles of blocks) and at most two rows per SM: the
-    // scoring kernel keeps the blocks itself, one CTA per row, which saves the
-    // selection launch.  Longer rows score faster spread over every SM, and
-    // many rows select faster in the selection kernel's one-CTA-per-row grid.
-    const bool fuse = L.ldb <= kFuseMaxBlocks && n_q <= 2 * sms;
-    if (fuse) {
-        p.fuse = 1;
-        p.m = m;
-        p.mm = L.mm;
-        p.sel_blocks = blocks;
-        p.sel_nblocks = nblocks;
-        p.sel_plan = plan;
-        p.sel_blocks_out = blocks_out;
-        p.sel_nblocks_out = nblocks_out;
-    }
-    rc = run_score(kScoreBlocks, v, pmap, qmap, p, s);
+    BlockLevel lv;
+    std::memset(&lv, 0, sizeof lv);
+    lv.v = &v;
+    lv.m = m;
+    lv.mm = L.mm;
+    lv.ldb = L.ldb;
+    lv.bkeys = reinterpret_cast<uint32_t*>(base + L.bkeys);
+    lv.blocks = reinterpret_cast<int32_t*>(base + L.blocks);
+    lv.nblocks = reinterpret_cast<int32_t*>(base + L.nblocks);
+    lv.plan = reinterpret_cast<int4*>(base + L.plan);
+    lv.blocks_out = blocks_out;
+    lv.nblocks_out = nblocks_out;
+    rc = block_stage(lv, Q, w, q_seq, q_pos, n_q, H, k, counts, 2, s);
     if (rc) return rc;
-    p.fuse = 0;
+    return token_stage(v, L, base, Q, w, q_seq, q_pos, n_q, H, k, idx, scores, counts, 2, 0, s);
+}
 
-    SelectParams sp;
-    std::memset(&sp, 0, sizeof sp);
-    sp.mode = kSelBlocks;
-    sp.keys = bkeys;
-    sp.ldk = L.ldb;
-    sp.rows = n_q;
-    sp.k = k;
-    sp.len = v.len;
-    sp.q_seq = q_seq;
-    sp.q_pos = q_pos;
-    sp.status = v.status;
-    sp.batch = v.batch;
-    sp.cap = v.cap;
-    sp.B = v.B;
-    sp.m = m;
-    sp.mm = L.mm;
-    sp.blocks = blocks;
-    sp.nblocks = nblocks;
-    sp.plan = plan;
-    sp.blocks_out = blocks_out;
-    sp.nblocks_out = nblocks_out;
-    if (!fuse) {
-        PhaseScope ps(HISA_PHASE_BLOCK_SELECT, s);
-        rc = cuda_status(launch_select(sp, v.nblk, sms, s));
-    }
-    if (rc) return rc;
+// Three-level search: a second index kv2 over the same keys with blocks of
+// bf = kv2->B / kv->B first-level blocks (superblocks).
+struct TreeWs {
+    HisaWs L;            // first level and tokens
+    size_t bkeys2, sblocks, nsblocks, plan2, total;
+    int ldb2, ws;        // superblock score-key row length, kept superblocks per row
+};
 
-    // stage 2: score the kept blocks' tokens, keep the top-k tokens
-    rc = prep_f8(v, Q, w, n_q, H, base + L.q8, reinterpret_cast<float*>(base + L.w8), &qmap, p, s);
-    if (rc) return rc;
-    p.out = tkeys;
-    p.ldo = L.ldt;
-    p.tiles_per_row = L.ldt / 128;
-    p.blocks = blocks;
-    p.plan_in = plan;
-    p.mm = L.mm;
-    rc = run_score(kScoreHisa, v, kmap, qmap, p, s);
-    if (rc) return rc;
+TreeWs tree_ws(const KvView& v, const KvView& v2, int n_q, int H, int W, int m) {
+    TreeWs T;
+    T.L = hisa_ws(v, n_q, H, m);
+    T.ws = W < v2.nblk ? W : v2.nblk;
+    T.ldb2 = static_cast<int>(round_up(v2.nblk, 128));
+    Carve c;
+    c.off = T.L.total;
+    T.bkeys2 = c.take(static_cast<size_t>(n_q) * T.ldb2 * 4);
+    T.sblocks = c.take(static_cast<size_t>(n_q) * T.ws * 4);
+    T.nsblocks = c.take(static_cast<size_t>(n_q) * 4);
+    T.plan2 = c.take(static_cast<size_t>(n_q) * 16);
+    T.total = c.off;
+    return T;
+}
 
-    sp.mode = kSelHisaTokens;
-    sp.keys = tkeys;
-    sp.ldk = L.ldt;
-    sp.idx = idx;
-    sp.scores = scores;
-    sp.blocks_out = nullptr;
-    sp.nblocks_out = nullptr;
-    PhaseScope ps(HISA_PHASE_TOKEN_SELECT, s);
-    return cuda_status(launch_select(sp, L.mm * v.B, sms, s));
+// kv2 must index the same keys as kv with a block size that is a multiple of kv's.
+int check_tree(const hisa_kv* kv, const hisa_kv* kv2, KvView* v, KvView* v2) {
+    int rc = check_kv(kv, v);
+    if (rc) return rc;
+    rc = check_kv(kv2, v2);
+    if (rc) return rc;
+    if (kv2->keys != kv->keys || kv2->key_scale != kv->key_scale || kv2->len != kv->len ||
+        kv2->batch != kv->batch || kv2->cap != kv->cap || kv2->d != kv->d || kv2->dtype != kv->dtype ||
+        kv2->pool != kv->pool || kv2->B % kv->B != 0)
+        return HISA_E_INVAL;
+    if (v2->nblk > kParentBits) return HISA_E_UNSUPPORTED;
+    return HISA_OK;
 }
 
 // Scratch of hisa_select_static: a file-scope device array, one per device
@@ -507,6 +599,78 @@ FlatWs flat_ws(const KvView& v, int n_q, int H) {
     take_q8(c, v, n_q, H, &f.q8, &f.w8);
     f.total = c.off;
     return f;
+}
+
+size_t hisa_tree_workspace_bytes(const hisa_kv* kv, const hisa_kv* kv2, int n_q, int H, int W, int m,
+                                 int k) {
+    (void)k;
+    KvView v, v2;
+    if (check_tree(kv, kv2, &v, &v2) || n_q < 0 || m < 1 || W < 1 || H < 1 || H > 128) return 0;
+    return tree_ws(v, v2, n_q, H, W, m).total;
+}
+
+int hisa_tree_select(const hisa_kv* kv, const hisa_kv* kv2, const uint16_t* Q, const float* w,
+                     const int32_t* q_seq, const int32_t* q_pos, int n_q, int H, int W, int m, int k,
+                     int32_t* idx, float* scores, int32_t* sblocks, int32_t* nsblocks, int32_t* blocks,
+                     int32_t* nblocks, uint64_t* counts, void* ws, size_t ws_bytes,
+                     hisa_stream_t stream) {
+    KvView v, v2;
+    int rc = check_tree(kv, kv2, &v, &v2);
+    if (rc) return rc;
+    if (!select_block_size_ok(v.B)) return HISA_E_UNSUPPORTED;
+    if (m < 1 || W < 1) return HISA_E_INVAL;
+    rc = check_queries(Q, w, q_seq, n_q, H, k, idx);
+    if (rc) return rc;
+    if (n_q == 0) return HISA_OK;
+    const TreeWs T = tree_ws(v, v2, n_q, H, W, m);
+    if (!ws || !aligned(ws, 256) || ws_bytes < T.total) return HISA_E_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    if (counts && cudaMemsetAsync(counts, 0, sizeof(uint64_t) * 3 * n_q, s) != cudaSuccess)
+        return HISA_E_CUDA;
+    // level 2: superblocks, the own one plus the best W - 1
+    BlockLevel l2;
+    std::memset(&l2, 0, sizeof l2);
+    l2.v = &v2;
+    l2.m = W;
+    l2.mm = T.ws;
+    l2.ldb = T.ldb2;
+    l2.bkeys = reinterpret_cast<uint32_t*>(base + T.bkeys2);
+    l2.blocks = reinterpret_cast<int32_t*>(base + T.sblocks);
+    l2.nblocks = reinterpret_cast<int32_t*>(base + T.nsblocks);
+    l2.plan = reinterpret_cast<int4*>(base + T.plan2);
+    l2.blocks_out = sblocks;
+    l2.nblocks_out = nsblocks;
+    rc = block_stage(l2, Q, w, q_seq, q_pos, n_q, H, k, counts, 3, s);
+    if (rc) return rc;
+    // level 1: the blocks under the kept superblocks, the own one plus the best m - 1
+    BlockLevel l1;
+    std::memset(&l1, 0, sizeof l1);
+    l1.v = &v;
+    l1.m = m;
+    l1.mm = T.L.mm;
+    l1.ldb = T.L.ldb;
+    l1.bkeys = reinterpret_cast<uint32_t*>(base + T.L.bkeys);
+    l1.blocks = reinterpret_cast<int32_t*>(base + T.L.blocks);
+    l1.nblocks = reinterpret_cast<int32_t*>(base + T.L.nblocks);
+    l1.plan = reinterpret_cast<int4*>(base + T.L.plan);
+    l1.blocks_out = blocks;
+    l1.nblocks_out = nblocks;
+    l1.parent = l2.blocks;
+    l1.parent_ld = T.ws;
+    l1.bf = v2.B / v.B;
+    l1.counts_col = 1;
+    rc = block_stage(l1, Q, w, q_seq, q_pos, n_q, H, k, counts, 3, s);
+    if (rc) return rc;
+    return token_stage(v, T.L, base, Q, w, q_seq, q_pos, n_q, H, k, idx, scores, counts, 3, 1, s);
+}
+
+int hisa_pool_tail(const hisa_kv* kv, hisa_stream_t stream) {
+    KvView v;
+    const int rc = check_kv(kv, &v);
+    if (rc) return rc;
+    PhaseScope ps(HISA_PHASE_APPEND, reinterpret_cast<cudaStream_t>(stream));
+    return cuda_status(launch_pool_tail(v, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 size_t dsa_flat_workspace_bytes(const hisa_kv* kv, int n_q, int H, int k) {

@@ -41,10 +41,18 @@ struct ScoreParams {
     const int32_t* blocks;
     const int4* plan_in;
     int mm;
+    // kScoreBlocks under a kept-superblock list (three-level search): block
+    // c of a row is a candidate only if superblock c / bf is in the row's
+    // parent[row, 0 .. parent_ld) (-1 padded); null: every block is
+    const int32_t* parent;
+    int parent_ld, bf;
     // score keys [n_q, ldo] (order-preserving; 0 = masked slot)
     uint32_t* out;
     int ldo;
-    unsigned long long* counts;   // [n_q, 2] or null: representatives / token slots scored
+    unsigned long long* counts;   // null, or per row: representatives scored at
+                                  // counts[row * counts_ld + counts_col] (blocks
+                                  // mode), token slots scored one column further
+    int counts_ld, counts_col;
     int tiles_per_row;            // tile slots per row (upper bound)
     long long total_tiles;        // n_q * tiles_per_row
     int stages;                   // bf16 operand stages
@@ -68,6 +76,7 @@ struct ScoreParams {
 };
 
 constexpr int kFuseMaxBlocks = 512;
+constexpr int kParentBits = 32768;    // superblocks a kept-superblock mask can cover
 
 enum SelectMode : int {
     kSelBlocks = 0,      // keep own block + best m-1 others -> blocks list
@@ -97,11 +106,14 @@ struct SelectParams {
     float* scores;      // [rows, k] or null
     int32_t* blocks_out;     // [rows, mm] or null (mode 0 copy for inspection)
     int32_t* nblocks_out;    // [rows] or null
+    int tree;                // mode 0 over masked candidates: no keep-everything shortcut
 };
 
 cudaError_t launch_pool(const KvView& kv, cudaStream_t s);
 cudaError_t launch_append(const KvView& kv, const void* tok, const float* tok_scale,
                           cudaStream_t s);
+// Re-pool each sequence's trailing block (the one holding key len - 1).
+cudaError_t launch_pool_tail(const KvView& kv, cudaStream_t s);
 
 // Scoring: tensor maps built by the caller.  `keys_map` covers keys
 // ([batch*cap, d], bf16 swizzled 128B boxes, or e4m3 plain boxes) or, for

@@ -150,6 +150,30 @@ __global__ void __launch_bounds__(kPoolThreads) append_kernel(KvView kv, const v
     if (threadIdx.x == 0) kv.len[b] = pos + 1;
 }
 
+// Re-pool the trailing block of each sequence (the block holding key
+// len - 1), e.g. a coarser index over keys another index's append just grew.
+template <int D, bool E4M3, bool MAX>
+__global__ void __launch_bounds__(kPoolThreads) tail_kernel(KvView kv) {
+    __shared__ __align__(16) float partial[PoolShape<D, E4M3>::kGroups * D];
+    const int b = blockIdx.x;
+    const int n = kv.len[b];
+    if (n < 0 || n > kv.cap) {
+        if (threadIdx.x == 0) set_status(kv.status, HISA_DEV_BAD_LEN);
+        return;
+    }
+    if (n == 0) return;
+    const int j = (n - 1) / kv.B;
+    const int s0 = j * kv.B;
+    block_mean<D, E4M3, MAX>(kv, b, j, s0, n - s0, partial);
+}
+
+template <int D, bool E4M3>
+cudaError_t launch_tail_t(const KvView& kv, cudaStream_t s) {
+    if (kv.pool_max) tail_kernel<D, E4M3, true><<<kv.batch, kPoolThreads, 0, s>>>(kv);
+    else tail_kernel<D, E4M3, false><<<kv.batch, kPoolThreads, 0, s>>>(kv);
+    return cudaGetLastError();
+}
+
 template <int D, bool E4M3>
 cudaError_t launch_pool_t(const KvView& kv, cudaStream_t s) {
     dim3 grid(kv.nblk, kv.batch);
@@ -167,6 +191,11 @@ cudaError_t launch_append_t(const KvView& kv, const void* tok, const float* tok_
 }
 
 }  // namespace
+
+cudaError_t launch_pool_tail(const KvView& kv, cudaStream_t s) {
+    if (kv.d == 128) return kv.e4m3 ? launch_tail_t<128, true>(kv, s) : launch_tail_t<128, false>(kv, s);
+    return kv.e4m3 ? launch_tail_t<64, true>(kv, s) : launch_tail_t<64, false>(kv, s);
+}
 
 cudaError_t launch_pool(const KvView& kv, cudaStream_t s) {
     if (kv.d == 128) return kv.e4m3 ? launch_pool_t<128, true>(kv, s) : launch_pool_t<128, false>(kv, s);

@@ -59,7 +59,8 @@ struct Layout {
 
 // Fused block selection scratch: the row's block score keys, a 256-bin
 // histogram, scan / result words.
-constexpr int kSelScratch = kFuseMaxBlocks * 4 + 256 * 4 + 16 * 4;
+constexpr int kParentWords = kParentBits / 32;   // kept-superblock bitmap
+constexpr int kSelScratch = kFuseMaxBlocks * 4 + 256 * 4 + 16 * 4 + kParentWords * 4;
 
 // Accumulators of n columns that fit a CTA's share of TMEM's 512 columns (up to four).
 __host__ __device__ inline int acc_count(int n, int per_sm) {
@@ -355,9 +356,9 @@ __device__ __forceinline__ uint32_t epi_scan(uint32_t v, int e, uint32_t* misc) 
     return before + incl - v;
 }
 
-// The kk-th largest of the keys s[0..n) (0 < kk < n, every key nonzero):
-// four 8-bit radix rounds from the top.  Returns T; *take_eq = how many keys
-// equal to T are among the top kk.
+// The kk-th largest of the nonzero keys s[0..n) (0 < kk < their count; key
+// 0 marks a masked slot): four 8-bit radix rounds from the top.  Returns T;
+// *take_eq = how many keys equal to T are among the top kk.
 __device__ uint32_t epi_threshold(const uint32_t* s, int n, int kk, uint32_t* hist, uint32_t* misc, int e,
                                   int* take_eq) {
     uint32_t prefix = 0, mask = 0;
@@ -368,7 +369,7 @@ __device__ uint32_t epi_threshold(const uint32_t* s, int n, int kk, uint32_t* hi
         epi_bar();
         for (int c = e; c < n; c += 128) {
             const uint32_t x = s[c];
-            if ((x & mask) == prefix) atomicAdd(&hist[(x >> shift) & 255u], 1u);
+            if (x != 0u && (x & mask) == prefix) atomicAdd(&hist[(x >> shift) & 255u], 1u);
         }
         epi_bar();
         // thread e owns bins 255 - 2e and 254 - 2e (highest first)
@@ -875,6 +876,7 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
         uint32_t* sKeys = reinterpret_cast<uint32_t*>(smem + L.sel);  // fused selection
         uint32_t* sHist = sKeys + kFuseMaxBlocks;
         uint32_t* sMisc = sHist + 256;
+        uint32_t* sPar = sMisc + 16;                                   // kept superblocks (bits)
         int it = 0, cur_row = -1;
         RowInfo R;
         R.nt = 0;
@@ -906,6 +908,18 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
                         set_status(p.status, HISA_DEV_BAD_QUERY);
                     }
                 }
+                if (MODE == kScoreBlocks && p.parent && ti < R.nt) {
+                    // the row's kept superblocks as a bitmap
+                    epi_bar();
+                    const int nwords = ((R.lim - 1) / p.bf) / 32 + 1;
+                    for (int i = e; i < nwords; i += 128) sPar[i] = 0u;
+                    epi_bar();
+                    for (int i = e; i < p.parent_ld; i += 128) {
+                        const int v = p.parent[static_cast<size_t>(row) * p.parent_ld + i];
+                        if (v >= 0 && v < nwords * 32) atomicOr(&sPar[v >> 5], 1u << (v & 31));
+                    }
+                    epi_bar();
+                }
                 if (ti < R.nt) {
                     __syncwarp();
                     for (int h = lane; h < 128; h += 32)
@@ -922,6 +936,10 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
             bool valid;
             if (MODE == kScoreBlocks) {
                 valid = c < R.lim;
+                if (p.parent && valid) {
+                    const int sb = c / p.bf;
+                    valid = (sPar[sb >> 5] >> (sb & 31)) & 1u;
+                }
             } else if (MODE == kScoreFlat) {
                 valid = c <= R.t;
             } else {
@@ -960,7 +978,8 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
                 const bool slot = MODE == kScoreBlocks ? valid : c < R.lim;
                 const int n = __popc(__ballot_sync(0xffffffffu, slot));
                 if (lane == 0 && n)
-                    atomicAdd(p.counts + 2 * row + (MODE == kScoreBlocks ? 0 : 1),
+                    atomicAdd(p.counts + static_cast<size_t>(row) * p.counts_ld + p.counts_col +
+                                  (MODE == kScoreBlocks ? 0 : 1),
                               static_cast<unsigned long long>(n));
             }
             if (fuse && ti == R.nt - 1) {
@@ -969,25 +988,34 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
                 const int nb = R.lim;                  // visible blocks; the own block is nb - 1
                 int32_t* bl = p.sel_blocks + static_cast<size_t>(row) * p.mm;
                 int32_t* bd = p.sel_blocks_out ? p.sel_blocks_out + static_cast<size_t>(row) * p.mm : nullptr;
-                const int keep = nb <= p.m ? nb : p.m;
-                if (nb <= p.m) {
-                    for (int i = e; i < p.mm; i += 128) {
-                        const int v = i < nb ? i : -1;
-                        bl[i] = v;
-                        if (bd) bd[i] = v;
-                    }
-                } else {
-                    if (p.m > 1) {
-                        int take_eq;
-                        const uint32_t T = epi_threshold(sKeys, nb - 1, p.m - 1, sHist, sMisc, e, &take_eq);
-                        epi_emit(sKeys, nb - 1, T, take_eq, bl, bd, sMisc, e);
-                    }
-                    for (int i = p.m - 1 + e; i < p.mm; i += 128) {
-                        const int v = i == p.m - 1 ? nb - 1 : -1;   // own block last
-                        bl[i] = v;
-                        if (bd) bd[i] = v;
-                    }
+                // candidates: the nonzero keys of blocks 0 .. nb - 2 (a kept-superblock
+                // list masks the others to 0)
+                uint32_t nv = static_cast<uint32_t>(nb - 1);
+                if (p.parent) {
+                    nv = 0;
+                    for (int c = e; c < nb - 1; c += 128) nv += sKeys[c] != 0u;
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) nv += __shfl_xor_sync(0xffffffffu, nv, o);
+                    if (lane == 0) sMisc[12 + (e >> 5)] = nv;
+                    epi_bar();
+                    nv = sMisc[12] + sMisc[13] + sMisc[14] + sMisc[15];
+                    epi_bar();
                 }
+                const int kk = p.m - 1;
+                const int kept = static_cast<int>(nv) <= kk ? static_cast<int>(nv) : kk;
+                if (static_cast<int>(nv) <= kk) {
+                    if (nv > 0) epi_emit(sKeys, nb - 1, 0u, 0, bl, bd, sMisc, e);   // every candidate
+                } else if (kk > 0) {
+                    int take_eq;
+                    const uint32_t T = epi_threshold(sKeys, nb - 1, kk, sHist, sMisc, e, &take_eq);
+                    epi_emit(sKeys, nb - 1, T, take_eq, bl, bd, sMisc, e);
+                }
+                for (int i = kept + e; i < p.mm; i += 128) {
+                    const int v = i == kept ? nb - 1 : -1;   // own block last
+                    bl[i] = v;
+                    if (bd) bd[i] = v;
+                }
+                const int keep = kept + 1;
                 if (e == 0) {
                     p.sel_nblocks[row] = keep;
                     if (p.sel_nblocks_out) p.sel_nblocks_out[row] = keep;

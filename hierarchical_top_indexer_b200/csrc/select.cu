@@ -299,7 +299,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectPara
         }
     }
 
-    if (bad || (p.mode == kSelBlocks && nb <= p.m)) {
+    if (bad || (p.mode == kSelBlocks && nb <= p.m && !p.tree)) {
         if (rank == 0) {
             if (p.mode == kSelBlocks) {
                 // bad row: nothing kept; short row: every visible block kept
@@ -558,7 +558,7 @@ __global__ void __launch_bounds__(kRowThreads) select_row_kernel(const SelectPar
             n = t + 1;
         }
     }
-    if (bad || (p.mode == kSelBlocks && nb <= p.m)) {
+    if (bad || (p.mode == kSelBlocks && nb <= p.m && !p.tree)) {
         if (p.mode == kSelBlocks) {
             const int keep = bad ? 0 : nb;
             for (int r = tid; r < p.mm; r += kRowThreads) {

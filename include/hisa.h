@@ -194,6 +194,44 @@ int hisa_select_inspect(const hisa_kv* kv, const uint16_t* Q, const float* w,
                         uint64_t* counts, void* ws, size_t ws_bytes, hisa_stream_t stream);
 
 /*
+ * hisa_tree_select — three-level search: superblocks, blocks, tokens.
+ * Blog "Hierarchical Indexing Makes Sparse Attention Actually Fast", "HISA's
+ * Approach": a multi-level summary of the cache searched top down, keeping
+ * the best branches at every level.
+ *   kv2    a second index over the same keys (keys, key_scale, len, batch,
+ *          cap, d, dtype and pool equal to kv's) whose block size is
+ *          bf = kv2->B / kv->B first-level blocks (a superblock); its own
+ *          pooled / pooled_hl, built by hisa_pool_blocks(kv2) and kept
+ *          current after each hisa_append(kv, ...) by hisa_pool_tail(kv2)
+ *   W      superblocks kept per row: the own superblock plus the best W - 1
+ *   m, k   blocks kept among the visible blocks under the kept superblocks
+ *          (the own block plus the best m - 1), then tokens, as hisa_select
+ *   sblocks [n_q, min(W, kv2 blocks)] out (or NULL): kept superblocks,
+ *          ascending, -1 padded; nsblocks [n_q] out (or NULL)
+ *   blocks [n_q, min(m, kv blocks)], nblocks [n_q]: out (or NULL), as
+ *          hisa_select_inspect
+ *   counts [n_q, 3] out (or NULL), zeroed by the call: superblocks scored,
+ *          blocks scored, token slots scored
+ * W covering every superblock gives hisa_select's result.  kv2 may hold up to
+ * 32768 superblocks per sequence (HISA_E_UNSUPPORTED beyond).
+ */
+size_t hisa_tree_workspace_bytes(const hisa_kv* kv, const hisa_kv* kv2, int n_q, int H, int W,
+                                 int m, int k);
+int hisa_tree_select(const hisa_kv* kv, const hisa_kv* kv2, const uint16_t* Q, const float* w,
+                     const int32_t* q_seq, const int32_t* q_pos, int n_q, int H, int W, int m,
+                     int k, int32_t* idx, float* scores, int32_t* sblocks, int32_t* nsblocks,
+                     int32_t* blocks, int32_t* nblocks, uint64_t* counts, void* ws,
+                     size_t ws_bytes, hisa_stream_t stream);
+
+/*
+ * hisa_pool_tail — re-pool each sequence's trailing block (the block that
+ * holds key len[b] - 1) from the keys.  For a coarser index over keys that
+ * hisa_append on a finer index sharing them has just grown; len is read,
+ * not changed.
+ */
+int hisa_pool_tail(const hisa_kv* kv, hisa_stream_t stream);
+
+/*
  * hisa_select_static — hisa_select without a caller workspace.  The pages
  * have no counterpart: this is a deployment convenience of this library.
  * The scratch hisa_select keeps in `ws` lives instead in one fixed device

@@ -146,3 +146,18 @@ def test_pool_mode_is_checked(hisa):
     lib = hisa.lib()
     assert lib.hisa_pool_blocks(ctypes.byref(_kv(hisa, pool=2)), None) == hisa.HISA_E_INVAL
     assert lib.hisa_pool_blocks(ctypes.byref(_kv(hisa, pool=-1)), None) == hisa.HISA_E_INVAL
+
+
+def test_tree_index_must_share_the_keys(hisa):
+    lib = hisa.lib()
+    P = ctypes.c_void_p
+    kv = _kv(hisa, cap=4096, B=128)
+    good2 = _kv(hisa, cap=4096, B=512, pooled=64, pooled_hl=80)
+    assert lib.hisa_tree_workspace_bytes(ctypes.byref(kv), ctypes.byref(good2), 4, 64, 2, 4, 64) > 0
+    bad_b = _kv(hisa, cap=4096, B=200, pooled=64, pooled_hl=80)          # not a multiple of 128
+    bad_keys = _kv(hisa, cap=4096, B=512, keys=32, pooled=64, pooled_hl=80)
+    for bad in (bad_b, bad_keys):
+        assert lib.hisa_tree_workspace_bytes(ctypes.byref(kv), ctypes.byref(bad), 4, 64, 2, 4, 64) == 0
+        assert lib.hisa_tree_select(ctypes.byref(kv), ctypes.byref(bad), P(16), P(16), P(16), None,
+                                    4, 64, 2, 4, 64, P(16), None, None, None, None, None, None,
+                                    P(256), 1 << 30, None) == hisa.HISA_E_INVAL
