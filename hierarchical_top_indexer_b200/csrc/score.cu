@@ -356,9 +356,10 @@ __device__ __forceinline__ uint32_t epi_scan(uint32_t v, int e, uint32_t* misc) 
     return before + incl - v;
 }
 
-// The kk-th largest of the nonzero keys s[0..n) (0 < kk < their count; key
-// 0 marks a masked slot): four 8-bit radix rounds from the top.  Returns T;
-// *take_eq = how many keys equal to T are among the top kk.
+// The kk-th largest of the keys s[0..n) (0 < kk < their count; with MASKED,
+// key 0 marks a masked slot and is not counted): four 8-bit radix rounds from
+// the top.  Returns T; *take_eq = how many keys equal to T are among the top kk.
+template <bool MASKED>
 __device__ uint32_t epi_threshold(const uint32_t* s, int n, int kk, uint32_t* hist, uint32_t* misc, int e,
                                   int* take_eq) {
     uint32_t prefix = 0, mask = 0;
@@ -369,7 +370,7 @@ __device__ uint32_t epi_threshold(const uint32_t* s, int n, int kk, uint32_t* hi
         epi_bar();
         for (int c = e; c < n; c += 128) {
             const uint32_t x = s[c];
-            if (x != 0u && (x & mask) == prefix) atomicAdd(&hist[(x >> shift) & 255u], 1u);
+            if ((!MASKED || x != 0u) && (x & mask) == prefix) atomicAdd(&hist[(x >> shift) & 255u], 1u);
         }
         epi_bar();
         // thread e owns bins 255 - 2e and 254 - 2e (highest first)
@@ -446,7 +447,8 @@ __device__ void epi_emit(const uint32_t* s, int n, uint32_t T, int take_eq, int3
     }
 }
 
-template <int MODE, bool E4M3, int D>
+// PAR (block scoring only): a kept-superblock list masks the blocks outside it.
+template <int MODE, bool E4M3, int D, bool PAR>
 __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(MODE, E4M3, D) ? 2 : 1)
     score_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap qmap,
                  const ScoreParams p) {
@@ -908,7 +910,7 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
                         set_status(p.status, HISA_DEV_BAD_QUERY);
                     }
                 }
-                if (MODE == kScoreBlocks && p.parent && ti < R.nt) {
+                if (MODE == kScoreBlocks && PAR && ti < R.nt) {
                     // the row's kept superblocks as a bitmap
                     epi_bar();
                     const int nwords = ((R.lim - 1) / p.bf) / 32 + 1;
@@ -936,7 +938,7 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
             bool valid;
             if (MODE == kScoreBlocks) {
                 valid = c < R.lim;
-                if (p.parent && valid) {
+                if (PAR && valid) {
                     const int sb = c / p.bf;
                     valid = (sPar[sb >> 5] >> (sb & 31)) & 1u;
                 }
@@ -991,7 +993,7 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
                 // candidates: the nonzero keys of blocks 0 .. nb - 2 (a kept-superblock
                 // list masks the others to 0)
                 uint32_t nv = static_cast<uint32_t>(nb - 1);
-                if (p.parent) {
+                if (PAR) {
                     nv = 0;
                     for (int c = e; c < nb - 1; c += 128) nv += sKeys[c] != 0u;
 #pragma unroll
@@ -1004,10 +1006,17 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
                 const int kk = p.m - 1;
                 const int kept = static_cast<int>(nv) <= kk ? static_cast<int>(nv) : kk;
                 if (static_cast<int>(nv) <= kk) {
-                    if (nv > 0) epi_emit(sKeys, nb - 1, 0u, 0, bl, bd, sMisc, e);   // every candidate
+                    if (PAR) {
+                        if (nv > 0) epi_emit(sKeys, nb - 1, 0u, 0, bl, bd, sMisc, e);   // every unmasked one
+                    } else {
+                        for (int i = e; i < kept; i += 128) {                         // every candidate
+                            bl[i] = i;
+                            if (bd) bd[i] = i;
+                        }
+                    }
                 } else if (kk > 0) {
                     int take_eq;
-                    const uint32_t T = epi_threshold(sKeys, nb - 1, kk, sHist, sMisc, e, &take_eq);
+                    const uint32_t T = epi_threshold<PAR>(sKeys, nb - 1, kk, sHist, sMisc, e, &take_eq);
                     epi_emit(sKeys, nb - 1, T, take_eq, bl, bd, sMisc, e);
                 }
                 for (int i = kept + e; i < p.mm; i += 128) {
@@ -1140,14 +1149,14 @@ __global__ void __launch_bounds__(128) qsplit_kernel(const uint16_t* __restrict_
     }
 }
 
-template <int MODE, bool E4M3, int D>
+template <int MODE, bool E4M3, int D, bool PAR = false>
 cudaError_t launch_t(const CUtensorMap& amap, const CUtensorMap& qmap, const ScoreParams& p, int grid,
                      cudaStream_t s) {
     const size_t smem = score_smem_bytes(MODE, E4M3, D, p.npad, p.stages, p.stages8);
     // the swizzled TMA destinations (operand stages, query heads) start on 1024-byte boundaries
     const Layout L = score_layout(MODE, E4M3, D, p.npad, p.stages, p.stages8);
     if ((L.a | L.q) & 1023u) return cudaErrorInvalidValue;
-    auto* fn = score_kernel<MODE, E4M3, D>;
+    auto* fn = score_kernel<MODE, E4M3, D, PAR>;
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
@@ -1213,9 +1222,13 @@ int score_config(int mode, bool e4m3, int d, int npad, int* stages, int* stages8
 
 cudaError_t launch_score(int mode, bool e4m3, int d, const CUtensorMap& amap, const CUtensorMap& qmap,
                          const ScoreParams& p, int grid, cudaStream_t s) {
-    if (mode == kScoreBlocks)
+    if (mode == kScoreBlocks) {
+        if (p.parent)
+            return d == 128 ? launch_t<kScoreBlocks, false, 128, true>(amap, qmap, p, grid, s)
+                            : launch_t<kScoreBlocks, false, 64, true>(amap, qmap, p, grid, s);
         return d == 128 ? launch_t<kScoreBlocks, false, 128>(amap, qmap, p, grid, s)
                         : launch_t<kScoreBlocks, false, 64>(amap, qmap, p, grid, s);
+    }
     if (mode == kScoreFlat) {
         if (e4m3)
             return d == 128 ? launch_t<kScoreFlat, true, 128>(amap, qmap, p, grid, s)
