@@ -380,7 +380,8 @@ def _phase_ms(hisa, fn, phase, n):
 
 def run_workloads(args, dev, peaks):
     """Select-only timings on the other workloads: HISA against the flat scan
-    (speedup, mean IoU) at 64K prefill and 128K e4m3 decode, and the streaming
+    (speedup, mean IoU) at 64K prefill and 128K e4m3 decode, the three-level
+    search at 128K, a block size / pooling sweep at 32K, and the streaming
     append + select step at 128K.  Parity on these sizes is in the GPU tests."""
     import torch
     import hierarchical_top_indexer_b200 as hisa
@@ -438,6 +439,7 @@ def run_workloads(args, dev, peaks):
     case, r = one(3)
     r["l2"] = "flushed between calls (cache 528 MiB)"
     out[case.name] = r
+    out["tree_" + case.name] = run_tree(case, dev, n, flush, stream, r["hisa_ms_per_select"])
 
     # block size / kept-block count / pooling sweep at a fixed candidate
     # budget m * B = 8192 on the 32K decode workload: quality (IoU with the
@@ -494,6 +496,48 @@ def run_workloads(args, dev, peaks):
                       "steps_per_s": steps / (sum(st) / 1e3),
                       "l2": "cache (32 MiB) L2-resident; no flush: each step follows the last"}
     return out
+
+
+def run_tree(case, dev, n, flush, stream, two_level_ms):
+    """Three-level search (superblocks of bf blocks, W kept superblocks, then
+    the top m blocks under them, then the top k tokens) against the flat scan
+    on one workload: select time, work per row and mean IoU."""
+    import torch
+    import hierarchical_top_indexer_b200 as hisa
+    from tests.parity import iou
+
+    kv = hisa.KVCache.from_case(case, device=dev)
+    hisa.hisa_pool_blocks(kv)
+    Q = torch.from_numpy(case.Q.view(np.int16)).view(torch.bfloat16).to(dev)
+    w = torch.from_numpy(case.w).to(dev)
+    qs = torch.from_numpy(case.q_seq).to(dev)
+    n_q, H, m, k = case.n_q, case.H, case.m, case.k
+    fws = hisa.workspace(hisa.dsa_flat_workspace_bytes(kv, n_q, H, k), dev)
+    fidx = hisa.dsa_flat_select(kv, Q, w, qs, None, k, ws=fws).cpu().numpy()
+    del fws
+    nb = -(-case.cap // case.B)
+    rows = []
+    for bf, W in ((8, 32), (8, 64), (16, 32)):
+        kv2 = hisa.superblock_index(kv, bf)
+        hisa.hisa_pool_blocks(kv2)
+        ws = hisa.workspace(hisa.hisa_tree_workspace_bytes(kv, kv2, n_q, H, W, m, k), dev)
+        idx = torch.empty((n_q, k), dtype=torch.int32, device=dev)
+        run = lambda: hisa.hisa_tree_select(kv, kv2, Q, w, qs, None, W, m, k, ws=ws, idx=idx)
+        ms = _median_ms(run, n, flush, stream)
+        mi = float(np.mean([iou(a, b) for a, b in zip(idx.cpu().numpy(), fidx)]))
+        assert kv.status_bits() == 0, f"device status {kv.status_bits():#x}"
+        nb2 = kv2.nblk
+        rows.append({"bf": bf, "W": W, "m": m, "ms_per_select": ms,
+                     "selections_per_s": n_q / (ms / 1e3), "mean_iou_tree_vs_flat": mi,
+                     "scores_per_row": {"superblocks": nb2, "blocks": min(W, nb2) * bf,
+                                        "tokens": min(m, nb) * case.B}})
+        del kv2, ws
+        torch.cuda.empty_cache()
+    del kv
+    torch.cuda.empty_cache()
+    return {"two_level_ms_per_select": two_level_ms,
+            "two_level_scores_per_row": {"blocks": nb, "tokens": min(m, nb) * case.B},
+            "levels": rows, "l2": "flushed between calls"}
 
 
 def run_select_only(args):

@@ -38,10 +38,11 @@ HISA_DEV_BAD_QUERY, HISA_DEV_CAPACITY, HISA_DEV_BAD_LEN, HISA_DEV_TIMEOUT = 0x1,
 
 EXPORTS = ("hisa_pool_blocks", "hisa_append", "hisa_select_workspace_bytes", "hisa_select",
            "hisa_select_inspect", "hisa_select_static", "hisa_tree_workspace_bytes",
-           "hisa_tree_select", "hisa_pool_tail", "dsa_flat_workspace_bytes", "dsa_flat_select", "hisa_topk_f32",
+           "hisa_tree_select", "hisa_pool_tail", "hisa_cp_workspace_bytes", "hisa_cp_blocks",
+           "hisa_cp_tokens", "hisa_merge_topk", "dsa_flat_workspace_bytes", "dsa_flat_select", "hisa_topk_f32",
            "hisa_profile_enable", "hisa_profile_read", "hisa_status_string", "hisa_last_cuda_error")
 PHASES = ("block_score", "block_select", "token_score", "token_select", "flat_score",
-          "flat_select", "pool", "append", "topk", "qsplit")
+          "flat_select", "pool", "append", "topk", "qsplit", "merge")
 
 
 class hisa_kv(ctypes.Structure):
@@ -67,6 +68,12 @@ _lib.hisa_tree_workspace_bytes.restype = _Z
 _lib.hisa_tree_select.argtypes = [_KVP, _KVP, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P,
                                   _P, _P, _P, _Z, _P]
 _lib.hisa_pool_tail.argtypes = [_KVP, _P]
+_lib.hisa_cp_workspace_bytes.argtypes = [_KVP, ctypes.c_int32, _I, _I, _I, _I]
+_lib.hisa_cp_workspace_bytes.restype = _Z
+_lib.hisa_cp_blocks.argtypes = [_KVP, ctypes.c_int32, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _Z, _P]
+_lib.hisa_cp_tokens.argtypes = [_KVP, ctypes.c_int32, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P,
+                                _Z, _P]
+_lib.hisa_merge_topk.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _P]
 _lib.dsa_flat_workspace_bytes.argtypes = [_KVP, _I, _I, _I]
 _lib.dsa_flat_workspace_bytes.restype = _Z
 _lib.dsa_flat_select.argtypes = [_KVP, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _Z, _P]
@@ -78,7 +85,7 @@ _lib.hisa_status_string.restype = ctypes.c_char_p
 _lib.hisa_last_cuda_error.argtypes = []
 _lib.hisa_last_cuda_error.restype = ctypes.c_char_p
 for _f in ("hisa_pool_blocks", "hisa_append", "hisa_select", "hisa_select_inspect", "hisa_select_static",
-           "hisa_tree_select", "hisa_pool_tail",
+           "hisa_tree_select", "hisa_pool_tail", "hisa_cp_blocks", "hisa_cp_tokens", "hisa_merge_topk",
            "dsa_flat_select", "hisa_topk_f32", "hisa_profile_enable", "hisa_profile_read"):
     getattr(_lib, _f).restype = _I
 
@@ -174,6 +181,17 @@ class KVCache:
         kv = cls(case.batch, case.cap, case.d, B or case.B, case.dtype, device, pool)
         return kv.load(torch.from_numpy(case.keys), torch.from_numpy(case.lens),
                        None if case.key_scale is None else torch.from_numpy(case.key_scale))
+
+    @classmethod
+    def shard_of_case(cls, case, tok_off: int, cap: int, device="cuda", pool: str = "mean",
+                      B: Optional[int] = None):
+        """The context-parallel shard of a seeded case that holds global
+        positions [tok_off, tok_off + cap) of every sequence."""
+        kv = cls(case.batch, cap, case.d, B or case.B, case.dtype, device, pool)
+        keys = torch.from_numpy(case.keys[:, tok_off:tok_off + cap])
+        lens = torch.from_numpy(case.lens.astype("int64").clip(tok_off, tok_off + cap) - tok_off)
+        sc = None if case.key_scale is None else torch.from_numpy(case.key_scale[:, tok_off:tok_off + cap])
+        return kv.load(keys, lens.to(torch.int32), sc)
 
     def status_bits(self) -> int:
         return int(self.status.item()) & 0xFFFFFFFF
@@ -297,7 +315,8 @@ def hisa_tree_workspace_bytes(kv: KVCache, kv2: KVCache, n_q: int, H: int, W: in
 
 
 def hisa_tree_select(kv: KVCache, kv2: KVCache, Q, w, q_seq, q_pos, W: int, m: int, k: int,
-                     inspect: bool = False, ws: Optional[torch.Tensor] = None, stream=None):
+                     inspect: bool = False, ws: Optional[torch.Tensor] = None,
+                     idx: Optional[torch.Tensor] = None, stream=None):
     """Three-level search (superblocks of kv2, blocks of kv, tokens).  Returns
     idx [n_q, k], or with inspect=True a dict with scores, kept superblocks and
     blocks and the per-row work counters."""
@@ -305,7 +324,7 @@ def hisa_tree_select(kv: KVCache, kv2: KVCache, Q, w, q_seq, q_pos, W: int, m: i
     n_q, H = Q.shape[0], Q.shape[1]
     dev = kv.device
     ws = workspace(hisa_tree_workspace_bytes(kv, kv2, n_q, H, W, m, k), dev) if ws is None else ws
-    idx = torch.empty((n_q, k), dtype=torch.int32, device=dev)
+    idx = torch.empty((n_q, k), dtype=torch.int32, device=dev) if idx is None else idx
     out = {}
     if inspect:
         out = dict(scores=torch.empty((n_q, k), dtype=torch.float32, device=dev),
@@ -349,6 +368,79 @@ def hisa_topk_f32(x: torch.Tensor, k: int, stream=None) -> torch.Tensor:
     idx = torch.empty((rows, k), dtype=torch.int32, device=x.device)
     _check("hisa_topk_f32", _lib.hisa_topk_f32(_ptr(x), rows, n, k, _ptr(idx), _stream(stream)))
     return idx
+
+
+def hisa_cp_workspace_bytes(kv: KVCache, tok_off: int, n_q: int, H: int, m: int, k: int) -> int:
+    return int(_lib.hisa_cp_workspace_bytes(kv.struct, tok_off, n_q, H, m, k))
+
+
+def hisa_cp_blocks(kv: KVCache, tok_off: int, Q, w, q_seq, q_pos, m: int,
+                   ws: Optional[torch.Tensor] = None, stream=None):
+    """One shard's block candidates: (ids [n_q, m] global block ids, scores
+    [n_q, m]); the own block, on the shard holding the query, scores +inf."""
+    Q, w, q_seq, q_pos = _queries(kv, Q, w, q_seq, q_pos)
+    n_q, H = Q.shape[0], Q.shape[1]
+    ws = workspace(hisa_cp_workspace_bytes(kv, tok_off, n_q, H, m, 1), kv.device) if ws is None else ws
+    ids = torch.empty((n_q, m), dtype=torch.int32, device=kv.device)
+    sc = torch.empty((n_q, m), dtype=torch.float32, device=kv.device)
+    _check("hisa_cp_blocks", _lib.hisa_cp_blocks(
+        kv.struct, tok_off, _ptr(Q), _ptr(w), _ptr(q_seq), _ptr(q_pos), n_q, H, m, _ptr(ids), _ptr(sc),
+        _ptr(ws), ws.numel(), _stream(stream)))
+    return ids, sc
+
+
+def hisa_cp_tokens(kv: KVCache, tok_off: int, Q, w, q_seq, q_pos, m: int, k: int, kept: torch.Tensor,
+                   ws: Optional[torch.Tensor] = None, stream=None):
+    """One shard's token candidates under the merged kept blocks kept [n_q, m]:
+    (idx [n_q, k] global token indices, scores [n_q, k])."""
+    Q, w, q_seq, q_pos = _queries(kv, Q, w, q_seq, q_pos)
+    n_q, H = Q.shape[0], Q.shape[1]
+    ws = workspace(hisa_cp_workspace_bytes(kv, tok_off, n_q, H, m, k), kv.device) if ws is None else ws
+    kept = _dev(kept, torch.int32, kv.device)
+    idx = torch.empty((n_q, k), dtype=torch.int32, device=kv.device)
+    sc = torch.empty((n_q, k), dtype=torch.float32, device=kv.device)
+    _check("hisa_cp_tokens", _lib.hisa_cp_tokens(
+        kv.struct, tok_off, _ptr(Q), _ptr(w), _ptr(q_seq), _ptr(q_pos), n_q, H, m, k, _ptr(kept),
+        _ptr(idx), _ptr(sc), _ptr(ws), ws.numel(), _stream(stream)))
+    return idx, sc
+
+
+def hisa_merge_topk(ids: torch.Tensor, scores: torch.Tensor, k: int, stream=None):
+    """Top-k of the (id, score) lists ids / scores [lists, rows, n] per row,
+    by (score desc, id asc): (idx [rows, k], scores [rows, k])."""
+    ids = ids.to(torch.int32).contiguous()
+    scores = scores.to(torch.float32).contiguous()
+    lists, rows, n = ids.shape
+    idx = torch.empty((rows, k), dtype=torch.int32, device=ids.device)
+    sc = torch.empty((rows, k), dtype=torch.float32, device=ids.device)
+    _check("hisa_merge_topk", _lib.hisa_merge_topk(_ptr(ids), _ptr(scores), lists, rows, n, k, _ptr(idx),
+                                                   _ptr(sc), _stream(stream)))
+    return idx, sc
+
+
+def _gather_ranks(t: torch.Tensor, group=None) -> torch.Tensor:
+    """[world, *t.shape]: every rank's t in rank order."""
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    if dist.get_backend(group) == "nccl":
+        out = torch.empty((world,) + tuple(t.shape), dtype=t.dtype, device=t.device)
+        dist.all_gather_into_tensor(out, t.contiguous(), group=group)
+        return out
+    parts = [torch.empty_like(t) for _ in range(world)]
+    dist.all_gather(parts, t.contiguous(), group=group)
+    return torch.stack(parts)
+
+
+def hisa_cp_select(kv: KVCache, tok_off: int, Q, w, q_seq, q_pos, m: int, k: int, group=None,
+                   ws: Optional[torch.Tensor] = None):
+    """Context-parallel hisa_select on the current stream: this rank holds the
+    shard at tok_off, the ranks of `group` hold ascending shards in rank
+    order.  Two all-gathers of (id, score) pairs; the result (idx, scores)
+    equals hisa_select's on the whole sequence, on every rank."""
+    ids, sc = hisa_cp_blocks(kv, tok_off, Q, w, q_seq, q_pos, m, ws=ws)
+    kept, _ = hisa_merge_topk(_gather_ranks(ids, group), _gather_ranks(sc, group), m)
+    tid, tsc = hisa_cp_tokens(kv, tok_off, Q, w, q_seq, q_pos, m, k, kept, ws=ws)
+    return hisa_merge_topk(_gather_ranks(tid, group), _gather_ranks(tsc, group), k)
 
 
 def hisa_profile_enable(on: bool = True):

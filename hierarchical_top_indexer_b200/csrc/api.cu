@@ -381,7 +381,8 @@ int block_stage(const BlockLevel& lv, const uint16_t* Q, const float* w, const i
 // Token level: score the kept blocks' tokens, keep the top k.
 int token_stage(const KvView& v, const HisaWs& L, uint8_t* base, const uint16_t* Q, const float* w,
                 const int32_t* q_seq, const int32_t* q_pos, int n_q, int H, int k, int32_t* idx,
-                float* scores, uint64_t* counts, int counts_ld, int counts_col, cudaStream_t s) {
+                float* scores, uint64_t* counts, int counts_ld, int counts_col, int id_off,
+                cudaStream_t s) {
     int32_t* blocks = reinterpret_cast<int32_t*>(base + L.blocks);
     int4* plan = reinterpret_cast<int4*>(base + L.plan);
     uint32_t* tkeys = reinterpret_cast<uint32_t*>(base + L.tkeys);
@@ -421,6 +422,7 @@ int token_stage(const KvView& v, const HisaWs& L, uint8_t* base, const uint16_t*
     sp.plan = plan;
     sp.idx = idx;
     sp.scores = scores;
+    sp.id_off = id_off;
     PhaseScope ps(HISA_PHASE_TOKEN_SELECT, s);
     return cuda_status(launch_select(sp, L.mm * v.B, sm_count(), s));
 }
@@ -456,7 +458,7 @@ int hisa_select_impl(const hisa_kv* kv, const uint16_t* Q, const float* w, const
     lv.nblocks_out = nblocks_out;
     rc = block_stage(lv, Q, w, q_seq, q_pos, n_q, H, k, counts, 2, s);
     if (rc) return rc;
-    return token_stage(v, L, base, Q, w, q_seq, q_pos, n_q, H, k, idx, scores, counts, 2, 0, s);
+    return token_stage(v, L, base, Q, w, q_seq, q_pos, n_q, H, k, idx, scores, counts, 2, 0, 0, s);
 }
 
 // Three-level search: a second index kv2 over the same keys with blocks of
@@ -519,6 +521,19 @@ int static_scratch(void** out) {
         }
     }
     *out = p;
+    return HISA_OK;
+}
+
+// A shard: global positions [tok_off, tok_off + cap) of every sequence, on
+// block boundaries, with at most kRowKeys blocks (one selection CTA per row).
+int check_cp(const hisa_kv* kv, int32_t tok_off, KvView* v) {
+    const int rc = check_kv(kv, v);
+    if (rc) return rc;
+    if (!select_block_size_ok(v->B)) return HISA_E_UNSUPPORTED;
+    if (tok_off < 0 || tok_off % v->B != 0 || v->cap % v->B != 0 ||
+        static_cast<long long>(tok_off) + v->cap > 0x7fffffffLL)
+        return HISA_E_INVAL;
+    if (v->nblk > kRowKeys) return HISA_E_UNSUPPORTED;
     return HISA_OK;
 }
 
@@ -662,7 +677,135 @@ int hisa_tree_select(const hisa_kv* kv, const hisa_kv* kv2, const uint16_t* Q, c
     l1.counts_col = 1;
     rc = block_stage(l1, Q, w, q_seq, q_pos, n_q, H, k, counts, 3, s);
     if (rc) return rc;
-    return token_stage(v, T.L, base, Q, w, q_seq, q_pos, n_q, H, k, idx, scores, counts, 3, 1, s);
+    return token_stage(v, T.L, base, Q, w, q_seq, q_pos, n_q, H, k, idx, scores, counts, 3, 1, 0, s);
+}
+
+// ---------------------------------------------------- context parallelism
+
+size_t hisa_cp_workspace_bytes(const hisa_kv* kv, int32_t tok_off, int n_q, int H, int m, int k) {
+    (void)k;
+    KvView v;
+    if (check_cp(kv, tok_off, &v) || n_q < 0 || m < 1 || H < 1 || H > 128) return 0;
+    return hisa_ws(v, n_q, H, m).total;
+}
+
+int hisa_cp_blocks(const hisa_kv* kv, int32_t tok_off, const uint16_t* Q, const float* w,
+                   const int32_t* q_seq, const int32_t* q_pos, int n_q, int H, int m, int32_t* cand_ids,
+                   float* cand_scores, void* ws, size_t ws_bytes, hisa_stream_t stream) {
+    KvView v;
+    int rc = check_cp(kv, tok_off, &v);
+    if (rc) return rc;
+    if (m < 1) return HISA_E_INVAL;
+    rc = check_queries(Q, w, q_seq, n_q, H, m, cand_ids);
+    if (rc) return rc;
+    if (n_q == 0) return HISA_OK;
+    if (!q_pos || !cand_scores || !aligned(q_pos, 4) || !aligned(cand_scores, 4)) return HISA_E_INVAL;
+    const HisaWs L = hisa_ws(v, n_q, H, m);
+    if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return HISA_E_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t* bkeys = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + L.bkeys);
+    CUtensorMap pmap, qmap;
+    if (!make_map(&pmap, v.pooled_hl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  static_cast<uint64_t>(v.batch) * v.nblk, 2 * v.d, 128, 64,
+                  CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !query_map(&qmap, Q, n_q, H, v.d))
+        return HISA_E_CUDA;
+    // the shard's visible blocks scored into the workspace ...
+    ScoreParams p = score_params(v, w, q_seq, q_pos, n_q, H);
+    p.out = bkeys;
+    p.ldo = L.ldb;
+    p.tiles_per_row = L.ldb / 128;
+    p.cp = 1;
+    p.tok_off = tok_off;
+    rc = run_score(kScoreBlocks, v, pmap, qmap, p, s);
+    if (rc) return rc;
+    // ... and the best m - 1 of them but the own block, then the own block
+    SelectParams sp;
+    std::memset(&sp, 0, sizeof sp);
+    sp.mode = kSelCpBlocks;
+    sp.keys = bkeys;
+    sp.ldk = L.ldb;
+    sp.rows = n_q;
+    sp.k = m;
+    sp.m = m;
+    sp.len = v.len;
+    sp.q_seq = q_seq;
+    sp.q_pos = q_pos;
+    sp.status = v.status;
+    sp.batch = v.batch;
+    sp.cap = v.cap;
+    sp.B = v.B;
+    sp.id_off = tok_off / v.B;
+    sp.idx = cand_ids;
+    sp.scores = cand_scores;
+    PhaseScope ps(HISA_PHASE_BLOCK_SELECT, s);
+    return cuda_status(launch_select(sp, v.nblk, sm_count(), s));
+}
+
+int hisa_cp_tokens(const hisa_kv* kv, int32_t tok_off, const uint16_t* Q, const float* w,
+                   const int32_t* q_seq, const int32_t* q_pos, int n_q, int H, int m, int k,
+                   const int32_t* kept, int32_t* idx, float* scores, void* ws, size_t ws_bytes,
+                   hisa_stream_t stream) {
+    KvView v;
+    int rc = check_cp(kv, tok_off, &v);
+    if (rc) return rc;
+    if (m < 1) return HISA_E_INVAL;
+    rc = check_queries(Q, w, q_seq, n_q, H, k, idx);
+    if (rc) return rc;
+    if (n_q == 0) return HISA_OK;
+    if (!q_pos || !kept || !aligned(q_pos, 4) || !aligned(kept, 4) || (scores && !aligned(scores, 4)))
+        return HISA_E_INVAL;
+    const HisaWs L = hisa_ws(v, n_q, H, m);
+    if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return HISA_E_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    CpLocalizeParams lp;
+    std::memset(&lp, 0, sizeof lp);
+    lp.kept = kept;
+    lp.m = m;
+    lp.q_seq = q_seq;
+    lp.q_pos = q_pos;
+    lp.len = v.len;
+    lp.status = v.status;
+    lp.batch = v.batch;
+    lp.cap = v.cap;
+    lp.B = v.B;
+    lp.tok_off = tok_off;
+    lp.rows = n_q;
+    lp.mm = L.mm;
+    lp.blocks = reinterpret_cast<int32_t*>(base + L.blocks);
+    lp.nblocks = reinterpret_cast<int32_t*>(base + L.nblocks);
+    lp.plan = reinterpret_cast<int4*>(base + L.plan);
+    {
+        PhaseScope ps(HISA_PHASE_BLOCK_SELECT, s);
+        rc = cuda_status(launch_cp_localize(lp, s));
+        if (rc) return rc;
+    }
+    return token_stage(v, L, base, Q, w, q_seq, q_pos, n_q, H, k, idx, scores, nullptr, 2, 0, tok_off, s);
+}
+
+int hisa_merge_topk(const int32_t* ids, const float* scores, int lists, int rows, int n, int k,
+                    int32_t* idx, float* out_scores, hisa_stream_t stream) {
+    if (lists < 1 || rows < 0 || n < 0 || k < 1) return HISA_E_INVAL;
+    if (static_cast<long long>(lists) * n > kRowKeys) return HISA_E_UNSUPPORTED;
+    if (rows == 0) return HISA_OK;
+    if (!ids || !scores || !idx || !aligned(ids, 4) || !aligned(scores, 4) || !aligned(idx, 4) ||
+        (out_scores && !aligned(out_scores, 4)))
+        return HISA_E_INVAL;
+    SelectParams sp;
+    std::memset(&sp, 0, sizeof sp);
+    sp.mode = kSelMerge;
+    sp.x = scores;
+    sp.ids = ids;
+    sp.lists = lists;
+    sp.n = n;
+    sp.rows = rows;
+    sp.k = k;
+    sp.idx = idx;
+    sp.scores = out_scores;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    PhaseScope ps(HISA_PHASE_MERGE, s);
+    return cuda_status(launch_select(sp, lists * n, sm_count(), s));
 }
 
 int hisa_pool_tail(const hisa_kv* kv, hisa_stream_t stream) {

@@ -73,6 +73,11 @@ struct ScoreParams {
     int4* sel_plan;               // [n_q]
     int32_t* sel_blocks_out;      // [n_q, mm] or null
     int32_t* sel_nblocks_out;     // [n_q] or null
+    // kScoreBlocks over one context-parallel shard (cp = 1): the cache holds
+    // the global positions [tok_off, tok_off + cap) of every sequence, q_pos
+    // are global positions, and a row's candidates are the shard's blocks
+    // that cp_visible_blocks admits
+    int cp, tok_off;
 };
 
 constexpr int kFuseMaxBlocks = 512;
@@ -82,8 +87,44 @@ enum SelectMode : int {
     kSelBlocks = 0,      // keep own block + best m-1 others -> blocks list
     kSelHisaTokens = 1,  // keep top-k of the kept blocks' token slots
     kSelFlatTokens = 2,  // keep top-k of keys 0..t
-    kSelF32Rows = 3      // keep top-k of n given fp32 values per row
+    kSelF32Rows = 3,     // keep top-k of n given fp32 values per row
+    kSelCpBlocks = 4,    // one shard's block candidates: best m-1 visible blocks
+                         // but the own one, then the own block (score +inf)
+    kSelMerge = 5        // top-k of `lists` (id, score) lists per row
 };
+
+// Rows of up to kRowKeys slots are selected by one CTA (the context-parallel
+// modes only ever take that path).
+constexpr int kRowKeys = 24576;
+
+// Context parallelism: a shard holds the global positions [tok_off, tok_off +
+// cap) of every sequence (tok_off and cap multiples of B).  For the query row
+// i at global position q_pos[i], returns how many of the shard's blocks it
+// sees (0: its prefix ends before the shard), with *own = 1 when the shard
+// holds the query position (the last visible block is then the row's own
+// block) and *tl = q_pos - tok_off; -1 for an invalid row (bad sequence, a
+// negative position, or a position past the sequence's end).
+__device__ __forceinline__ int cp_visible_blocks(const int32_t* q_seq, const int32_t* q_pos,
+                                                 const int32_t* len, int batch, int cap, int B,
+                                                 int tok_off, int i, int* seq_out, int* own, int* tl) {
+    const int b = q_seq[i];
+    *seq_out = b;
+    *own = 0;
+    *tl = -1;
+    if (b < 0 || b >= batch) return -1;
+    const int n = len[b];
+    const int t = q_pos[i];
+    if (n < 0 || n > cap || t < 0) return -1;
+    const long long l = static_cast<long long>(t) - tok_off;
+    if (l < 0) return 0;
+    *tl = static_cast<int>(l);
+    if (l < n) {
+        *own = 1;
+        return static_cast<int>(l) / B + 1;
+    }
+    return n == cap ? cap / B : -1;   // a full shard is wholly visible
+}
+
 
 struct SelectParams {
     int mode;
@@ -107,7 +148,33 @@ struct SelectParams {
     int32_t* blocks_out;     // [rows, mm] or null (mode 0 copy for inspection)
     int32_t* nblocks_out;    // [rows] or null
     int tree;                // mode 0 over masked candidates: no keep-everything shortcut
+    int id_off;              // added to every emitted id (modes 1, 4: a shard's first
+                             // token / block); mode 4 also reads tok_off = id_off * B
+    // mode 5: ids [lists, rows, n] (-1: empty) and their scores x [lists, rows, n];
+    // the concatenated lists of a row must ascend in id
+    const int32_t* ids;
+    int lists;
 };
+
+// Context-parallel token plan: from each row's merged global block list
+// kept [rows, m] (ascending, -1 padded), the visible blocks of the shard at
+// tok_off, as local ids into blocks [rows, mm] with counts nblocks and plans
+// {sequence, position for the token masks, count, 0}.  A valid row always
+// has its own block (global id q_pos / B) among the kept ones; a row without
+// it is invalid on every shard (plan position -1, HISA_DEV_BAD_QUERY).
+struct CpLocalizeParams {
+    const int32_t* kept;
+    int m;
+    const int32_t* q_seq;
+    const int32_t* q_pos;
+    const int32_t* len;
+    uint32_t* status;
+    int batch, cap, B, tok_off, rows, mm;
+    int32_t* blocks;
+    int32_t* nblocks;
+    int4* plan;
+};
+cudaError_t launch_cp_localize(const CpLocalizeParams& p, cudaStream_t s);
 
 cudaError_t launch_pool(const KvView& kv, cudaStream_t s);
 cudaError_t launch_append(const KvView& kv, const void* tok, const float* tok_scale,

@@ -130,13 +130,16 @@ __host__ __device__ inline uint32_t tmem_columns(int cols) {
     return c;
 }
 
+// Block scoring variants (a template parameter, so that each compiles alone).
+constexpr int kBlocksPlain = 0, kBlocksMasked = 1, kBlocksShard = 2;
+
 // A query row: sequence, position, candidate slots, candidate tiles (0 if
 // the row is invalid).
 struct RowInfo {
     int b, t, lim, nt;
 };
 
-template <int MODE>
+template <int MODE, int BV>
 __device__ __forceinline__ RowInfo load_row(const ScoreParams& p, int row) {
     RowInfo R;
     R.lim = 0;
@@ -147,6 +150,15 @@ __device__ __forceinline__ RowInfo load_row(const ScoreParams& p, int row) {
         R.t = pl.y;
         if (R.t < 0) return R;
         R.lim = pl.z * p.B;                 // kept token slots
+    } else if (MODE == kScoreBlocks && BV == kBlocksShard) {
+        int own;
+        const int vis = cp_visible_blocks(p.q_seq, p.q_pos, p.len, p.batch, p.cap, p.B, p.tok_off, row,
+                                          &R.b, &own, &R.t);
+        if (vis <= 0) {
+            R.t = -1;
+            return R;
+        }
+        R.lim = vis;                        // the shard's visible blocks
     } else {
         R.t = query_position(p.q_seq, p.q_pos, p.len, p.batch, p.cap, row, &R.b);
         if (R.t < 0) return R;
@@ -447,8 +459,10 @@ __device__ void epi_emit(const uint32_t* s, int n, uint32_t T, int take_eq, int3
     }
 }
 
-// PAR (block scoring only): a kept-superblock list masks the blocks outside it.
-template <int MODE, bool E4M3, int D, bool PAR>
+// BV (block scoring only): every visible block is a candidate (kBlocksPlain),
+// a kept-superblock list masks the blocks outside it (kBlocksMasked), or the
+// cache is a context-parallel shard (kBlocksShard).
+template <int MODE, bool E4M3, int D, int BV>
 __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(MODE, E4M3, D) ? 2 : 1)
     score_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap qmap,
                  const ScoreParams p) {
@@ -456,6 +470,7 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
     constexpr int kOps = (MODE == kScoreBlocks) ? 2 : 1;
     constexpr bool kF8 = uses_f8(MODE, E4M3, D);          // fp8 operands straight from TMA
     constexpr bool kConv = E4M3 && !kF8;                  // e4m3 widened to bf16 by converter warps
+    constexpr bool PAR = MODE == kScoreBlocks && BV == kBlocksMasked;
     constexpr int kStageBytes = kF8 ? kTileRows * D : kOps * kHalves * kHalfBytes;
     constexpr int kStage8Bytes = kTileRows * D;
 
@@ -561,7 +576,7 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
             TileCursor cur(g0, tpr);
             while (cur.g < g1 && ok) {
                 const int row = cur.row;
-                R = load_row<MODE>(p, row);
+                R = load_row<MODE, BV>(p, row);
                 const long long left = g1 - cur.g;
                 const int t_end = static_cast<int>(R.nt < cur.ti + left ? R.nt : cur.ti + left);
                 if (cur.ti >= t_end) {
@@ -681,7 +696,7 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
             const int ti = cur.ti;
             if (row != cur_row) {
                 cur_row = row;
-                R = load_row<MODE>(p, row);
+                R = load_row<MODE, BV>(p, row);
                 if (ti < R.nt) {
                     // new row with work here: its query heads and block-id windows
                     const int qs = qloads & 1;
@@ -812,7 +827,7 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
                 const int ti = cur.ti;
                 if (row != cur_row) {
                     cur_row = row;
-                    R = load_row<MODE>(p, row);
+                    R = load_row<MODE, BV>(p, row);
                     if (ti < R.nt) {
                         if (qloads > 0) umma_commit(qempty + ((qloads - 1) & 1));
                         if (!mbar_wait(qfull + (qloads & 1), (qloads >> 1) & 1, abort_flag)) {
@@ -890,7 +905,7 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
             const int ti = cur.ti;
             if (row != cur_row) {
                 cur_row = row;
-                R = load_row<MODE>(p, row);
+                R = load_row<MODE, BV>(p, row);
                 if (MODE == kScoreHisa && R.nt > 0) {
                     own0 = R.lim - p.B;
                     own_t = R.t % p.B;
@@ -1048,7 +1063,7 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
             const int ti = cur.ti;
             if (row != cur_row) {
                 cur_row = row;
-                R = load_row<MODE>(p, row);
+                R = load_row<MODE, BV>(p, row);
             }
             if (ti >= R.nt) {
                 cur.next_row();
@@ -1149,14 +1164,14 @@ __global__ void __launch_bounds__(128) qsplit_kernel(const uint16_t* __restrict_
     }
 }
 
-template <int MODE, bool E4M3, int D, bool PAR = false>
+template <int MODE, bool E4M3, int D, int BV = kBlocksPlain>
 cudaError_t launch_t(const CUtensorMap& amap, const CUtensorMap& qmap, const ScoreParams& p, int grid,
                      cudaStream_t s) {
     const size_t smem = score_smem_bytes(MODE, E4M3, D, p.npad, p.stages, p.stages8);
     // the swizzled TMA destinations (operand stages, query heads) start on 1024-byte boundaries
     const Layout L = score_layout(MODE, E4M3, D, p.npad, p.stages, p.stages8);
     if ((L.a | L.q) & 1023u) return cudaErrorInvalidValue;
-    auto* fn = score_kernel<MODE, E4M3, D, PAR>;
+    auto* fn = score_kernel<MODE, E4M3, D, BV>;
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
@@ -1223,9 +1238,12 @@ int score_config(int mode, bool e4m3, int d, int npad, int* stages, int* stages8
 cudaError_t launch_score(int mode, bool e4m3, int d, const CUtensorMap& amap, const CUtensorMap& qmap,
                          const ScoreParams& p, int grid, cudaStream_t s) {
     if (mode == kScoreBlocks) {
+        if (p.cp)
+            return d == 128 ? launch_t<kScoreBlocks, false, 128, kBlocksShard>(amap, qmap, p, grid, s)
+                            : launch_t<kScoreBlocks, false, 64, kBlocksShard>(amap, qmap, p, grid, s);
         if (p.parent)
-            return d == 128 ? launch_t<kScoreBlocks, false, 128, true>(amap, qmap, p, grid, s)
-                            : launch_t<kScoreBlocks, false, 64, true>(amap, qmap, p, grid, s);
+            return d == 128 ? launch_t<kScoreBlocks, false, 128, kBlocksMasked>(amap, qmap, p, grid, s)
+                            : launch_t<kScoreBlocks, false, 64, kBlocksMasked>(amap, qmap, p, grid, s);
         return d == 128 ? launch_t<kScoreBlocks, false, 128>(amap, qmap, p, grid, s)
                         : launch_t<kScoreBlocks, false, 64>(amap, qmap, p, grid, s);
     }

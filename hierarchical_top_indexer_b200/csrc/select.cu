@@ -473,7 +473,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectPara
         const int Bsz = p.B;
         compact(keys, nl, T, take_eq, eq_base, out_base, sh, [&](int pos, int c, uint32_t x) {
             const int slot = s0 + c;
-            idx[pos] = blk ? blk[slot / Bsz] * Bsz + slot % Bsz : slot;
+            idx[pos] = (blk ? blk[slot / Bsz] * Bsz + slot % Bsz : slot) + p.id_off;
             if (sc) sc[pos] = key_score(x);
         });
         if (rank == 0)
@@ -492,7 +492,6 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectPara
 
 constexpr int kRowThreads = 512;
 constexpr int kRowWarps = kRowThreads / 32;
-constexpr int kRowKeys = 24576;
 
 constexpr int kRowBlocks = 2048;   // kept-block ids staged in shared memory
 
@@ -537,16 +536,25 @@ __global__ void __launch_bounds__(kRowThreads) select_row_kernel(const SelectPar
     const int row = blockIdx.x;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-    int n = 0, kk = p.k, b = 0, t = 0, nb = 0;
+    int n = 0, kk = p.k, b = 0, t = 0, nb = 0, cp_own = 0;
     bool bad = false;
     if (p.mode == kSelF32Rows) {
         n = p.n;
+    } else if (p.mode == kSelMerge) {
+        n = p.lists * p.n;
     } else if (p.mode == kSelHisaTokens) {
         const int4 pl = p.plan[row];
         b = pl.x;
         t = pl.y;
         bad = t < 0;
         n = pl.z * p.B;
+    } else if (p.mode == kSelCpBlocks) {
+        // the shard's visible blocks but the own one compete for m - 1 places
+        nb = cp_visible_blocks(p.q_seq, p.q_pos, p.len, p.batch, p.cap, p.B, p.id_off * p.B, row, &b,
+                               &cp_own, &t);
+        bad = nb < 0;
+        n = bad ? 0 : nb - cp_own;
+        kk = p.m - 1;
     } else {
         t = query_position(p.q_seq, p.q_pos, p.len, p.batch, p.cap, row, &b);
         bad = t < 0;
@@ -589,14 +597,27 @@ __global__ void __launch_bounds__(kRowThreads) select_row_kernel(const SelectPar
 
     // 1. stage the keys; count, min, max of the nonzero ones
     uint32_t cnt = 0, mn = 0xFFFFFFFFu, mx = 0u;
-    if (p.mode == kSelF32Rows) {
+    // slot c of a merged row: list c / n, entry c % n
+    auto merge_at = [&](int c) {
+        const int l = c / p.n;
+        return (static_cast<size_t>(l) * p.rows + row) * p.n + (c - l * p.n);
+    };
+    if (p.mode == kSelF32Rows || p.mode == kSelMerge) {
         const float* x = p.x + static_cast<size_t>(row) * p.n;
         for (int c = tid; c < n; c += kRowThreads) {
-            const uint32_t v = score_key(x[c]);
+            uint32_t v;
+            if (p.mode == kSelMerge) {
+                const size_t o = merge_at(c);
+                v = p.ids[o] < 0 ? 0u : score_key(p.x[o]);   // an empty entry never competes
+            } else {
+                v = score_key(x[c]);
+            }
             ks[c] = v;
-            cnt += v != 0u;
-            mn = min(mn, v);
-            mx = max(mx, v);
+            if (v != 0u) {
+                ++cnt;
+                mn = min(mn, v);
+                mx = max(mx, v);
+            }
         }
     } else {
         const uint4* g4 = reinterpret_cast<const uint4*>(p.keys + static_cast<size_t>(row) * p.ldk);
@@ -786,9 +807,11 @@ __global__ void __launch_bounds__(kRowThreads) select_row_kernel(const SelectPar
                 } else {
                     if (blk) {
                         const int bi = pow2 ? c >> lgB : c / Bsz;
-                        idx[at] = blk[bi] * Bsz + (c - bi * Bsz);
+                        idx[at] = blk[bi] * Bsz + (c - bi * Bsz) + p.id_off;
+                    } else if (p.mode == kSelMerge) {
+                        idx[at] = p.ids[merge_at(c)];
                     } else {
-                        idx[at] = c;
+                        idx[at] = c + p.id_off;
                     }
                     if (sc) sc[at] = key_score(x);
                 }
@@ -810,7 +833,17 @@ __global__ void __launch_bounds__(kRowThreads) select_row_kernel(const SelectPar
             p.plan[row] = make_int4(b, t, keep, 0);
         }
     } else {
-        for (int r = static_cast<int>(kept) + tid; r < p.k; r += kRowThreads) {
+        int r0 = static_cast<int>(kept);
+        if (cp_own) {
+            // the shard holds the row's own block: it follows the m - 1 others,
+            // marked with an infinite score so that every merge keeps it
+            if (tid == 0) {
+                idx[r0] = p.id_off + nb - 1;
+                if (sc) sc[r0] = __int_as_float(0x7f800000);
+            }
+            ++r0;
+        }
+        for (int r = r0 + tid; r < p.k; r += kRowThreads) {
             idx[r] = -1;
             if (sc) sc[r] = __int_as_float(0x7fc00000);
         }
@@ -859,10 +892,70 @@ cudaError_t launch_t(const SelectParams& p, int csize, int chunk, cudaStream_t s
     return cudaLaunchKernelEx(&cfg, fn, p);
 }
 
+// One warp per row: the shard's visible blocks among the row's merged global
+// block list, in order (an ordered compaction by ballots).
+__global__ void __launch_bounds__(128) cp_localize_kernel(const CpLocalizeParams p) {
+    grid_dependency_wait();
+    grid_launch_dependents();
+    const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= p.rows) return;
+    int b, own, tl;
+    const int vis = cp_visible_blocks(p.q_seq, p.q_pos, p.len, p.batch, p.cap, p.B, p.tok_off, row, &b,
+                                      &own, &tl);
+    const int blk0 = p.tok_off / p.B;
+    const int32_t* kept = p.kept + static_cast<size_t>(row) * p.m;
+    int32_t* out = p.blocks + static_cast<size_t>(row) * p.mm;
+    const int t = p.q_pos[row];
+    const int g_own = t >= 0 ? t / p.B : -2;
+    bool has_own = false;
+    for (int base = 0; base < p.m; base += 32) {
+        const int j = base + lane;
+        has_own |= __any_sync(0xffffffffu, j < p.m && kept[j] == g_own);
+    }
+    const bool valid = vis >= 0 && has_own;
+    int cnt = 0;
+    if (valid && vis > 0)
+        for (int base = 0; base < p.m; base += 32) {
+            const int j = base + lane;
+            const int g = j < p.m ? kept[j] : -1;
+            const bool mine = g >= blk0 && g - blk0 < vis;
+            const unsigned bal = __ballot_sync(0xffffffffu, mine);
+            const int at = cnt + __popc(bal & ((1u << lane) - 1u));
+            if (mine && at < p.mm) out[at] = g - blk0;
+            cnt += __popc(bal);
+        }
+    cnt = min(cnt, p.mm);
+    for (int j = cnt + lane; j < p.mm; j += 32) out[j] = -1;
+    if (lane == 0) {
+        p.nblocks[row] = cnt;
+        // the own block is the last kept one on the shard that holds the query
+        // position; elsewhere every kept block is visible as a whole
+        p.plan[row] = make_int4(b, !valid ? -1 : (own ? tl : p.cap - 1), cnt, 0);
+        if (!valid) set_status(p.status, HISA_DEV_BAD_QUERY);
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_cp_localize(const CpLocalizeParams& p, cudaStream_t s) {
+    if (p.rows <= 0) return cudaSuccess;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>((p.rows + 3) / 4));
+    cfg.blockDim = dim3(128);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, cp_localize_kernel, p);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
 
 cudaError_t launch_select(const SelectParams& p, int max_n, int sms, cudaStream_t s) {
     if (p.rows <= 0) return cudaSuccess;
+    if ((p.mode == kSelCpBlocks || p.mode == kSelMerge) && max_n > kRowKeys) return cudaErrorInvalidValue;
     if (max_n <= kRowKeys) {
         const cudaError_t e = launch_row(p, max_n, s);
         return e == cudaSuccess ? cudaGetLastError() : e;

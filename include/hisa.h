@@ -232,6 +232,65 @@ int hisa_tree_select(const hisa_kv* kv, const hisa_kv* kv2, const uint16_t* Q, c
 int hisa_pool_tail(const hisa_kv* kv, hisa_stream_t stream);
 
 /*
+ * Context parallelism: one sequence longer than a GPU holds, split by token
+ * range over R ranks.  The pages motivate contexts of 64K to 1M tokens and
+ * beyond (blog "What This Means for Long-Context Inference"; gptget.net
+ * summary, limitations: texts beyond millions of tokens) but give no
+ * multi-GPU design; this decomposition is this library's.  Each rank's
+ * hisa_kv is a shard: keys[b, s] holds global position tok_off + s of
+ * sequence b, for every sequence, with tok_off and cap multiples of B and
+ * len[b] the shard's own length (a shard before the one holding the end of
+ * a sequence is full).  q_pos are GLOBAL positions and are required.
+ * The result equals hisa_select on the whole sequence:
+ *   1. hisa_cp_blocks on every rank: the shard's candidates, [n_q, m]
+ *      (global block id, score) pairs, ascending in id, -1 / NaN padded:
+ *      the best m - 1 blocks visible to the row other than its own block,
+ *      then, on the rank holding the query position, the own block with
+ *      score +inf.
+ *   2. all-gather the pairs in rank order (ranks own ascending ranges) into
+ *      [R, n_q, m], and hisa_merge_topk(lists = R, n = m, k = m): the kept
+ *      global block ids [n_q, m] (the own block always among them).
+ *   3. hisa_cp_tokens on every rank with those ids: the top-k of the
+ *      shard's tokens in the kept blocks, as (global index, score) pairs.
+ *   4. all-gather [R, n_q, k] and hisa_merge_topk(lists = R, n = k, k).
+ * Exactness: every block and token is scored by the same kernel as in
+ * hisa_select, and the best kk of a union of lists is the best kk of the
+ * union of each list's best kk, so each merge is exact (ties: lower id).
+ * Rows the shard cannot see (query before the shard) give no candidates.
+ * An invalid row (bad sequence, a position past the sequence end) gives -1
+ * rows and sets HISA_DEV_BAD_QUERY: in hisa_cp_blocks on a shard that sees
+ * it, and in hisa_cp_tokens on every shard (a valid row always has its own
+ * block, global id q_pos / B, among the merged kept blocks).
+ * Limits: at most 24576 blocks per shard; lists * n <= 24576 in a merge.
+ * Errors as hisa_select; HISA_E_INVAL also for a missing q_pos, or tok_off
+ * or cap not on block boundaries.  Workspace: hisa_cp_workspace_bytes,
+ * reused by both calls of one rank.
+ */
+size_t hisa_cp_workspace_bytes(const hisa_kv* kv, int32_t tok_off, int n_q, int H, int m, int k);
+int hisa_cp_blocks(const hisa_kv* kv, int32_t tok_off, const uint16_t* Q, const float* w,
+                   const int32_t* q_seq, const int32_t* q_pos, int n_q, int H, int m,
+                   int32_t* cand_ids, float* cand_scores, void* ws, size_t ws_bytes,
+                   hisa_stream_t stream);
+int hisa_cp_tokens(const hisa_kv* kv, int32_t tok_off, const uint16_t* Q, const float* w,
+                   const int32_t* q_seq, const int32_t* q_pos, int n_q, int H, int m, int k,
+                   const int32_t* kept, int32_t* idx, float* scores, void* ws, size_t ws_bytes,
+                   hisa_stream_t stream);
+
+/*
+ * hisa_merge_topk — top-k of several (id, score) lists per row, by (score
+ * desc, id asc): the exchange step of context parallelism.  ids and scores
+ * are [lists, rows, n] (device, row-major; the layout an all-gather in list
+ * order produces); id -1 marks an empty entry (its score is ignored).  The
+ * concatenation of a row's lists must ascend in id (each list ascending and
+ * the lists' id ranges ascending), which is what makes the lower-id rule the
+ * lower-slot rule.  Out: idx [rows, k] ascending then -1, out_scores
+ * [rows, k] (NaN under padding) or NULL.  Scores must not be NaN for
+ * non-empty entries.  HISA_E_UNSUPPORTED if lists * n > 24576.
+ */
+int hisa_merge_topk(const int32_t* ids, const float* scores, int lists, int rows, int n, int k,
+                    int32_t* idx, float* out_scores, hisa_stream_t stream);
+
+/*
  * hisa_select_static — hisa_select without a caller workspace.  The pages
  * have no counterpart: this is a deployment convenience of this library.
  * The scratch hisa_select keeps in `ws` lives instead in one fixed device
@@ -304,7 +363,8 @@ enum hisa_phase {
     HISA_PHASE_APPEND = 7,        /* hisa_append */
     HISA_PHASE_TOPK = 8,          /* hisa_topk_f32 */
     HISA_PHASE_QSPLIT = 9,        /* query heads split for fp8 scoring (e4m3 keys, d = 128) */
-    HISA_NUM_PHASES = 10
+    HISA_PHASE_MERGE = 10,        /* hisa_merge_topk */
+    HISA_NUM_PHASES = 11
 };
 int hisa_profile_enable(int on);
 int hisa_profile_read(float* ms, int* launches, int reset);

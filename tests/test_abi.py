@@ -161,3 +161,39 @@ def test_tree_index_must_share_the_keys(hisa):
         assert lib.hisa_tree_select(ctypes.byref(kv), ctypes.byref(bad), P(16), P(16), P(16), None,
                                     4, 64, 2, 4, 64, P(16), None, None, None, None, None, None,
                                     P(256), 1 << 30, None) == hisa.HISA_E_INVAL
+
+
+def test_context_parallel_shard_checks(hisa):
+    lib = hisa.lib()
+    P = ctypes.c_void_p
+    kv = _kv(hisa, cap=4096, B=128)
+    assert lib.hisa_cp_workspace_bytes(ctypes.byref(kv), 8192, 4, 64, 8, 64) > 0
+    # shard offsets and capacities on block boundaries only
+    assert lib.hisa_cp_workspace_bytes(ctypes.byref(kv), 100, 4, 64, 8, 64) == 0
+    assert lib.hisa_cp_workspace_bytes(ctypes.byref(kv), -128, 4, 64, 8, 64) == 0
+    odd = _kv(hisa, cap=4000, B=128)
+    assert lib.hisa_cp_workspace_bytes(ctypes.byref(odd), 0, 4, 64, 8, 64) == 0
+    args = (P(16), P(16), P(16))
+    # global query positions are required
+    assert lib.hisa_cp_blocks(ctypes.byref(kv), 0, *args, None, 4, 64, 8, P(16), P(16), P(256), 1 << 30,
+                              None) == hisa.HISA_E_INVAL
+    assert lib.hisa_cp_blocks(ctypes.byref(kv), 100, *args, P(16), 4, 64, 8, P(16), P(16), P(256),
+                              1 << 30, None) == hisa.HISA_E_INVAL
+    assert lib.hisa_cp_blocks(ctypes.byref(kv), 0, *args, P(16), 4, 64, 0, P(16), P(16), P(256), 1 << 30,
+                              None) == hisa.HISA_E_INVAL
+    assert lib.hisa_cp_blocks(ctypes.byref(kv), 0, *args, P(16), 4, 64, 8, P(16), P(16), P(256), 16,
+                              None) == hisa.HISA_E_WORKSPACE
+    assert lib.hisa_cp_tokens(ctypes.byref(kv), 0, *args, P(16), 4, 64, 8, 64, None, P(16), P(16),
+                              P(256), 1 << 30, None) == hisa.HISA_E_INVAL
+    assert lib.hisa_cp_blocks(ctypes.byref(kv), 0, *args, P(16), 0, 64, 8, P(16), P(16), None, 0,
+                              None) == hisa.HISA_OK
+
+
+def test_merge_checks(hisa):
+    lib = hisa.lib()
+    P = ctypes.c_void_p
+    assert lib.hisa_merge_topk(P(16), P(16), 0, 4, 8, 4, P(16), None, None) == hisa.HISA_E_INVAL
+    assert lib.hisa_merge_topk(P(16), P(16), 2, 4, 8, 0, P(16), None, None) == hisa.HISA_E_INVAL
+    assert lib.hisa_merge_topk(None, P(16), 2, 4, 8, 4, P(16), None, None) == hisa.HISA_E_INVAL
+    assert lib.hisa_merge_topk(P(16), P(16), 4, 4, 8192, 4, P(16), None, None) == hisa.HISA_E_UNSUPPORTED
+    assert lib.hisa_merge_topk(P(16), P(16), 2, 0, 8, 4, P(16), None, None) == hisa.HISA_OK
