@@ -59,8 +59,11 @@ def _bind(lib):
     lib.hisa_oracle_topk_f32.argtypes = [P, I, I, I, P]
     lib.hisa_oracle_tree_select.argtypes = [P, P, I, I, I, I, I, I, I, P, P, P, P, P, I, I, I, I,
                                             I, I, P, P, P, P, P, P, P]
+    lib.hisa_oracle_sparse_attn.argtypes = [P, I, P, P, P, I, I, I, P, P, I, I, ctypes.c_double, I,
+                                            P, P]
     for f in ("hisa_oracle_pool", "hisa_oracle_select", "hisa_oracle_refine",
-              "hisa_oracle_flat", "hisa_oracle_topk_f32", "hisa_oracle_tree_select"):
+              "hisa_oracle_flat", "hisa_oracle_topk_f32", "hisa_oracle_tree_select",
+              "hisa_oracle_sparse_attn"):
         getattr(lib, f).restype = I
     return lib
 
@@ -215,3 +218,29 @@ def topk_f32(x, k: int, lib=None) -> np.ndarray:
     if rc:
         raise ValueError(f"hisa_oracle_topk_f32 rc={rc}")
     return idx
+
+
+def sparse_attn(Qa, K, V, lens, q_seq, idx, scale: float, threads: Optional[int] = None,
+                lib=None):
+    """Attention of each query row over its selected entries (the plain
+    definition, in double).  Qa [n_q, Ha, d], K, V [batch, cap, d] as bf16
+    bits (uint16); idx [n_q, k] (-1 or >= len: skipped).  Returns (out
+    [n_q, Ha, d], lse [n_q, Ha])."""
+    lib = lib or load()
+    Qa = _c(Qa, np.uint16)
+    K = _c(K, np.uint16)
+    V = _c(V, np.uint16)
+    lens = _c(lens, np.int32)
+    q_seq = _c(q_seq, np.int32)
+    idx = _c(idx, np.int32)
+    n_q, Ha, d = Qa.shape
+    batch, cap, _ = K.shape
+    k = idx.shape[1]
+    out = np.empty((n_q, Ha, d))
+    lse = np.empty((n_q, Ha))
+    rc = lib.hisa_oracle_sparse_attn(_p(Qa), Ha, _p(K), _p(V), _p(lens), batch, cap, d, _p(q_seq),
+                                     _p(idx), n_q, k, float(scale), threads or default_threads(),
+                                     _p(out), _p(lse))
+    if rc:
+        raise ValueError(f"hisa_oracle_sparse_attn rc={rc}")
+    return out, lse

@@ -606,3 +606,73 @@ int hisa_oracle_topk_f32(const float* x, int rows, int n, int k, int32_t* idx) {
     free(items);
     return 0;
 }
+
+/* ----------------------------------------------------- sparse attention */
+
+/* The consumer of the selection (blog "Hierarchical Indexing Makes Sparse
+ * Attention Actually Fast", "How Fine-Grained Sparse Attention Works Today":
+ * the second stage attends to the selected top-K tokens only).  A synthetic
+ * multi-query operator, by its definition: for row i (sequence b) and head h,
+ * over the list entries j whose index s_j satisfies 0 <= s_j < len[b],
+ *     a_j = scale * Qa[i,h] . K[b, s_j]
+ *     out[i,h] = sum_j exp(a_j) V[b, s_j] / sum_j exp(a_j)
+ *     lse[i,h] = log sum_j exp(a_j)
+ * in double (the exponentials are taken relative to the largest a_j, which
+ * changes nothing but the range).  No valid entry: out = 0, lse = -inf. */
+typedef struct {
+    const uint16_t* Qa; const uint16_t* K; const uint16_t* V;
+    const int32_t* lens; const int32_t* q_seq; const int32_t* idx;
+    int Ha, batch, cap, d, k;
+    double scale;
+    double* out; double* lse;
+} attn_job_t;
+
+static void attn_row(void* ctx, int i, void* scratch) {
+    const attn_job_t* J = (const attn_job_t*)ctx;
+    double* a = (double*)scratch;             /* [k] */
+    double* x = a + J->k;                     /* [d] */
+    const int b = J->q_seq[i];
+    const int n = (b >= 0 && b < J->batch) ? J->lens[b] : 0;
+    for (int h = 0; h < J->Ha; ++h) {
+        double* o = J->out + ((size_t)i * J->Ha + h) * J->d;
+        for (int e = 0; e < J->d; ++e) o[e] = 0.0;
+        const uint16_t* q = J->Qa + ((size_t)i * J->Ha + h) * J->d;
+        double amax = -INFINITY;
+        for (int j = 0; j < J->k; ++j) {
+            const int s = J->idx[(size_t)i * J->k + j];
+            if (s < 0 || s >= n) { a[j] = NAN; continue; }
+            const uint16_t* kr = J->K + ((size_t)b * J->cap + s) * J->d;
+            double z = 0.0;
+            for (int e = 0; e < J->d; ++e) z += bf16_value(q[e]) * bf16_value(kr[e]);
+            a[j] = J->scale * z;
+            if (a[j] > amax) amax = a[j];
+        }
+        if (amax == -INFINITY) {
+            if (J->lse) J->lse[(size_t)i * J->Ha + h] = -INFINITY;
+            continue;
+        }
+        double sum = 0.0;
+        for (int e = 0; e < J->d; ++e) x[e] = 0.0;
+        for (int j = 0; j < J->k; ++j) {
+            if (isnan(a[j])) continue;
+            const int s = J->idx[(size_t)i * J->k + j];
+            const double p = exp(a[j] - amax);
+            const uint16_t* vr = J->V + ((size_t)b * J->cap + s) * J->d;
+            sum += p;
+            for (int e = 0; e < J->d; ++e) x[e] += p * bf16_value(vr[e]);
+        }
+        for (int e = 0; e < J->d; ++e) o[e] = x[e] / sum;
+        if (J->lse) J->lse[(size_t)i * J->Ha + h] = amax + log(sum);
+    }
+}
+
+int hisa_oracle_sparse_attn(const uint16_t* Qa, int Ha, const uint16_t* K, const uint16_t* V,
+                            const int32_t* lens, int batch, int cap, int d, const int32_t* q_seq,
+                            const int32_t* idx, int n_q, int k, double scale, int n_threads,
+                            double* out, double* lse) {
+    if (!Qa || !K || !V || !lens || !q_seq || !idx || !out || Ha < 1 || batch < 1 || cap < 1 ||
+        d < 1 || n_q < 0 || k < 1)
+        return 1;
+    attn_job_t J = {Qa, K, V, lens, q_seq, idx, Ha, batch, cap, d, k, scale, out, lse};
+    return for_rows(attn_row, &J, n_q, n_threads, sizeof(double) * ((size_t)k + (size_t)d));
+}

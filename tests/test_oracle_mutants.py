@@ -12,7 +12,7 @@ import pytest
 
 import oracle
 from hisa_inputs import bf16_bits, make_case
-from tests import brute
+from tests import attn_pins, brute
 
 MUTANTS = {
     "relu_dropped": ("acc += w[h] * (z > 0.0 ? z : 0.0);", "acc += w[h] * z;"),
@@ -34,6 +34,11 @@ MUTANTS = {
                                        "skept[J->W - 1] = (int32_t)items[J->W - 1].i;"),
     "tree_children_skip_last": ("j < (long)(skept[r] + 1) * bf && j < nb - 1; ++j",
                                 "j < (long)(skept[r] + 1) * bf - 1 && j < nb - 1; ++j"),
+    "attn_scale_dropped": ("a[j] = J->scale * z;", "a[j] = z;"),
+    "attn_entries_past_len_kept": ("if (s < 0 || s >= n) { a[j] = NAN; continue; }",
+                                   "if (s < 0) { a[j] = NAN; continue; }"),
+    "attn_lse_without_max": ("J->lse[(size_t)i * J->Ha + h] = amax + log(sum);",
+                             "J->lse[(size_t)i * J->Ha + h] = log(sum);"),
 }
 
 
@@ -70,6 +75,8 @@ def _pool_closed_form_fails(lib) -> bool:
 def _detects(lib) -> bool:
     """True if some pin rejects the library `lib`."""
     if _pool_closed_form_fails(lib):
+        return True
+    if attn_pins.any_fails(lib):
         return True
     for c in _cases():
         cache = oracle.Cache.of(c)
