@@ -469,6 +469,7 @@ def run_workloads(args, dev, peaks):
             del kv, ws
             torch.cuda.empty_cache()
     out["pool_sweep_decode-32k-b64"] = sweep
+    out["sparse_attention_decode-32k-b64"] = run_attention(dev, n, flush, stream, peaks)
 
     # streaming append + select for the new last position, one row per step
     case = make_config(4)
@@ -496,6 +497,54 @@ def run_workloads(args, dev, peaks):
                       "steps_per_s": steps / (sum(st) / 1e3),
                       "l2": "cache (32 MiB) L2-resident; no flush: each step follows the last"}
     return out
+
+
+def run_attention(dev, n, flush, stream, peaks):
+    """The consumer of the selection on the 32K decode workload: each of the
+    64 rows attends with 128 query heads (d = 128, one shared key and value
+    head) over the 2048 tokens hisa_select kept.  Key and value caches are
+    their own seeded N(0, 1) bf16 tensors [64, 32768, 128], drawn on the
+    device.  Reports the attention call's time and roofline next to the
+    indexer's select time on the same rows."""
+    import torch
+    import hierarchical_top_indexer_b200 as hisa
+    from hisa_inputs import make_config
+
+    case = make_config(1)
+    kv = hisa.KVCache.from_case(case, device=dev)
+    hisa.hisa_pool_blocks(kv)
+    Q = torch.from_numpy(case.Q.view(np.int16)).view(torch.bfloat16).to(dev)
+    w = torch.from_numpy(case.w).to(dev)
+    qs = torch.from_numpy(case.q_seq).to(dev)
+    n_q, Ha, D, k = case.n_q, 128, 128, case.k
+    ws = hisa.workspace(hisa.hisa_select_workspace_bytes(kv, n_q, case.H, case.m, k), dev)
+    idx = torch.empty((n_q, k), dtype=torch.int32, device=dev)
+    sel = lambda: hisa.hisa_select(kv, Q, w, qs, None, case.m, k, ws=ws, idx=idx)
+    sel_ms = _median_ms(sel, n, flush, stream)
+    g = torch.Generator(device=dev).manual_seed(20260331)
+    Kc = torch.randn((case.batch, case.cap, D), generator=g, device=dev).to(torch.bfloat16)
+    Vc = torch.randn((case.batch, case.cap, D), generator=g, device=dev).to(torch.bfloat16)
+    Qa = torch.randn((n_q, Ha, D), generator=g, device=dev).to(torch.bfloat16)
+    lens = kv.len.clone()
+    aws = hisa.workspace(hisa.hisa_sparse_attn_workspace_bytes(n_q, k), dev)
+    out = torch.empty((n_q, Ha, D), dtype=torch.float32, device=dev)
+    lse = torch.empty((n_q, Ha), dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    att = lambda: hisa.hisa_sparse_attn(Qa, Kc, Vc, lens, qs, idx, ws=aws, out=out, lse=lse, status=status)
+    att_ms = _median_ms(att, n, flush, stream)
+    assert int(status.item()) == 0 and kv.status_bits() == 0
+    nbytes = n_q * (k * 2 * D * 2 + Ha * D * 2 + Ha * D * 4 + Ha * 4 + k * 4)
+    flops = n_q * 2 * Ha * k * 2 * D
+    gbs = nbytes / (att_ms / 1e3) / 1e9
+    del Kc, Vc, kv
+    torch.cuda.empty_cache()
+    return {"rows": n_q, "heads": Ha, "d": D, "k": k,
+            "attn_ms_per_call": att_ms, "hisa_select_ms_per_call": sel_ms,
+            "indexer_share": sel_ms / (sel_ms + att_ms),
+            "attn_roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                              "frac": gbs / peaks["hbm_gbs"], "algorithmic_bytes_per_call": nbytes,
+                              "TFLOP/s": flops / (att_ms / 1e3) / 1e12},
+            "l2": "flushed between calls (key and value caches 512 MiB each)"}
 
 
 def run_tree(case, dev, n, flush, stream, two_level_ms):
@@ -688,6 +737,8 @@ def main(argv=None, backend: str = "nccl"):
     ap.add_argument("--select-only", default=None,
                     help="time only hisa_select on this workload (a name from hisa_inputs)")
     ap.add_argument("--flat", action="store_true", help="with --select-only: dsa_flat_select")
+    ap.add_argument("--attn-only", action="store_true",
+                    help="time only the sparse attention over the 32K decode selection")
     ap.add_argument("--workload-steps", type=int, default=20,
                     help="timed selects per extra workload (0: skip them)")
     args = ap.parse_args(argv)
@@ -700,6 +751,15 @@ def main(argv=None, backend: str = "nccl"):
             line = run_reference(args, rank, world)
             if line is not None:
                 print(json.dumps(line), flush=True)
+            return 0
+
+        if args.attn_only:
+            if rank == 0:
+                import torch
+                dev = torch.device("cuda", 0)
+                flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+                print(json.dumps(run_attention(dev, args.steps, flush, torch.cuda.current_stream(),
+                                               measured_peaks())), flush=True)
             return 0
 
         if args.select_only:

@@ -39,10 +39,11 @@ HISA_DEV_BAD_QUERY, HISA_DEV_CAPACITY, HISA_DEV_BAD_LEN, HISA_DEV_TIMEOUT = 0x1,
 EXPORTS = ("hisa_pool_blocks", "hisa_append", "hisa_select_workspace_bytes", "hisa_select",
            "hisa_select_inspect", "hisa_select_static", "hisa_tree_workspace_bytes",
            "hisa_tree_select", "hisa_pool_tail", "hisa_cp_workspace_bytes", "hisa_cp_blocks",
-           "hisa_cp_tokens", "hisa_merge_topk", "dsa_flat_workspace_bytes", "dsa_flat_select", "hisa_topk_f32",
+           "hisa_cp_tokens", "hisa_merge_topk", "hisa_sparse_attn_workspace_bytes", "hisa_sparse_attn",
+           "dsa_flat_workspace_bytes", "dsa_flat_select", "hisa_topk_f32",
            "hisa_profile_enable", "hisa_profile_read", "hisa_status_string", "hisa_last_cuda_error")
 PHASES = ("block_score", "block_select", "token_score", "token_select", "flat_score",
-          "flat_select", "pool", "append", "topk", "qsplit", "merge")
+          "flat_select", "pool", "append", "topk", "qsplit", "merge", "attn")
 
 
 class hisa_kv(ctypes.Structure):
@@ -74,6 +75,10 @@ _lib.hisa_cp_blocks.argtypes = [_KVP, ctypes.c_int32, _P, _P, _P, _P, _I, _I, _I
 _lib.hisa_cp_tokens.argtypes = [_KVP, ctypes.c_int32, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P,
                                 _Z, _P]
 _lib.hisa_merge_topk.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _P]
+_lib.hisa_sparse_attn_workspace_bytes.argtypes = [_I, _I]
+_lib.hisa_sparse_attn_workspace_bytes.restype = _Z
+_lib.hisa_sparse_attn.argtypes = [_P, _I, _P, _P, _P, _I, _I, _I, _P, _P, _I, _I, ctypes.c_float, _P, _P,
+                                  _P, _P, _Z, _P]
 _lib.dsa_flat_workspace_bytes.argtypes = [_KVP, _I, _I, _I]
 _lib.dsa_flat_workspace_bytes.restype = _Z
 _lib.dsa_flat_select.argtypes = [_KVP, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _Z, _P]
@@ -86,7 +91,7 @@ _lib.hisa_last_cuda_error.argtypes = []
 _lib.hisa_last_cuda_error.restype = ctypes.c_char_p
 for _f in ("hisa_pool_blocks", "hisa_append", "hisa_select", "hisa_select_inspect", "hisa_select_static",
            "hisa_tree_select", "hisa_pool_tail", "hisa_cp_blocks", "hisa_cp_tokens", "hisa_merge_topk",
-           "dsa_flat_select", "hisa_topk_f32", "hisa_profile_enable", "hisa_profile_read"):
+           "hisa_sparse_attn", "dsa_flat_select", "hisa_topk_f32", "hisa_profile_enable", "hisa_profile_read"):
     getattr(_lib, _f).restype = _I
 
 
@@ -416,6 +421,34 @@ def hisa_merge_topk(ids: torch.Tensor, scores: torch.Tensor, k: int, stream=None
     _check("hisa_merge_topk", _lib.hisa_merge_topk(_ptr(ids), _ptr(scores), lists, rows, n, k, _ptr(idx),
                                                    _ptr(sc), _stream(stream)))
     return idx, sc
+
+
+def hisa_sparse_attn_workspace_bytes(n_q: int, k: int) -> int:
+    return int(_lib.hisa_sparse_attn_workspace_bytes(n_q, k))
+
+
+def hisa_sparse_attn(Qa: torch.Tensor, K: torch.Tensor, V: torch.Tensor, lens: torch.Tensor,
+                     q_seq: torch.Tensor, idx: torch.Tensor, scale: Optional[float] = None,
+                     ws: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                     lse: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
+                     stream=None):
+    """Attention of each query row over its selected tokens: Qa [n_q, Ha, 128]
+    bf16 heads sharing the key and value heads K, V [batch, cap, 128] bf16;
+    idx [n_q, k] (hisa_select's output).  Returns (out [n_q, Ha, 128] fp32,
+    lse [n_q, Ha] fp32); `status` (int32 [1], device) collects device errors."""
+    n_q, Ha, d = Qa.shape
+    batch, cap, _ = K.shape
+    k = idx.shape[1]
+    dev = Qa.device
+    scale = (1.0 / d ** 0.5) if scale is None else float(scale)
+    ws = workspace(hisa_sparse_attn_workspace_bytes(n_q, k), dev) if ws is None else ws
+    out = torch.empty((n_q, Ha, d), dtype=torch.float32, device=dev) if out is None else out
+    lse = torch.empty((n_q, Ha), dtype=torch.float32, device=dev) if lse is None else lse
+    status = torch.zeros(1, dtype=torch.int32, device=dev) if status is None else status
+    _check("hisa_sparse_attn", _lib.hisa_sparse_attn(
+        _ptr(Qa), Ha, _ptr(K), _ptr(V), _ptr(lens), batch, cap, d, _ptr(q_seq), _ptr(idx), n_q, k,
+        scale, _ptr(out), _ptr(lse), _ptr(status), _ptr(ws), ws.numel(), _stream(stream)))
+    return out, lse
 
 
 def _gather_ranks(t: torch.Tensor, group=None) -> torch.Tensor:

@@ -4,6 +4,7 @@
 // for hisa_select_static, whose scratch is one fixed device array below.
 #include <atomic>
 #include <climits>
+#include <cmath>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -806,6 +807,49 @@ int hisa_merge_topk(const int32_t* ids, const float* scores, int lists, int rows
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     PhaseScope ps(HISA_PHASE_MERGE, s);
     return cuda_status(launch_select(sp, lists * n, sm_count(), s));
+}
+
+size_t hisa_sparse_attn_workspace_bytes(int n_q, int k) {
+    if (n_q < 0 || k < 1) return 0;
+    return attn_workspace_bytes(n_q, k);
+}
+
+int hisa_sparse_attn(const uint16_t* Qa, int Ha, const uint16_t* Kc, const uint16_t* Vc, const int32_t* len,
+                     int batch, int cap, int d, const int32_t* q_seq, const int32_t* idx, int n_q, int k,
+                     float scale, float* out, float* lse, uint32_t* status, void* ws, size_t ws_bytes,
+                     hisa_stream_t stream) {
+    if (n_q < 0 || k < 1 || batch < 1 || cap < 1 || !(scale > 0.f) || !std::isfinite(scale)) return HISA_E_INVAL;
+    if (Ha < 1 || Ha > 128 || d != 128) return HISA_E_UNSUPPORTED;
+    if (n_q == 0) return HISA_OK;
+    if (!Qa || !Kc || !Vc || !len || !q_seq || !idx || !out || !status) return HISA_E_INVAL;
+    if (!aligned(Qa, 16) || !aligned(Kc, 16) || !aligned(Vc, 16) || !aligned(out, 16) || !aligned(len, 4) ||
+        !aligned(q_seq, 4) || !aligned(idx, 4) || !aligned(status, 4) || (lse && !aligned(lse, 4)))
+        return HISA_E_INVAL;
+    if (!ws || !aligned(ws, 256) || ws_bytes < attn_workspace_bytes(n_q, k)) return HISA_E_WORKSPACE;
+    AttnParams p;
+    std::memset(&p, 0, sizeof p);
+    p.q = Qa;
+    p.kc = Kc;
+    p.vc = Vc;
+    p.idx = idx;
+    p.q_seq = q_seq;
+    p.len = len;
+    p.batch = batch;
+    p.cap = cap;
+    p.n_q = n_q;
+    p.Ha = Ha;
+    p.k = k;
+    p.T = (k + 127) / 128;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.out = out;
+    p.lse = lse;
+    p.status = status;
+    attn_carve(p, ws);
+    const int sms = sm_count();
+    if (sms <= 0) return HISA_E_CUDA;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    PhaseScope ps(HISA_PHASE_ATTN, s);
+    return cuda_status(launch_attn(p, sms, s));
 }
 
 int hisa_pool_tail(const hisa_kv* kv, hisa_stream_t stream) {

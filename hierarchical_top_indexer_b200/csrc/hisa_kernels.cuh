@@ -176,6 +176,28 @@ struct CpLocalizeParams {
 };
 cudaError_t launch_cp_localize(const CpLocalizeParams& p, cudaStream_t s);
 
+// Sparse attention over selected tokens (attn.cu): Ha <= 128 query heads of
+// d = 128 sharing one key and one value head, k selected entries per row.
+struct AttnParams {
+    const uint16_t* q;       // [n_q, Ha, 128] bf16
+    const uint16_t* kc;      // [batch, cap, 128] bf16
+    const uint16_t* vc;      // [batch, cap, 128] bf16
+    const int32_t* idx;      // [n_q, k]
+    const int32_t* q_seq;    // [n_q]
+    const int32_t* len;      // [batch]
+    int batch, cap, n_q, Ha, k, T;   // T = tiles of 128 entries per row
+    float scale_log2;        // softmax scale * log2(e)
+    float* part_o;           // workspace: [n_q * T, 128, 128] unnormalised segment outputs
+    float* part_ml;          // workspace: [n_q * T, 2, 128] segment max (log2 domain), sum
+    int32_t* seg_len;        // workspace: [n_q * T] tiles of the segment starting there
+    float* out;              // [n_q, Ha, 128]
+    float* lse;              // [n_q, Ha] or null
+    uint32_t* status;
+};
+size_t attn_workspace_bytes(int n_q, int k);
+void attn_carve(AttnParams& p, void* ws);
+cudaError_t launch_attn(const AttnParams& p, int sms, cudaStream_t s);
+
 cudaError_t launch_pool(const KvView& kv, cudaStream_t s);
 cudaError_t launch_append(const KvView& kv, const void* tok, const float* tok_scale,
                           cudaStream_t s);

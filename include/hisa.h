@@ -277,6 +277,38 @@ int hisa_cp_tokens(const hisa_kv* kv, int32_t tok_off, const uint16_t* Q, const 
                    hisa_stream_t stream);
 
 /*
+ * hisa_sparse_attn — the consumer of the selection: attention of each query
+ * row over the tokens it selected (HISA blog, "How Fine-Grained Sparse
+ * Attention Works Today": the second stage attends only to the top-K tokens;
+ * arXiv abstract: the indices feed the sparse attention operator).  A
+ * synthetic multi-query operator: Ha query heads (1..128) of d = 128 share
+ * one key head and one value head.  For row i (sequence b = q_seq[i]) and
+ * head h, over the entries j with 0 <= idx[i, j] < len[b]:
+ *     s_j = scale * Qa[i, h] . Kc[b, idx[i, j]]
+ *     out[i, h] = sum_j exp(s_j) Vc[b, idx[i, j]] / sum_j exp(s_j)
+ *     lse[i, h] = log sum_j exp(s_j)
+ * Other entries (-1 padding, or past len[b]) are skipped; a repeated index
+ * counts once per entry.  A row with no valid entry gives out = 0 and
+ * lse = -inf.
+ *   Qa [n_q, Ha, 128] bf16; Kc, Vc [batch, cap, 128] bf16 (16-byte aligned);
+ *   len [batch] int32; q_seq [n_q]; idx [n_q, k] (hisa_select's output);
+ *   out [n_q, Ha, 128] fp32 (16-byte aligned); lse [n_q, Ha] or NULL;
+ *   status: a device word for HISA_DEV_TIMEOUT; all device memory, caller
+ *   owned.  Workspace: hisa_sparse_attn_workspace_bytes(n_q, k).
+ * Numerics: Qa Kc^T on the bf16 tensor cores into fp32, softmax weights in
+ * fp32 rounded to bf16 for the weights-times-values product (fp32
+ * accumulate); the sum of weights is taken over the rounded weights.
+ * Errors: HISA_E_INVAL (sizes, pointers, alignment, scale not finite and
+ * positive), HISA_E_UNSUPPORTED (d != 128, Ha outside 1..128),
+ * HISA_E_WORKSPACE, HISA_E_CUDA.
+ */
+size_t hisa_sparse_attn_workspace_bytes(int n_q, int k);
+int hisa_sparse_attn(const uint16_t* Qa, int Ha, const uint16_t* Kc, const uint16_t* Vc, const int32_t* len,
+                     int batch, int cap, int d, const int32_t* q_seq, const int32_t* idx, int n_q, int k,
+                     float scale, float* out, float* lse, uint32_t* status, void* ws, size_t ws_bytes,
+                     hisa_stream_t stream);
+
+/*
  * hisa_merge_topk — top-k of several (id, score) lists per row, by (score
  * desc, id asc): the exchange step of context parallelism.  ids and scores
  * are [lists, rows, n] (device, row-major; the layout an all-gather in list
@@ -364,7 +396,8 @@ enum hisa_phase {
     HISA_PHASE_TOPK = 8,          /* hisa_topk_f32 */
     HISA_PHASE_QSPLIT = 9,        /* query heads split for fp8 scoring (e4m3 keys, d = 128) */
     HISA_PHASE_MERGE = 10,        /* hisa_merge_topk */
-    HISA_NUM_PHASES = 11
+    HISA_PHASE_ATTN = 11,         /* hisa_sparse_attn */
+    HISA_NUM_PHASES = 12
 };
 int hisa_profile_enable(int on);
 int hisa_profile_read(float* ms, int* launches, int reset);
