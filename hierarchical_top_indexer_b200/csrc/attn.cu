@@ -9,37 +9,42 @@
 //     o[i, h] = sum_j softmax_j(scale * qa[i, h] . K[b, idx[i, j]]) V[b, idx[i, j]]
 // over the entries j with 0 <= idx[i, j] < len[b] (the others are padding).
 //
-// Layout of one CTA (288 threads): warps 0-3 gather, warp 4 issues the
-// tcgen05 MMAs, warps 5-8 run the softmax (one thread per head).  A CTA
+// Layout of one CTA (416 threads): warps 0-3 gather, warp 4 issues the
+// tcgen05 MMAs, warps 5-12 run the softmax (two threads per head, one per
+// half of the tile's 128 columns).  A CTA
 // takes a contiguous range of (row, 128-token tile) slots; a run of tiles of
 // one row is a segment, whose unnormalised output, running max and sum go to
 // the workspace, and combine_kernel merges a row's segments.
-//   gather:  per tile, thread r copies token r's key and value rows (256 B
-//            each) with 16-byte cp.async into the 128-byte swizzled operand
-//            layout (zero rows for padding entries).
+//   gather:  per tile, the key and value rows (256 B each) of the tile's 128
+//            tokens, by 16-byte cp.async into the 128-byte swizzled operand
+//            layout, half a warp per row (zero rows for padding entries).
 //   MMA:     S = Qa K^T (M = 128 heads, N = 128 tokens, K = 128) into one of
 //            two TMEM buffers; then O += P V (K = 128 tokens, V read
 //            MN-major) into a third.
 //   softmax: per tile, the head's row of S: max, p = 2^(s - max) rounded to
-//            bf16 into the P operand, running sum; when the max grows, the
-//            head's row of O is rescaled in TMEM before the next P V.
+//            bf16 into the P operand, running sum (of the unrounded p); when
+//            the max grows, the head's row of O is rescaled in TMEM before
+//            the next P V.
 #include "hisa_kernels.cuh"
 
 namespace hisa {
 
 namespace {
 
-constexpr int kAttnThreads = 288;
-constexpr int kWarpMmaA = 4;   // warps 0-3 gather, 5-8 softmax
+constexpr int kAttnThreads = 416;
+constexpr int kWarpMmaA = 4;    // warps 0-3 gather
+constexpr int kWarpSoft0 = 5;   // warps 5-12 softmax
 constexpr int kAttnStages = 2;
 constexpr int kOperandBytes = 128 * 256;            // one 128 x 128 bf16 operand
-constexpr int kAttnSmem = kOperandBytes * (2 + 2 * kAttnStages) + 1024 + 256;
+constexpr int kAttnSmem = kOperandBytes * (2 + 2 * kAttnStages) + 1024 + 4096;
 
 struct AttnLayout {
     static constexpr int q = 0;
     static constexpr int k0 = kOperandBytes;                       // K of stage s: k0 + s * 2 * op
     static constexpr int p = kOperandBytes * (1 + 2 * kAttnStages);
     static constexpr int bars = kOperandBytes * (2 + 2 * kAttnStages);
+    static constexpr int red = bars + 256;         // [2][2][128] fp32 maxima of the halves
+    static constexpr int lred = red + 2048;        // [2][128] fp32 sums of the halves
 };
 
 // Byte offset of 16-byte chunk c (0..15) of row r (0..127) of a 128 x 128
@@ -81,6 +86,13 @@ __device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t saddr) {
 // bf16 x bf16 -> fp32, M = N = 128, A K-major; B K-major or MN-major.
 __host__ __device__ constexpr uint32_t idesc_attn(bool b_mn_major) {
     return idesc_bf16_f32(128) | (b_mn_major ? (1u << 16) : 0u);
+}
+
+// 2^x by the hardware approximation (about 2^-22 relative; 2^-inf = 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -139,13 +151,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
     uint64_t* full = bars;                  // [stages] a tile's K and V landed (128 copy arrivals)
     uint64_t* empty = full + kAttnStages;   // [stages] the tile's P V is done (commit)
     uint64_t* sfull = empty + kAttnStages;  // [2] S buffer written (commit)
-    uint64_t* sempty = sfull + 2;           // [2] S buffer read (4 softmax warps)
+    uint64_t* sempty = sfull + 2;           // [2] S buffer read (8 softmax warps)
     uint64_t* qfull = sempty + 2;           // the segment's query heads landed (128 arrivals)
     uint64_t* qempty = qfull + 1;           // the segment's last S MMA is done (commit)
-    uint64_t* pfull = qempty + 1;           // P written and O corrected (4 softmax warps)
+    uint64_t* pfull = qempty + 1;           // P written and O corrected (8 softmax warps)
     uint64_t* ofull = pfull + 1;            // a P V is done (commit)
     uint64_t* done = ofull + 1;             // every MMA issued is done (commit)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+    uint64_t* xbar = done + 1;              // [2] both halves' maxima written (8 softmax warps)
+    uint64_t* lbar = xbar + 2;              // both halves' sums written (8 softmax warps)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lbar + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -162,11 +176,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
             }
             for (int b = 0; b < 2; ++b) {
                 mbar_init(sfull + b, 1);
-                mbar_init(sempty + b, 4);
+                mbar_init(sempty + b, 8);
+                mbar_init(xbar + b, 8);
             }
+            mbar_init(lbar, 8);
             mbar_init(qfull, 128);
             mbar_init(qempty, 1);
-            mbar_init(pfull, 4);
+            mbar_init(pfull, 8);
             mbar_init(ofull, 1);
             mbar_init(done, 1);
             *abort_flag = 0;
@@ -188,7 +204,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
 
     if (warp < 4) {
         // ---------------------------------------------------------- gather
-        const int r = threadIdx.x;   // head (query rows) / token slot (tiles)
+        // Warp w copies rows 32 w .. 32 w + 31 of each operand; one copy
+        // instruction moves two whole 256-byte rows (lanes 0-15 the first,
+        // 16-31 the second), so every request is a contiguous run.
+        const int rbase = warp * 32;
+        const int c = lane & 15;
         bool ok = true;
         int it = 0, qn = 0;
         for (long long g = g0; g < g1 && ok;) {
@@ -200,31 +220,40 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
                 break;
             }
             {
-                const bool hv = r < p.Ha;
-                const uint16_t* src = hv ? p.q + (static_cast<size_t>(sg.row) * p.Ha + r) * 128 : p.q;
                 const uint32_t dst = smem_addr(sQ);
-#pragma unroll
-                for (int c = 0; c < 16; ++c) cp_async_16(dst + sw128_off(r, c), src + (hv ? 8 * c : 0), hv ? 16u : 0u);
+#pragma unroll 4
+                for (int i = 0; i < 16; ++i) {
+                    const int r = rbase + 2 * i + (lane >> 4);
+                    const bool hv = r < p.Ha;
+                    const uint16_t* src = p.q + (hv ? (static_cast<size_t>(sg.row) * p.Ha + r) * 128 + 8 * c : 0);
+                    cp_async_16(dst + sw128_off(r, c), src, hv ? 16u : 0u);
+                }
                 cp_async_arrive_noinc(qfull);
             }
             ++qn;
             for (int j = 0; j < sg.n; ++j, ++it) {
                 const int st = it % kAttnStages, use = it / kAttnStages;
+                // this lane's token (row rbase + lane), read before the wait for a free stage
+                const int slot = (sg.t0 + j) * 128 + rbase + lane;
+                int tok = slot < p.k ? p.idx[static_cast<size_t>(sg.row) * p.k + slot] : -1;
                 if (use > 0 && !warp_wait_a(empty + st, (use - 1) & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
-                const int slot = (sg.t0 + j) * 128 + r;
-                int tok = slot < p.k ? p.idx[static_cast<size_t>(sg.row) * p.k + slot] : -1;
                 const bool v = tok >= 0 && tok < len_b;
                 if (!v) tok = 0;
-                const size_t off = (static_cast<size_t>(v ? b : 0) * p.cap + tok) * 128;
                 const uint32_t dk = smem_addr(smem + AttnLayout::k0 + st * 2 * kOperandBytes);
                 const uint32_t dv = dk + kOperandBytes;
-#pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    cp_async_16(dk + sw128_off(r, c), p.kc + off + 8 * c, v ? 16u : 0u);
-                    cp_async_16(dv + sw128_off(r, c), p.vc + off + 8 * c, v ? 16u : 0u);
+#pragma unroll 4
+                for (int i = 0; i < 16; ++i) {
+                    // row rr's token and validity (not this lane's own)
+                    const int rr = 2 * i + (lane >> 4);
+                    const int t_i = __shfl_sync(0xffffffffu, tok, rr);
+                    const bool v_i = __shfl_sync(0xffffffffu, v ? 1 : 0, rr) != 0;
+                    const size_t off = (static_cast<size_t>(v_i ? b : 0) * p.cap + t_i) * 128 + 8 * c;
+                    const uint32_t o = sw128_off(rbase + rr, c);
+                    cp_async_16(dk + o, p.kc + off, v_i ? 16u : 0u);
+                    cp_async_16(dv + o, p.vc + off, v_i ? 16u : 0u);
                 }
                 cp_async_arrive_noinc(full + st);
             }
@@ -243,6 +272,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
                 if (!mbar_wait(full + st, use & 1, abort_flag)) return false;
                 const uint32_t buf = sc & 1;
                 if (sc >= 2 && !mbar_wait(sempty + buf, ((sc >> 1) - 1) & 1, abort_flag)) return false;
+                // the tile arrived by cp.async (generic proxy); the MMAs read it through the async proxy
+                fence_async_smem();
                 tc_fence_after();
                 const uint32_t bk = smem_addr(smem + AttnLayout::k0 + st * 2 * kOperandBytes);
 #pragma unroll
@@ -262,6 +293,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
                     break;
                 }
                 ++qn;
+                fence_async_smem();
                 tc_fence_after();
                 ok = issue_s(it);
                 for (int j = 0; j < sg.n && ok; ++j) {
@@ -295,12 +327,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
         __syncwarp();
     } else {
         // --------------------------------------------------------- softmax
+        // Warps 5-12.  Warp w reads the TMEM lanes of its quadrant (heads
+        // h = 32 (w mod 4) + lane) and the columns of its half (w - 5) / 4:
+        // tokens 64 half .. + 63 of S and P, value dims 64 half .. + 63 of O.
+        // The two halves of a head exchange their maxima (and, at the end of
+        // a segment, their sums) through shared memory and a bounded barrier.
         const int quad = warp & 3;
+        const int half = (warp - kWarpSoft0) >> 2;
         const int h = quad * 32 + lane;
         const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+        const uint32_t col0 = static_cast<uint32_t>(half * 64);
         const uint32_t p_row = smem_addr(sP);
+        float* red = reinterpret_cast<float*>(smem + AttnLayout::red);     // [2][2 halves][128]
+        float* lred = reinterpret_cast<float*>(smem + AttnLayout::lred);   // [2 halves][128]
+        const float c2 = p.scale_log2;
         bool ok = true;
-        uint32_t sc = 0, ow = 0;
+        uint32_t sc = 0, ow = 0, xn = 0, ln = 0;
         for (long long g = g0; g < g1 && ok;) {
             const Seg sg = next_seg(g, g1, T);
             int b;
@@ -308,29 +350,45 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
             float m = -INFINITY, l = 0.f;
             for (int j = 0; j < sg.n; ++j) {
                 const uint32_t buf = sc & 1;
+                // the tile's entries of this half, read before the wait for S
+                const int base = (sg.t0 + j) * 128 + half * 64;
+                const bool va = attn_valid(p, sg.row, base + lane, len_b);
+                const bool vb = attn_valid(p, sg.row, base + 32 + lane, len_b);
                 if (!warp_wait_a(sfull + buf, (sc >> 1) & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const int base = (sg.t0 + j) * 128;
-                uint32_t mask[4];
-#pragma unroll
-                for (int w = 0; w < 4; ++w) mask[w] = __ballot_sync(0xffffffffu, attn_valid(p, sg.row, base + 32 * w + lane, len_b));
-                const uint32_t ts = tmem_base + lane_off + buf * 128;
-                // pass 1: the tile's maximum (log2 domain)
+                const uint32_t mw[2] = {__ballot_sync(0xffffffffu, va), __ballot_sync(0xffffffffu, vb)};
+                const bool dense = (mw[0] & mw[1]) == 0xffffffffu;
+                const uint32_t ts = tmem_base + lane_off + buf * 128 + col0;
+                // pass 1: this half's maximum (raw logits; the scale is positive)
                 float mx = -INFINITY;
 #pragma unroll 1
-                for (int c = 0; c < 8; ++c) {
+                for (int c = 0; c < 4; ++c) {
                     float v[16];
                     tmem_ld16(ts + c * 16, v);
+                    if (dense) {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int col = c * 16 + i;
-                        if ((mask[col >> 5] >> (col & 31)) & 1u) mx = fmaxf(mx, v[i] * p.scale_log2);
+                        for (int i = 0; i < 16; ++i) mx = fmaxf(mx, v[i]);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            if ((mw[c >> 1] >> ((c & 1) * 16 + i)) & 1u) mx = fmaxf(mx, v[i]);
                     }
                 }
-                const float m_new = fmaxf(m, mx);
+                mx *= c2;
+                // the row maximum from both halves
+                const uint32_t xb = xn & 1;
+                red[(xb * 2 + half) * 128 + h] = mx;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(xbar + xb);
+                if (!warp_wait_a(xbar + xb, (xn >> 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                ++xn;
+                const float m_new = fmaxf(m, fmaxf(mx, red[(xb * 2 + (half ^ 1)) * 128 + h]));
                 // the previous P V must be done before P is rewritten or O rescaled
                 if (j > 0) {
                     if (!warp_wait_a(ofull, ow & 1, abort_flag)) {
@@ -343,11 +401,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
                     // warp rescales together when any of its heads' maxima grew
                     const bool grew = m_new > m && m > -INFINITY;
                     if (__any_sync(0xffffffffu, grew)) {
-                        const float alpha = grew ? exp2f(m - m_new) : 1.f;
+                        const float alpha = grew ? ex2_approx(m - m_new) : 1.f;
                         l *= alpha;
-                        const uint32_t to = tmem_base + lane_off + 256;
+                        const uint32_t to = tmem_base + lane_off + 256 + col0;
 #pragma unroll 1
-                        for (int c = 0; c < 8; ++c) {
+                        for (int c = 0; c < 4; ++c) {
                             float v[16];
                             tmem_ld16(to + c * 16, v);
                             uint32_t u[16];
@@ -358,30 +416,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
                         tmem_st_wait();
                     }
                 }
-                // pass 2: p = 2^(s - max) in bf16 into the P operand, and its sum
+                // pass 2: p = 2^(s c2 - max) in bf16 into this half of the P row, and its sum
+                const bool live = m_new > -INFINITY;
                 float psum = 0.f;
 #pragma unroll 1
-                for (int c = 0; c < 8; ++c) {
+                for (int c = 0; c < 4; ++c) {
                     float v[16];
                     tmem_ld16(ts + c * 16, v);
+                    float e[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const bool on = live && (dense || ((mw[c >> 1] >> ((c & 1) * 16 + i)) & 1u));
+                        e[i] = on ? ex2_approx(fmaf(v[i], c2, -m_new)) : 0.f;
+                        psum += e[i];
+                    }
                     uint32_t w8[8];
 #pragma unroll
-                    for (int i = 0; i < 16; i += 2) {
-                        float e[2];
-#pragma unroll
-                        for (int q = 0; q < 2; ++q) {
-                            const int col = c * 16 + i + q;
-                            const bool on = ((mask[col >> 5] >> (col & 31)) & 1u) && m_new > -INFINITY;
-                            e[q] = on ? exp2f(v[i + q] * p.scale_log2 - m_new) : 0.f;
-                        }
-                        w8[i >> 1] = pack_bf16(e[0], e[1]);
-                        const __nv_bfloat162 pr = *reinterpret_cast<const __nv_bfloat162*>(&w8[i >> 1]);
-                        psum += __low2float(pr) + __high2float(pr);
-                    }
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(p_row + sw128_off(h, 2 * c)),
+                    for (int i = 0; i < 8; ++i) w8[i] = pack_bf16(e[2 * i], e[2 * i + 1]);
+                    const int chunk = half * 8 + 2 * c;
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(p_row + sw128_off(h, chunk)),
                                  "r"(w8[0]), "r"(w8[1]), "r"(w8[2]), "r"(w8[3])
                                  : "memory");
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(p_row + sw128_off(h, 2 * c + 1)),
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(p_row + sw128_off(h, chunk + 1)),
                                  "r"(w8[4]), "r"(w8[5]), "r"(w8[6]), "r"(w8[7])
                                  : "memory");
                 }
@@ -405,25 +461,35 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const AttnParams 
             ++ow;
             tc_fence_after();
             const size_t slot = static_cast<size_t>(sg.row) * T + sg.t0;
-            float* po = p.part_o + (slot * 128 + h) * 128;
-            const uint32_t to = tmem_base + lane_off + 256;
+            float* po = p.part_o + (slot * 128 + h) * 128 + col0;
+            const uint32_t to = tmem_base + lane_off + 256 + col0;
 #pragma unroll 1
-            for (int c = 0; c < 8; ++c) {
+            for (int c = 0; c < 4; ++c) {
                 float v[16];
                 tmem_ld16(to + c * 16, v);
 #pragma unroll
                 for (int i = 0; i < 16; i += 4)
                     *reinterpret_cast<float4*>(po + c * 16 + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
             }
-            p.part_ml[slot * 256 + h] = m;
-            p.part_ml[slot * 256 + 128 + h] = l;
-            if (h == 0) p.seg_len[slot] = sg.n;
+            // the head's sum over both halves
+            lred[half * 128 + h] = l;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(lbar);
+            if (!warp_wait_a(lbar, ln & 1, abort_flag)) {
+                ok = false;
+                break;
+            }
+            ++ln;
+            if (half == 0) {
+                p.part_ml[slot * 256 + h] = m;
+                p.part_ml[slot * 256 + 128 + h] = l + lred[128 + h];
+                if (h == 0) p.seg_len[slot] = sg.n;
+            }
             tc_fence_before();
             g += sg.n;
         }
         if (!ok) attn_abort(abort_flag, p.status);
     }
-
     tc_fence_before();
     __syncthreads();
     if (warp == kWarpMmaA) {

@@ -295,9 +295,11 @@ int hisa_cp_tokens(const hisa_kv* kv, int32_t tok_off, const uint16_t* Q, const 
  *   out [n_q, Ha, 128] fp32 (16-byte aligned); lse [n_q, Ha] or NULL;
  *   status: a device word for HISA_DEV_TIMEOUT; all device memory, caller
  *   owned.  Workspace: hisa_sparse_attn_workspace_bytes(n_q, k).
- * Numerics: Qa Kc^T on the bf16 tensor cores into fp32, softmax weights in
- * fp32 rounded to bf16 for the weights-times-values product (fp32
- * accumulate); the sum of weights is taken over the rounded weights.
+ * Numerics: Qa Kc^T on the bf16 tensor cores into fp32; softmax weights in
+ * fp32 (hardware 2^x, about 2^-22 relative), rounded to bf16 for the
+ * weights-times-values product (fp32 accumulate); the normalising sum is
+ * taken over the fp32 weights.  Each output is then within 2^-9 (plus fp32
+ * rounding) of max |v| over the row's entries of the exact value.
  * Errors: HISA_E_INVAL (sizes, pointers, alignment, scale not finite and
  * positive), HISA_E_UNSUPPORTED (d != 128, Ha outside 1..128),
  * HISA_E_WORKSPACE, HISA_E_CUDA.

@@ -1,11 +1,11 @@
 """Sparse attention over selected tokens against the oracle (plain definition
 in double).  Tolerance from the arithmetic: the logits are exact bf16
-products summed in fp32; the softmax weights are rounded to bf16 (relative
-error <= 2^-9 each) before the weights-times-values product, and the sum of
-weights is taken over the same rounded weights, so each output is a convex
-combination of the selected value rows whose weights are off by at most
-about 2^-8 relative: |out - out_ref| <= 2^-8 * max |v| over the row's
-entries (plus fp32 accumulation), and |lse - lse_ref| <= 2^-8."""
+products summed in fp32; the softmax weights w_j (normalised by their fp32
+sum) are rounded to bf16 (relative error <= 2^-9 each) before the
+weights-times-values product, so out = sum_j w_j (1 + d_j) v_j with
+sum_j w_j = 1 and |d_j| <= 2^-9, and the hardware 2^x adds about 2^-22:
+|out - out_ref| <= 2^-9 * max |v| over the row's entries plus fp32
+accumulation; the tests allow 2^-8 * max |v| + 1e-5, and 2^-8 on lse."""
 import math
 
 import numpy as np
