@@ -490,8 +490,10 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectPara
 // Rows of up to kRowKeys slots: one CTA of kRowThreads, keys staged in shared
 // memory, the same four steps without any cross-CTA exchange.
 
-constexpr int kRowThreads = 512;
+constexpr int kRowThreads = 1024;
 constexpr int kRowWarps = kRowThreads / 32;
+constexpr int kRowBinsPer = kBins / kRowThreads;   // histogram bins each thread scans
+static_assert(kBins % kRowThreads == 0, "bins split evenly over the threads");
 
 constexpr int kRowBlocks = 2048;   // kept-block ids staged in shared memory
 
@@ -506,7 +508,7 @@ struct RowShared {
     uint32_t bc[8];
 };
 
-// Exclusive block scan of one value per thread (512 threads).
+// Exclusive block scan of one value per thread (kRowThreads threads).
 __device__ __forceinline__ uint32_t row_scan(uint32_t v, uint32_t* wtot, uint32_t* total) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint32_t incl = v;
@@ -677,18 +679,21 @@ __global__ void __launch_bounds__(kRowThreads) select_row_kernel(const SelectPar
                 if (x != 0u && x >= lo && x <= hi) atomicAdd(&sh.hist[(x - lo) >> shift], 1u);
             }
             __syncthreads();
-            // thread t owns bins 2047-4t .. 2044-4t (highest first)
-            const int b0 = kBins - 1 - 4 * tid;
-            const uint32_t h0 = sh.hist[b0], h1 = sh.hist[b0 - 1], h2 = sh.hist[b0 - 2], h3 = sh.hist[b0 - 3];
-            const uint32_t loc = h0 + h1 + h2 + h3;
+            // thread t owns kRowBinsPer consecutive bins from the top (highest first)
+            const int b0 = kBins - 1 - kRowBinsPer * tid;
+            uint32_t hs[kRowBinsPer], loc = 0;
+#pragma unroll
+            for (int q = 0; q < kRowBinsPer; ++q) {
+                hs[q] = sh.hist[b0 - q];
+                loc += hs[q];
+            }
             uint32_t tot;
             const uint32_t excl = row_scan(loc, sh.wd, &tot);
             const uint32_t kr = static_cast<uint32_t>(krem);
             if (excl < kr && kr <= excl + loc) {
-                const uint32_t hs[4] = {h0, h1, h2, h3};
                 uint32_t run = excl;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
+                for (int q = 0; q < kRowBinsPer; ++q) {
                     if (run < kr && kr <= run + hs[q]) {
                         sh.bc[0] = static_cast<uint32_t>(b0 - q);
                         sh.bc[1] = kr - run;
