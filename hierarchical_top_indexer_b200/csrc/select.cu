@@ -487,28 +487,29 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectPara
 
 // ------------------------------------------------ single-CTA rows
 //
-// Rows of up to kRowKeys slots: one CTA of kRowThreads, keys staged in shared
+// Rows of up to kRowKeys slots: one CTA of NT threads, keys staged in shared
 // memory, the same four steps without any cross-CTA exchange.
 
-constexpr int kRowThreads = 1024;
-constexpr int kRowWarps = kRowThreads / 32;
-constexpr int kRowBinsPer = kBins / kRowThreads;   // histogram bins each thread scans
-static_assert(kBins % kRowThreads == 0, "bins split evenly over the threads");
+// The kernel is instantiated for 1024 threads (rows up to two per SM: more
+// warps per row shorten each phase) and 512 (many rows: more CTAs per SM).
 
 constexpr int kRowBlocks = 2048;   // kept-block ids staged in shared memory
 
+template <int NT>
 struct RowShared {
+    static constexpr int kWarps = NT / 32;
     int32_t blk[kRowBlocks];
     uint32_t hist[kBins];
     unsigned long long members[kMembersCap];
-    uint32_t wa[kRowWarps];
-    uint32_t wb[kRowWarps];
-    uint32_t wc[kRowWarps];
-    uint32_t wd[kRowWarps];
+    uint32_t wa[kWarps];
+    uint32_t wb[kWarps];
+    uint32_t wc[kWarps];
+    uint32_t wd[kWarps];
     uint32_t bc[8];
 };
 
-// Exclusive block scan of one value per thread (kRowThreads threads).
+// Exclusive block scan of one value per thread (NT threads).
+template <int NT>
 __device__ __forceinline__ uint32_t row_scan(uint32_t v, uint32_t* wtot, uint32_t* total) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint32_t incl = v;
@@ -521,7 +522,7 @@ __device__ __forceinline__ uint32_t row_scan(uint32_t v, uint32_t* wtot, uint32_
     __syncthreads();
     uint32_t before = 0, tot = 0;
 #pragma unroll
-    for (int w = 0; w < kRowWarps; ++w) {
+    for (int w = 0; w < NT / 32; ++w) {
         const uint32_t x = wtot[w];
         before += w < warp ? x : 0u;
         tot += x;
@@ -530,9 +531,14 @@ __device__ __forceinline__ uint32_t row_scan(uint32_t v, uint32_t* wtot, uint32_
     return before + incl - v;
 }
 
-__global__ void __launch_bounds__(kRowThreads) select_row_kernel(const SelectParams p) {
+template <int NT>
+__global__ void __launch_bounds__(NT) select_row_kernel(const SelectParams p) {
+    constexpr int kRowThreads = NT;
+    constexpr int kRowWarps = NT / 32;
+    constexpr int kRowBinsPer = kBins / NT;   // histogram bins each thread scans
+    static_assert(kBins % NT == 0, "bins split evenly over the threads");
     extern __shared__ uint32_t ks[];
-    __shared__ RowShared sh;
+    __shared__ RowShared<NT> sh;
     grid_dependency_wait();
     grid_launch_dependents();
     const int row = blockIdx.x;
@@ -688,7 +694,7 @@ __global__ void __launch_bounds__(kRowThreads) select_row_kernel(const SelectPar
                 loc += hs[q];
             }
             uint32_t tot;
-            const uint32_t excl = row_scan(loc, sh.wd, &tot);
+            const uint32_t excl = row_scan<NT>(loc, sh.wd, &tot);
             const uint32_t kr = static_cast<uint32_t>(krem);
             if (excl < kr && kr <= excl + loc) {
                 uint32_t run = excl;
@@ -855,14 +861,15 @@ __global__ void __launch_bounds__(kRowThreads) select_row_kernel(const SelectPar
     }
 }
 
-cudaError_t launch_row(const SelectParams& p, int max_n, cudaStream_t s) {
+template <int NT>
+cudaError_t launch_row_t(const SelectParams& p, int max_n, cudaStream_t s) {
     const size_t smem = static_cast<size_t>(max_n > 4 ? max_n : 4) * sizeof(uint32_t);
-    cudaError_t e = cudaFuncSetAttribute(select_row_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(select_row_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(p.rows));
-    cfg.blockDim = dim3(kRowThreads);
+    cfg.blockDim = dim3(NT);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
@@ -870,7 +877,11 @@ cudaError_t launch_row(const SelectParams& p, int max_n, cudaStream_t s) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, select_row_kernel, p);
+    return cudaLaunchKernelEx(&cfg, select_row_kernel<NT>, p);
+}
+
+cudaError_t launch_row(const SelectParams& p, int max_n, int sms, cudaStream_t s) {
+    return p.rows <= 2 * sms ? launch_row_t<1024>(p, max_n, s) : launch_row_t<512>(p, max_n, s);
 }
 
 template <bool STAGE>
@@ -962,7 +973,7 @@ cudaError_t launch_select(const SelectParams& p, int max_n, int sms, cudaStream_
     if (p.rows <= 0) return cudaSuccess;
     if ((p.mode == kSelCpBlocks || p.mode == kSelMerge) && max_n > kRowKeys) return cudaErrorInvalidValue;
     if (max_n <= kRowKeys) {
-        const cudaError_t e = launch_row(p, max_n, s);
+        const cudaError_t e = launch_row(p, max_n, sms, s);
         return e == cudaSuccess ? cudaGetLastError() : e;
     }
     // cluster size: enough CTAs to stage the longest row, and more while
