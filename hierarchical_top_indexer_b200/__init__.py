@@ -127,6 +127,9 @@ def _stream(stream=None):
 
 
 def _dev(x, dtype, device):
+    if isinstance(x, torch.Tensor) and x.dtype == dtype and x.is_cuda and x.is_contiguous() and \
+            x.device.index == (device.index if device.index is not None else torch.cuda.current_device()):
+        return x
     if not isinstance(x, torch.Tensor):
         x = torch.as_tensor(x)
     if x.dtype != dtype:
@@ -241,8 +244,8 @@ def hisa_select(kv: KVCache, Q, w, q_seq, q_pos, m: int, k: int, want_scores: bo
     """Two-stage HISA selection.  Returns idx [n_q, k] (and scores if asked)."""
     Q, w, q_seq, q_pos = _queries(kv, Q, w, q_seq, q_pos)
     n_q, H = Q.shape[0], Q.shape[1]
-    need = hisa_select_workspace_bytes(kv, n_q, H, m, k)
-    ws = workspace(need, kv.device) if ws is None else ws
+    if ws is None:
+        ws = workspace(hisa_select_workspace_bytes(kv, n_q, H, m, k), kv.device)
     idx = torch.empty((n_q, k), dtype=torch.int32, device=kv.device) if idx is None else idx
     if want_scores and scores is None:
         scores = torch.empty((n_q, k), dtype=torch.float32, device=kv.device)

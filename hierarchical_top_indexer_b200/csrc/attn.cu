@@ -575,7 +575,7 @@ cudaError_t launch_attn(const AttnParams& p, int sms, cudaStream_t s) {
     if (p.n_q <= 0) return cudaSuccess;
     const long long tiles = static_cast<long long>(p.n_q) * p.T;
     const int grid = static_cast<int>(tiles < sms ? tiles : sms);
-    cudaError_t e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem);
+    cudaError_t e = smem_limit(reinterpret_cast<const void*>(attn_kernel), kAttnSmem);
     if (e != cudaSuccess) return e;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

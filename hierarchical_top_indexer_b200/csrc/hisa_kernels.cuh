@@ -1,6 +1,10 @@
 // Internal interface between the C-ABI layer (api.cu) and the kernels.
 #pragma once
 
+#include <map>
+#include <mutex>
+#include <utility>
+
 #include "hisa_device.cuh"
 
 namespace hisa {
@@ -197,6 +201,28 @@ struct AttnParams {
 size_t attn_workspace_bytes(int n_q, int k);
 void attn_carve(AttnParams& p, void* ws);
 cudaError_t launch_attn(const AttnParams& p, int sms, cudaStream_t s);
+
+// Raise a kernel's dynamic shared-memory limit to at least `bytes` on the
+// current device, once: the attribute call costs microseconds of host time,
+// so it is made only the first time a kernel needs a larger limit there.
+inline cudaError_t smem_limit(const void* fn, size_t bytes) {
+    static std::mutex mu;
+    static std::map<std::pair<const void*, int>, size_t> have;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    {
+        std::lock_guard<std::mutex> g(mu);
+        const auto it = have.find({fn, dev});
+        if (it != have.end() && it->second >= bytes) return cudaSuccess;
+    }
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> g(mu);
+    size_t& h = have[{fn, dev}];
+    if (h < bytes) h = bytes;
+    return cudaSuccess;
+}
 
 cudaError_t launch_pool(const KvView& kv, cudaStream_t s);
 cudaError_t launch_append(const KvView& kv, const void* tok, const float* tok_scale,

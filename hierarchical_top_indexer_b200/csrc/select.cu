@@ -864,8 +864,7 @@ __global__ void __launch_bounds__(NT) select_row_kernel(const SelectParams p) {
 template <int NT>
 cudaError_t launch_row_t(const SelectParams& p, int max_n, cudaStream_t s) {
     const size_t smem = static_cast<size_t>(max_n > 4 ? max_n : 4) * sizeof(uint32_t);
-    cudaError_t e = cudaFuncSetAttribute(select_row_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    cudaError_t e = smem_limit(reinterpret_cast<const void*>(select_row_kernel<NT>), smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(p.rows));
@@ -888,8 +887,7 @@ template <bool STAGE>
 cudaError_t launch_t(const SelectParams& p, int csize, int chunk, cudaStream_t s) {
     const size_t smem = STAGE ? static_cast<size_t>(chunk) * sizeof(uint32_t) : 0;
     auto* fn = select_kernel<STAGE>;
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    cudaError_t e = smem_limit(reinterpret_cast<const void*>(fn), smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(p.rows * csize));
