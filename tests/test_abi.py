@@ -197,3 +197,27 @@ def test_merge_checks(hisa):
     assert lib.hisa_merge_topk(None, P(16), 2, 4, 8, 4, P(16), None, None) == hisa.HISA_E_INVAL
     assert lib.hisa_merge_topk(P(16), P(16), 4, 4, 8192, 4, P(16), None, None) == hisa.HISA_E_UNSUPPORTED
     assert lib.hisa_merge_topk(P(16), P(16), 2, 0, 8, 4, P(16), None, None) == hisa.HISA_OK
+
+
+def test_sparse_attention_checks(hisa):
+    lib = hisa.lib()
+    P = ctypes.c_void_p
+    ok = dict(Qa=P(16), Ha=128, Kc=P(16), Vc=P(16), len=P(16), batch=2, cap=64, d=128, q_seq=P(16),
+              idx=P(16), n_q=4, k=32, scale=0.1, out=P(16), lse=None, status=P(16), ws=P(256),
+              ws_bytes=1 << 30, stream=None)
+
+    def call(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return lib.hisa_sparse_attn(*a.values())
+    assert lib.hisa_sparse_attn_workspace_bytes(4, 32) > 0
+    assert lib.hisa_sparse_attn_workspace_bytes(4, 0) == 0
+    assert call(d=64) == hisa.HISA_E_UNSUPPORTED
+    assert call(Ha=129) == hisa.HISA_E_UNSUPPORTED
+    assert call(scale=0.0) == hisa.HISA_E_INVAL
+    assert call(scale=float("inf")) == hisa.HISA_E_INVAL
+    assert call(k=0) == hisa.HISA_E_INVAL
+    assert call(idx=None) == hisa.HISA_E_INVAL
+    assert call(out=P(20)) == hisa.HISA_E_INVAL              # output rows need 16-byte alignment
+    assert call(ws_bytes=16) == hisa.HISA_E_WORKSPACE
+    assert call(n_q=0, Qa=None) == hisa.HISA_OK
