@@ -1,4 +1,4 @@
-"""Context-parallel selection across two gloo ranks on CPU, as torchrun would
+"""Context-parallel selection across two and three gloo ranks on CPU, as torchrun would
 start them.  Each rank holds one token-range shard of every sequence, and
 hisa_cp_select's exchange (two all-gathers of (id, score) lists in rank order,
 each merged by the rule score desc, id asc) must hand every rank the selection
@@ -16,7 +16,12 @@ import numpy as np
 import torch.multiprocessing as mp
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-B, LR, M, K = 64, 512, 4, 64
+B, M, K = 64, 4, 64
+
+
+def _shard_len(world):
+    """Shards on block boundaries that together cover the 1024-token sequence."""
+    return -(-1024 // (world * B)) * B
 
 
 def _case():
@@ -34,11 +39,12 @@ def _free_port():
 class ShardSteps:
     """numpy stand-ins for the three library calls on the shard at tok_off."""
 
-    def __init__(self, case, tok_off):
+    def __init__(self, case, tok_off, lr):
         from hisa_inputs import bf16_to_f32
         self.keys = bf16_to_f32(case.keys).astype(np.float64)      # [batch, cap, d]
         self.tok_off = tok_off
-        self.n = np.clip(case.lens.astype(np.int64), tok_off, tok_off + LR) - tok_off
+        self.lr = lr
+        self.n = np.clip(case.lens.astype(np.int64), tok_off, tok_off + lr) - tok_off
 
     def _score(self, Q, w, x):
         return float((np.maximum(Q @ x, 0.0) * w).sum())
@@ -50,7 +56,7 @@ class ShardSteps:
             return 0, 0
         if tl < n:
             return tl // B + 1, 1
-        return (LR // B, 0) if n == LR else None
+        return (self.lr // B, 0) if n == self.lr else None
 
     def blocks(self, kv, tok_off, Q, w, qs, qp, m, ws=None):
         import torch
@@ -122,18 +128,23 @@ def _rank_main(rank, world, port, out_dir):
     import hierarchical_top_indexer_b200 as hisa
     dist.init_process_group("gloo", rank=rank, world_size=world)
     case = _case()
-    steps = ShardSteps(case, rank * LR)
+    lr = _shard_len(world)
+    steps = ShardSteps(case, rank * lr, lr)
     hisa.hisa_cp_blocks, hisa.hisa_cp_tokens, hisa.hisa_merge_topk = steps.blocks, steps.tokens, steps.merge
     from hisa_inputs import bf16_to_f32
     Q = torch.from_numpy(bf16_to_f32(case.Q))
-    idx, sc = hisa.hisa_cp_select(None, rank * LR, Q, torch.from_numpy(case.w),
+    idx, sc = hisa.hisa_cp_select(None, rank * lr, Q, torch.from_numpy(case.w),
                                   torch.from_numpy(case.q_seq), torch.from_numpy(case.q_pos), M, K)
     dist.destroy_process_group()
     with open(os.path.join(out_dir, f"rank{rank}.json"), "w") as f:
         json.dump({"idx": idx.tolist()}, f)
 
 
-def test_two_rank_exchange_gives_the_whole_sequence_selection(tmp_path):
+import pytest
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_rank_exchange_gives_the_whole_sequence_selection(tmp_path, world):
     sys.path.insert(0, ROOT)
     from tests.test_abi import build_module
     build = build_module()
@@ -141,9 +152,9 @@ def test_two_rank_exchange_gives_the_whole_sequence_selection(tmp_path):
         build.build()
     import oracle
     case = _case()
-    mp.start_processes(_rank_main, args=(2, _free_port(), str(tmp_path)), nprocs=2, join=True,
+    mp.start_processes(_rank_main, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True,
                        start_method="spawn")
-    got = [np.array(json.load(open(tmp_path / f"rank{r}.json"))["idx"]) for r in range(2)]
+    got = [np.array(json.load(open(tmp_path / f"rank{r}.json"))["idx"]) for r in range(world)]
     ora = oracle.hisa_select(oracle.Cache.of(case), case.Q, case.w, case.q_seq, case.q_pos, B, M, K)
     for g in got:
         np.testing.assert_array_equal(g, ora["idx"])

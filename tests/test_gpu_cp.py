@@ -158,3 +158,33 @@ def _pooled(case):
     kv = h.KVCache.from_case(case)
     h.hisa_pool_blocks(kv)
     return kv
+
+
+@pytest.mark.parametrize("lists,n,k", [(3, 50, 40), (2, 128, 300), (4, 7, 5)])
+def test_merge_rule_by_definition(lists, n, k):
+    """hisa_merge_topk against a sort by (score desc, id asc) of the non-empty
+    entries, with exact ties across lists, empty entries and k above the count."""
+    rng = np.random.default_rng(lists * 100 + n)
+    rows = 6
+    ids = np.full((lists, rows, n), -1, np.int32)
+    sc = np.zeros((lists, rows, n), np.float32)
+    for r in range(rows):
+        base = 0
+        for l in range(lists):
+            cnt = int(rng.integers(0, n + 1))
+            ids[l, r, :cnt] = base + np.sort(rng.choice(1000, cnt, replace=False))
+            sc[l, r, :cnt] = rng.integers(0, 6, cnt).astype(np.float32) * 0.5   # many exact ties
+            base += 1000                                                       # list ranges ascend
+    h = lib()
+    idx, out = h.hisa_merge_topk(torch.from_numpy(ids).cuda(), torch.from_numpy(sc).cuda(), k)
+    torch.cuda.synchronize()
+    idx, out = idx.cpu().numpy(), out.cpu().numpy()
+    for r in range(rows):
+        ent = sorted((-float(sc[l, r, j]), int(ids[l, r, j])) for l in range(lists) for j in range(n)
+                     if ids[l, r, j] >= 0)[:k]
+        want = sorted(g for _, g in ent)
+        got = [g for g in idx[r] if g >= 0]
+        assert got == want
+        assert np.all(idx[r, len(want):] == -1) and np.all(np.isnan(out[r, len(want):]))
+        score_of = {g: -s for s, g in ent}
+        assert all(out[r, i] == score_of[g] for i, g in enumerate(got))
