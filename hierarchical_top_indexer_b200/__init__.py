@@ -41,7 +41,8 @@ EXPORTS = ("hisa_pool_blocks", "hisa_append", "hisa_select_workspace_bytes", "hi
            "hisa_tree_select", "hisa_pool_tail", "hisa_cp_workspace_bytes", "hisa_cp_blocks",
            "hisa_cp_tokens", "hisa_merge_topk", "hisa_sparse_attn_workspace_bytes", "hisa_sparse_attn",
            "dsa_flat_workspace_bytes", "dsa_flat_select", "hisa_topk_f32",
-           "hisa_profile_enable", "hisa_profile_read", "hisa_status_string", "hisa_last_cuda_error")
+           "hisa_profile_enable", "hisa_profile_read", "hisa_status_string", "hisa_last_cuda_error",
+           "hisa_selftest_wait")
 PHASES = ("block_score", "block_select", "token_score", "token_select", "flat_score",
           "flat_select", "pool", "append", "topk", "qsplit", "merge", "attn")
 
@@ -83,6 +84,8 @@ _lib.dsa_flat_workspace_bytes.argtypes = [_KVP, _I, _I, _I]
 _lib.dsa_flat_workspace_bytes.restype = _Z
 _lib.dsa_flat_select.argtypes = [_KVP, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _Z, _P]
 _lib.hisa_topk_f32.argtypes = [_P, _I, _I, _I, _P, _P]
+_lib.hisa_selftest_wait.argtypes = [_P, _P]
+_lib.hisa_selftest_wait.restype = _I
 _lib.hisa_profile_enable.argtypes = [_I]
 _lib.hisa_profile_read.argtypes = [_P, _P, _I]
 _lib.hisa_status_string.argtypes = [_I]
@@ -477,6 +480,12 @@ def hisa_cp_select(kv: KVCache, tok_off: int, Q, w, q_seq, q_pos, m: int, k: int
     kept, _ = hisa_merge_topk(_gather_ranks(ids, group), _gather_ranks(sc, group), m)
     tid, tsc = hisa_cp_tokens(kv, tok_off, Q, w, q_seq, q_pos, m, k, kept, ws=ws)
     return hisa_merge_topk(_gather_ranks(tid, group), _gather_ranks(tsc, group), k)
+
+
+def hisa_selftest_wait(status: torch.Tensor, stream=None):
+    """Launch one warp whose bounded wait must run out and set HISA_DEV_TIMEOUT
+    in `status` (int32 [1], device)."""
+    _check("hisa_selftest_wait", _lib.hisa_selftest_wait(_ptr(status), _stream(stream)))
 
 
 def hisa_profile_enable(on: bool = True):

@@ -852,6 +852,11 @@ int hisa_sparse_attn(const uint16_t* Qa, int Ha, const uint16_t* Kc, const uint1
     return cuda_status(launch_attn(p, sms, s));
 }
 
+int hisa_selftest_wait(uint32_t* status, hisa_stream_t stream) {
+    if (!status || !aligned(status, 4)) return HISA_E_INVAL;
+    return cuda_status(launch_wait_probe(status, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int hisa_pool_tail(const hisa_kv* kv, hisa_stream_t stream) {
     KvView v;
     const int rc = check_kv(kv, &v);

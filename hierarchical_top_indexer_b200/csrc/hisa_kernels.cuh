@@ -202,6 +202,9 @@ size_t attn_workspace_bytes(int n_q, int k);
 void attn_carve(AttnParams& p, void* ws);
 cudaError_t launch_attn(const AttnParams& p, int sms, cudaStream_t s);
 
+// One warp waiting on an mbarrier that never completes (diag.cu).
+cudaError_t launch_wait_probe(uint32_t* status, cudaStream_t s);
+
 // Raise a kernel's dynamic shared-memory limit to at least `bytes` on the
 // current device, once: the attribute call costs microseconds of host time,
 // so it is made only the first time a kernel needs a larger limit there.

@@ -404,6 +404,16 @@ enum hisa_phase {
 int hisa_profile_enable(int on);
 int hisa_profile_read(float* ms, int* launches, int reset);
 
+/*
+ * hisa_selftest_wait — failure detection check (no counterpart on the pages).
+ * Launches one warp that waits on an mbarrier nothing completes, with the
+ * same bounded wait every library kernel uses: after its 2 s limit the wait
+ * gives up, HISA_DEV_TIMEOUT is OR-ed into the device word `status`, and the
+ * kernel returns, leaving the context usable.  No fault, trap or hang is
+ * involved.  HISA_E_INVAL for a NULL or unaligned status.
+ */
+int hisa_selftest_wait(uint32_t* status, hisa_stream_t stream);
+
 /* Human-readable name of a return code. */
 const char* hisa_status_string(int code);
 
