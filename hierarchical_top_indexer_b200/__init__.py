@@ -474,8 +474,9 @@ def hisa_cp_select(kv: KVCache, tok_off: int, Q, w, q_seq, q_pos, m: int, k: int
                    ws: Optional[torch.Tensor] = None):
     """Context-parallel hisa_select on the current stream: this rank holds the
     shard at tok_off, the ranks of `group` hold ascending shards in rank
-    order.  Two all-gathers of (id, score) pairs; the result (idx, scores)
-    equals hisa_select's on the whole sequence, on every rank."""
+    order.  Every rank passes the same query rows (Q, w, q_seq, global q_pos)
+    and the same m and k.  Two all-gathers of (id, score) pairs; the result
+    (idx, scores) equals hisa_select's on the whole sequence, on every rank."""
     ids, sc = hisa_cp_blocks(kv, tok_off, Q, w, q_seq, q_pos, m, ws=ws)
     kept, _ = hisa_merge_topk(_gather_ranks(ids, group), _gather_ranks(sc, group), m)
     tid, tsc = hisa_cp_tokens(kv, tok_off, Q, w, q_seq, q_pos, m, k, kept, ws=ws)

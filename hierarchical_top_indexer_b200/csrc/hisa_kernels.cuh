@@ -208,6 +208,9 @@ cudaError_t launch_wait_probe(uint32_t* status, cudaStream_t s);
 // Raise a kernel's dynamic shared-memory limit to at least `bytes` on the
 // current device, once: the attribute call costs microseconds of host time,
 // so it is made only the first time a kernel needs a larger limit there.
+// (A cudaDeviceReset discards the attribute but not this record; a process
+// that resets a device it keeps using would see the next large launch fail
+// with an invalid-value error.)
 inline cudaError_t smem_limit(const void* fn, size_t bytes) {
     static std::mutex mu;
     static std::map<std::pair<const void*, int>, size_t> have;
