@@ -36,6 +36,15 @@ WORKLOAD = dict(cfg=1, name="decode-32k-b64")
 L2_FLUSH_BYTES = 256 << 20
 
 
+def iou(a_row, b_row) -> float:
+    """|A & B| / |A | B| of two index rows, -1 padding excluded."""
+    a = set(int(v) for v in a_row if v >= 0)
+    b = set(int(v) for v in b_row if v >= 0)
+    if not a and not b:
+        return 1.0
+    return len(a & b) / len(a | b)
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -288,7 +297,6 @@ def run_gpu(args, rank, world):
     flat_ms = time_calls(lambda: hisa.dsa_flat_select(kv, qc, wc, q_seq, None, k,
                                                       ws=fws, idx=fidx), n_flat)
     torch.cuda.synchronize()
-    from tests.parity import iou
     hi, fi = hidx.cpu().numpy(), fidx.cpu().numpy()
     mean_iou = float(np.mean([iou(a, b) for a, b in zip(hi, fi)]))
 
@@ -386,7 +394,6 @@ def run_workloads(args, dev, peaks):
     import torch
     import hierarchical_top_indexer_b200 as hisa
     from hisa_inputs import make_config
-    from tests.parity import iou
 
     stream = torch.cuda.current_stream()
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -553,7 +560,6 @@ def run_tree(case, dev, n, flush, stream, two_level_ms):
     on one workload: select time, work per row and mean IoU."""
     import torch
     import hierarchical_top_indexer_b200 as hisa
-    from tests.parity import iou
 
     kv = hisa.KVCache.from_case(case, device=dev)
     hisa.hisa_pool_blocks(kv)

@@ -221,11 +221,20 @@ def hisa_append(kv: KVCache, tok: torch.Tensor, tok_scale: Optional[torch.Tensor
 
 
 def _queries(kv, Q, w, q_seq, q_pos):
-    Q = _dev(Q, torch.bfloat16, kv.device)
-    w = _dev(w, torch.float32, kv.device)
-    q_seq = _dev(q_seq, torch.int32, kv.device)
-    q_pos = None if q_pos is None else _dev(q_pos, torch.int32, kv.device)
+    dev = kv.keys.device
+    Q = _dev(Q, torch.bfloat16, dev)
+    w = _dev(w, torch.float32, dev)
+    q_seq = _dev(q_seq, torch.int32, dev)
+    q_pos = None if q_pos is None else _dev(q_pos, torch.int32, dev)
     return Q, w, q_seq, q_pos
+
+
+def _check_ws(fn: str, kv, ws: Optional[torch.Tensor]):
+    """A caller's workspace: its byte size is passed as numel(), so it must be
+    a contiguous byte tensor on the cache's device."""
+    if ws is not None and (ws.dtype != torch.uint8 or not ws.is_contiguous()
+                           or ws.device != kv.keys.device):
+        raise ValueError(f"{fn}: ws must be a contiguous uint8 tensor on {kv.keys.device}")
 
 
 def hisa_select_workspace_bytes(kv: KVCache, n_q: int, H: int, m: int, k: int) -> int:
@@ -249,6 +258,8 @@ def hisa_select(kv: KVCache, Q, w, q_seq, q_pos, m: int, k: int, want_scores: bo
     n_q, H = Q.shape[0], Q.shape[1]
     if ws is None:
         ws = workspace(hisa_select_workspace_bytes(kv, n_q, H, m, k), kv.device)
+    _check_out("hisa_select", kv, n_q, k, idx, scores)
+    _check_ws("hisa_select", kv, ws)
     idx = torch.empty((n_q, k), dtype=torch.int32, device=kv.device) if idx is None else idx
     if want_scores and scores is None:
         scores = torch.empty((n_q, k), dtype=torch.float32, device=kv.device)
@@ -276,24 +287,52 @@ def hisa_select_inspect(kv: KVCache, Q, w, q_seq, q_pos, m: int, k: int, stream=
     return dict(idx=idx, scores=scores, blocks=blocks, nblocks=nblocks, counts=counts)
 
 
+def _same_device(t: torch.Tensor, kv: KVCache) -> bool:
+    return t.device == kv.keys.device
+
+
+def _check_out(fn: str, kv: KVCache, n_q: int, k: int, idx: Optional[torch.Tensor],
+               scores: Optional[torch.Tensor]):
+    """Caller-owned outputs: the library writes n_q * k entries to each, so a
+    short or misplaced buffer must be refused here, before any launch."""
+    for name, t, dt in (("idx", idx, torch.int32), ("scores", scores, torch.float32)):
+        if t is None:
+            continue
+        if t.dtype != dt or not t.is_contiguous() or not _same_device(t, kv):
+            raise ValueError(f"{fn}: {name} must be a contiguous {dt} tensor on {kv.keys.device}")
+        if t.numel() < n_q * k:
+            raise ValueError(f"{fn}: {name} holds {t.numel()} entries, needs n_q * k = {n_q * k}")
+
+
 def hisa_select_static(kv: KVCache, Q: torch.Tensor, w: torch.Tensor, q_seq: torch.Tensor,
                        q_pos: Optional[torch.Tensor], m: int, k: int, idx: torch.Tensor,
                        scores: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """hisa_select with the library's fixed scratch array instead of a workspace.
 
     Every tensor must already be on the cache's device with its final dtype and
-    layout (Q bf16 [n_q, H, d], w fp32 [n_q, H], q_seq / q_pos / idx int32,
-    scores fp32 or None): this wrapper converts and allocates nothing, and
-    neither does the library call.  Calls on one device share the scratch, so
-    they must be ordered on one stream."""
-    for t, dt in ((Q, torch.bfloat16), (w, torch.float32), (q_seq, torch.int32),
-                  (q_pos, torch.int32), (idx, torch.int32), (scores, torch.float32)):
-        if t is not None and (t.dtype != dt or t.device.type != kv.device.type
-                              or not t.is_contiguous()):
-            raise ValueError("hisa_select_static takes contiguous tensors of the final dtype "
-                             "on the cache's device")
+    layout (Q bf16 [n_q, H, d], w fp32 [n_q, H], q_seq / q_pos int32 [n_q], idx
+    int32 and scores fp32 (or None) of at least n_q * k entries): this wrapper
+    converts and allocates nothing, and neither does the library call.  It is
+    also the only guard of those shapes, since the C call cannot see tensor
+    sizes: anything else raises ValueError before the call.  Calls on one
+    device share the scratch, so they must be ordered on one stream."""
+    fn = "hisa_select_static"
+    for name, t, dt in (("Q", Q, torch.bfloat16), ("w", w, torch.float32), ("q_seq", q_seq, torch.int32),
+                        ("q_pos", q_pos, torch.int32)):
+        if t is not None and (t.dtype != dt or not t.is_contiguous() or not _same_device(t, kv)):
+            raise ValueError(f"{fn}: {name} must be a contiguous {dt} tensor on {kv.keys.device}")
+    if Q.dim() != 3 or Q.shape[2] != kv.d:
+        raise ValueError(f"{fn}: Q must be [n_q, H, {kv.d}], got {tuple(Q.shape)}")
     n_q, H = Q.shape[0], Q.shape[1]
-    _check("hisa_select_static", _lib.hisa_select_static(
+    if tuple(w.shape) != (n_q, H):
+        raise ValueError(f"{fn}: w must be [{n_q}, {H}], got {tuple(w.shape)}")
+    for name, t in (("q_seq", q_seq), ("q_pos", q_pos)):
+        if t is not None and t.numel() != n_q:
+            raise ValueError(f"{fn}: {name} must hold n_q = {n_q} entries, got {t.numel()}")
+    if idx is None:
+        raise ValueError(f"{fn}: idx is required (the call allocates nothing)")
+    _check_out(fn, kv, n_q, k, idx, scores)
+    _check(fn, _lib.hisa_select_static(
         kv.struct, _ptr(Q), _ptr(w), _ptr(q_seq), _ptr(q_pos), n_q, H, m, k, _ptr(idx),
         _ptr(scores), _stream(stream)))
     return idx
@@ -333,7 +372,9 @@ def hisa_tree_select(kv: KVCache, kv2: KVCache, Q, w, q_seq, q_pos, W: int, m: i
     blocks and the per-row work counters."""
     Q, w, q_seq, q_pos = _queries(kv, Q, w, q_seq, q_pos)
     n_q, H = Q.shape[0], Q.shape[1]
-    dev = kv.device
+    dev = kv.keys.device
+    _check_out("hisa_tree_select", kv, n_q, k, idx, None)
+    _check_ws("hisa_tree_select", kv, ws)
     ws = workspace(hisa_tree_workspace_bytes(kv, kv2, n_q, H, W, m, k), dev) if ws is None else ws
     idx = torch.empty((n_q, k), dtype=torch.int32, device=dev) if idx is None else idx
     out = {}
@@ -363,6 +404,8 @@ def dsa_flat_select(kv: KVCache, Q, w, q_seq, q_pos, k: int, want_scores: bool =
     n_q, H = Q.shape[0], Q.shape[1]
     need = dsa_flat_workspace_bytes(kv, n_q, H, k)
     ws = workspace(need, kv.device) if ws is None else ws
+    _check_out("dsa_flat_select", kv, n_q, k, idx, scores)
+    _check_ws("dsa_flat_select", kv, ws)
     idx = torch.empty((n_q, k), dtype=torch.int32, device=kv.device) if idx is None else idx
     if want_scores and scores is None:
         scores = torch.empty((n_q, k), dtype=torch.float32, device=kv.device)
@@ -391,6 +434,7 @@ def hisa_cp_blocks(kv: KVCache, tok_off: int, Q, w, q_seq, q_pos, m: int,
     [n_q, m]); the own block, on the shard holding the query, scores +inf."""
     Q, w, q_seq, q_pos = _queries(kv, Q, w, q_seq, q_pos)
     n_q, H = Q.shape[0], Q.shape[1]
+    _check_ws("hisa_cp_blocks", kv, ws)
     ws = workspace(hisa_cp_workspace_bytes(kv, tok_off, n_q, H, m, 1), kv.device) if ws is None else ws
     ids = torch.empty((n_q, m), dtype=torch.int32, device=kv.device)
     sc = torch.empty((n_q, m), dtype=torch.float32, device=kv.device)
@@ -406,6 +450,7 @@ def hisa_cp_tokens(kv: KVCache, tok_off: int, Q, w, q_seq, q_pos, m: int, k: int
     (idx [n_q, k] global token indices, scores [n_q, k])."""
     Q, w, q_seq, q_pos = _queries(kv, Q, w, q_seq, q_pos)
     n_q, H = Q.shape[0], Q.shape[1]
+    _check_ws("hisa_cp_tokens", kv, ws)
     ws = workspace(hisa_cp_workspace_bytes(kv, tok_off, n_q, H, m, k), kv.device) if ws is None else ws
     kept = _dev(kept, torch.int32, kv.device)
     idx = torch.empty((n_q, k), dtype=torch.int32, device=kv.device)

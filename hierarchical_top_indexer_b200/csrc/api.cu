@@ -2,7 +2,6 @@
 // layout, TMA tensor maps and kernel launches.  No allocation happens here:
 // every buffer belongs to the caller, and so does the scratch space, except
 // for hisa_select_static, whose scratch is one fixed device array below.
-#include <atomic>
 #include <climits>
 #include <cmath>
 #include <cstring>
@@ -500,28 +499,60 @@ int check_tree(const hisa_kv* kv, const hisa_kv* kv2, KvView* v, KvView* v2) {
 }
 
 // Scratch of hisa_select_static: a file-scope device array, one per device
-// (the runtime gives every device its own copy when it loads this module).
-// Its address is looked up once per device and cached.
+// (the runtime gives every device's context its own copy when it loads this
+// module).  Its address is looked up once per device context and cached with
+// that context's unique id, so a context re-created after a cudaDeviceReset
+// gets a fresh lookup instead of a dangling address.
 static __device__ __align__(256) uint8_t g_static_scratch[HISA_STATIC_SCRATCH_BYTES];
 
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+template <class Fn>
+Fn driver_fn(const char* name) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+        return nullptr;
+    return reinterpret_cast<Fn>(p);
+}
+
+// Unique id of the calling thread's current context (0 if there is none yet).
+unsigned long long current_ctx_id() {
+    static CtxGetCurrentFn get_ctx = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+    static CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_ctx || !get_id || get_ctx(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
+
 constexpr int kMaxDevices = 64;
-std::atomic<void*> g_static_scratch_ptr[kMaxDevices];
+struct StaticScratchSlot {
+    unsigned long long ctx_id = 0;
+    void* ptr = nullptr;
+};
+StaticScratchSlot g_static_scratch_slot[kMaxDevices];
 std::mutex g_static_scratch_mu;
 
 // Device address of the current device's copy of g_static_scratch.
 int static_scratch(void** out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HISA_E_CUDA;
-    void* p = g_static_scratch_ptr[dev].load(std::memory_order_acquire);
-    if (!p) {
-        std::lock_guard<std::mutex> lock(g_static_scratch_mu);
-        p = g_static_scratch_ptr[dev].load(std::memory_order_relaxed);
-        if (!p) {
-            if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return HISA_E_CUDA;
-            g_static_scratch_ptr[dev].store(p, std::memory_order_release);
-        }
+    std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+    StaticScratchSlot& slot = g_static_scratch_slot[dev];
+    const unsigned long long id = current_ctx_id();
+    if (id == 0 || id != slot.ctx_id || !slot.ptr) {
+        void* p = nullptr;   // the lookup creates the context if there is none yet
+        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return HISA_E_CUDA;
+        const unsigned long long now = current_ctx_id();
+        if (now == 0) return HISA_E_CUDA;
+        slot.ctx_id = now;
+        slot.ptr = p;
     }
-    *out = p;
+    *out = slot.ptr;
     return HISA_OK;
 }
 

@@ -16,9 +16,11 @@
 //   kScoreFlat    every key s <= t (the flat scan);
 //   kScoreHisa    the keys of the row's kept blocks (gathered block-wise by
 //                 TMA: a kept block is one or more contiguous tile rows).
-// e4m3 keys are staged as bytes, widened to bf16 in shared memory by four
-// converter warps (exact), and their per-token scale multiplies the score
-// (ReLU(s*x) = s*ReLU(x) for s > 0).
+// e4m3 keys with d = 128 are multiplied on the fp8 tensor cores as loaded
+// (kind::f8f6f4) against the query heads split into two e4m3 parts; e4m3 keys
+// with d = 64 are staged as bytes and widened to bf16 in shared memory by
+// four converter warps (exact).  Either way the per-token scale multiplies
+// the finished score (ReLU(s*x) = s*ReLU(x) for s > 0).
 //
 // Work split: the (row, tile) pairs are laid out row-major with a fixed
 // number of tile slots per row; CTA c takes the c-th contiguous range, so all
@@ -29,7 +31,7 @@
 //   warp 0       TMA producer (keys / representatives, query heads)
 //   warp 1       TMEM owner and UMMA issuer
 //   warps 2-5    epilogue (TMEM -> registers -> score key -> global)
-//   warps 6-9    e4m3 -> bf16 converters (e4m3 keys only)
+//   warps 6-9    e4m3 -> bf16 converters (e4m3 keys with d = 64 only)
 // Every mbarrier wait is bounded; on expiry the CTA raises HISA_DEV_TIMEOUT,
 // drains its outstanding copies and returns.
 #include "hisa_kernels.cuh"

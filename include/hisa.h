@@ -343,7 +343,10 @@ int hisa_merge_topk(const int32_t* ids, const float* scores, int lists, int rows
  *   Setup: the first call on a device, with that device current, looks up
  *   the array's device address (cudaGetSymbolAddress, which loads the
  *   library's device code if it is not loaded yet); later calls on that
- *   device reuse it.  Make that first call before any stream capture.
+ *   device reuse it while the device's context lives.  The address is kept
+ *   with the context's unique id: after a cudaDeviceReset the next call is a
+ *   first call again and looks the address up anew.  Make the first call on
+ *   a device (and the first after a reset) before any stream capture.
  *   Contents: nothing in the array needs to start at zero; every byte a call
  *   reads was written earlier in the same call.
  *   Races: all calls on one device share the one array.  Two calls whose

@@ -92,6 +92,27 @@ def hisa_row(keys, key_scale, dtype, Q, w, b, t, i, B, m, k, pool="mean"):
     return dict(idx=kept, scores=[val[s] for s in kept], blocks=chosen, block_scores=S)
 
 
+def refine_row(keys, key_scale, dtype, Q, w, b, t, i, B, k, blocks):
+    """Token-level refinement on a GIVEN list of block ids (any order, -1 for
+    an empty entry): slot r * B + o holds the exact score of token
+    blocks[r] * B + o when that token is visible (<= t), else None; idx is the
+    top-k of the visible slots by definition (ties: lower token index)."""
+    q, ww = query_values(Q, w, i)
+    cand, items = [], []
+    for j in blocks:
+        for o in range(B):
+            s = j * B + o
+            if j >= 0 and s <= t:
+                v = score(q, ww, key_values(keys, key_scale, dtype, b, s))
+                cand.append(v)
+                items.append((v, s))
+            else:
+                cand.append(None)
+    kept = keep_by_definition(items, k)
+    val = {s: v for v, s in items}
+    return dict(idx=kept, scores=[val[s] for s in kept], cand=cand)
+
+
 def flat_row(keys, key_scale, dtype, Q, w, b, t, i, k):
     q, ww = query_values(Q, w, i)
     cand = [(score(q, ww, key_values(keys, key_scale, dtype, b, s)), s) for s in range(t + 1)]

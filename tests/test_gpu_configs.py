@@ -6,7 +6,8 @@ import pytest
 import torch
 
 from hisa_inputs import make_config
-from tests.gpu_util import check_flat, check_hisa, device_case, lib, run_flat, run_hisa
+from tests.gpu_util import (AppendRecorder, check_flat, check_hisa, device_case, lib, run_flat,
+                            run_hisa)
 from tests.parity import iou
 
 pytestmark = pytest.mark.gpu
@@ -44,19 +45,23 @@ def test_config_parity(cfg, hisa_rows, flat_rows):
 
 def test_streaming_append_config():
     """512 appends at 128K: after every append, select for the new last
-    position; the incremental index must equal a re-pool, and the selections
-    must satisfy the parity rule against the oracle run on the grown cache."""
+    position.  Every step is checked: the block the append changed equals a
+    from-scratch re-pool of that block bit for bit (and the oracle's mean
+    within the pooled tolerance), and all 512 selections satisfy the parity
+    rule against the oracle, which pools the grown cache from scratch for
+    each row."""
     h = lib()
     case = make_config(4)
     steps = case.append_keys.shape[0]
     kv = device_case(case)
     L0 = int(case.lens[0])
-    idx_all, sc_all, blocks_all, nblk_all = [], [], [], []
+    idx_all, sc_all, blocks_all, nblk_all, counts_all = [], [], [], [], []
+    rec = AppendRecorder()
     qs = torch.zeros(1, dtype=torch.int32, device="cuda")
-    ws = h.workspace(h.hisa_select_workspace_bytes(kv, 1, case.H, case.m, case.k))
     for s in range(steps):
         tok = torch.from_numpy(case.append_keys[s].view(np.int16)).cuda()
         h.hisa_append(kv, tok)
+        rec.record(kv)
         Q = torch.from_numpy(case.append_Q[s].view(np.int16)).view(torch.bfloat16).cuda()
         w = torch.from_numpy(case.append_w[s]).cuda()
         r = h.hisa_select_inspect(kv, Q, w, qs, None, case.m, case.k)
@@ -64,8 +69,10 @@ def test_streaming_append_config():
         sc_all.append(r["scores"])
         blocks_all.append(r["blocks"])
         nblk_all.append(r["nblocks"])
+        counts_all.append(r["counts"])
     torch.cuda.synchronize()
     assert kv.len.item() == L0 + steps and kv.status_bits() == 0
+    assert rec.verify(kv) == steps                  # every append against a re-pool
     inc = kv.pooled.clone()
     h.hisa_pool_blocks(kv)
     torch.cuda.synchronize()
@@ -80,6 +87,13 @@ def test_streaming_append_config():
     grown.q_pos = (L0 + np.arange(steps)).astype(np.int32)
     gpu = dict(idx=torch.cat(idx_all).cpu().numpy(), scores=torch.cat(sc_all).cpu().numpy(),
                blocks=torch.cat(blocks_all).cpu().numpy(), nblocks=torch.cat(nblk_all).cpu().numpy())
-    rows = np.concatenate([np.arange(0, steps, 8), [steps - 1]])
+    rows = np.arange(steps)                          # all 512 steps
     _, swaps = check_hisa(grown, gpu, rows)
+    assert len(swaps) == steps
     assert sum(a + b for a, b in swaps) <= max(2, len(rows) // 8)
+    counts = torch.cat(counts_all).cpu().numpy()
+    for s in range(steps):
+        t = L0 + s
+        assert tuple(counts[s]) == (t // case.B + 1, min(case.m, t // case.B + 1) * case.B)
+    assert kv.status_bits() == 0
+    print(f"streaming: {steps}/{steps} steps checked against the oracle, {steps} appends re-pooled")

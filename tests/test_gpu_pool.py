@@ -5,48 +5,9 @@ import torch
 
 import oracle
 from hisa_inputs import bf16_bits, make_case
-from tests.gpu_util import device_case, lib
+from tests.gpu_util import AppendRecorder, check_pooled, device_case, lib
 
 pytestmark = pytest.mark.gpu
-
-
-def pooled_tol(case, ora_pooled, B):
-    """|delta| <= 1e-5 * (|mu| + mean|v|) per element: the fp32 sum of n <= B
-    terms is within about n * 2^-24 * sum|v| of the exact sum."""
-    from hisa_inputs import bf16_to_f32, e4m3_to_f32
-    if case.dtype == "bf16":
-        v = np.abs(bf16_to_f32(case.keys).astype(np.float64))
-    else:
-        v = np.abs((e4m3_to_f32(case.keys) * case.key_scale[..., None]).astype(np.float64))
-    mav = np.zeros_like(ora_pooled)
-    for b in range(case.batch):
-        n = int(case.lens[b])
-        for j in range(-(-n // B)):
-            mav[b, j] = v[b, j * B:min((j + 1) * B, n)].mean(0)
-    return 1e-5 * (np.abs(ora_pooled) + mav)
-
-
-def check_pooled(case, kv):
-    B = case.B
-    got = kv.pooled.cpu().numpy().astype(np.float64)
-    ora = oracle.pool(oracle.Cache.of(case), B)
-    tol = pooled_tol(case, ora, B)
-    for b in range(case.batch):
-        nbv = -(-int(case.lens[b]) // B)
-        d = np.abs(got[b, :nbv] - ora[b, :nbv])
-        assert np.all(d <= tol[b, :nbv]), f"seq {b}: max excess {(d - tol[b, :nbv]).max()}"
-    # hi/lo split of the fp32 mean
-    hl = kv.pooled_hl.view(torch.int16).cpu().numpy().view(np.uint16).astype(np.uint32)
-    hi = (hl[..., :case.d] << 16).view(np.float32)
-    lo = (hl[..., case.d:] << 16).view(np.float32)
-    g32 = kv.pooled.cpu().numpy()
-    for b in range(case.batch):
-        nbv = -(-int(case.lens[b]) // B)
-        assert np.array_equal(bf16_bits(g32[b, :nbv]), hl[b, :nbv, :case.d].astype(np.uint16))
-        assert np.array_equal(bf16_bits(g32[b, :nbv] - hi[b, :nbv]),
-                              hl[b, :nbv, case.d:].astype(np.uint16))
-        assert np.all(np.abs((hi + lo)[b, :nbv] - g32[b, :nbv]) <= 2.0 ** -15 * np.abs(g32[b, :nbv]) + 1e-30)
-    return ora
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
@@ -89,12 +50,15 @@ def test_append_equals_repool_bit_exact(dtype, B):
     case = make_case(batch=2, L=[1000, 640], H=2, d=128, B=B, m=4, k=8, dtype=dtype, seed=7,
                      append_steps=steps, cap=1400)
     kv = device_case(case)
+    rec = AppendRecorder()
     for s in range(steps):
         tok = torch.from_numpy(case.append_keys[s].view(np.int16 if dtype == "bf16" else np.uint8)).cuda()
         sc = None if dtype == "bf16" else torch.from_numpy(case.append_scale[s]).cuda()
         h.hisa_append(kv, tok, sc)
+        rec.record(kv)
     torch.cuda.synchronize()
     assert kv.len.cpu().tolist() == [1300, 940]
+    assert rec.verify(kv) == 2 * steps          # every append, both sequences
     inc_p = kv.pooled.clone()
     inc_hl = kv.pooled_hl.clone()
     h.hisa_pool_blocks(kv)            # from scratch over the grown cache
@@ -162,11 +126,14 @@ def test_append_equals_repool_max_pooling(dtype):
                      append_steps=steps, cap=1300)
     kv = h.KVCache.from_case(case, pool="max")
     h.hisa_pool_blocks(kv)
+    rec = AppendRecorder()
     for s in range(steps):
         tok = torch.from_numpy(case.append_keys[s].view(np.int16 if dtype == "bf16" else np.uint8)).cuda()
         sc = None if dtype == "bf16" else torch.from_numpy(case.append_scale[s]).cuda()
         h.hisa_append(kv, tok, sc)
+        rec.record(kv)
     torch.cuda.synchronize()
+    assert rec.verify(kv, pool="max") == 2 * steps
     inc = kv.pooled.clone()
     inc_hl = kv.pooled_hl.clone()
     h.hisa_pool_blocks(kv)

@@ -34,6 +34,10 @@ MUTANTS = {
                                        "skept[J->W - 1] = (int32_t)items[J->W - 1].i;"),
     "tree_children_skip_last": ("j < (long)(skept[r] + 1) * bf && j < nb - 1; ++j",
                                 "j < (long)(skept[r] + 1) * bf - 1 && j < nb - 1; ++j"),
+    "refine_cand_layout_transposed": ("if (cand) cand[(size_t)r * J->B + o] = v;",
+                                      "if (cand) cand[(size_t)o * J->mm + r] = v;"),
+    "refine_skips_last_given_block": ("for (int r = 0; r < nblk; ++r) {",
+                                      "for (int r = 0; r + 1 < nblk; ++r) {"),
     "attn_scale_dropped": ("a[j] = J->scale * z;", "a[j] = z;"),
     "attn_entries_past_len_kept": ("if (s < 0 || s >= n) { a[j] = NAN; continue; }",
                                    "if (s < 0) { a[j] = NAN; continue; }"),
@@ -72,6 +76,26 @@ def _pool_closed_form_fails(lib) -> bool:
     return False
 
 
+def _refine_fails(lib) -> bool:
+    c = make_case(batch=1, L=30, H=2, d=4, B=4, m=3, k=5, seed=313, positions=np.array([29, 17]))
+    cache = oracle.Cache.of(c)
+    given = [[2, -1, 7, 0], [4, 1, -1, 3]]       # row 0 (t = 29): own block 7 partial
+    r = oracle.hisa_refine(cache, c.Q, c.w, c.q_seq, c.q_pos, c.B, 5, np.array(given, np.int32),
+                           np.array([4, 4], np.int32), threads=1, lib=lib)
+    for i in range(c.n_q):
+        ref = brute.refine_row(c.keys, c.key_scale, c.dtype, c.Q, c.w, int(c.q_seq[i]),
+                               int(c.q_pos[i]), i, c.B, 5, given[i])
+        if [x for x in r["idx"][i] if x >= 0] != ref["idx"]:
+            return True
+        for slot, v in enumerate(ref["cand"]):
+            got = r["cand_scores"][i][slot]
+            if (v is None) != bool(np.isnan(got)):
+                return True
+            if v is not None and abs(got - float(v)) > 1e-12 * (1 + abs(float(v))):
+                return True
+    return False
+
+
 def _detects(lib) -> bool:
     """True if some pin rejects the library `lib`."""
     if _pool_closed_form_fails(lib):
@@ -95,6 +119,10 @@ def _detects(lib) -> bool:
             fref = brute.flat_row(c.keys, c.key_scale, c.dtype, c.Q, c.w, b, t, i, c.k)
             if [x for x in f["idx"][i] if x >= 0] != fref["idx"]:
                 return True
+    # refinement on given block lists (unsorted, -1 entries, the partial own
+    # block) against the exact brute force, candidate scores slot by slot
+    if _refine_fails(lib):
+        return True
     # max-pooled representatives against the exact brute force
     c = make_case(batch=1, L=24, H=2, d=4, B=4, m=2, k=5, seed=311, positions=np.array([23, 13]))
     cache = oracle.Cache.of(c)

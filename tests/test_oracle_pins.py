@@ -293,6 +293,68 @@ def test_refine_on_own_blocks_reproduces_select():
     assert np.array_equal(r["idx"], rr["idx"])
 
 
+def _given_block_sets(rng, nb_vis, nb_all, mm):
+    """Block lists a refinement may be handed (distinct ids, as every caller
+    gives): unsorted, with -1 entries, with blocks past the query position,
+    with the own (partial) block anywhere."""
+    own = nb_vis - 1
+    sets = []
+    perm = [int(j) for j in rng.permutation(nb_vis)[:mm]]
+    if own not in perm:
+        perm[-1] = own
+    sets.append(perm)                                        # unsorted, own block inside
+    holes = list(perm)
+    holes[0] = -1
+    if len(holes) > 2:
+        holes[len(holes) // 2] = -1
+    sets.append(holes)                                       # -1 entries between ids
+    future = [int(j) for j in rng.choice(nb_all - 1, size=min(mm, nb_all - 1) - 1, replace=False)]
+    future = [nb_all - 1] + future                           # wholly past t when t < its start
+    sets.append(future)
+    sets.append([own] + [-1] * (mm - 1))                     # only the partial own block
+    return sets
+
+
+@pytest.mark.parametrize("seed", range(5))
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+def test_refine_matches_exact_bruteforce_on_given_blocks(seed, dtype):
+    # Token-level refinement on a block set the oracle did not choose itself
+    # (the GPU's blocks in the token half of the parity rule): per slot
+    # r * B + o the exact score of token blocks[r] * B + o, NaN for -1
+    # entries and tokens past t; idx the top-k of the visible slots.
+    rng = np.random.default_rng(400 + seed)
+    B = int(rng.choice([2, 4, 8]))
+    L = int(rng.integers(3 * B + 1, 48))
+    nb_all = -(-L // B)
+    pos = np.unique(np.concatenate([rng.integers(B + 1, L, size=2), [L - 1]]))
+    c = make_case(batch=2, L=L, H=int(rng.integers(1, 4)), d=int(rng.choice([4, 8])), B=B, m=3,
+                  k=5, dtype=dtype, seed=450 + seed, positions=pos)
+    cache = oracle.Cache.of(c)
+    for i in range(c.n_q):
+        b, t = int(c.q_seq[i]), int(c.q_pos[i])
+        nb_vis = t // B + 1
+        mm = int(rng.integers(2, nb_vis + 1)) if nb_vis > 1 else 1
+        for blocks in _given_block_sets(rng, nb_vis, nb_all, max(mm, 2)):
+            for k in (1, int(rng.integers(2, 3 * B)), L + 3):
+                Qi, wi = c.Q[i:i + 1], c.w[i:i + 1]
+                r = oracle.hisa_refine(cache, Qi, wi, c.q_seq[i:i + 1], c.q_pos[i:i + 1], B, k,
+                                       np.array([blocks], np.int32), np.array([len(blocks)], np.int32),
+                                       threads=1)
+                ref = brute.refine_row(c.keys, c.key_scale, c.dtype, c.Q, c.w, b, t, i, B, k, blocks)
+                cs = r["cand_scores"][0]
+                assert cs.shape == (len(blocks) * B,)
+                for slot, v in enumerate(ref["cand"]):
+                    if v is None:
+                        assert np.isnan(cs[slot]), (slot, blocks, t)
+                    else:
+                        assert abs(cs[slot] - float(v)) <= 1e-12 * (1 + abs(float(v))), (slot, blocks)
+                got = [x for x in r["idx"][0] if x >= 0]
+                assert got == ref["idx"], (blocks, t, k)
+                assert list(r["idx"][0][len(got):]) == [-1] * (k - len(got))
+                np.testing.assert_allclose(r["score"][0][:len(got)], [float(v) for v in ref["scores"]],
+                                           rtol=1e-12, atol=1e-15)
+
+
 def test_topk_f32_rule_by_definition():
     rng = np.random.default_rng(3)
     x = rng.integers(-3, 4, size=(20, 37)).astype(np.float32) * 0.5   # many ties

@@ -1,7 +1,16 @@
 """hisa_select_static: the selection with the library's fixed scratch array in
-place of a caller workspace.  It runs the same kernels as hisa_select, so two
-calls in a row must reproduce hisa_select's output exactly, allocate no
-memory, and reject a request larger than the array before launching anything.
+place of a caller workspace, for callers that cannot allocate device memory
+while they select (an engine that has handed all free memory to its KV pages
+up front, or a C caller with no allocator).  It runs the same kernels as
+hisa_select, so calls in a row must reproduce hisa_select's output exactly,
+allocate no memory, and reject a request larger than the array before
+launching anything.
+
+"Allocates no memory" is checked two ways: torch's allocator counter, and
+the device's free memory (cudaMemGetInfo), which also sees any cudaMalloc or
+cudaMallocAsync the library itself might make.  The first call on a device
+looks up the array's address, which can load the library's device code, so
+the free-memory check brackets the calls after that first one.
 
 This file is collected last on purpose: the static array is shared by every
 call on the device, so the test also shows that earlier tests leave nothing
@@ -35,12 +44,16 @@ def test_static_scratch_matches_workspace_call(cfg):
     torch.cuda.synchronize()
     ref_idx, ref_sc = ref_idx.cpu().numpy(), ref_sc.cpu().numpy()
 
-    outs = [_outputs(case), _outputs(case)]
+    outs = [_outputs(case), _outputs(case), _outputs(case)]
     torch.cuda.synchronize()
     before = torch.cuda.memory_allocated()
-    for idx, sc in outs:
+    h.hisa_select_static(kv, Q, w, qs, qp, case.m, case.k, *outs[0])
+    torch.cuda.synchronize()
+    free_before = torch.cuda.mem_get_info()[0]
+    for idx, sc in outs[1:]:
         h.hisa_select_static(kv, Q, w, qs, qp, case.m, case.k, idx, sc)
     torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free_before
     assert torch.cuda.memory_allocated() == before
     for idx, sc in outs:
         got_idx, got_sc = idx.cpu().numpy(), sc.cpu().numpy()
