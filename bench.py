@@ -187,6 +187,23 @@ def traffic_record():
 # --------------------------------------------------------------------- GPU
 
 
+def capture_steps(fns, dev):
+    """One CUDA graph per step: fns[i]() is captured as it would run (the
+    library's launches, with their programmatic-launch edges), so replaying it
+    puts no host work between a step's kernels.  The library allocates and
+    synchronises nothing inside a call, so its calls capture as they are."""
+    import torch
+    cap = torch.cuda.Stream(dev)
+    graphs = []
+    for fn in fns:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            fn()
+        graphs.append(g)
+    torch.cuda.synchronize()
+    return graphs
+
+
 def run_gpu(args, rank, world):
     import torch
     import hierarchical_top_indexer_b200 as hisa
@@ -220,20 +237,22 @@ def run_gpu(args, rank, world):
     Qs = torch.from_numpy(case.append_Q.view(np.int16)).view(torch.bfloat16).to(dev)
     Ws = torch.from_numpy(case.append_w).to(dev)
     q_seq = torch.arange(batch, dtype=torch.int32, device=dev)
-    ws = hisa.workspace(hisa.hisa_select_workspace_bytes(kv, batch, H, m, k), dev)
+    ws = hisa.workspace(hisa.hisa_decode_step_workspace_bytes(kv, H, m, k), dev)
     idx = torch.empty((2, batch, k), dtype=torch.int32, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     nsets = Qs.shape[0]
 
     def step(s, out):
-        hisa.hisa_append(kv, toks[s])
-        hisa.hisa_select(kv, Qs[s % nsets], Ws[s % nsets], q_seq, None, m, k, ws=ws, idx=out)
+        # one decode step: every sequence's new key appended, then its new
+        # last position selected (hisa_decode_step = hisa_append + hisa_select)
+        hisa.hisa_decode_step(kv, toks[s], Qs[s % nsets], Ws[s % nsets], m, k, ws=ws, idx=out)
 
     for s in range(W):
         step(s, idx[s % 2])
         flush.fill_(7)
     torch.cuda.synchronize()
+    graphs = capture_steps([lambda s=W + i: step(s, idx[s % 2]) for i in range(K)], dev)
 
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(K)]
@@ -244,9 +263,8 @@ def run_gpu(args, rank, world):
     with ClockSampler(dev.index) as clk:
         wall0 = time.perf_counter()
         for i in range(K):
-            s = W + i
             ev[i][0].record(stream)
-            step(s, idx[s % 2])
+            graphs[i].replay()
             ev[i][1].record(stream)
             flush.fill_(7)
         torch.cuda.synchronize()
@@ -303,34 +321,7 @@ def run_gpu(args, rank, world):
     # end to end through the public API with host buffers
     e2e = None
     if E > 0:
-        ptok = torch.from_numpy(case.append_keys.view(np.int16)).view(torch.bfloat16).pin_memory()
-        pQ = torch.from_numpy(case.append_Q.view(np.int16)).view(torch.bfloat16).pin_memory()
-        pW = torch.from_numpy(case.append_w).pin_memory()
-        pidx = torch.empty((batch, k), dtype=torch.int32).pin_memory()
-        dtok = torch.empty_like(toks[0])
-        dQ = torch.empty_like(Qs[0])
-        dW = torch.empty_like(Ws[0])
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(E)]
-        base = W + K + n_prof + 1
-        for i, (a, b) in enumerate(evs):
-            s = base + i
-            a.record(stream)
-            dtok.copy_(ptok[s], non_blocking=True)
-            dQ.copy_(pQ[s % nsets], non_blocking=True)
-            dW.copy_(pW[s % nsets], non_blocking=True)
-            hisa.hisa_append(kv, dtok)
-            out = hisa.hisa_select(kv, dQ, dW, q_seq, None, m, k, ws=ws, idx=hidx)
-            pidx.copy_(out, non_blocking=True)
-            b.record(stream)
-            b.synchronize()
-            flush.fill_(7)
-        torch.cuda.synchronize()
-        e2e_ms = float(sum(a.elapsed_time(b) for a, b in evs))
-        e2e = {"value": batch * E / (e2e_ms / 1e3), "unit": "selections/s",
-               "h2d_bytes_per_step": int(dtok.numel() * 2 + dQ.numel() * 2 + dW.numel() * 4),
-               "d2h_bytes_per_step": int(pidx.numel() * 4), "steps": E,
-               "path": "pinned host -> hisa_append + hisa_select (python binding of the C ABI) -> pinned host"}
+        e2e = run_e2e(hisa, kv, case, toks, Qs, Ws, q_seq, ws, stream, W + K + n_prof + 1, E)
     assert kv.status_bits() == 0, f"device status {kv.status_bits():#x}"
 
     peaks = measured_peaks()
@@ -350,6 +341,70 @@ def run_gpu(args, rank, world):
         kernels=kernels, tok_bytes=tok_bytes, achieved=achieved, peaks=peaks,
         pool_gbs=pool_gbs, pool_ms=float(np.median(pool_ms)), hisa_sel_ms=hisa_sel_ms,
         flat_ms=flat_ms, mean_iou=mean_iou, e2e=e2e, case=case)
+
+
+def run_e2e(hisa, kv, case, toks, Qs, Ws, q_seq, ws, stream, base, E):
+    """The decode step end to end through the public calls: every step copies
+    its inputs (new keys, Q, w) from pinned host memory to the device, runs
+    hisa_decode_step, and copies its 64 x 2048 indices back to
+    pinned host memory.  Steps are pipelined the way a serving loop would run
+    them: host-to-device copies on one stream, the kernels on the launching
+    stream, device-to-host copies on a third, two device slots for inputs and
+    outputs, events for every dependency.  One event pair brackets all E
+    steps; the caches (512 MiB of keys) exceed L2, so no flush is needed."""
+    import torch
+    dev = kv.keys.device
+    batch, k, m = case.batch, case.k, case.m
+    nsets = Qs.shape[0]
+    ptok = torch.from_numpy(case.append_keys.view(np.int16)).view(torch.bfloat16).pin_memory()
+    pQ = torch.from_numpy(case.append_Q.view(np.int16)).view(torch.bfloat16).pin_memory()
+    pW = torch.from_numpy(case.append_w).pin_memory()
+    pidx = torch.empty((E, batch, k), dtype=torch.int32).pin_memory()
+    dtok = [torch.empty_like(toks[0]) for _ in range(2)]
+    dQ = [torch.empty_like(Qs[0]) for _ in range(2)]
+    dW = [torch.empty_like(Ws[0]) for _ in range(2)]
+    didx = [torch.empty((batch, k), dtype=torch.int32, device=dev) for _ in range(2)]
+    h2d, d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(E)]
+    ev_done = [torch.cuda.Event() for _ in range(E)]
+    ev_out = [torch.cuda.Event() for _ in range(E)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    host0 = time.perf_counter()
+    t0.record(stream)
+    h2d.wait_event(t0)
+    d2h.wait_event(t0)
+    for s in range(E):
+        j, src = s % 2, base + s
+        with torch.cuda.stream(h2d):
+            if s >= 2:
+                h2d.wait_event(ev_done[s - 2])          # step s - 2 no longer reads slot j
+            dtok[j].copy_(ptok[src], non_blocking=True)
+            dQ[j].copy_(pQ[src % nsets], non_blocking=True)
+            dW[j].copy_(pW[src % nsets], non_blocking=True)
+            ev_in[s].record(h2d)
+        stream.wait_event(ev_in[s])
+        if s >= 2:
+            stream.wait_event(ev_out[s - 2])            # step s - 2's indices have left slot j
+        hisa.hisa_decode_step(kv, dtok[j], dQ[j], dW[j], m, k, ws=ws, idx=didx[j])
+        ev_done[s].record(stream)
+        with torch.cuda.stream(d2h):
+            d2h.wait_event(ev_done[s])
+            pidx[s].copy_(didx[j], non_blocking=True)
+            ev_out[s].record(d2h)
+    stream.wait_event(ev_out[E - 1])
+    t1.record(stream)
+    host_enqueue = time.perf_counter() - host0
+    t1.synchronize()
+    e2e_ms = t0.elapsed_time(t1)
+    return {"value": batch * E / (e2e_ms / 1e3), "unit": "selections/s",
+            "h2d_bytes_per_step": int(dtok[0].numel() * 2 + dQ[0].numel() * 2 + dW[0].numel() * 4),
+            "d2h_bytes_per_step": int(didx[0].numel() * 4), "steps": E,
+            "ms_per_step": e2e_ms / E, "host_enqueue_ms_per_step": host_enqueue * 1e3 / E,
+            "path": "pinned host -> hisa_decode_step (python binding of the C ABI, plain calls, "
+                    "no graphs) -> pinned host; copies on their own streams, overlapping the "
+                    "previous and next steps' kernels",
+            "l2": "not flushed: the key cache (512 MiB) exceeds L2"}
 
 
 # ------------------------------------------------------ other workloads
@@ -486,23 +541,29 @@ def run_workloads(args, dev, peaks):
     toks = torch.from_numpy(case.append_keys.view(np.int16)).view(torch.bfloat16).to(dev)
     AQ = torch.from_numpy(case.append_Q.view(np.int16)).view(torch.bfloat16).to(dev)
     AW = torch.from_numpy(case.append_w).to(dev)
-    qs = torch.zeros(1, dtype=torch.int32, device=dev)
-    ws = hisa.workspace(hisa.hisa_select_workspace_bytes(kv, 1, case.H, case.m, case.k), dev)
+    ws = hisa.workspace(hisa.hisa_decode_step_workspace_bytes(kv, case.H, case.m, case.k), dev)
     idx = torch.empty((1, case.k), dtype=torch.int32, device=dev)
+    # one graph per step (the step is a chain of short launches on an
+    # L2-resident cache: launch-bound)
+    graphs = capture_steps([lambda s=s: hisa.hisa_decode_step(kv, toks[s], AQ[s], AW[s], case.m, case.k,
+                                                                ws=ws, idx=idx)
+                            for s in range(steps)], dev)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(steps)]
     for s, (a, b) in enumerate(evs):
         a.record(stream)
-        hisa.hisa_append(kv, toks[s])
-        hisa.hisa_select(kv, AQ[s], AW[s], qs, None, case.m, case.k, ws=ws, idx=idx)
+        graphs[s].replay()
         b.record(stream)
     torch.cuda.synchronize()
+    del graphs
     assert kv.status_bits() == 0, f"device status {kv.status_bits():#x}"
     st = [a.elapsed_time(b) for a, b in evs]
     out[case.name] = {"steps": steps, "us_per_step_mean": 1e3 * float(np.mean(st)),
                       "us_per_step_median": 1e3 * float(np.median(st)),
                       "steps_per_s": steps / (sum(st) / 1e3),
-                      "l2": "cache (32 MiB) L2-resident; no flush: each step follows the last"}
+                      "l2": "cache (32 MiB) L2-resident; no flush: each step follows the last",
+                      "step": "hisa_decode_step (1 key appended, 1 row selected), replayed from a "
+                              "CUDA graph per step"}
     return out
 
 
@@ -796,7 +857,9 @@ def main(argv=None, backend: str = "nccl"):
             "config": {"workload": WORKLOAD["name"], "batch": case.batch, "L": 32768,
                        "H_I": case.H, "d_I": case.d, "B": case.B, "m": case.m, "k": case.k,
                        "key_dtype": "bf16", "parallelism": f"replicas x{world}" if world > 1 else "1 gpu",
-                       "step": "hisa_append (64 keys) + hisa_select (64 rows at the new last position)",
+                       "step": "hisa_decode_step: 64 keys appended (trailing block means updated) + "
+                               "64 rows selected at the new last positions (= hisa_append + hisa_select)",
+                       "launch": "each timed step replayed from a CUDA graph captured from the same calls",
                        "l2": "flushed between timed steps (256 MiB write, outside the timed events)"},
             "clocks": r["clocks"],
             "gpu_launches": r["launches"],

@@ -37,6 +37,7 @@ HISA_STATIC_SCRATCH_BYTES = 8 << 20
 HISA_DEV_BAD_QUERY, HISA_DEV_CAPACITY, HISA_DEV_BAD_LEN, HISA_DEV_TIMEOUT = 0x1, 0x2, 0x4, 0x8
 
 EXPORTS = ("hisa_pool_blocks", "hisa_append", "hisa_select_workspace_bytes", "hisa_select",
+           "hisa_decode_step_workspace_bytes", "hisa_decode_step",
            "hisa_select_inspect", "hisa_select_static", "hisa_tree_workspace_bytes",
            "hisa_tree_select", "hisa_pool_tail", "hisa_cp_workspace_bytes", "hisa_cp_blocks",
            "hisa_cp_tokens", "hisa_merge_topk", "hisa_sparse_attn_workspace_bytes", "hisa_sparse_attn",
@@ -62,6 +63,9 @@ _lib.hisa_append.argtypes = [_KVP, _P, _P, _P]
 _lib.hisa_select_workspace_bytes.argtypes = [_KVP, _I, _I, _I, _I]
 _lib.hisa_select_workspace_bytes.restype = _Z
 _lib.hisa_select.argtypes = [_KVP, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _Z, _P]
+_lib.hisa_decode_step_workspace_bytes.argtypes = [_KVP, _I, _I, _I]
+_lib.hisa_decode_step_workspace_bytes.restype = _Z
+_lib.hisa_decode_step.argtypes = [_KVP, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _Z, _P]
 _lib.hisa_select_inspect.argtypes = [_KVP, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P,
                                      _P, _Z, _P]
 _lib.hisa_select_static.argtypes = [_KVP, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P]
@@ -92,7 +96,8 @@ _lib.hisa_status_string.argtypes = [_I]
 _lib.hisa_status_string.restype = ctypes.c_char_p
 _lib.hisa_last_cuda_error.argtypes = []
 _lib.hisa_last_cuda_error.restype = ctypes.c_char_p
-for _f in ("hisa_pool_blocks", "hisa_append", "hisa_select", "hisa_select_inspect", "hisa_select_static",
+for _f in ("hisa_pool_blocks", "hisa_append", "hisa_select", "hisa_decode_step", "hisa_select_inspect",
+           "hisa_select_static",
            "hisa_tree_select", "hisa_pool_tail", "hisa_cp_blocks", "hisa_cp_tokens", "hisa_merge_topk",
            "hisa_sparse_attn", "dsa_flat_select", "hisa_topk_f32", "hisa_profile_enable", "hisa_profile_read"):
     getattr(_lib, _f).restype = _I
@@ -266,6 +271,44 @@ def hisa_select(kv: KVCache, Q, w, q_seq, q_pos, m: int, k: int, want_scores: bo
     _check("hisa_select", _lib.hisa_select(
         kv.struct, _ptr(Q), _ptr(w), _ptr(q_seq), _ptr(q_pos), n_q, H, m, k, _ptr(idx),
         _ptr(scores), _ptr(ws), ws.numel(), _stream(stream)))
+    return (idx, scores) if want_scores else idx
+
+
+def hisa_decode_step_workspace_bytes(kv: KVCache, H: int, m: int, k: int) -> int:
+    return int(_lib.hisa_decode_step_workspace_bytes(kv.struct, H, m, k))
+
+
+def hisa_decode_step(kv: KVCache, tok: torch.Tensor, Q, w, m: int, k: int,
+                     tok_scale: Optional[torch.Tensor] = None, want_scores: bool = False,
+                     ws: Optional[torch.Tensor] = None, idx: Optional[torch.Tensor] = None,
+                     scores: Optional[torch.Tensor] = None, stream=None):
+    """hisa_append(kv, tok) then hisa_select for every sequence's new last
+    position (query row b = sequence b), in one call.  Returns idx [batch, k]
+    (and scores if asked)."""
+    fn = "hisa_decode_step"
+    dev = kv.keys.device
+    Q = _dev(Q, torch.bfloat16, dev)
+    w = _dev(w, torch.float32, dev)
+    n_q, H = kv.batch, Q.shape[1]
+    if Q.dim() != 3 or Q.shape[0] != n_q or Q.shape[2] != kv.d or tuple(w.shape) != (n_q, H):
+        raise ValueError(f"{fn}: Q must be [{n_q}, H, {kv.d}] and w [{n_q}, H]")
+    tdt = torch.bfloat16 if kv.dtype == "bf16" else torch.uint8
+    if tok.dtype not in (tdt, torch.int16) or not tok.is_contiguous() or tok.device != dev or \
+            tok.numel() != n_q * kv.d:
+        raise ValueError(f"{fn}: tok must be a contiguous [{n_q}, {kv.d}] {tdt} tensor on {dev}")
+    if kv.dtype == "e4m3" and (tok_scale is None or tok_scale.dtype != torch.float32 or
+                               tok_scale.numel() != n_q or tok_scale.device != dev):
+        raise ValueError(f"{fn}: tok_scale must be fp32 [{n_q}] on {dev}")
+    _check_out(fn, kv, n_q, k, idx, scores)
+    _check_ws(fn, kv, ws)
+    if ws is None:
+        ws = workspace(hisa_decode_step_workspace_bytes(kv, H, m, k), dev)
+    idx = torch.empty((n_q, k), dtype=torch.int32, device=dev) if idx is None else idx
+    if want_scores and scores is None:
+        scores = torch.empty((n_q, k), dtype=torch.float32, device=dev)
+    _check(fn, _lib.hisa_decode_step(
+        kv.struct, _ptr(tok), _ptr(tok_scale), _ptr(Q), _ptr(w), H, m, k, _ptr(idx), _ptr(scores),
+        _ptr(ws), ws.numel(), _stream(stream)))
     return (idx, scores) if want_scores else idx
 
 

@@ -2,6 +2,7 @@
 // layout, TMA tensor maps and kernel launches.  No allocation happens here:
 // every buffer belongs to the caller, and so does the scratch space, except
 // for hisa_select_static, whose scratch is one fixed device array below.
+#include <atomic>
 #include <climits>
 #include <cmath>
 #include <cstring>
@@ -46,6 +47,23 @@ bool make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, size_t
     const cuuint32_t estr[2] = {1, 1};
     return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The block representatives as a 3-D tensor [batch, nblk, 2d] bf16 with
+// boxes of [1, 128, 64]: a box that runs past a sequence's nblk rows is
+// zero-filled there instead of reading the next sequence's rows.
+bool pooled_map(CUtensorMap* map, const KvView& v) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(2 * v.d), static_cast<cuuint64_t>(v.nblk),
+                                static_cast<cuuint64_t>(v.batch)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(2 * v.d) * 2,
+                                   static_cast<cuuint64_t>(v.nblk) * 2 * v.d * 2};
+    const cuuint32_t box[3] = {64, 128, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, v.pooled_hl, dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -102,10 +120,15 @@ struct PhaseScope {
     }
 };
 
+// SMs of the current device (looked up once per device).
 int sm_count() {
+    constexpr int kDevs = 64;
+    static std::atomic<int> cached[kDevs];
     int dev = 0, n = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (dev >= 0 && dev < kDevs && (n = cached[dev].load(std::memory_order_relaxed)) > 0) return n;
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    if (dev >= 0 && dev < kDevs) cached[dev].store(n, std::memory_order_relaxed);
     return n;
 }
 
@@ -278,15 +301,22 @@ int run_score(int mode, const KvView& v, const CUtensorMap& amap, const CUtensor
     return cuda_status(launch_score(mode, e4m3, v.d, amap, qmap, p, grid, s));
 }
 
-// fp8 scoring of e4m3 keys (d = 128): split the query heads into the
-// workspace and aim the query tensor map and the weights at them.
+// fp8 scoring of e4m3 keys (d = 128): the query heads split into the
+// workspace (launch_qsplit; already done by the caller when split = false),
+// and the query tensor map and the weights aimed at them.
+int split_queries(const KvView& v, const uint16_t* Q, const float* w, int n_q, int H, uint8_t* q8, float* w8,
+                  cudaStream_t s) {
+    if (!f8_keys(v)) return HISA_OK;
+    PhaseScope ps(HISA_PHASE_QSPLIT, s);
+    return cuda_status(launch_qsplit(Q, w, n_q, H, npad_of(H), q8, w8, s));
+}
+
 int prep_f8(const KvView& v, const uint16_t* Q, const float* w, int n_q, int H, uint8_t* q8, float* w8,
-            CUtensorMap* qmap, ScoreParams& p, cudaStream_t s) {
+            CUtensorMap* qmap, ScoreParams& p, cudaStream_t s, bool split = true) {
     if (!f8_keys(v)) return HISA_OK;
     const int npad = npad_of(H);
-    {
-        PhaseScope ps(HISA_PHASE_QSPLIT, s);
-        const int rc = cuda_status(launch_qsplit(Q, w, n_q, H, npad, q8, w8, s));
+    if (split) {
+        const int rc = split_queries(v, Q, w, n_q, H, q8, w8, s);
         if (rc) return rc;
     }
     if (!make_map(qmap, q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(n_q) * 2 * npad, 128,
@@ -312,6 +342,10 @@ struct BlockLevel {
     const int32_t* parent;   // kept superblocks [n_q, parent_ld] or null
     int parent_ld, bf;
     int counts_col;
+    // the decode step: row b is sequence b, whose new key the append kernel
+    // launched just before writes (the caller guarantees the conditions of
+    // the one-CTA-per-row block stage)
+    int app;
 };
 
 int block_stage(const BlockLevel& lv, const uint16_t* Q, const float* w, const int32_t* q_seq,
@@ -319,11 +353,7 @@ int block_stage(const BlockLevel& lv, const uint16_t* Q, const float* w, const i
                 cudaStream_t s) {
     const KvView& v = *lv.v;
     CUtensorMap pmap, qmap;
-    if (!make_map(&pmap, v.pooled_hl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-                  static_cast<uint64_t>(v.batch) * v.nblk, 2 * v.d, 128, 64,
-                  CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !query_map(&qmap, Q, n_q, H, v.d))
-        return HISA_E_CUDA;
+    if (!pooled_map(&pmap, v) || !query_map(&qmap, Q, n_q, H, v.d)) return HISA_E_CUDA;
     const int sms = sm_count();
     ScoreParams p = score_params(v, w, q_seq, q_pos, n_q, H);
     p.out = lv.bkeys;
@@ -340,6 +370,11 @@ int block_stage(const BlockLevel& lv, const uint16_t* Q, const float* w, const i
     // selection launch.  Longer rows score faster spread over every SM, and
     // many rows select faster in the selection kernel's one-CTA-per-row grid.
     const bool fuse = lv.ldb <= kFuseMaxBlocks && n_q <= 2 * sms;
+    if (lv.app) {
+        if (!fuse) return HISA_E_UNSUPPORTED;
+        p.app = 1;
+        p.len_w = v.len;
+    }
     if (fuse) {
         p.fuse = 1;
         p.m = lv.m;
@@ -382,7 +417,7 @@ int block_stage(const BlockLevel& lv, const uint16_t* Q, const float* w, const i
 int token_stage(const KvView& v, const HisaWs& L, uint8_t* base, const uint16_t* Q, const float* w,
                 const int32_t* q_seq, const int32_t* q_pos, int n_q, int H, int k, int32_t* idx,
                 float* scores, uint64_t* counts, int counts_ld, int counts_col, int id_off,
-                cudaStream_t s) {
+                cudaStream_t s, bool split = true) {
     int32_t* blocks = reinterpret_cast<int32_t*>(base + L.blocks);
     int4* plan = reinterpret_cast<int4*>(base + L.plan);
     uint32_t* tkeys = reinterpret_cast<uint32_t*>(base + L.tkeys);
@@ -393,7 +428,7 @@ int token_stage(const KvView& v, const HisaWs& L, uint8_t* base, const uint16_t*
     p.counts = reinterpret_cast<unsigned long long*>(counts);
     p.counts_ld = counts_ld;
     p.counts_col = counts_col;
-    int rc = prep_f8(v, Q, w, n_q, H, base + L.q8, reinterpret_cast<float*>(base + L.w8), &qmap, p, s);
+    int rc = prep_f8(v, Q, w, n_q, H, base + L.q8, reinterpret_cast<float*>(base + L.w8), &qmap, p, s, split);
     if (rc) return rc;
     p.out = tkeys;
     p.ldo = L.ldt;
@@ -427,23 +462,18 @@ int token_stage(const KvView& v, const HisaWs& L, uint8_t* base, const uint16_t*
     return cuda_status(launch_select(sp, L.mm * v.B, sm_count(), s));
 }
 
-int hisa_select_impl(const hisa_kv* kv, const uint16_t* Q, const float* w, const int32_t* q_seq,
-                     const int32_t* q_pos, int n_q, int H, int m, int k, int32_t* idx, float* scores,
-                     int32_t* blocks_out, int32_t* nblocks_out, uint64_t* counts, void* ws,
-                     size_t ws_bytes, cudaStream_t s) {
-    KvView v;
-    int rc = check_kv(kv, &v);
-    if (rc) return rc;
-    if (!select_block_size_ok(v.B)) return HISA_E_UNSUPPORTED;
-    if (m < 1) return HISA_E_INVAL;
-    rc = check_queries(Q, w, q_seq, n_q, H, k, idx);
-    if (rc) return rc;
-    if (n_q == 0) return HISA_OK;
-    const HisaWs L = hisa_ws(v, n_q, H, m);
-    if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return HISA_E_WORKSPACE;
-    uint8_t* base = static_cast<uint8_t*>(ws);
+// The two stages on validated arguments (q_seq NULL: row i is sequence i).
+int select_stages(const KvView& v, const HisaWs& L, uint8_t* base, const uint16_t* Q, const float* w,
+                  const int32_t* q_seq, const int32_t* q_pos, int n_q, int H, int m, int k, int32_t* idx,
+                  float* scores, int32_t* blocks_out, int32_t* nblocks_out, uint64_t* counts,
+                  cudaStream_t s) {
+    int rc;
     if (counts && cudaMemsetAsync(counts, 0, sizeof(uint64_t) * 2 * n_q, s) != cudaSuccess)
         return HISA_E_CUDA;
+    // fp8 keys: the query split depends on the inputs alone, so it goes first
+    // rather than between the two stages
+    rc = split_queries(v, Q, w, n_q, H, base + L.q8, reinterpret_cast<float*>(base + L.w8), s);
+    if (rc) return rc;
     BlockLevel lv;
     std::memset(&lv, 0, sizeof lv);
     lv.v = &v;
@@ -458,7 +488,25 @@ int hisa_select_impl(const hisa_kv* kv, const uint16_t* Q, const float* w, const
     lv.nblocks_out = nblocks_out;
     rc = block_stage(lv, Q, w, q_seq, q_pos, n_q, H, k, counts, 2, s);
     if (rc) return rc;
-    return token_stage(v, L, base, Q, w, q_seq, q_pos, n_q, H, k, idx, scores, counts, 2, 0, 0, s);
+    return token_stage(v, L, base, Q, w, q_seq, q_pos, n_q, H, k, idx, scores, counts, 2, 0, 0, s, false);
+}
+
+int hisa_select_impl(const hisa_kv* kv, const uint16_t* Q, const float* w, const int32_t* q_seq,
+                     const int32_t* q_pos, int n_q, int H, int m, int k, int32_t* idx, float* scores,
+                     int32_t* blocks_out, int32_t* nblocks_out, uint64_t* counts, void* ws,
+                     size_t ws_bytes, cudaStream_t s) {
+    KvView v;
+    int rc = check_kv(kv, &v);
+    if (rc) return rc;
+    if (!select_block_size_ok(v.B)) return HISA_E_UNSUPPORTED;
+    if (m < 1) return HISA_E_INVAL;
+    rc = check_queries(Q, w, q_seq, n_q, H, k, idx);
+    if (rc) return rc;
+    if (n_q == 0) return HISA_OK;
+    const HisaWs L = hisa_ws(v, n_q, H, m);
+    if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return HISA_E_WORKSPACE;
+    return select_stages(v, L, static_cast<uint8_t*>(ws), Q, w, q_seq, q_pos, n_q, H, m, k, idx, scores,
+                         blocks_out, nblocks_out, counts, s);
 }
 
 // Three-level search: a second index kv2 over the same keys with blocks of
@@ -613,6 +661,69 @@ int hisa_select_inspect(const hisa_kv* kv, const uint16_t* Q, const float* w, co
                             counts, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
+size_t hisa_decode_step_workspace_bytes(const hisa_kv* kv, int H, int m, int k) {
+    (void)k;
+    KvView v;
+    if (check_kv(kv, &v) || m < 1 || H < 1 || H > 128) return 0;
+    return hisa_ws(v, v.batch, H, m).total;
+}
+
+int hisa_decode_step(const hisa_kv* kv, const void* tok, const float* tok_scale, const uint16_t* Q,
+                     const float* w, int H, int m, int k, int32_t* idx, float* scores, void* ws,
+                     size_t ws_bytes, hisa_stream_t stream) {
+    KvView v;
+    int rc = check_kv(kv, &v);
+    if (rc) return rc;
+    if (!select_block_size_ok(v.B)) return HISA_E_UNSUPPORTED;
+    if (m < 1 || k < 1) return HISA_E_INVAL;
+    if (H < 1 || H > 128) return HISA_E_UNSUPPORTED;
+    if (!tok || !aligned(tok, 16) || (v.e4m3 && (!tok_scale || !aligned(tok_scale, 4)))) return HISA_E_INVAL;
+    if (!Q || !w || !idx || !aligned(Q, 16) || !aligned(w, 4) || !aligned(idx, 4) ||
+        (scores && !aligned(scores, 4)))
+        return HISA_E_INVAL;
+    const int n_q = v.batch;
+    const HisaWs L = hisa_ws(v, n_q, H, m);
+    if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return HISA_E_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    const int sms = sm_count();
+    if (sms <= 0) return HISA_E_CUDA;
+    if (L.ldb > kFuseMaxBlocks || n_q > 2 * sms) {
+        // rows too long (or too many) for one CTA per row: the append and the
+        // selection as separate launches, with the same results
+        {
+            PhaseScope ps(HISA_PHASE_APPEND, s);
+            rc = cuda_status(launch_append(v, tok, tok_scale, s));
+            if (rc) return rc;
+        }
+        return select_stages(v, L, base, Q, w, nullptr, nullptr, n_q, H, m, k, idx, scores, nullptr,
+                             nullptr, nullptr, s);
+    }
+    BlockLevel lv;
+    std::memset(&lv, 0, sizeof lv);
+    lv.v = &v;
+    lv.m = m;
+    lv.mm = L.mm;
+    lv.ldb = L.ldb;
+    lv.bkeys = reinterpret_cast<uint32_t*>(base + L.bkeys);
+    lv.blocks = reinterpret_cast<int32_t*>(base + L.blocks);
+    lv.nblocks = reinterpret_cast<int32_t*>(base + L.nblocks);
+    lv.plan = reinterpret_cast<int4*>(base + L.plan);
+    lv.app = 1;
+    rc = split_queries(v, Q, w, n_q, H, base + L.q8, reinterpret_cast<float*>(base + L.w8), s);
+    if (rc) return rc;
+    {
+        // the append, which the block scoring does not wait for (see
+        // ScoreParams::app); it goes right before that kernel
+        PhaseScope ps(HISA_PHASE_APPEND, s);
+        rc = cuda_status(launch_append(v, tok, tok_scale, s, true));
+        if (rc) return rc;
+    }
+    rc = block_stage(lv, Q, w, nullptr, nullptr, n_q, H, k, nullptr, 2, s);
+    if (rc) return rc;
+    return token_stage(v, L, base, Q, w, nullptr, nullptr, n_q, H, k, idx, scores, nullptr, 2, 0, 0, s, false);
+}
+
 int hisa_select_static(const hisa_kv* kv, const uint16_t* Q, const float* w, const int32_t* q_seq,
                        const int32_t* q_pos, int n_q, int H, int m, int k, int32_t* idx,
                        float* scores, hisa_stream_t stream) {
@@ -737,11 +848,7 @@ int hisa_cp_blocks(const hisa_kv* kv, int32_t tok_off, const uint16_t* Q, const 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint32_t* bkeys = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + L.bkeys);
     CUtensorMap pmap, qmap;
-    if (!make_map(&pmap, v.pooled_hl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-                  static_cast<uint64_t>(v.batch) * v.nblk, 2 * v.d, 128, 64,
-                  CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !query_map(&qmap, Q, n_q, H, v.d))
-        return HISA_E_CUDA;
+    if (!pooled_map(&pmap, v) || !query_map(&qmap, Q, n_q, H, v.d)) return HISA_E_CUDA;
     // the shard's visible blocks scored into the workspace ...
     ScoreParams p = score_params(v, w, q_seq, q_pos, n_q, H);
     p.out = bkeys;

@@ -96,6 +96,17 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
         : "memory");
 }
 
+// 3-D box at (c0, c1, c2); coordinates past a dimension's end read as zero
+// and move no memory.
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int32_t c0, int32_t c1, int32_t c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
 // Same, with an L2 eviction-priority hint (a createpolicy value).
 __device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* map, uint64_t* bar,
                                                  int32_t c0, int32_t c1, uint64_t policy) {
@@ -295,10 +306,11 @@ __device__ __forceinline__ void set_status(uint32_t* status, uint32_t bits) {
 }
 
 // Position of query row i (or -1 when outside its sequence's prefix).
+// q_seq NULL: row i is sequence i (the decode step's rows).
 __device__ __forceinline__ int query_position(const int32_t* q_seq, const int32_t* q_pos,
                                               const int32_t* len, int batch, int cap, int i,
                                               int* seq_out) {
-    const int b = q_seq[i];
+    const int b = q_seq ? q_seq[i] : i;
     *seq_out = b;
     if (b < 0 || b >= batch) return -1;
     const int n = len[b];

@@ -77,6 +77,14 @@ struct ScoreParams {
     int4* sel_plan;               // [n_q]
     int32_t* sel_blocks_out;      // [n_q, mm] or null
     int32_t* sel_nblocks_out;     // [n_q] or null
+    // kScoreBlocks in the decode step (app = 1, fuse = 1): row b is sequence
+    // b, whose new key the append kernel launched just before is writing at
+    // position len[b] (concurrently: it only changes the representative of
+    // the row's own block, which is kept whatever its score); the row selects
+    // for position len[b] (cap - 1 for a full sequence, which appends
+    // nothing), and after waiting for the append the kernel advances len[b]
+    int app;
+    int32_t* len_w;               // the cache's lengths (app = 1)
     // kScoreBlocks over one context-parallel shard (cp = 1): the cache holds
     // the global positions [tok_off, tok_off + cap) of every sequence, q_pos
     // are global positions, and a row's candidates are the shard's blocks
@@ -231,8 +239,10 @@ inline cudaError_t smem_limit(const void* fn, size_t bytes) {
 }
 
 cudaError_t launch_pool(const KvView& kv, cudaStream_t s);
+// step = true: the decode step's append, which leaves len to the scoring
+// kernel that follows it (see append_kernel).
 cudaError_t launch_append(const KvView& kv, const void* tok, const float* tok_scale,
-                          cudaStream_t s);
+                          cudaStream_t s, bool step = false);
 // Re-pool each sequence's trailing block (the one holding key len - 1).
 cudaError_t launch_pool_tail(const KvView& kv, cudaStream_t s);
 

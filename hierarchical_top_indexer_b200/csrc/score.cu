@@ -34,7 +34,7 @@
 //   warps 6-9    e4m3 -> bf16 converters (e4m3 keys with d = 64 only)
 // Every mbarrier wait is bounded; on expiry the CTA raises HISA_DEV_TIMEOUT,
 // drains its outstanding copies and returns.
-#include "hisa_kernels.cuh"
+#include "hisa_pool.cuh"
 
 namespace hisa {
 
@@ -132,13 +132,15 @@ __host__ __device__ inline uint32_t tmem_columns(int cols) {
     return c;
 }
 
-// Block scoring variants (a template parameter, so that each compiles alone).
-constexpr int kBlocksPlain = 0, kBlocksMasked = 1, kBlocksShard = 2;
+// Block scoring variants (a template parameter, so that each compiles alone):
+// kBlocksAppend is the decode step (row b = sequence b, scored while the
+// append kernel launched before it writes the new keys; see ScoreParams::app).
+constexpr int kBlocksPlain = 0, kBlocksMasked = 1, kBlocksShard = 2, kBlocksAppend = 3;
 
 // A query row: sequence, position, candidate slots, candidate tiles (0 if
-// the row is invalid).
+// the row is invalid); app: the decode step appends a key at t first.
 struct RowInfo {
-    int b, t, lim, nt;
+    int b, t, lim, nt, app;
 };
 
 template <int MODE, int BV>
@@ -146,7 +148,20 @@ __device__ __forceinline__ RowInfo load_row(const ScoreParams& p, int row) {
     RowInfo R;
     R.lim = 0;
     R.nt = 0;
-    if (MODE == kScoreHisa) {
+    R.app = 0;
+    if (MODE == kScoreBlocks && BV == kBlocksAppend) {
+        // decode step: the new key goes to position len[b] (nothing is
+        // appended to a full sequence, whose last position is then cap - 1)
+        R.b = row;
+        const int n = p.len[row];
+        if (n < 0 || n > p.cap) {
+            R.t = -1;
+            return R;
+        }
+        R.app = n < p.cap;
+        R.t = R.app ? n : p.cap - 1;
+        R.lim = R.t / p.B + 1;
+    } else if (MODE == kScoreHisa) {
         const int4 pl = p.plan_in[row];     // written by the block selection
         R.b = pl.x;
         R.t = pl.y;
@@ -276,11 +291,16 @@ __device__ __forceinline__ float head_sum(uint32_t taddr, const float* wv) {
 #pragma unroll
         for (int c = 0; c < kG; c += 16)
             if (g + c < NP) tmem_ld16_nowait(taddr + g + c, r + c);
+        // the group's head weights load while the TMEM loads are in flight
+        float4 wg[kG / 4];
+#pragma unroll
+        for (int h = 0; h < kG; h += 4)
+            if (g + h < NP) wg[h / 4] = lds_f32x4(wv + g + h);
         tmem_ld_wait();
 #pragma unroll
         for (int h = 0; h < kG; h += 4)
             if (g + h < NP) {
-                const float4 w4 = lds_f32x4(wv + g + h);
+                const float4 w4 = wg[h / 4];
                 a[0] = fmaf(w4.x, fmaxf(__uint_as_float(r[h]), 0.f), a[0]);
                 a[1] = fmaf(w4.y, fmaxf(__uint_as_float(r[h + 1]), 0.f), a[1]);
                 a[2] = fmaf(w4.z, fmaxf(__uint_as_float(r[h + 2]), 0.f), a[2]);
@@ -305,11 +325,15 @@ __device__ __forceinline__ float head_sum2(uint32_t taddr, const float* wv) {
                 tmem_ld16_nowait(taddr + g + c, r1 + c);
                 tmem_ld16_nowait(taddr + NP + g + c, r2 + c);
             }
+        float4 wg[kG / 4];
+#pragma unroll
+        for (int h = 0; h < kG; h += 4)
+            if (g + h < NP) wg[h / 4] = lds_f32x4(wv + g + h);
         tmem_ld_wait();
 #pragma unroll
         for (int h = 0; h < kG; h += 4) {
             if (g + h >= NP) break;
-            const float4 w4 = lds_f32x4(wv + g + h);
+            const float4 w4 = wg[h / 4];
             a[0] = fmaf(w4.x, fmaxf(__uint_as_float(r1[h]) + __uint_as_float(r2[h]), 0.f), a[0]);
             a[1] = fmaf(w4.y, fmaxf(__uint_as_float(r1[h + 1]) + __uint_as_float(r2[h + 1]), 0.f), a[1]);
             a[2] = fmaf(w4.z, fmaxf(__uint_as_float(r1[h + 2]) + __uint_as_float(r2[h + 2]), 0.f), a[2]);
@@ -405,10 +429,10 @@ __device__ uint32_t epi_threshold(const uint32_t* s, int n, int kk, uint32_t* hi
     return prefix;
 }
 
-// Writes the slots of the top kk keys of s[0..n) in ascending order to out
-// (and dbg) given T and take_eq from epi_threshold.
-__device__ void epi_emit(const uint32_t* s, int n, uint32_t T, int take_eq, int32_t* out, int32_t* dbg,
-                         uint32_t* misc, int e) {
+// Writes the slots of the keys of s[0..n) above T, plus the first take_eq
+// equal to T, in ascending order to out (and dbg).
+__device__ __noinline__ void epi_emit(const uint32_t* s, int n, uint32_t T, int take_eq, int32_t* out,
+                                      int32_t* dbg, uint32_t* misc, int e) {
     const int w = e >> 5, l = e & 31;
     const int per = ((n + 3) / 4 + 31) & ~31;
     const int w0 = w * per;
@@ -461,6 +485,7 @@ __device__ void epi_emit(const uint32_t* s, int n, uint32_t T, int take_eq, int3
     }
 }
 
+
 // BV (block scoring only): every visible block is a candidate (kBlocksPlain),
 // a kept-superblock list masks the blocks outside it (kBlocksMasked), or the
 // cache is a context-parallel shard (kBlocksShard).
@@ -473,6 +498,7 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
     constexpr bool kF8 = uses_f8(MODE, E4M3, D);          // fp8 operands straight from TMA
     constexpr bool kConv = E4M3 && !kF8;                  // e4m3 widened to bf16 by converter warps
     constexpr bool PAR = MODE == kScoreBlocks && BV == kBlocksMasked;
+    constexpr bool APP = MODE == kScoreBlocks && BV == kBlocksAppend;
     constexpr int kStageBytes = kF8 ? kTileRows * D : kOps * kHalves * kHalfBytes;
     constexpr int kStage8Bytes = kTileRows * D;
 
@@ -554,8 +580,10 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    // everything above overlaps the previous kernel; its outputs are read below
-    grid_dependency_wait();
+    // everything above overlaps the previous kernel; its outputs are read
+    // below.  In the decode step the previous kernel is the append, which this
+    // kernel does not wait for here (see ScoreParams::app).
+    if (!APP) grid_dependency_wait();
     grid_launch_dependents();
 
     if (warp == kWarpProducer) {
@@ -578,6 +606,22 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
             TileCursor cur(g0, tpr);
             while (cur.g < g1 && ok) {
                 const int row = cur.row;
+                // kept-block ids of the row's first window, loaded together
+                // with the row's plan rather than after it (one L2 round trip
+                // per row start instead of two); the ids are read within the
+                // row's [0, mm) entries and only used where the plan says so
+                constexpr int kPre = kTabSubs / 32;
+                int pre[kPre];
+                if constexpr (MODE == kScoreHisa) {
+                    const int32_t* brow = p.blocks + static_cast<size_t>(row) * p.mm;
+                    const int wmax = min(tpr - cur.ti, kTabSubs / nsub) * nsub;
+#pragma unroll
+                    for (int q = 0; q < kPre; ++q) {
+                        const int j = lane + 32 * q;
+                        const int slot = (cur.ti + j / nsub) * kTileRows + (j % nsub) * BR;
+                        pre[q] = j < wmax ? __ldg(brow + min(slot / p.B, p.mm - 1)) : 0;
+                    }
+                }
                 R = load_row<MODE, BV>(p, row);
                 const long long left = g1 - cur.g;
                 const int t_end = static_cast<int>(R.nt < cur.ti + left ? R.nt : cur.ti + left);
@@ -606,8 +650,19 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
                 for (int t = cur.ti; t < t_end && ok;) {
                     const int nwin = min(t_end - t, kTabSubs / nsub);
                     if (MODE == kScoreHisa) {
-                        for (int j = lane; j < nwin * nsub; j += 32)
-                            sTab[j] = tile_sub_row<MODE>(p, R, row, t + j / nsub, j % nsub, BR);
+                        if (t == cur.ti) {
+#pragma unroll
+                            for (int q = 0; q < kPre; ++q) {
+                                const int j = lane + 32 * q;
+                                if (j < nwin * nsub) {
+                                    const int slot = (t + j / nsub) * kTileRows + (j % nsub) * BR;
+                                    sTab[j] = R.b * p.cap + (slot < R.lim ? pre[q] : 0) * p.B + slot % p.B;
+                                }
+                            }
+                        } else {
+                            for (int j = lane; j < nwin * nsub; j += 32)
+                                sTab[j] = tile_sub_row<MODE>(p, R, row, t + j / nsub, j % nsub, BR);
+                        }
                         __syncwarp();
                     }
                     if (lane == 0) {
@@ -618,16 +673,19 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
                                 ok = false;
                                 break;
                             }
+
                             uint64_t* fb = full + ring.slot;
                             uint8_t* dst = sA + ring.slot * kStageBytes;
                             mbar_arrive_expect_tx(fb, kStageBytes);
                             if (MODE == kScoreBlocks) {
+                                // [batch, nblk, 2d] boxes: the rows past the sequence's
+                                // blocks are zero-filled, not read
 #pragma unroll
                                 for (int op = 0; op < 2; ++op)
 #pragma unroll
                                     for (int kh = 0; kh < kHalves; ++kh)
-                                        tma_load_2d(dst + (op * kHalves + kh) * kHalfBytes, &amap, fb,
-                                                    op * D + kh * 64, R.b * p.nblk + (t + k) * kTileRows);
+                                        tma_load_3d(dst + (op * kHalves + kh) * kHalfBytes, &amap, fb,
+                                                    op * D + kh * 64, (t + k) * kTileRows, R.b);
                             } else {
                                 for (int sub = 0; sub < nsub; ++sub) {
                                     const int srow = MODE == kScoreHisa
@@ -754,8 +812,8 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
                     for (int op = 0; op < 2; ++op)
 #pragma unroll
                         for (int kh = 0; kh < kHalves; ++kh)
-                            tma_load_2d(sA + ss * kStageBytes + (op * kHalves + kh) * kHalfBytes, &amap, fb,
-                                        op * D + kh * 64, R.b * p.nblk + ti * kTileRows);
+                            tma_load_3d(sA + ss * kStageBytes + (op * kHalves + kh) * kHalfBytes, &amap, fb,
+                                        op * D + kh * 64, ti * kTileRows, R.b);
                 }
             } else {
                 if (lane == 0) mbar_arrive_expect_tx(fb, E4M3 ? kStage8Bytes : kStageBytes);
@@ -1046,6 +1104,10 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
                     p.sel_nblocks[row] = keep;
                     if (p.sel_nblocks_out) p.sel_nblocks_out[row] = keep;
                     p.sel_plan[row] = make_int4(R.b, R.t, keep, 0);
+                    if (APP && R.app) {
+                        grid_dependency_wait();    // the append kernel has finished
+                        p.len_w[R.b] = R.t + 1;
+                    }
                 }
                 epi_bar();
             }
@@ -1113,8 +1175,9 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
     if (warp == kWarpMma) tmem_dealloc(tmem_base, ncols);
 }
 
-// Query heads for fp8 scoring (see launch_qsplit).  One CTA per query row,
-// one warp per head, four elements per lane.  The power of two puts the
+// Query heads for fp8 scoring (see launch_qsplit).  CTA (row, g) splits the
+// heads 4g .. 4g + 3 of one query row, one warp per head (all their loads in
+// flight at once), four elements per lane.  The power of two puts the
 // head's largest |q| in (224, 448] (e4m3's largest finite value is 448), so
 // q1 = e4m3(q * 2^e) and q2 = e4m3(q * 2^e - q1) hold the bf16 value exactly
 // unless part of it falls below e4m3's smallest step (2^-9).
@@ -1124,7 +1187,7 @@ __global__ void __launch_bounds__(128) qsplit_kernel(const uint16_t* __restrict_
     const int row = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     grid_dependency_wait();
     grid_launch_dependents();
-    for (int h = warp; h < npad; h += 4) {
+    for (int h = blockIdx.y * 4 + warp; h < npad; h += 4 * gridDim.y) {
         uint32_t* o1 = reinterpret_cast<uint32_t*>(q8 + (static_cast<size_t>(row) * 2 * npad + h) * 128);
         uint32_t* o2 = reinterpret_cast<uint32_t*>(q8 + (static_cast<size_t>(row) * 2 * npad + npad + h) * 128);
         if (h >= H) {
@@ -1174,8 +1237,7 @@ cudaError_t launch_t(const CUtensorMap& amap, const CUtensorMap& qmap, const Sco
     const Layout L = score_layout(MODE, E4M3, D, p.npad, p.stages, p.stages8);
     if ((L.a | L.q) & 1023u) return cudaErrorInvalidValue;
     auto* fn = score_kernel<MODE, E4M3, D, BV>;
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    cudaError_t e = smem_limit(reinterpret_cast<const void*>(fn), smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
@@ -1197,7 +1259,7 @@ cudaError_t launch_qsplit(const uint16_t* Q, const float* w, int n_q, int H, int
                           float* w8, cudaStream_t s) {
     if (n_q == 0) return cudaSuccess;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(n_q));
+    cfg.gridDim = dim3(static_cast<unsigned>(n_q), static_cast<unsigned>((npad + 3) / 4));
     cfg.blockDim = dim3(128);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
@@ -1240,6 +1302,9 @@ int score_config(int mode, bool e4m3, int d, int npad, int* stages, int* stages8
 cudaError_t launch_score(int mode, bool e4m3, int d, const CUtensorMap& amap, const CUtensorMap& qmap,
                          const ScoreParams& p, int grid, cudaStream_t s) {
     if (mode == kScoreBlocks) {
+        if (p.app)   // the decode step: whole rows per CTA (fuse = 1)
+            return d == 128 ? launch_t<kScoreBlocks, false, 128, kBlocksAppend>(amap, qmap, p, grid, s)
+                            : launch_t<kScoreBlocks, false, 64, kBlocksAppend>(amap, qmap, p, grid, s);
         if (p.cp)
             return d == 128 ? launch_t<kScoreBlocks, false, 128, kBlocksShard>(amap, qmap, p, grid, s)
                             : launch_t<kScoreBlocks, false, 64, kBlocksShard>(amap, qmap, p, grid, s);

@@ -487,11 +487,15 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelectPara
 
 // ------------------------------------------------ single-CTA rows
 //
-// Rows of up to kRowKeys slots: one CTA of NT threads, keys staged in shared
-// memory, the same four steps without any cross-CTA exchange.
-
-// The kernel is instantiated for 1024 threads (rows up to two per SM: more
-// warps per row shorten each phase) and 512 (many rows: more CTAs per SM).
+// Rows of up to kRowKeys slots: one CTA of NT threads; thread t holds the KPT
+// consecutive slots t*KPT .. t*KPT + KPT - 1 of the row in registers, so every
+// pass over the row (count / min / max, histogram, bin members, compaction)
+// reads registers, and the ordered compaction needs a single block-wide scan
+// of a thread's (greater-than, equal-to) counts.  Every block-wide scan or
+// reduction is one barrier: warp totals go to shared memory and each warp
+// then reduces or scans all of them with shuffles.
+// NT = 1024 serves few rows (up to two per SM: more warps per row shorten
+// each phase), NT = 512 many rows (more CTAs per SM).
 
 constexpr int kRowBlocks = 2048;   // kept-block ids staged in shared memory
 
@@ -504,13 +508,17 @@ struct RowShared {
     uint32_t wa[kWarps];
     uint32_t wb[kWarps];
     uint32_t wc[kWarps];
-    uint32_t wd[kWarps];
+    uint32_t wd[kWarps];     // the compaction's scan (wa..wc may still be read then)
+    uint32_t nmem;
     uint32_t bc[8];
 };
 
-// Exclusive block scan of one value per thread (NT threads).
+// Exclusive block scan of one value per thread (NT threads, thread order);
+// *total = the sum over the block.  One barrier; wtot must not be read or
+// written by another scan until the caller's next barrier.
 template <int NT>
-__device__ __forceinline__ uint32_t row_scan(uint32_t v, uint32_t* wtot, uint32_t* total) {
+__device__ __forceinline__ uint32_t block_scan(uint32_t v, uint32_t* wtot, uint32_t* total) {
+    constexpr int NW = NT / 32;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint32_t incl = v;
 #pragma unroll
@@ -520,43 +528,52 @@ __device__ __forceinline__ uint32_t row_scan(uint32_t v, uint32_t* wtot, uint32_
     }
     if (lane == 31) wtot[warp] = incl;
     __syncthreads();
-    uint32_t before = 0, tot = 0;
+    // every warp scans the NW warp totals
+    uint32_t t = lane < NW ? wtot[lane] : 0u;
+    uint32_t ti = t;
 #pragma unroll
-    for (int w = 0; w < NT / 32; ++w) {
-        const uint32_t x = wtot[w];
-        before += w < warp ? x : 0u;
-        tot += x;
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t x = __shfl_up_sync(0xffffffffu, ti, o);
+        if (lane >= o) ti += x;
     }
-    *total = tot;
+    *total = __shfl_sync(0xffffffffu, ti, 31);
+    const uint32_t before = __shfl_sync(0xffffffffu, ti - t, warp);   // exclusive prefix of this warp
     return before + incl - v;
 }
 
-template <int NT>
-__global__ void __launch_bounds__(NT) select_row_kernel(const SelectParams p) {
-    constexpr int kRowThreads = NT;
-    constexpr int kRowWarps = NT / 32;
-    constexpr int kRowBinsPer = kBins / NT;   // histogram bins each thread scans
+// Outputs of a row are staged in shared memory and written out in order with
+// 16-byte stores when the row's k entries fit (stage_k = k, a multiple of 4;
+// 0 = write each entry where it goes).
+// MODE >= 0 fixes the selection mode at compile time (the token rows of the
+// HISA path, so that their code carries no other mode's branches); -1 reads
+// it from p.
+template <int NT, int KPT, int MODE>
+__global__ void __launch_bounds__(NT, NT >= 1024 ? 1 : 2) select_row_kernel(const SelectParams p, int stage_k) {
+    static_assert(KPT % 4 == 0, "slots per thread in 16-byte groups");
+    static_assert(NT * KPT <= 65535, "packed (gt, eq) counts fit 16 bits each");
+    constexpr int kBinsPer = kBins / NT;   // histogram bins each thread scans
     static_assert(kBins % NT == 0, "bins split evenly over the threads");
-    extern __shared__ uint32_t ks[];
     __shared__ RowShared<NT> sh;
+    extern __shared__ __align__(16) int32_t stage_out[];   // [stage_k] ids, then [stage_k] scores
     grid_dependency_wait();
     grid_launch_dependents();
     const int row = blockIdx.x;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int mode = MODE >= 0 ? MODE : p.mode;
 
     int n = 0, kk = p.k, b = 0, t = 0, nb = 0, cp_own = 0;
     bool bad = false;
-    if (p.mode == kSelF32Rows) {
+    if (mode == kSelF32Rows) {
         n = p.n;
-    } else if (p.mode == kSelMerge) {
+    } else if (mode == kSelMerge) {
         n = p.lists * p.n;
-    } else if (p.mode == kSelHisaTokens) {
+    } else if (mode == kSelHisaTokens) {
         const int4 pl = p.plan[row];
         b = pl.x;
         t = pl.y;
         bad = t < 0;
         n = pl.z * p.B;
-    } else if (p.mode == kSelCpBlocks) {
+    } else if (mode == kSelCpBlocks) {
         // the shard's visible blocks but the own one compete for m - 1 places
         nb = cp_visible_blocks(p.q_seq, p.q_pos, p.len, p.batch, p.cap, p.B, p.id_off * p.B, row, &b,
                                &cp_own, &t);
@@ -566,7 +583,7 @@ __global__ void __launch_bounds__(NT) select_row_kernel(const SelectParams p) {
     } else {
         t = query_position(p.q_seq, p.q_pos, p.len, p.batch, p.cap, row, &b);
         bad = t < 0;
-        if (p.mode == kSelBlocks) {
+        if (mode == kSelBlocks) {
             nb = t / p.B + 1;
             n = nb - 1;
             kk = p.m - 1;
@@ -574,10 +591,10 @@ __global__ void __launch_bounds__(NT) select_row_kernel(const SelectParams p) {
             n = t + 1;
         }
     }
-    if (bad || (p.mode == kSelBlocks && nb <= p.m && !p.tree)) {
-        if (p.mode == kSelBlocks) {
+    if (bad || (mode == kSelBlocks && nb <= p.m && !p.tree)) {
+        if (mode == kSelBlocks) {
             const int keep = bad ? 0 : nb;
-            for (int r = tid; r < p.mm; r += kRowThreads) {
+            for (int r = tid; r < p.mm; r += NT) {
                 const int v = r < keep ? r : -1;
                 p.blocks[static_cast<size_t>(row) * p.mm + r] = v;
                 if (p.blocks_out) p.blocks_out[static_cast<size_t>(row) * p.mm + r] = v;
@@ -589,63 +606,67 @@ __global__ void __launch_bounds__(NT) select_row_kernel(const SelectParams p) {
                 if (bad) set_status(p.status, HISA_DEV_BAD_QUERY);
             }
         } else {
-            for (int r = tid; r < p.k; r += kRowThreads) {
+            for (int r = tid; r < p.k; r += NT) {
                 p.idx[static_cast<size_t>(row) * p.k + r] = -1;
                 if (p.scores) p.scores[static_cast<size_t>(row) * p.k + r] = __int_as_float(0x7fc00000);
             }
-            if (tid == 0 && bad && p.mode != kSelHisaTokens) set_status(p.status, HISA_DEV_BAD_QUERY);
+            if (tid == 0 && bad && mode != kSelHisaTokens) set_status(p.status, HISA_DEV_BAD_QUERY);
         }
         return;
     }
 
     // kept-block ids of a HISA row (slot c belongs to block blk[c / B])
-    const bool blk_smem = p.mode == kSelHisaTokens && p.mm <= kRowBlocks;
+    const bool blk_smem = mode == kSelHisaTokens && p.mm <= kRowBlocks;
     if (blk_smem)
-        for (int r = tid; r < p.mm; r += kRowThreads) sh.blk[r] = p.blocks[static_cast<size_t>(row) * p.mm + r];
+        for (int r = tid; r < p.mm; r += NT) sh.blk[r] = p.blocks[static_cast<size_t>(row) * p.mm + r];
+    for (int i = tid; i < kBins; i += NT) sh.hist[i] = 0u;
+    if (tid == 0) sh.nmem = 0u;
 
-    // 1. stage the keys; count, min, max of the nonzero ones
-    uint32_t cnt = 0, mn = 0xFFFFFFFFu, mx = 0u;
+    // 1. this thread's slots c0 .. c0 + KPT - 1 (key 0 past n); count, min, max
+    const int c0 = tid * KPT;
     // slot c of a merged row: list c / n, entry c % n
     auto merge_at = [&](int c) {
         const int l = c / p.n;
         return (static_cast<size_t>(l) * p.rows + row) * p.n + (c - l * p.n);
     };
-    if (p.mode == kSelF32Rows || p.mode == kSelMerge) {
-        const float* x = p.x + static_cast<size_t>(row) * p.n;
-        for (int c = tid; c < n; c += kRowThreads) {
-            uint32_t v;
-            if (p.mode == kSelMerge) {
-                const size_t o = merge_at(c);
-                v = p.ids[o] < 0 ? 0u : score_key(p.x[o]);   // an empty entry never competes
-            } else {
-                v = score_key(x[c]);
-            }
-            ks[c] = v;
-            if (v != 0u) {
-                ++cnt;
-                mn = min(mn, v);
-                mx = max(mx, v);
-            }
-        }
-    } else {
-        const uint4* g4 = reinterpret_cast<const uint4*>(p.keys + static_cast<size_t>(row) * p.ldk);
-        const int n4 = (n + 3) >> 2;
-#pragma unroll 4
-        for (int c4 = tid; c4 < n4; c4 += kRowThreads) {
-            const uint4 v = __ldcg(g4 + c4);
-            const uint32_t xs[4] = {v.x, v.y, v.z, v.w};
+    uint32_t x[KPT];
+    if (mode == kSelF32Rows || mode == kSelMerge) {
+        const float* xr = p.x + static_cast<size_t>(row) * p.n;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int c = 4 * c4 + j;
-                const uint32_t x = c < n ? xs[j] : 0u;
-                if (c < n) ks[c] = x;
-                if (x != 0u) {
-                    ++cnt;
-                    mn = min(mn, x);
-                    mx = max(mx, x);
+        for (int e = 0; e < KPT; ++e) {
+            const int c = c0 + e;
+            uint32_t v = 0u;
+            if (c < n) {
+                if (mode == kSelMerge) {
+                    const size_t o = merge_at(c);
+                    v = p.ids[o] < 0 ? 0u : score_key(p.x[o]);   // an empty entry never competes
+                } else {
+                    v = score_key(xr[c]);
                 }
             }
+            x[e] = v;
         }
+    } else {
+        // rows are ldk (a multiple of 128) keys apart: a 4-key group that
+        // starts below n lies inside the row
+        const uint4* g4 = reinterpret_cast<const uint4*>(p.keys + static_cast<size_t>(row) * p.ldk + c0);
+#pragma unroll
+        for (int q = 0; q < KPT / 4; ++q) {
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (c0 + 4 * q < n) v = __ldg(g4 + q);   // L1 keeps the half of each sector the next load uses
+            x[4 * q] = c0 + 4 * q < n ? v.x : 0u;
+            x[4 * q + 1] = c0 + 4 * q + 1 < n ? v.y : 0u;
+            x[4 * q + 2] = c0 + 4 * q + 2 < n ? v.z : 0u;
+            x[4 * q + 3] = c0 + 4 * q + 3 < n ? v.w : 0u;
+        }
+    }
+    uint32_t cnt = 0, mn = 0xFFFFFFFFu, mx = 0u;
+#pragma unroll
+    for (int e = 0; e < KPT; ++e) {
+        const uint32_t v = x[e];
+        cnt += v != 0u;
+        mn = v != 0u ? min(mn, v) : mn;
+        mx = max(mx, v);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -659,17 +680,24 @@ __global__ void __launch_bounds__(NT) select_row_kernel(const SelectParams p) {
         sh.wc[warp] = mx;
     }
     __syncthreads();
-    uint32_t nvalid = 0;
-    mn = 0xFFFFFFFFu;
-    mx = 0u;
+    {
+        constexpr int NW = NT / 32;
+        cnt = lane < NW ? sh.wa[lane] : 0u;
+        mn = lane < NW ? sh.wb[lane] : 0xFFFFFFFFu;
+        mx = lane < NW ? sh.wc[lane] : 0u;
 #pragma unroll
-    for (int w = 0; w < kRowWarps; ++w) {
-        nvalid += sh.wa[w];
-        mn = min(mn, sh.wb[w]);
-        mx = max(mx, sh.wc[w]);
+        for (int o = 16; o > 0; o >>= 1) {
+            cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+            mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+            mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        }
     }
+    const uint32_t nvalid = cnt;
 
-    // 2-3. the k-th largest key T and how many keys == T are kept
+    // 2-3. the k-th largest key T and how many keys == T are kept: a
+    // 2048-bin histogram over [lo, hi] finds the bin of the k-th key; a bin of
+    // at most kMembersCap keys is ranked by counting, a crowded one becomes
+    // the next [lo, hi]
     uint32_t T = 0;
     int take_eq = 0;
     if (kk > 0 && nvalid > static_cast<uint32_t>(kk)) {
@@ -678,28 +706,27 @@ __global__ void __launch_bounds__(NT) select_row_kernel(const SelectParams p) {
         for (;;) {
             const uint32_t span = hi - lo;
             const int shift = span == 0 ? 0 : max(0, 32 - __clz(span) - kBinBits);
-            for (int i = tid; i < kBins; i += kRowThreads) sh.hist[i] = 0;
-            __syncthreads();
-            for (int c = tid; c < n; c += kRowThreads) {
-                const uint32_t x = ks[c];
-                if (x != 0u && x >= lo && x <= hi) atomicAdd(&sh.hist[(x - lo) >> shift], 1u);
+#pragma unroll
+            for (int e = 0; e < KPT; ++e) {
+                const uint32_t v = x[e];
+                if (v != 0u && v >= lo && v <= hi) atomicAdd(&sh.hist[(v - lo) >> shift], 1u);
             }
             __syncthreads();
-            // thread t owns kRowBinsPer consecutive bins from the top (highest first)
-            const int b0 = kBins - 1 - kRowBinsPer * tid;
-            uint32_t hs[kRowBinsPer], loc = 0;
+            // thread t owns kBinsPer consecutive bins from the top (highest first)
+            const int b0 = kBins - 1 - kBinsPer * tid;
+            uint32_t hs[kBinsPer], loc = 0;
 #pragma unroll
-            for (int q = 0; q < kRowBinsPer; ++q) {
+            for (int q = 0; q < kBinsPer; ++q) {
                 hs[q] = sh.hist[b0 - q];
                 loc += hs[q];
             }
             uint32_t tot;
-            const uint32_t excl = row_scan<NT>(loc, sh.wd, &tot);
+            const uint32_t excl = block_scan<NT>(loc, sh.wc, &tot);
             const uint32_t kr = static_cast<uint32_t>(krem);
             if (excl < kr && kr <= excl + loc) {
                 uint32_t run = excl;
 #pragma unroll
-                for (int q = 0; q < kRowBinsPer; ++q) {
+                for (int q = 0; q < kBinsPer; ++q) {
                     if (run < kr && kr <= run + hs[q]) {
                         sh.bc[0] = static_cast<uint32_t>(b0 - q);
                         sh.bc[1] = kr - run;
@@ -708,7 +735,6 @@ __global__ void __launch_bounds__(NT) select_row_kernel(const SelectParams p) {
                     run += hs[q];
                 }
             }
-            if (tid == 0) sh.bc[3] = 0;
             __syncthreads();
             const uint32_t bin = sh.bc[0];
             krem = static_cast<int>(sh.bc[1]);
@@ -721,16 +747,17 @@ __global__ void __launch_bounds__(NT) select_row_kernel(const SelectParams p) {
                 break;
             }
             if (nmem <= static_cast<uint32_t>(kMembersCap)) {
-                for (int c = tid; c < n; c += kRowThreads) {
-                    const uint32_t x = ks[c];
-                    if (x != 0u && x >= blo && x <= bhi) {
-                        const uint32_t at = atomicAdd(&sh.bc[3], 1u);
-                        sh.members[at] = (static_cast<unsigned long long>(x) << 32) | static_cast<uint32_t>(c);
+#pragma unroll
+                for (int e = 0; e < KPT; ++e) {
+                    const uint32_t v = x[e];
+                    if (v != 0u && v >= blo && v <= bhi) {
+                        const uint32_t at = atomicAdd(&sh.nmem, 1u);
+                        sh.members[at] = (static_cast<unsigned long long>(v) << 32) | static_cast<uint32_t>(c0 + e);
                     }
                 }
                 __syncthreads();
-                const int m = static_cast<int>(sh.bc[3]);
-                for (int i = tid; i < m; i += kRowThreads) {
+                const int m = static_cast<int>(sh.nmem);
+                for (int i = tid; i < m; i += NT) {
                     const uint32_t xi = static_cast<uint32_t>(sh.members[i] >> 32);
                     int above = 0, equal = 0;
                     for (int j = 0; j < m; ++j) {
@@ -748,103 +775,96 @@ __global__ void __launch_bounds__(NT) select_row_kernel(const SelectParams p) {
                 take_eq = static_cast<int>(sh.bc[5]);
                 break;
             }
-            lo = blo;   // crowded bin: narrow the range and repeat
+            // crowded bin: narrow the range and repeat (nobody reads the
+            // histogram after the barrier above)
+            lo = blo;
             hi = bhi;
+            for (int i = tid; i < kBins; i += NT) sh.hist[i] = 0u;
             __syncthreads();
         }
     }
 
-    // 4. ordered compaction: warp w owns a contiguous slot range
-    const int per_warp = ((n + kRowWarps - 1) / kRowWarps + 31) & ~31;
-    const int w0 = warp * per_warp;
-    const int w1 = min(n, w0 + per_warp);
+    // 4. ordered compaction: one scan of the packed (> T, == T) counts gives
+    // each thread its first output position and its first equal-key rank
+    const bool any = kk > 0;
     uint32_t gt = 0, eq = 0;
-    if (kk > 0) {
-        for (int base = w0; base < w1; base += 32) {
-            const int c = base + lane;
-            const uint32_t x = c < w1 ? ks[c] : 0u;
-            gt += __popc(__ballot_sync(0xffffffffu, x != 0u && x > T));
-            eq += __popc(__ballot_sync(0xffffffffu, x != 0u && x == T));
+    if (any) {
+#pragma unroll
+        for (int e = 0; e < KPT; ++e) {
+            gt += x[e] != 0u && x[e] > T;
+            eq += x[e] != 0u && x[e] == T;
         }
     }
-    __syncthreads();   // bc / wa reuse below
-    if (lane == 0) {
-        sh.wa[warp] = gt;
-        sh.wb[warp] = eq;
-    }
-    __syncthreads();
-    uint32_t eq_run = 0, pos = 0, kept = 0;
-    {
-        uint32_t eqb = 0, off = 0;
-        for (int w = 0; w < kRowWarps; ++w) {
-            const uint32_t e = sh.wb[w];
-            const int room = take_eq - static_cast<int>(eqb);
-            const uint32_t take = room <= 0 ? 0u : (static_cast<uint32_t>(room) < e ? room : e);
-            if (w == warp) {
-                eq_run = eqb;
-                pos = off;
-            }
-            eqb += e;
-            off += sh.wa[w] + take;
-        }
-        kept = off;
-    }
-    const unsigned lt = (1u << lane) - 1u;
-    int32_t* blist = p.mode == kSelBlocks ? p.blocks + static_cast<size_t>(row) * p.mm : nullptr;
-    int32_t* bdbg = p.mode == kSelBlocks && p.blocks_out ? p.blocks_out + static_cast<size_t>(row) * p.mm : nullptr;
-    int32_t* idx = p.mode != kSelBlocks ? p.idx + static_cast<size_t>(row) * p.k : nullptr;
-    float* sc = p.mode != kSelBlocks && p.scores ? p.scores + static_cast<size_t>(row) * p.k : nullptr;
-    const int32_t* blk = p.mode != kSelHisaTokens ? nullptr
+    uint32_t tot;
+    const uint32_t excl = block_scan<NT>((gt << 16) | eq, sh.wd, &tot);
+    const uint32_t gt_before = excl >> 16, eq_before = excl & 0xFFFFu;
+    const uint32_t te = static_cast<uint32_t>(take_eq);
+    const int kept = static_cast<int>((tot >> 16) + min(tot & 0xFFFFu, te));
+
+    int32_t* blist = mode == kSelBlocks ? p.blocks + static_cast<size_t>(row) * p.mm : nullptr;
+    int32_t* bdbg = mode == kSelBlocks && p.blocks_out ? p.blocks_out + static_cast<size_t>(row) * p.mm : nullptr;
+    int32_t* const idx_g = mode != kSelBlocks ? p.idx + static_cast<size_t>(row) * p.k : nullptr;
+    float* const sc_g = mode != kSelBlocks && p.scores ? p.scores + static_cast<size_t>(row) * p.k : nullptr;
+    // token rows with staging: emit into shared memory, write out below
+    const bool staged = stage_k > 0 && mode != kSelBlocks && mode != kSelCpBlocks;
+    int32_t* idx = staged ? stage_out : idx_g;
+    float* sc = !sc_g ? nullptr : staged ? reinterpret_cast<float*>(stage_out + stage_k) : sc_g;
+    const int32_t* blk = mode != kSelHisaTokens ? nullptr
                          : blk_smem ? sh.blk
                                     : p.blocks + static_cast<size_t>(row) * p.mm;
     const int Bsz = p.B;
     const bool pow2 = (Bsz & (Bsz - 1)) == 0;
     const int lgB = __ffs(Bsz) - 1;
-    if (kk > 0) {
-        for (int base = w0; base < w1; base += 32) {
-            const int c = base + lane;
-            const uint32_t x = c < w1 ? ks[c] : 0u;
-            const bool is_gt = x != 0u && x > T;
-            const bool is_eq = x != 0u && x == T;
-            const unsigned eqm = __ballot_sync(0xffffffffu, is_eq);
-            const uint32_t eq_rank = eq_run + __popc(eqm & lt);
-            const bool sel = is_gt || (is_eq && eq_rank < static_cast<uint32_t>(take_eq));
-            const unsigned selm = __ballot_sync(0xffffffffu, sel);
-            if (sel) {
-                const int at = static_cast<int>(pos + __popc(selm & lt));
-                if (blist) {
-                    blist[at] = c;
-                    if (bdbg) bdbg[at] = c;
+    if (any) {
+        uint32_t pos = gt_before + min(eq_before, te);
+        uint32_t eqr = eq_before;
+        // a thread's KPT slots start at a multiple of KPT, so they lie in one
+        // kept block when KPT divides B: their ids are consecutive from one lookup
+        const bool one_blk = blk && Bsz % KPT == 0;
+        const int bi0 = one_blk ? (pow2 ? c0 >> lgB : c0 / Bsz) : 0;
+        const int id0 = one_blk ? blk[bi0] * Bsz + (c0 - bi0 * Bsz) + p.id_off : 0;
+#pragma unroll
+        for (int e = 0; e < KPT; ++e) {
+            const uint32_t v = x[e];
+            const bool is_eq = v != 0u && v == T;
+            const bool sel = (v != 0u && v > T) || (is_eq && eqr < te);
+            eqr += is_eq;
+            const int c = c0 + e;
+            const int at = static_cast<int>(pos);
+            pos += sel;
+            if (!sel) continue;
+            if (blist) {
+                blist[at] = c;
+                if (bdbg) bdbg[at] = c;
+            } else {
+                if (one_blk) {
+                    idx[at] = id0 + e;
+                } else if (blk) {
+                    const int bi = pow2 ? c >> lgB : c / Bsz;
+                    idx[at] = blk[bi] * Bsz + (c - bi * Bsz) + p.id_off;
+                } else if (mode == kSelMerge) {
+                    idx[at] = p.ids[merge_at(c)];
                 } else {
-                    if (blk) {
-                        const int bi = pow2 ? c >> lgB : c / Bsz;
-                        idx[at] = blk[bi] * Bsz + (c - bi * Bsz) + p.id_off;
-                    } else if (p.mode == kSelMerge) {
-                        idx[at] = p.ids[merge_at(c)];
-                    } else {
-                        idx[at] = c + p.id_off;
-                    }
-                    if (sc) sc[at] = key_score(x);
+                    idx[at] = c + p.id_off;
                 }
+                if (sc) sc[at] = key_score(v);
             }
-            eq_run += __popc(eqm);
-            pos += __popc(selm);
         }
     }
-    if (p.mode == kSelBlocks) {
-        for (int r = static_cast<int>(kept) + tid; r < p.mm; r += kRowThreads) {
-            const int v = r == static_cast<int>(kept) ? nb - 1 : -1;   // own block last
+    if (mode == kSelBlocks) {
+        for (int r = kept + tid; r < p.mm; r += NT) {
+            const int v = r == kept ? nb - 1 : -1;   // own block last
             blist[r] = v;
             if (bdbg) bdbg[r] = v;
         }
         if (tid == 0) {
-            const int keep = static_cast<int>(kept) + 1;
+            const int keep = kept + 1;
             p.nblocks[row] = keep;
             if (p.nblocks_out) p.nblocks_out[row] = keep;
             p.plan[row] = make_int4(b, t, keep, 0);
         }
     } else {
-        int r0 = static_cast<int>(kept);
+        int r0 = kept;
         if (cp_own) {
             // the shard holds the row's own block: it follows the m - 1 others,
             // marked with an infinite score so that every merge keeps it
@@ -854,17 +874,37 @@ __global__ void __launch_bounds__(NT) select_row_kernel(const SelectParams p) {
             }
             ++r0;
         }
-        for (int r = r0 + tid; r < p.k; r += kRowThreads) {
+        for (int r = r0 + tid; r < p.k; r += NT) {
             idx[r] = -1;
             if (sc) sc[r] = __int_as_float(0x7fc00000);
+        }
+        if (staged) {
+            __syncthreads();
+            const int4* si = reinterpret_cast<const int4*>(stage_out);
+            int4* gi = reinterpret_cast<int4*>(idx_g);
+            for (int r = tid; r < p.k / 4; r += NT) gi[r] = si[r];
+            if (sc_g) {
+                const int4* ss = reinterpret_cast<const int4*>(stage_out + stage_k);
+                int4* gs = reinterpret_cast<int4*>(sc_g);
+                for (int r = tid; r < p.k / 4; r += NT) gs[r] = ss[r];
+            }
         }
     }
 }
 
-template <int NT>
-cudaError_t launch_row_t(const SelectParams& p, int max_n, cudaStream_t s) {
-    const size_t smem = static_cast<size_t>(max_n > 4 ? max_n : 4) * sizeof(uint32_t);
-    cudaError_t e = smem_limit(reinterpret_cast<const void*>(select_row_kernel<NT>), smem);
+// Token rows whose k outputs (ids and scores) fit in this much shared
+// memory, with k a multiple of 4 and 16-byte aligned rows, are staged.
+constexpr int kStageBytes = 64 * 1024;
+
+template <int NT, int KPT, int MODE>
+cudaError_t launch_row_m(const SelectParams& p, cudaStream_t s) {
+    const bool tokens = p.mode != kSelBlocks && p.mode != kSelCpBlocks;
+    const int per = p.scores ? 8 : 4;
+    const bool aligned16 = (reinterpret_cast<uintptr_t>(p.idx) % 16 == 0) &&
+                           (!p.scores || reinterpret_cast<uintptr_t>(p.scores) % 16 == 0);
+    const int stage_k = tokens && p.k % 4 == 0 && aligned16 && p.k * per <= kStageBytes ? p.k : 0;
+    const size_t smem = static_cast<size_t>(stage_k) * per;
+    cudaError_t e = smem_limit(reinterpret_cast<const void*>(select_row_kernel<NT, KPT, MODE>), smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(p.rows));
@@ -876,11 +916,28 @@ cudaError_t launch_row_t(const SelectParams& p, int max_n, cudaStream_t s) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, select_row_kernel<NT>, p);
+    return cudaLaunchKernelEx(&cfg, select_row_kernel<NT, KPT, MODE>, p, stage_k);
 }
 
+template <int NT, int KPT>
+cudaError_t launch_row_t(const SelectParams& p, cudaStream_t s) {
+    return p.mode == kSelHisaTokens ? launch_row_m<NT, KPT, kSelHisaTokens>(p, s) : launch_row_m<NT, KPT, -1>(p, s);
+}
+
+// Threads per row: 1024 while there are at most two rows per SM, else 512
+// (rows over 512 * 32 slots keep 1024); slots per thread: the fewest that
+// cover the longest row.
 cudaError_t launch_row(const SelectParams& p, int max_n, int sms, cudaStream_t s) {
-    return p.rows <= 2 * sms ? launch_row_t<1024>(p, max_n, s) : launch_row_t<512>(p, max_n, s);
+    const bool wide = p.rows <= 2 * sms || max_n > 512 * 32;
+    if (wide) {
+        if (max_n <= 1024 * 4) return launch_row_t<1024, 4>(p, s);
+        if (max_n <= 1024 * 8) return launch_row_t<1024, 8>(p, s);
+        if (max_n <= 1024 * 16) return launch_row_t<1024, 16>(p, s);
+        return launch_row_t<1024, 24>(p, s);
+    }
+    if (max_n <= 512 * 8) return launch_row_t<512, 8>(p, s);
+    if (max_n <= 512 * 16) return launch_row_t<512, 16>(p, s);
+    return launch_row_t<512, 32>(p, s);
 }
 
 template <bool STAGE>

@@ -179,6 +179,33 @@ int hisa_select(const hisa_kv* kv, const uint16_t* Q, const float* w, const int3
                 float* scores, void* ws, size_t ws_bytes, hisa_stream_t stream);
 
 /*
+ * hisa_decode_step — one decode step of a batch: hisa_append, then
+ * hisa_select for every sequence's new last position, in one call.
+ * HISA blog "Hierarchical Indexing Makes Sparse Attention Actually Fast",
+ * "HISA's Approach" (the summary is kept current as tokens are appended) and
+ * the two stages of hisa_select (arXiv abstract, stages (1) and (2)).
+ *   tok        [batch, d]  the new key of each sequence (bf16 or e4m3 codes)
+ *   tok_scale  [batch]     fp32 scales (E4M3) or NULL
+ *   Q [batch, H, d] bf16, w [batch, H] fp32: query row b belongs to sequence b
+ *   idx [batch, k] int32 out, scores [batch, k] fp32 out or NULL: as hisa_select
+ *   ws  workspace of at least hisa_decode_step_workspace_bytes(...) bytes
+ * Results (idx, scores, keys, key scales, pooled, pooled_hl, len, status) are
+ * those of hisa_append(kv, tok, tok_scale) followed by hisa_select(kv, Q, w,
+ * q_seq = 0..batch-1, q_pos = NULL, m, k), bit for bit.  Rows of at most
+ * 4 x 128 blocks and batches of at most two rows per SM run the append inside
+ * the block-scoring kernel (no separate launch): each row writes its key,
+ * recomputes its trailing block's representative and scores its blocks in
+ * one CTA.  Other sizes run the two calls' launches.  A full sequence is left
+ * as it is (HISA_DEV_CAPACITY) and selects for position cap - 1; a len[]
+ * outside [0, cap] sets HISA_DEV_BAD_LEN and HISA_DEV_BAD_QUERY and gives a
+ * -1 row.  Errors as hisa_append and hisa_select.
+ */
+size_t hisa_decode_step_workspace_bytes(const hisa_kv* kv, int H, int m, int k);
+int hisa_decode_step(const hisa_kv* kv, const void* tok, const float* tok_scale, const uint16_t* Q,
+                     const float* w, int H, int m, int k, int32_t* idx, float* scores, void* ws,
+                     size_t ws_bytes, hisa_stream_t stream);
+
+/*
  * hisa_select_inspect — hisa_select plus its intermediate results, for
  * verification of the two stages separately.
  *   blocks  [n_q, min(m, nblk)] int32 out (or NULL): kept block ids per row,
