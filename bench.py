@@ -687,6 +687,70 @@ def run_select_only(args):
             "ms_per_select": ms, "selections_per_s": n_q / (ms / 1e3)}
 
 
+def run_ncu_case(name: str, reps: int = 3):
+    """--ncu-case NAME: a fixed, untimed sequence of library calls on one
+    workload, L2 flushed between calls, for ncu captures filtered by kernel
+    name (each call kind `reps` times, in this order):
+      decode-32k-b64          hisa_pool_blocks, hisa_decode_step, hisa_select,
+                              dsa_flat_select (pool, append, block scoring,
+                              token scoring, top-k, flat scoring, cluster top-k)
+      decode-128k-b32-e4m3    hisa_pool_blocks, hisa_select (e4m3 pool, fp8 scoring)
+      prefill-64k-chunk4096   hisa_select (stage 2 on L2-resident keys)
+      sparse-attention        hisa_sparse_attn over the decode-32k-b64 selection"""
+    import torch
+    import hierarchical_top_indexer_b200 as hisa
+    from hisa_inputs import CONFIGS, make_config
+    dev = torch.device("cuda", 0)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def rep(fn):
+        for _ in range(reps):
+            fn()
+            flush.fill_(7)
+
+    attn = name == "sparse-attention"
+    cfg = next(i for i, c in CONFIGS.items() if c["name"] == ("decode-32k-b64" if attn else name))
+    steps = reps + 1 if cfg == 1 else 0
+    case = make_config(cfg, cap=CONFIGS[cfg]["L"] + steps, append_steps=steps,
+                       append_query_sets=1) if steps else make_config(cfg)
+    kv = hisa.KVCache.from_case(case, device=dev)
+    Q = torch.from_numpy(case.Q.view(np.int16)).view(torch.bfloat16).to(dev)
+    w = torch.from_numpy(case.w).to(dev)
+    qs = torch.from_numpy(case.q_seq).to(dev)
+    qp = torch.from_numpy(case.q_pos).to(dev)
+    n_q, H, m, k = case.n_q, case.H, case.m, case.k
+    idx = torch.empty((n_q, k), dtype=torch.int32, device=dev)
+    ws = hisa.workspace(max(hisa.hisa_select_workspace_bytes(kv, n_q, H, m, k),
+                            hisa.dsa_flat_workspace_bytes(kv, n_q, H, k)), dev)
+    if not attn:
+        rep(lambda: hisa.hisa_pool_blocks(kv))
+    else:
+        hisa.hisa_pool_blocks(kv)
+    if cfg == 1 and not attn:
+        toks = torch.from_numpy(case.append_keys.view(np.int16)).view(torch.bfloat16).to(dev)
+        AQ = torch.from_numpy(case.append_Q[0].view(np.int16)).view(torch.bfloat16).to(dev)
+        AW = torch.from_numpy(case.append_w[0]).to(dev)
+        it = iter(range(steps))
+        rep(lambda: hisa.hisa_decode_step(kv, toks[next(it)], AQ, AW, m, k, ws=ws, idx=idx))
+    rep(lambda: hisa.hisa_select(kv, Q, w, qs, qp, m, k, ws=ws, idx=idx))
+    if cfg == 1 and not attn:
+        rep(lambda: hisa.dsa_flat_select(kv, Q, w, qs, qp, k, ws=ws, idx=idx))
+    if attn:
+        g = torch.Generator(device=dev)
+        g.manual_seed(20260331)
+        Ha, cap = 128, case.cap
+        Kc = torch.randn((case.batch, cap, 128), generator=g, device=dev).to(torch.bfloat16)
+        Vc = torch.randn((case.batch, cap, 128), generator=g, device=dev).to(torch.bfloat16)
+        Qa = torch.randn((n_q, Ha, 128), generator=g, device=dev).to(torch.bfloat16)
+        aws = hisa.workspace(hisa.hisa_sparse_attn_workspace_bytes(n_q, k), dev)
+        out = torch.empty((n_q, Ha, 128), dtype=torch.float32, device=dev)
+        lse = torch.empty((n_q, Ha), dtype=torch.float32, device=dev)
+        rep(lambda: hisa.hisa_sparse_attn(Qa, Kc, Vc, kv.len, qs, idx, ws=aws, out=out, lse=lse))
+    torch.cuda.synchronize()
+    assert kv.status_bits() == 0, f"device status {kv.status_bits():#x}"
+    return {"ncu_case": name, "reps": reps}
+
+
 # ----------------------------------------------------------- CPU baseline
 
 
@@ -804,6 +868,10 @@ def main(argv=None, backend: str = "nccl"):
     ap.add_argument("--select-only", default=None,
                     help="time only hisa_select on this workload (a name from hisa_inputs)")
     ap.add_argument("--flat", action="store_true", help="with --select-only: dsa_flat_select")
+    ap.add_argument("--ncu-case", default=None,
+                    choices=["decode-32k-b64", "decode-128k-b32-e4m3", "prefill-64k-chunk4096",
+                             "sparse-attention"],
+                    help="run a fixed untimed call sequence on one workload (for ncu captures)")
     ap.add_argument("--attn-only", action="store_true",
                     help="time only the sparse attention over the 32K decode selection")
     ap.add_argument("--workload-steps", type=int, default=20,
@@ -832,6 +900,11 @@ def main(argv=None, backend: str = "nccl"):
         if args.select_only:
             if rank == 0:
                 print(json.dumps(run_select_only(args)), flush=True)
+            return 0
+
+        if args.ncu_case:
+            if rank == 0:
+                print(json.dumps(run_ncu_case(args.ncu_case)), flush=True)
             return 0
 
         r = run_gpu(args, rank, world)

@@ -198,7 +198,19 @@ struct Carve {
 struct HisaWs {
     size_t bkeys, blocks, nblocks, plan, tkeys, q8, w8, total;
     int ldb, ldt, mm;
+    // block-centric token scoring (rows sharing their keys): the inverted index
+    bool bc;
+    size_t bc_cnt, bc_off, bc_rank, bc_pairs, bc_units, bc_nunits;
 };
+
+// Rows that share their keys (many rows per sequence, as a prefill chunk)
+// score their tokens block by block (score_bc.cu) where that kernel applies:
+// bf16 keys, B = 128, npad in {32, 64, 128}, H % 4 == 0.
+bool use_block_centric(const KvView& v, int n_q, int H, int mm) {
+    const int npad = (H + 15) / 16 * 16;
+    return !v.e4m3 && v.B == 128 && (npad == 32 || npad == 64 || npad == 128) && H % 4 == 0 &&
+           mm <= 2048 && n_q >= 256 && n_q >= 16 * v.batch && n_q < (1 << 21);
+}
 
 // e4m3 keys with d = 128 are scored on the fp8 tensor cores against split
 // query heads (launch_qsplit), which the workspace holds.
@@ -223,6 +235,17 @@ HisaWs hisa_ws(const KvView& v, int n_q, int H, int m) {
     w.plan = c.take(static_cast<size_t>(n_q) * 16);
     w.tkeys = c.take(static_cast<size_t>(n_q) * w.ldt * 4);
     take_q8(c, v, n_q, H, &w.q8, &w.w8);
+    w.bc = use_block_centric(v, n_q, H, w.mm);
+    if (w.bc) {
+        const size_t nbj = static_cast<size_t>(v.batch) * v.nblk;
+        const size_t pairs = static_cast<size_t>(n_q) * w.mm;
+        w.bc_cnt = c.take(nbj * 4);
+        w.bc_off = c.take(nbj * 4);
+        w.bc_rank = c.take(pairs * 4);
+        w.bc_pairs = c.take(pairs * 4);
+        w.bc_units = c.take(bc_max_units(n_q, w.mm, static_cast<int>(nbj)) * 16);
+        w.bc_nunits = c.take(4);
+    }
     w.total = c.off;
     return w;
 }
@@ -436,8 +459,45 @@ int token_stage(const KvView& v, const HisaWs& L, uint8_t* base, const uint16_t*
     p.blocks = blocks;
     p.plan_in = plan;
     p.mm = L.mm;
-    rc = run_score(kScoreHisa, v, kmap, qmap, p, s);
-    if (rc) return rc;
+    if (L.bc && id_off == 0) {
+        // block-centric: an inverted index of the kept lists, then one unit
+        // per (block, up to 32 rows that kept it)
+        BcParams bp;
+        std::memset(&bp, 0, sizeof bp);
+        bp.plan = plan;
+        bp.w = w;
+        bp.n_q = n_q;
+        bp.H = H;
+        bp.npad = npad_of(H);
+        bp.cap = v.cap;
+        bp.nblk = v.nblk;
+        bp.mm = L.mm;
+        bp.cnt = reinterpret_cast<int32_t*>(base + L.bc_cnt);
+        bp.off = reinterpret_cast<int32_t*>(base + L.bc_off);
+        bp.rank = reinterpret_cast<int32_t*>(base + L.bc_rank);
+        bp.pairs_w = reinterpret_cast<uint32_t*>(base + L.bc_pairs);
+        bp.units_w = reinterpret_cast<int4*>(base + L.bc_units);
+        bp.n_units_w = reinterpret_cast<int32_t*>(base + L.bc_nunits);
+        bp.pairs = bp.pairs_w;
+        bp.units = bp.units_w;
+        bp.n_units = bp.n_units_w;
+        bp.out = tkeys;
+        bp.ldo = L.ldt;
+        bp.status = v.status;
+        bp.counts = reinterpret_cast<unsigned long long*>(counts);
+        bp.counts_ld = counts_ld;
+        bp.counts_col = counts_col;
+        const int sms = sm_count();
+        if (sms <= 0) return HISA_E_CUDA;
+        PhaseScope ps(HISA_PHASE_TOKEN_SCORE, s);
+        rc = cuda_status(launch_bc_index(bp, blocks, v.batch * v.nblk, s));
+        if (rc) return rc;
+        rc = cuda_status(launch_bc_score(kmap, qmap, bp, sms, s));
+        if (rc) return rc;
+    } else {
+        rc = run_score(kScoreHisa, v, kmap, qmap, p, s);
+        if (rc) return rc;
+    }
     SelectParams sp;
     std::memset(&sp, 0, sizeof sp);
     sp.mode = kSelHisaTokens;

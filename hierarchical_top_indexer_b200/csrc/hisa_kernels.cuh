@@ -257,6 +257,34 @@ cudaError_t launch_score(int mode, bool e4m3, int d, const CUtensorMap& keys_map
 
 cudaError_t launch_select(const SelectParams& p, int max_n, int sms, cudaStream_t s);
 
+// Block-centric token scoring (score_bc.cu) for rows sharing their keys:
+// bf16 keys, B = 128, npad in {32, 64, 128}, H % 4 == 0, kept lists of at
+// most 2048 blocks.  Output: score keys [n_q, ldo] as kScoreHisa writes them.
+struct BcParams {
+    const int4* plan;        // [n_q] {sequence, position (-1: invalid), kept blocks, 0}
+    const float* w;          // [n_q, H]
+    int n_q, H, npad, cap, nblk, mm;
+    // inverted index of the kept lists (workspace), built by launch_bc_index
+    int32_t* cnt;            // [batch * nblk] pairs per block
+    int32_t* off;            // [batch * nblk] first pair of each block
+    int32_t* rank;           // [n_q * mm] a pair's place in its block's list
+    uint32_t* pairs_w;       // [n_q * mm] (row << 11) | r, grouped by block
+    int4* units_w;           // [bc_max_units] {b * nblk + j, first pair, pairs, 0}
+    int32_t* n_units_w;      // [1]
+    const uint32_t* pairs;   // read views of the three above
+    const int4* units;
+    const int32_t* n_units;
+    uint32_t* out;           // [n_q, ldo] score keys
+    int ldo;
+    uint32_t* status;
+    unsigned long long* counts;   // null, or the token slots scored per row go to
+    int counts_ld, counts_col;    // counts[row * counts_ld + counts_col + 1]
+};
+size_t bc_max_units(int n_q, int mm, int nbj);
+cudaError_t launch_bc_index(const BcParams& p, const int32_t* blocks, int nbj, cudaStream_t s);
+cudaError_t launch_bc_score(const CUtensorMap& kmap, const CUtensorMap& qmap, const BcParams& p, int sms,
+                            cudaStream_t s);
+
 // Query heads for scoring e4m3 keys (d = 128) on the fp8 tensor cores: every
 // head of Q [n_q, H, 128] bf16 is scaled by a power of two 2^e and split into
 // two e4m3 pieces, q * 2^e = q1 + q2; q8 [n_q, 2 * npad, 128] holds the q1

@@ -76,9 +76,13 @@ __host__ __device__ constexpr bool uses_f8(int mode, bool e4m3, int d) {
     return e4m3 && d == 128 && mode != kScoreBlocks;
 }
 
-// Columns of one accumulator: the H heads, or for fp8 the two query pieces.
+// Columns of one accumulator: the H heads (padded).  For fp8 scoring both
+// e4m3 pieces of a query head accumulate into the head's column.
 __host__ __device__ inline int acc_width(int mode, bool e4m3, int d, int npad) {
-    return uses_f8(mode, e4m3, d) ? 2 * npad : npad;
+    (void)mode;
+    (void)e4m3;
+    (void)d;
+    return npad;
 }
 
 __host__ __device__ constexpr int score_threads(int mode, bool e4m3, int d) {
@@ -92,9 +96,6 @@ __host__ __device__ constexpr bool two_per_sm_kind(int mode, bool e4m3, int d) {
     return mode != kScoreBlocks && !(e4m3 && !uses_f8(mode, e4m3, d));
 }
 
-__host__ __device__ inline int ctas_per_sm(int mode, bool e4m3, int d, int npad) {
-    return two_per_sm_kind(mode, e4m3, d) && acc_width(mode, e4m3, d, npad) <= 128 ? 2 : 1;
-}
 
 __host__ __device__ inline Layout score_layout(int mode, bool e4m3, int d, int npad, int sa, int s8) {
     const int halves = d / 64;
@@ -123,6 +124,14 @@ __host__ __device__ inline Layout score_layout(int mode, bool e4m3, int d, int n
     off += 16;
     L.total = off;
     return L;
+}
+
+// Two CTAs per SM when the kind allows it, the accumulators fit half of TMEM
+// and two operand stages fit half of the shared memory (wide heads at
+// d = 128 do not: one CTA then takes the whole SM).
+__host__ __device__ inline int ctas_per_sm(int mode, bool e4m3, int d, int npad) {
+    if (!two_per_sm_kind(mode, e4m3, d) || acc_width(mode, e4m3, d, npad) > 128) return 1;
+    return score_layout(mode, e4m3, d, npad, 2, 0).total + 1024 <= static_cast<uint32_t>(kSmem2) ? 2 : 1;
 }
 
 // TMEM allocation for `cols` accumulator columns: a power of two, at least 32.
@@ -308,52 +317,6 @@ __device__ __forceinline__ float head_sum(uint32_t taddr, const float* wv) {
             }
     }
     return (a[0] + a[1]) + (a[2] + a[3]);
-}
-
-// fp8 accumulators: columns [0, NP) hold q1 . x and [NP, 2 NP) hold q2 . x per
-// head; sum_h w'_h * ReLU(q1 . x + q2 . x), w' carrying the query scale 2^-e.
-template <int NP>
-__device__ __forceinline__ float head_sum2(uint32_t taddr, const float* wv) {
-    float a[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int g = 0; g < NP; g += 32) {
-        constexpr int kG = NP < 32 ? NP : 32;
-        uint32_t r1[kG], r2[kG];
-#pragma unroll
-        for (int c = 0; c < kG; c += 16)
-            if (g + c < NP) {
-                tmem_ld16_nowait(taddr + g + c, r1 + c);
-                tmem_ld16_nowait(taddr + NP + g + c, r2 + c);
-            }
-        float4 wg[kG / 4];
-#pragma unroll
-        for (int h = 0; h < kG; h += 4)
-            if (g + h < NP) wg[h / 4] = lds_f32x4(wv + g + h);
-        tmem_ld_wait();
-#pragma unroll
-        for (int h = 0; h < kG; h += 4) {
-            if (g + h >= NP) break;
-            const float4 w4 = wg[h / 4];
-            a[0] = fmaf(w4.x, fmaxf(__uint_as_float(r1[h]) + __uint_as_float(r2[h]), 0.f), a[0]);
-            a[1] = fmaf(w4.y, fmaxf(__uint_as_float(r1[h + 1]) + __uint_as_float(r2[h + 1]), 0.f), a[1]);
-            a[2] = fmaf(w4.z, fmaxf(__uint_as_float(r1[h + 2]) + __uint_as_float(r2[h + 2]), 0.f), a[2]);
-            a[3] = fmaf(w4.w, fmaxf(__uint_as_float(r1[h + 3]) + __uint_as_float(r2[h + 3]), 0.f), a[3]);
-        }
-    }
-    return (a[0] + a[1]) + (a[2] + a[3]);
-}
-
-__device__ __forceinline__ float head_sum2_any(int npad, uint32_t taddr, const float* wv) {
-    switch (npad) {
-        case 16: return head_sum2<16>(taddr, wv);
-        case 32: return head_sum2<32>(taddr, wv);
-        case 48: return head_sum2<48>(taddr, wv);
-        case 64: return head_sum2<64>(taddr, wv);
-        case 80: return head_sum2<80>(taddr, wv);
-        case 96: return head_sum2<96>(taddr, wv);
-        case 112: return head_sum2<112>(taddr, wv);
-        default: return head_sum2<128>(taddr, wv);
-    }
 }
 
 __device__ __forceinline__ float head_sum_any(int npad, uint32_t taddr, const float* wv) {
@@ -874,7 +837,7 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
         }
     } else if (warp == kWarpMma) {
         if (lane == 0) {
-            const uint32_t idesc = kF8 ? idesc_e4m3_f32(static_cast<uint32_t>(NW))
+            const uint32_t idesc = kF8 ? idesc_e4m3_f32(static_cast<uint32_t>(npad))
                                        : idesc_bf16_f32(static_cast<uint32_t>(npad));
             int it = 0, qloads = 0, cur_row = -1;
             uint32_t q_base = 0;
@@ -913,11 +876,16 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * NW);
                 const uint32_t a_base = smem_addr(sA + s * kStageBytes);
                 if (kF8) {
-                    // 128 candidates x (q1 | q2 pieces of the heads) x 128 bytes: four K = 32 steps
+                    // 128 candidates x npad heads x 128 bytes: four K = 32 steps,
+                    // each for the q1 piece and then the q2 piece of every head
+                    // (rows npad .. 2 npad - 1 of the split heads) into the same
+                    // accumulator: D = K (q1 + q2)^T
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_e4m3(d_tmem, sw128_kmajor_desc(a_base + kk * 32), sw128_kmajor_desc(q_base + kk * 32),
-                                  idesc, kk ? 1u : 0u);
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t adesc = sw128_kmajor_desc(a_base + kk * 32);
+                        umma_e4m3(d_tmem, adesc, sw128_kmajor_desc(q_base + kk * 32), idesc, kk ? 1u : 0u);
+                        umma_e4m3(d_tmem, adesc, sw128_kmajor_desc(q_base + npad * 128 + kk * 32), idesc, 1u);
+                    }
                 } else {
 #pragma unroll
                 for (int kh = 0; kh < kHalves; ++kh) {
@@ -1028,7 +996,7 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
                 tc_fence_after();
                 const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                                        static_cast<uint32_t>(a * NW);
-                acc = kF8 ? head_sum2_any(npad, taddr, wv) : head_sum_any(npad, taddr, wv);
+                acc = head_sum_any(npad, taddr, wv);
                 tc_fence_before();
             } else if (ok) {
                 ok = false;

@@ -548,7 +548,7 @@ __device__ __forceinline__ uint32_t block_scan(uint32_t v, uint32_t* wtot, uint3
 // HISA path, so that their code carries no other mode's branches); -1 reads
 // it from p.
 template <int NT, int KPT, int MODE>
-__global__ void __launch_bounds__(NT, NT >= 1024 ? 1 : 2) select_row_kernel(const SelectParams p, int stage_k) {
+__global__ void __launch_bounds__(NT, NT >= 1024 ? 1 : (NT >= 512 ? 2 : 4)) select_row_kernel(const SelectParams p, int stage_k) {
     static_assert(KPT % 4 == 0, "slots per thread in 16-byte groups");
     static_assert(NT * KPT <= 65535, "packed (gt, eq) counts fit 16 bits each");
     constexpr int kBinsPer = kBins / NT;   // histogram bins each thread scans
@@ -924,10 +924,13 @@ cudaError_t launch_row_t(const SelectParams& p, cudaStream_t s) {
     return p.mode == kSelHisaTokens ? launch_row_m<NT, KPT, kSelHisaTokens>(p, s) : launch_row_m<NT, KPT, -1>(p, s);
 }
 
-// Threads per row: 1024 while there are at most two rows per SM, else 512
-// (rows over 512 * 32 slots keep 1024); slots per thread: the fewest that
-// cover the longest row.
+// Threads per row: 256 for rows of at most 1024 slots; otherwise 1024 while
+// there are at most two rows per SM, else 512 (rows over 512 * 32 slots keep
+// 1024); slots per thread: the fewest that cover the longest row.
 cudaError_t launch_row(const SelectParams& p, int max_n, int sms, cudaStream_t s) {
+    // short rows (block selection at long contexts, merges): 256 threads, whose
+    // barriers and scans are cheaper in a chain of latency-bound phases
+    if (max_n <= 256 * 4) return launch_row_t<256, 4>(p, s);
     const bool wide = p.rows <= 2 * sms || max_n > 512 * 32;
     if (wide) {
         if (max_n <= 1024 * 4) return launch_row_t<1024, 4>(p, s);

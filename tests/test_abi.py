@@ -221,3 +221,31 @@ def test_sparse_attention_checks(hisa):
     assert call(out=P(20)) == hisa.HISA_E_INVAL              # output rows need 16-byte alignment
     assert call(ws_bytes=16) == hisa.HISA_E_WORKSPACE
     assert call(n_q=0, Qa=None) == hisa.HISA_OK
+
+
+def test_decode_step_checks_before_any_launch(hisa):
+    """hisa_decode_step rejects bad arguments on the host (no CUDA call is
+    possible on this machine, so reaching one would return HISA_E_CUDA)."""
+    lib = hisa.lib()
+    P = ctypes.c_void_p
+    kv = _kv(hisa, cap=32768, B=128)
+
+    def step(kvp=ctypes.byref(kv), tok=P(16), tok_scale=None, Q=P(16), w=P(16), H=64, m=64, k=2048,
+             idx=P(16), scores=None, ws=P(256), ws_bytes=1 << 30):
+        return lib.hisa_decode_step(kvp, tok, tok_scale, Q, w, H, m, k, idx, scores, ws, ws_bytes, None)
+
+    assert step(kvp=None) == hisa.HISA_E_INVAL
+    assert step(tok=None) == hisa.HISA_E_INVAL
+    assert step(tok=P(8)) == hisa.HISA_E_INVAL                      # misaligned key rows
+    assert step(kvp=ctypes.byref(_kv(hisa, cap=32768, dtype=1, key_scale=16))) == hisa.HISA_E_INVAL  # e4m3 without scales
+    assert step(Q=None) == hisa.HISA_E_INVAL
+    assert step(idx=None) == hisa.HISA_E_INVAL
+    assert step(scores=P(2)) == hisa.HISA_E_INVAL
+    assert step(m=0) == hisa.HISA_E_INVAL
+    assert step(k=0) == hisa.HISA_E_INVAL
+    assert step(H=0) == hisa.HISA_E_UNSUPPORTED
+    assert step(kvp=ctypes.byref(_kv(hisa, B=100))) == hisa.HISA_E_UNSUPPORTED
+    assert step(ws=None) == hisa.HISA_E_WORKSPACE
+    assert step(ws_bytes=16) == hisa.HISA_E_WORKSPACE
+    need = lib.hisa_decode_step_workspace_bytes(ctypes.byref(kv), 64, 64, 2048)
+    assert need == lib.hisa_select_workspace_bytes(ctypes.byref(kv), kv.batch, 64, 64, 2048) > 0
