@@ -274,18 +274,21 @@ def run_gpu(args, rank, world):
     step_ms = [a.elapsed_time(b) for a, b in ev]
     total_ms = float(sum(step_ms))
     total_ms = max_over_ranks(total_ms, world, dev)
-    # Per-kernel durations: the same steps again with an event pair around
-    # every launch (separate pass: those events stop the launches from
-    # overlapping, so the timed steps above run without them).
+    # Per-kernel durations: the same steps again, captured as graphs like the
+    # timed ones but with an event pair around every launch (separate pass:
+    # those events stop the launches from overlapping, so the timed steps
+    # above run without them).
     hisa.hisa_profile_enable(True)
     hisa.hisa_profile_read(reset=True)
-    for i in range(n_prof):
-        s = W + K + i
-        step(s, idx[s % 2])
+    pgraphs = capture_steps([lambda s=W + K + i: step(s, idx[s % 2]) for i in range(n_prof)], dev)
+    torch.cuda.synchronize()
+    for g in pgraphs:
+        g.replay()
         flush.fill_(7)
     torch.cuda.synchronize()
     phases = hisa.hisa_profile_read(reset=True)
     hisa.hisa_profile_enable(False)
+    del pgraphs
     launches = sum(n for _, n in phases.values()) * K // n_prof
 
     # select-only comparison: HISA vs the flat scan on the same rows
@@ -345,26 +348,50 @@ def run_gpu(args, rank, world):
 
 def run_e2e(hisa, kv, case, toks, Qs, Ws, q_seq, ws, stream, base, E):
     """The decode step end to end through the public calls: every step copies
-    its inputs (new keys, Q, w) from pinned host memory to the device, runs
-    hisa_decode_step, and copies its 64 x 2048 indices back to
-    pinned host memory.  Steps are pipelined the way a serving loop would run
-    them: host-to-device copies on one stream, the kernels on the launching
-    stream, device-to-host copies on a third, two device slots for inputs and
-    outputs, events for every dependency.  One event pair brackets all E
-    steps; the caches (512 MiB of keys) exceed L2, so no flush is needed."""
+    its inputs (new keys, Q, w: one packed pinned buffer per step) from host
+    to device, runs hisa_decode_step, and copies its 64 x 2048 indices back to
+    pinned host memory.  As a serving loop would, each step's three parts are
+    captured once as CUDA graphs (the copy in, the call, the copy out) and
+    replayed on three streams, with events for every dependency: the copy in
+    of step s overlaps the kernels of step s - 1, the copy out of step s those
+    of step s + 1; two device slots hold the inputs and outputs in flight.
+    One event pair brackets all E steps; the caches (512 MiB of keys) exceed
+    L2, so no flush is needed."""
     import torch
     dev = kv.keys.device
-    batch, k, m = case.batch, case.k, case.m
+    batch, k, m, H, d = case.batch, case.k, case.m, case.H, case.d
     nsets = Qs.shape[0]
-    ptok = torch.from_numpy(case.append_keys.view(np.int16)).view(torch.bfloat16).pin_memory()
-    pQ = torch.from_numpy(case.append_Q.view(np.int16)).view(torch.bfloat16).pin_memory()
-    pW = torch.from_numpy(case.append_w).pin_memory()
-    pidx = torch.empty((E, batch, k), dtype=torch.int32).pin_memory()
-    dtok = [torch.empty_like(toks[0]) for _ in range(2)]
-    dQ = [torch.empty_like(Qs[0]) for _ in range(2)]
-    dW = [torch.empty_like(Ws[0]) for _ in range(2)]
+    n_tok, n_q, n_w = batch * d * 2, batch * H * d * 2, batch * H * 4     # bytes
+    n_in = n_tok + n_q + n_w
+    pin_in = torch.empty((E, n_in), dtype=torch.uint8).pin_memory()
+    for i in range(E):
+        src = base + i
+        pin_in[i, :n_tok] = torch.from_numpy(case.append_keys[src].view(np.uint8).reshape(-1))
+        pin_in[i, n_tok:n_tok + n_q] = torch.from_numpy(case.append_Q[src % nsets].view(np.uint8).reshape(-1))
+        pin_in[i, n_tok + n_q:] = torch.from_numpy(case.append_w[src % nsets].view(np.uint8).reshape(-1))
+    pin_out = torch.empty((E, batch, k), dtype=torch.int32).pin_memory()
+    dev_in = [torch.empty(n_in, dtype=torch.uint8, device=dev) for _ in range(2)]
     didx = [torch.empty((batch, k), dtype=torch.int32, device=dev) for _ in range(2)]
-    h2d, d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    views = [(b[:n_tok].view(torch.bfloat16).view(batch, d),
+              b[n_tok:n_tok + n_q].view(torch.bfloat16).view(batch, H, d),
+              b[n_tok + n_q:].view(torch.float32).view(batch, H)) for b in dev_in]
+    s_in, s_out, cap = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    g_in, g_cmp, g_out = [], [], []
+    for i in range(E):
+        j = i % 2
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s_in):
+            dev_in[j].copy_(pin_in[i], non_blocking=True)
+        g_in.append(g)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            tok, Q, w = views[j]
+            hisa.hisa_decode_step(kv, tok, Q, w, m, k, ws=ws, idx=didx[j])
+        g_cmp.append(g)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s_out):
+            pin_out[i].copy_(didx[j], non_blocking=True)
+        g_out.append(g)
     ev_in = [torch.cuda.Event() for _ in range(E)]
     ev_done = [torch.cuda.Event() for _ in range(E)]
     ev_out = [torch.cuda.Event() for _ in range(E)]
@@ -372,38 +399,35 @@ def run_e2e(hisa, kv, case, toks, Qs, Ws, q_seq, ws, stream, base, E):
     torch.cuda.synchronize()
     host0 = time.perf_counter()
     t0.record(stream)
-    h2d.wait_event(t0)
-    d2h.wait_event(t0)
-    for s in range(E):
-        j, src = s % 2, base + s
-        with torch.cuda.stream(h2d):
-            if s >= 2:
-                h2d.wait_event(ev_done[s - 2])          # step s - 2 no longer reads slot j
-            dtok[j].copy_(ptok[src], non_blocking=True)
-            dQ[j].copy_(pQ[src % nsets], non_blocking=True)
-            dW[j].copy_(pW[src % nsets], non_blocking=True)
-            ev_in[s].record(h2d)
-        stream.wait_event(ev_in[s])
-        if s >= 2:
-            stream.wait_event(ev_out[s - 2])            # step s - 2's indices have left slot j
-        hisa.hisa_decode_step(kv, dtok[j], dQ[j], dW[j], m, k, ws=ws, idx=didx[j])
-        ev_done[s].record(stream)
-        with torch.cuda.stream(d2h):
-            d2h.wait_event(ev_done[s])
-            pidx[s].copy_(didx[j], non_blocking=True)
-            ev_out[s].record(d2h)
+    s_in.wait_event(t0)
+    s_out.wait_event(t0)
+    for i in range(E):                               # (a graph replays on the current stream)
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(ev_done[i - 2])      # step i - 2 no longer reads slot i % 2
+            g_in[i].replay()
+            ev_in[i].record(s_in)
+        stream.wait_event(ev_in[i])
+        if i >= 2:
+            stream.wait_event(ev_out[i - 2])         # step i - 2's indices have left slot i % 2
+        g_cmp[i].replay()
+        ev_done[i].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_done[i])
+            g_out[i].replay()
+            ev_out[i].record(s_out)
     stream.wait_event(ev_out[E - 1])
     t1.record(stream)
     host_enqueue = time.perf_counter() - host0
     t1.synchronize()
     e2e_ms = t0.elapsed_time(t1)
+    del g_in, g_cmp, g_out
     return {"value": batch * E / (e2e_ms / 1e3), "unit": "selections/s",
-            "h2d_bytes_per_step": int(dtok[0].numel() * 2 + dQ[0].numel() * 2 + dW[0].numel() * 4),
-            "d2h_bytes_per_step": int(didx[0].numel() * 4), "steps": E,
+            "h2d_bytes_per_step": int(n_in), "d2h_bytes_per_step": int(batch * k * 4), "steps": E,
             "ms_per_step": e2e_ms / E, "host_enqueue_ms_per_step": host_enqueue * 1e3 / E,
-            "path": "pinned host -> hisa_decode_step (python binding of the C ABI, plain calls, "
-                    "no graphs) -> pinned host; copies on their own streams, overlapping the "
-                    "previous and next steps' kernels",
+            "path": "pinned host -> hisa_decode_step (python binding of the C ABI) -> pinned host; "
+                    "each step's copy in, call and copy out captured as CUDA graphs and replayed "
+                    "on three streams, overlapping the neighbouring steps",
             "l2": "not flushed: the key cache (512 MiB) exceeds L2"}
 
 
@@ -942,8 +966,9 @@ def main(argv=None, backend: str = "nccl"):
                          "traffic": traffic, "peak_source": peaks["source"],
                          "algorithmic_bytes_per_launch": r["tok_bytes"]},
             "kernels": r["kernels"],
-            "kernels_note": "per-launch times from a separate pass of the same steps with an event "
-                            "pair around every launch",
+            "kernels_note": "per-launch times from a separate pass of the same steps, replayed from "
+                            "CUDA graphs with an event pair around every launch (L2 flushed "
+                            "between steps)",
             "pool": {"GB/s": r["pool_gbs"], "frac": r["pool_gbs"] / peaks["hbm_gbs"],
                      "ms": r["pool_ms"]},
             "flat_scan": {"ms_per_select": r["flat_ms"], "hisa_ms_per_select": r["hisa_sel_ms"],

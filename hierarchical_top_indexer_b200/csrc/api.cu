@@ -112,11 +112,20 @@ struct PhaseScope {
             stop = nullptr;
             return;
         }
-        cudaEventRecord(start, s);
+        record(start);
         P.pending.push_back({start, stop, phase});
     }
     ~PhaseScope() {
-        if (stop) cudaEventRecord(stop, s);
+        if (stop) record(stop);
+    }
+    // while the stream is captured into a CUDA graph the pair becomes event
+    // record nodes of the graph, timed each time the graph runs
+    void record(cudaEvent_t e) const {
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(s, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+            cudaEventRecordWithFlags(e, s, cudaEventRecordExternal);
+        else
+            cudaEventRecord(e, s);
     }
 };
 

@@ -18,7 +18,8 @@ struct PoolShape {
     static constexpr int kGroups = kPoolThreads / kLanes;   // rows read in parallel
 };
 
-__device__ __forceinline__ void dequant16(const uint4 raw, float scale, float (&v)[16]) {
+// 16 e4m3 keys -> fp32 (exact), before the key's scale is applied.
+__device__ __forceinline__ void e4m3x16(const uint4 raw, float (&v)[16]) {
     const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -26,11 +27,24 @@ __device__ __forceinline__ void dequant16(const uint4 raw, float scale, float (&
         const __nv_fp8x2_storage_t hi = static_cast<__nv_fp8x2_storage_t>(w[q] >> 16);
         const float2 a = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(lo, __NV_E4M3)));
         const float2 b = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(hi, __NV_E4M3)));
-        v[4 * q + 0] = a.x * scale;
-        v[4 * q + 1] = a.y * scale;
-        v[4 * q + 2] = b.x * scale;
-        v[4 * q + 3] = b.y * scale;
+        v[4 * q + 0] = a.x;
+        v[4 * q + 1] = a.y;
+        v[4 * q + 2] = b.x;
+        v[4 * q + 3] = b.y;
     }
+}
+
+// a0 = fma(x0, s, a0) and a1 = fma(x1, s, a1), each rounded to nearest: one
+// packed f32x2 instruction (sm_100) with the bits of two scalar fmas.
+__device__ __forceinline__ void fma2_scaled(float& a0, float& a1, float x0, float x1, float s) {
+    asm("{\n\t.reg .b64 acc, xs, ss;\n\t"
+        "mov.b64 acc, {%0, %1};\n\t"
+        "mov.b64 xs, {%2, %3};\n\t"
+        "mov.b64 ss, {%4, %4};\n\t"
+        "fma.rn.f32x2 acc, xs, ss, acc;\n\t"
+        "mov.b64 {%0, %1}, acc;\n\t}"
+        : "+f"(a0), "+f"(a1)
+        : "f"(x0), "f"(x1), "f"(s));
 }
 
 __device__ __forceinline__ void bf16x8(const uint4 raw, float (&v)[8]) {
@@ -46,7 +60,7 @@ __device__ __forceinline__ void bf16x8(const uint4 raw, float (&v)[8]) {
 // pooled row and its hi/lo split.  The arithmetic is that of kPoolThreads
 // "virtual" threads: virtual thread v (group v / kLanes, lane v % kLanes)
 // adds, in fp32 and in row order, the rows grp, grp + kGroups, ... of its
-// 16-byte column slice; then the group partial sums of each element are added
+// 16-byte column slice (an e4m3 row as acc = fma(x, scale, acc)); then the group partial sums of each element are added
 // in group order and divided by cnt.  NT real threads (NT divides
 // kPoolThreads) play the virtual threads v = tid, tid + NT, ..., so every NT
 // gives the same bits; `sync` is the barrier among the NT threads.  The loads
@@ -59,7 +73,9 @@ __device__ void block_mean(const KvView& kv, int b, int j, int s0, int cnt, floa
     using S = PoolShape<D, E4M3>;
     constexpr int V = S::kVec;
     constexpr int NV = kPoolThreads / NT;          // virtual threads per thread
-    constexpr int kUnroll = NV == 1 ? 8 : 4;       // rows per virtual thread per chunk
+    // rows per virtual thread per chunk (e4m3 rows dequantise into twice the
+    // registers: a shorter chunk keeps the pool kernel's occupancy)
+    constexpr int kUnroll = NV == 1 && !E4M3 ? 8 : 4;
     static_assert(kPoolThreads % NT == 0, "virtual threads split evenly");
     const size_t row0 = static_cast<size_t>(b) * kv.cap + s0;
     int lane[NV], grp[NV];
@@ -102,12 +118,21 @@ __device__ void block_mean(const KvView& kv, int b, int j, int s0, int cnt, floa
                 if (grp[u] + (i0 + i) * S::kGroups >= cnt) break;
                 float x[V];
                 if constexpr (E4M3) {
-                    dequant16(raw[u][i], sc[u][i], *reinterpret_cast<float(*)[16]>(x));
+                    // sum: acc + x * scale as one fma per element; max: of x * scale
+                    e4m3x16(raw[u][i], *reinterpret_cast<float(*)[16]>(x));
+                    if constexpr (MAX) {
+#pragma unroll
+                        for (int e = 0; e < V; ++e) acc[u][e] = fmaxf(acc[u][e], x[e] * sc[u][i]);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < V; e += 2)
+                            fma2_scaled(acc[u][e], acc[u][e + 1], x[e], x[e + 1], sc[u][i]);
+                    }
                 } else {
                     bf16x8(raw[u][i], *reinterpret_cast<float(*)[8]>(x));
-                }
 #pragma unroll
-                for (int e = 0; e < V; ++e) acc[u][e] = MAX ? fmaxf(acc[u][e], x[e]) : acc[u][e] + x[e];
+                    for (int e = 0; e < V; ++e) acc[u][e] = MAX ? fmaxf(acc[u][e], x[e]) : acc[u][e] + x[e];
+                }
             }
     }
 #pragma unroll

@@ -191,7 +191,11 @@ __device__ __forceinline__ RowInfo load_row(const ScoreParams& p, int row) {
         R.lim = MODE == kScoreBlocks ? R.t / p.B + 1   // visible blocks
                                      : R.t + 1;        // visible keys
     }
-    R.nt = (R.lim + kTileRows - 1) / kTileRows;
+    // the own block (the last visible one) is kept without a score: block
+    // scoring covers blocks 0 .. lim - 2, in at least one tile (a shard need
+    // not hold the own block: it scores all its visible blocks)
+    const int scored = (MODE == kScoreBlocks && BV != kBlocksShard) ? max(R.lim - 1, 1) : R.lim;
+    R.nt = (scored + kTileRows - 1) / kTileRows;
     return R;
 }
 
@@ -287,49 +291,31 @@ __device__ __forceinline__ float4 lds_f32x4(const float* p) {
     return v;
 }
 
-// sum_h w_h * ReLU(acc_h) over the NP head columns of one TMEM lane: loads
-// of up to 64 columns at a time, one wait per group, four interleaved partial
-// sums (fixed order).
-template <int NP>
-__device__ __forceinline__ float head_sum(uint32_t taddr, const float* wv) {
+// sum_h w_h * ReLU(acc_h) over the npad head columns of one TMEM lane, 16
+// columns (one TMEM load) at a time in a loop that is not unrolled: the code
+// stays a few cache lines, which is what the first tile after a cold start
+// waits for; four interleaved partial sums (fixed order: a[j] adds heads
+// j, j + 4, ... in turn).
+__device__ __forceinline__ float head_sum(int npad, uint32_t taddr, const float* wv) {
     float a[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+    for (int g = 0; g < npad; g += 16) {
+        uint32_t r[16];
+        tmem_ld16_nowait(taddr + g, r);
+        // the group's head weights load while the TMEM load is in flight
+        float4 wg[4];
 #pragma unroll
-    for (int g = 0; g < NP; g += 64) {
-        constexpr int kG = NP < 64 ? NP : 64;
-        uint32_t r[kG];
-#pragma unroll
-        for (int c = 0; c < kG; c += 16)
-            if (g + c < NP) tmem_ld16_nowait(taddr + g + c, r + c);
-        // the group's head weights load while the TMEM loads are in flight
-        float4 wg[kG / 4];
-#pragma unroll
-        for (int h = 0; h < kG; h += 4)
-            if (g + h < NP) wg[h / 4] = lds_f32x4(wv + g + h);
+        for (int q = 0; q < 4; ++q) wg[q] = lds_f32x4(wv + g + 4 * q);
         tmem_ld_wait();
 #pragma unroll
-        for (int h = 0; h < kG; h += 4)
-            if (g + h < NP) {
-                const float4 w4 = wg[h / 4];
-                a[0] = fmaf(w4.x, fmaxf(__uint_as_float(r[h]), 0.f), a[0]);
-                a[1] = fmaf(w4.y, fmaxf(__uint_as_float(r[h + 1]), 0.f), a[1]);
-                a[2] = fmaf(w4.z, fmaxf(__uint_as_float(r[h + 2]), 0.f), a[2]);
-                a[3] = fmaf(w4.w, fmaxf(__uint_as_float(r[h + 3]), 0.f), a[3]);
-            }
+        for (int q = 0; q < 4; ++q) {
+            a[0] = fmaf(wg[q].x, fmaxf(__uint_as_float(r[4 * q]), 0.f), a[0]);
+            a[1] = fmaf(wg[q].y, fmaxf(__uint_as_float(r[4 * q + 1]), 0.f), a[1]);
+            a[2] = fmaf(wg[q].z, fmaxf(__uint_as_float(r[4 * q + 2]), 0.f), a[2]);
+            a[3] = fmaf(wg[q].w, fmaxf(__uint_as_float(r[4 * q + 3]), 0.f), a[3]);
+        }
     }
     return (a[0] + a[1]) + (a[2] + a[3]);
-}
-
-__device__ __forceinline__ float head_sum_any(int npad, uint32_t taddr, const float* wv) {
-    switch (npad) {
-        case 16: return head_sum<16>(taddr, wv);
-        case 32: return head_sum<32>(taddr, wv);
-        case 48: return head_sum<48>(taddr, wv);
-        case 64: return head_sum<64>(taddr, wv);
-        case 80: return head_sum<80>(taddr, wv);
-        case 96: return head_sum<96>(taddr, wv);
-        case 112: return head_sum<112>(taddr, wv);
-        default: return head_sum<128>(taddr, wv);
-    }
 }
 
 // ---------------------------------------------- fused block selection
@@ -365,6 +351,7 @@ __device__ uint32_t epi_threshold(const uint32_t* s, int n, int kk, uint32_t* hi
                                   int* take_eq) {
     uint32_t prefix = 0, mask = 0;
     uint32_t krem = static_cast<uint32_t>(kk);
+#pragma unroll 1
     for (int shift = 24; shift >= 0; shift -= 8) {
         hist[e] = 0;
         hist[e + 128] = 0;
@@ -875,32 +862,31 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * NW);
                 const uint32_t a_base = smem_addr(sA + s * kStageBytes);
+                // (loops kept rolled: a few instructions of code for the cold start)
                 if (kF8) {
                     // 128 candidates x npad heads x 128 bytes: four K = 32 steps,
                     // each for the q1 piece and then the q2 piece of every head
                     // (rows npad .. 2 npad - 1 of the split heads) into the same
                     // accumulator: D = K (q1 + q2)^T
-#pragma unroll
+#pragma unroll 1
                     for (int kk = 0; kk < 4; ++kk) {
                         const uint64_t adesc = sw128_kmajor_desc(a_base + kk * 32);
                         umma_e4m3(d_tmem, adesc, sw128_kmajor_desc(q_base + kk * 32), idesc, kk ? 1u : 0u);
                         umma_e4m3(d_tmem, adesc, sw128_kmajor_desc(q_base + npad * 128 + kk * 32), idesc, 1u);
                     }
                 } else {
-#pragma unroll
-                for (int kh = 0; kh < kHalves; ++kh) {
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll 1
+                    for (int k = 0; k < kHalves * 4; ++k) {
+                        const int kh = k >> 2, kk = k & 3;
                         const uint64_t bdesc = sw128_kmajor_desc(q_base + kh * npad * 128 + kk * 32);
                         const uint64_t adesc = sw128_kmajor_desc(a_base + kh * kHalfBytes + kk * 32);
-                        umma_bf16(d_tmem, adesc, bdesc, idesc, (kh | kk) ? 1u : 0u);
+                        umma_bf16(d_tmem, adesc, bdesc, idesc, k ? 1u : 0u);
                         if (MODE == kScoreBlocks) {
                             const uint64_t ldesc =
                                 sw128_kmajor_desc(a_base + (kHalves + kh) * kHalfBytes + kk * 32);
                             umma_bf16(d_tmem, ldesc, bdesc, idesc, 1u);
                         }
                     }
-                }
                 }
                 umma_commit(empty + s);
                 umma_commit(tfull + a);
@@ -980,7 +966,7 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
             const int c = ti * kTileRows + r;
             bool valid;
             if (MODE == kScoreBlocks) {
-                valid = c < R.lim;
+                valid = c < (BV == kBlocksShard ? R.lim : R.lim - 1);   // the candidates
                 if (PAR && valid) {
                     const int sb = c / p.bf;
                     valid = (sPar[sb >> 5] >> (sb & 31)) & 1u;
@@ -996,7 +982,7 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
                 tc_fence_after();
                 const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                                        static_cast<uint32_t>(a * NW);
-                acc = head_sum_any(npad, taddr, wv);
+                acc = head_sum(npad, taddr, wv);
                 tc_fence_before();
             } else if (ok) {
                 ok = false;
@@ -1021,7 +1007,9 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
             else p.out[static_cast<size_t>(row) * p.ldo + c] = valid ? score_key(acc) : 0u;
             if (p.counts) {
                 const bool slot = MODE == kScoreBlocks ? valid : c < R.lim;
-                const int n = __popc(__ballot_sync(0xffffffffu, slot));
+                // the own block counts as a visible block once per row
+                const int own = MODE == kScoreBlocks && BV != kBlocksShard && ti == 0 && e == 0;
+                const int n = __popc(__ballot_sync(0xffffffffu, slot)) + own;
                 if (lane == 0 && n)
                     atomicAdd(p.counts + static_cast<size_t>(row) * p.counts_ld + p.counts_col +
                                   (MODE == kScoreBlocks ? 0 : 1),
