@@ -236,6 +236,19 @@ __device__ __forceinline__ void tmem_ld_wait() {
 // 128-byte swizzled layout (rows of 128 bytes, 8-row / 1024-byte atoms):
 // start address, leading offset 16 B (unused for this layout), stride
 // between 8-row groups 1024 B, descriptor version 1, swizzle mode 128B.
+// (a0, a1) = (fma(w0, x0, a0), fma(w1, x1, a1)), each rounded to nearest:
+// one packed f32x2 instruction (sm_100) with the bits of two scalar fmas.
+__device__ __forceinline__ void fma2(float& a0, float& a1, float w0, float w1, float x0, float x1) {
+    asm("{\n\t.reg .b64 acc, ws, xs;\n\t"
+        "mov.b64 acc, {%0, %1};\n\t"
+        "mov.b64 ws, {%2, %3};\n\t"
+        "mov.b64 xs, {%4, %5};\n\t"
+        "fma.rn.f32x2 acc, ws, xs, acc;\n\t"
+        "mov.b64 {%0, %1}, acc;\n\t}"
+        : "+f"(a0), "+f"(a1)
+        : "f"(w0), "f"(w1), "f"(x0), "f"(x1));
+}
+
 __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
     return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(1) << 16) |
            (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |

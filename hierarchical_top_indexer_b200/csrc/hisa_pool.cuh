@@ -34,17 +34,9 @@ __device__ __forceinline__ void e4m3x16(const uint4 raw, float (&v)[16]) {
     }
 }
 
-// a0 = fma(x0, s, a0) and a1 = fma(x1, s, a1), each rounded to nearest: one
-// packed f32x2 instruction (sm_100) with the bits of two scalar fmas.
+// a0 = fma(x0, s, a0) and a1 = fma(x1, s, a1) (one packed instruction).
 __device__ __forceinline__ void fma2_scaled(float& a0, float& a1, float x0, float x1, float s) {
-    asm("{\n\t.reg .b64 acc, xs, ss;\n\t"
-        "mov.b64 acc, {%0, %1};\n\t"
-        "mov.b64 xs, {%2, %3};\n\t"
-        "mov.b64 ss, {%4, %4};\n\t"
-        "fma.rn.f32x2 acc, xs, ss, acc;\n\t"
-        "mov.b64 {%0, %1}, acc;\n\t}"
-        : "+f"(a0), "+f"(a1)
-        : "f"(x0), "f"(x1), "f"(s));
+    fma2(a0, a1, x0, x1, s, s);
 }
 
 __device__ __forceinline__ void bf16x8(const uint4 raw, float (&v)[8]) {

@@ -309,10 +309,10 @@ __device__ __forceinline__ float head_sum(int npad, uint32_t taddr, const float*
         tmem_ld_wait();
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            a[0] = fmaf(wg[q].x, fmaxf(__uint_as_float(r[4 * q]), 0.f), a[0]);
-            a[1] = fmaf(wg[q].y, fmaxf(__uint_as_float(r[4 * q + 1]), 0.f), a[1]);
-            a[2] = fmaf(wg[q].z, fmaxf(__uint_as_float(r[4 * q + 2]), 0.f), a[2]);
-            a[3] = fmaf(wg[q].w, fmaxf(__uint_as_float(r[4 * q + 3]), 0.f), a[3]);
+            fma2(a[0], a[1], wg[q].x, wg[q].y, fmaxf(__uint_as_float(r[4 * q]), 0.f),
+                 fmaxf(__uint_as_float(r[4 * q + 1]), 0.f));
+            fma2(a[2], a[3], wg[q].z, wg[q].w, fmaxf(__uint_as_float(r[4 * q + 2]), 0.f),
+                 fmaxf(__uint_as_float(r[4 * q + 3]), 0.f));
         }
     }
     return (a[0] + a[1]) + (a[2] + a[3]);

@@ -82,10 +82,8 @@ __device__ __forceinline__ float bc_head_sum(int npad, uint32_t taddr, const flo
 #pragma unroll
         for (int h = 0; h < 32; h += 4) {
             const float4 w4 = *reinterpret_cast<const float4*>(wv + g + h);
-            a[0] = fmaf(w4.x, fmaxf(__uint_as_float(r[h]), 0.f), a[0]);
-            a[1] = fmaf(w4.y, fmaxf(__uint_as_float(r[h + 1]), 0.f), a[1]);
-            a[2] = fmaf(w4.z, fmaxf(__uint_as_float(r[h + 2]), 0.f), a[2]);
-            a[3] = fmaf(w4.w, fmaxf(__uint_as_float(r[h + 3]), 0.f), a[3]);
+            fma2(a[0], a[1], w4.x, w4.y, fmaxf(__uint_as_float(r[h]), 0.f), fmaxf(__uint_as_float(r[h + 1]), 0.f));
+            fma2(a[2], a[3], w4.z, w4.w, fmaxf(__uint_as_float(r[h + 2]), 0.f), fmaxf(__uint_as_float(r[h + 3]), 0.f));
         }
     }
     return (a[0] + a[1]) + (a[2] + a[3]);
@@ -154,6 +152,7 @@ __global__ void __launch_bounds__(kBcThreads, 1)
     const int u1 = static_cast<int>(static_cast<long long>(n_units) * (blockIdx.x + 1) / gridDim.x);
 
     if (warp == 0) {
+        const uint64_t keep = policy_evict_last();   // keys and queries are read again and again
         bool ok = true;
         int ua = 0, gq = 0;
         for (int u = u0; u < u1 && ok; ++u, ++ua) {
@@ -176,8 +175,8 @@ __global__ void __launch_bounds__(kBcThreads, 1)
                     const int krow = b * p.cap + j * kBcTile;
 #pragma unroll
                     for (int kh = 0; kh < 2; ++kh)
-                        tma_load_2d(sA + (ua & 1) * kBcABytes + kh * (kBcTile * 128), &kmap, afull + (ua & 1),
-                                    kh * 64, krow);
+                        tma_load_2d_hint(sA + (ua & 1) * kBcABytes + kh * (kBcTile * 128), &kmap,
+                                         afull + (ua & 1), kh * 64, krow, keep);
                 }
             }
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -213,8 +212,8 @@ __global__ void __launch_bounds__(kBcThreads, 1)
                         const int rq = q < nvalid ? md[q].x : row0;   // padding rows reuse a valid row
 #pragma unroll
                         for (int kh = 0; kh < 2; ++kh)
-                            tma_load_2d(sB + s * kBcBBytes + kh * (kBcN * 128) + q * npad * 128, &qmap,
-                                        bfull + s, kh * 64, rq * p.H);
+                            tma_load_2d_hint(sB + s * kBcBBytes + kh * (kBcN * 128) + q * npad * 128, &qmap,
+                                             bfull + s, kh * 64, rq * p.H, keep);
                     }
                 }
                 __syncwarp();
@@ -305,8 +304,10 @@ __global__ void __launch_bounds__(kBcThreads, 1)
                                            static_cast<uint32_t>(a * kBcN + pq * npad);
                     const float acc = bc_head_sum(npad, taddr, sW + m * kBcN + pq * npad);
                     const int s = md.w * kBcTile + token;
-                    p.out[static_cast<size_t>(md.x) * p.ldo + md.y * kBcTile + token] =
-                        s <= md.z ? score_key(acc) : 0u;
+                    // streamed past L2 (evict first), which keeps the keys and
+                    // the queries that the next units read there
+                    __stcs(p.out + static_cast<size_t>(md.x) * p.ldo + md.y * kBcTile + token,
+                           s <= md.z ? score_key(acc) : 0u);
                 }
                 tc_fence_before();
                 __syncwarp();

@@ -192,10 +192,11 @@ int hisa_select(const hisa_kv* kv, const uint16_t* Q, const float* w, const int3
  * Results (idx, scores, keys, key scales, pooled, pooled_hl, len, status) are
  * those of hisa_append(kv, tok, tok_scale) followed by hisa_select(kv, Q, w,
  * q_seq = 0..batch-1, q_pos = NULL, m, k), bit for bit.  Rows of at most
- * 4 x 128 blocks and batches of at most two rows per SM run the append inside
- * the block-scoring kernel (no separate launch): each row writes its key,
- * recomputes its trailing block's representative and scores its blocks in
- * one CTA.  Other sizes run the two calls' launches.  A full sequence is left
+ * 4 x 128 blocks and batches of at most two rows per SM run the append and
+ * the block scoring (one CTA per row, top-m kept in the same kernel) side by
+ * side: the block scoring does not read the appended block (the row's own
+ * block, kept without a score) and publishes the new lengths once the append
+ * kernel has finished.  Other sizes run the two calls' launches.  A full sequence is left
  * as it is (HISA_DEV_CAPACITY) and selects for position cap - 1; a len[]
  * outside [0, cap] sets HISA_DEV_BAD_LEN and HISA_DEV_BAD_QUERY and gives a
  * -1 row.  Errors as hisa_append and hisa_select.
