@@ -53,14 +53,16 @@ bool make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, size_t
 // The block representatives as a 3-D tensor [batch, nblk, 2d] bf16 with
 // boxes of [1, 128, 64]: a box that runs past a sequence's nblk rows is
 // zero-filled there instead of reading the next sequence's rows.
-bool pooled_map(CUtensorMap* map, const KvView& v) {
+// boxes of `rows` representatives (128: a tile; bf: the children of one
+// superblock in the gathered level of the three-level search)
+bool pooled_map(CUtensorMap* map, const KvView& v, int rows = 128) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(2 * v.d), static_cast<cuuint64_t>(v.nblk),
                                 static_cast<cuuint64_t>(v.batch)};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(2 * v.d) * 2,
                                    static_cast<cuuint64_t>(v.nblk) * 2 * v.d * 2};
-    const cuuint32_t box[3] = {64, 128, 1};
+    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(rows), 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, v.pooled_hl, dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -373,6 +375,9 @@ struct BlockLevel {
     int32_t* nblocks_out;
     const int32_t* parent;   // kept superblocks [n_q, parent_ld] or null
     int parent_ld, bf;
+    // gathered (the caller checked gathered_level()): score only the kept
+    // superblocks' children; parent_n = the kept superblocks per row
+    const int32_t* parent_n;
     int counts_col;
     // the decode step: row b is sequence b, whose new key the append kernel
     // launched just before writes (the caller guarantees the conditions of
@@ -385,23 +390,24 @@ int block_stage(const BlockLevel& lv, const uint16_t* Q, const float* w, const i
                 cudaStream_t s) {
     const KvView& v = *lv.v;
     CUtensorMap pmap, qmap;
-    if (!pooled_map(&pmap, v) || !query_map(&qmap, Q, n_q, H, v.d)) return HISA_E_CUDA;
+    if (!pooled_map(&pmap, v, lv.parent_n ? lv.bf : 128) || !query_map(&qmap, Q, n_q, H, v.d)) return HISA_E_CUDA;
     const int sms = sm_count();
     ScoreParams p = score_params(v, w, q_seq, q_pos, n_q, H);
     p.out = lv.bkeys;
     p.ldo = lv.ldb;
-    p.tiles_per_row = lv.ldb / 128;
+    p.tiles_per_row = lv.parent_n ? (lv.parent_ld * lv.bf + 127) / 128 : lv.ldb / 128;
     p.counts = reinterpret_cast<unsigned long long*>(counts);
     p.counts_ld = counts_ld;
     p.counts_col = lv.counts_col;
     p.parent = lv.parent;
     p.parent_ld = lv.parent_ld;
     p.bf = lv.bf;
+    p.parent_n = lv.parent_n;
     // Short rows (up to kFuseMaxBlocks = 4 tiles of blocks) and at most two rows per SM: the
     // scoring kernel keeps the blocks itself, one CTA per row, which saves the
     // selection launch.  Longer rows score faster spread over every SM, and
     // many rows select faster in the selection kernel's one-CTA-per-row grid.
-    const bool fuse = lv.ldb <= kFuseMaxBlocks && n_q <= 2 * sms;
+    const bool fuse = lv.parent_n ? true : lv.ldb <= kFuseMaxBlocks && n_q <= 2 * sms;
     if (lv.app) {
         if (!fuse) return HISA_E_UNSUPPORTED;
         p.app = 1;
@@ -686,6 +692,18 @@ int check_cp(const hisa_kv* kv, int32_t tok_off, KvView* v) {
     return HISA_OK;
 }
 
+// The level under the kept superblocks loads and scores only their children
+// when that is at most a quarter of the blocks (otherwise scoring every block
+// over all SMs and masking the others is as fast), a row's children fit one
+// fused CTA (at most kFuseMaxBlocks), runs of bf children start on whole
+// swizzle atoms (bf a power of two from 8 to 128) and there are at most two
+// rows per SM.
+bool gathered_level(int bf, int W, int nblk, int n_q) {
+    const long long children = static_cast<long long>(W) * bf;
+    return bf >= 8 && bf <= 128 && (bf & (bf - 1)) == 0 && W <= 256 && children <= kFuseMaxBlocks &&
+           4 * children <= nblk && n_q <= 2 * sm_count();
+}
+
 }  // namespace
 
 extern "C" {
@@ -887,6 +905,7 @@ int hisa_tree_select(const hisa_kv* kv, const hisa_kv* kv2, const uint16_t* Q, c
     l1.parent_ld = T.ws;
     l1.bf = v2.B / v.B;
     l1.counts_col = 1;
+    if (gathered_level(l1.bf, T.ws, v.nblk, n_q)) l1.parent_n = l2.nblocks;
     rc = block_stage(l1, Q, w, q_seq, q_pos, n_q, H, k, counts, 3, s);
     if (rc) return rc;
     return token_stage(v, T.L, base, Q, w, q_seq, q_pos, n_q, H, k, idx, scores, counts, 3, 1, 0, s);

@@ -50,6 +50,10 @@ struct ScoreParams {
     // parent[row, 0 .. parent_ld) (-1 padded); null: every block is
     const int32_t* parent;
     int parent_ld, bf;
+    // with parent_n (the kept superblocks per row) the kernel loads and
+    // scores only their children, bf per superblock (rows fused, bf a power
+    // of two from 8 to 128, parent_ld <= 256)
+    const int32_t* parent_n;
     // score keys [n_q, ldo] (order-preserving; 0 = masked slot)
     uint32_t* out;
     int ldo;

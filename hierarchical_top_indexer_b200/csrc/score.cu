@@ -144,7 +144,7 @@ __host__ __device__ inline uint32_t tmem_columns(int cols) {
 // Block scoring variants (a template parameter, so that each compiles alone):
 // kBlocksAppend is the decode step (row b = sequence b, scored while the
 // append kernel launched before it writes the new keys; see ScoreParams::app).
-constexpr int kBlocksPlain = 0, kBlocksMasked = 1, kBlocksShard = 2, kBlocksAppend = 3;
+constexpr int kBlocksPlain = 0, kBlocksMasked = 1, kBlocksShard = 2, kBlocksAppend = 3, kBlocksGathered = 4;
 
 // A query row: sequence, position, candidate slots, candidate tiles (0 if
 // the row is invalid); app: the decode step appends a key at t first.
@@ -193,8 +193,14 @@ __device__ __forceinline__ RowInfo load_row(const ScoreParams& p, int row) {
     }
     // the own block (the last visible one) is kept without a score: block
     // scoring covers blocks 0 .. lim - 2, in at least one tile (a shard need
-    // not hold the own block: it scores all its visible blocks)
-    const int scored = (MODE == kScoreBlocks && BV != kBlocksShard) ? max(R.lim - 1, 1) : R.lim;
+    // not hold the own block: it scores all its visible blocks); gathered,
+    // the row's slots are the children of its app = parent_n[row] kept
+    // superblocks, bf per superblock
+    int scored = (MODE == kScoreBlocks && BV != kBlocksShard) ? max(R.lim - 1, 1) : R.lim;
+    if (MODE == kScoreBlocks && BV == kBlocksGathered) {
+        R.app = min(max(p.parent_n[row], 0), p.parent_ld);
+        scored = max(R.app * p.bf, 1);
+    }
     R.nt = (scored + kTileRows - 1) / kTileRows;
     return R;
 }
@@ -380,9 +386,11 @@ __device__ uint32_t epi_threshold(const uint32_t* s, int n, int kk, uint32_t* hi
 }
 
 // Writes the slots of the keys of s[0..n) above T, plus the first take_eq
-// equal to T, in ascending order to out (and dbg).
+// equal to T, in ascending order to out (and dbg); with par, slot c is
+// written as block par[c / bf] * bf + c % bf.
 __device__ __noinline__ void epi_emit(const uint32_t* s, int n, uint32_t T, int take_eq, int32_t* out,
-                                      int32_t* dbg, uint32_t* misc, int e) {
+                                      int32_t* dbg, uint32_t* misc, int e, const int32_t* par = nullptr,
+                                      int bf = 1) {
     const int w = e >> 5, l = e & 31;
     const int per = ((n + 3) / 4 + 31) & ~31;
     const int w0 = w * per;
@@ -427,8 +435,9 @@ __device__ __noinline__ void epi_emit(const uint32_t* s, int n, uint32_t T, int 
         const unsigned selm = __ballot_sync(0xffffffffu, sel);
         if (sel) {
             const int at = static_cast<int>(pos + __popc(selm & lt));
-            out[at] = c;
-            if (dbg) dbg[at] = c;
+            const int id = par ? par[c / bf] * bf + c % bf : c;
+            out[at] = id;
+            if (dbg) dbg[at] = id;
         }
         eq_run += __popc(eqm);
         pos += __popc(selm);
@@ -437,8 +446,10 @@ __device__ __noinline__ void epi_emit(const uint32_t* s, int n, uint32_t T, int 
 
 
 // BV (block scoring only): every visible block is a candidate (kBlocksPlain),
-// a kept-superblock list masks the blocks outside it (kBlocksMasked), or the
-// cache is a context-parallel shard (kBlocksShard).
+// a kept-superblock list masks the blocks outside it (kBlocksMasked), only
+// the children of the kept superblocks are loaded and scored, bf at a time,
+// slot q * bf + c being child c of the q-th kept superblock (kBlocksGathered),
+// or the cache is a context-parallel shard (kBlocksShard).
 template <int MODE, bool E4M3, int D, int BV>
 __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(MODE, E4M3, D) ? 2 : 1)
     score_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap qmap,
@@ -448,6 +459,7 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
     constexpr bool kF8 = uses_f8(MODE, E4M3, D);          // fp8 operands straight from TMA
     constexpr bool kConv = E4M3 && !kF8;                  // e4m3 widened to bf16 by converter warps
     constexpr bool PAR = MODE == kScoreBlocks && BV == kBlocksMasked;
+    constexpr bool GAT = MODE == kScoreBlocks && BV == kBlocksGathered;
     constexpr bool APP = MODE == kScoreBlocks && BV == kBlocksAppend;
     constexpr int kStageBytes = kF8 ? kTileRows * D : kOps * kHalves * kHalfBytes;
     constexpr int kStage8Bytes = kTileRows * D;
@@ -579,6 +591,12 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
                     cur.next_row();
                     continue;
                 }
+                if constexpr (GAT) {
+                    // the row's kept superblocks, for lane 0's boxes
+                    for (int i = lane; i < R.app; i += 32)
+                        sTab[i] = p.parent[static_cast<size_t>(row) * p.parent_ld + i];
+                    __syncwarp();
+                }
                 const int qs = qloads & 1;
                 if (qloads >= 2 && !warp_wait(qempty + qs, ((qloads - 2) >> 1) & 1, abort_flag)) {
                     ok = false;
@@ -626,10 +644,24 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
 
                             uint64_t* fb = full + ring.slot;
                             uint8_t* dst = sA + ring.slot * kStageBytes;
-                            mbar_arrive_expect_tx(fb, kStageBytes);
-                            if (MODE == kScoreBlocks) {
+                            if (GAT) {
+                                // one run of bf representatives per kept superblock of the
+                                // tile (boxes of bf rows; runs past the list are not loaded
+                                // and their slots are masked)
+                                const int runs = kTileRows / p.bf;
+                                const int q0 = (t + k) * runs;
+                                const int nr = max(0, min(runs, R.app - q0));
+                                mbar_arrive_expect_tx(fb, static_cast<uint32_t>(nr * p.bf * 2 * kHalves * 128));
+                                for (int r = 0; r < nr; ++r)
+#pragma unroll 1
+                                    for (int h = 0; h < 2 * kHalves; ++h)
+                                        tma_load_3d(dst + h * kHalfBytes + r * p.bf * 128, &amap, fb,
+                                                    (h / kHalves) * D + (h % kHalves) * 64, sTab[q0 + r] * p.bf,
+                                                    R.b);
+                            } else if (MODE == kScoreBlocks) {
                                 // [batch, nblk, 2d] boxes: the rows past the sequence's
                                 // blocks are zero-filled, not read
+                                mbar_arrive_expect_tx(fb, kStageBytes);
 #pragma unroll
                                 for (int op = 0; op < 2; ++op)
 #pragma unroll
@@ -637,6 +669,7 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
                                         tma_load_3d(dst + (op * kHalves + kh) * kHalfBytes, &amap, fb,
                                                     op * D + kh * 64, (t + k) * kTileRows, R.b);
                             } else {
+                                mbar_arrive_expect_tx(fb, kStageBytes);
                                 for (int sub = 0; sub < nsub; ++sub) {
                                     const int srow = MODE == kScoreHisa
                                                          ? sTab[k * nsub + sub]
@@ -939,6 +972,13 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
                         set_status(p.status, HISA_DEV_BAD_QUERY);
                     }
                 }
+                if (GAT && ti < R.nt) {
+                    // the row's kept superblocks (slot q * bf + c: child c of the q-th)
+                    epi_bar();
+                    for (int i = e; i < R.app; i += 128)
+                        reinterpret_cast<int32_t*>(sPar)[i] = p.parent[static_cast<size_t>(row) * p.parent_ld + i];
+                    epi_bar();
+                }
                 if (MODE == kScoreBlocks && PAR && ti < R.nt) {
                     // the row's kept superblocks as a bitmap
                     epi_bar();
@@ -967,6 +1007,10 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
             bool valid;
             if (MODE == kScoreBlocks) {
                 valid = c < (BV == kBlocksShard ? R.lim : R.lim - 1);   // the candidates
+                if (GAT) {
+                    const int q = c / p.bf;
+                    valid = q < R.app && reinterpret_cast<const int32_t*>(sPar)[q] * p.bf + (c - q * p.bf) < R.lim - 1;
+                }
                 if (PAR && valid) {
                     const int sb = c / p.bf;
                     valid = (sPar[sb >> 5] >> (sb & 31)) & 1u;
@@ -1022,11 +1066,13 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
                 int32_t* bl = p.sel_blocks + static_cast<size_t>(row) * p.mm;
                 int32_t* bd = p.sel_blocks_out ? p.sel_blocks_out + static_cast<size_t>(row) * p.mm : nullptr;
                 // candidates: the nonzero keys of blocks 0 .. nb - 2 (a kept-superblock
-                // list masks the others to 0)
-                uint32_t nv = static_cast<uint32_t>(nb - 1);
-                if (PAR) {
+                // list masks the others to 0), or of the gathered slots
+                const int nsl = GAT ? R.app * p.bf : nb - 1;
+                const int32_t* par = GAT ? reinterpret_cast<const int32_t*>(sPar) : nullptr;
+                uint32_t nv = static_cast<uint32_t>(nsl);
+                if (PAR || GAT) {
                     nv = 0;
-                    for (int c = e; c < nb - 1; c += 128) nv += sKeys[c] != 0u;
+                    for (int c = e; c < nsl; c += 128) nv += sKeys[c] != 0u;
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) nv += __shfl_xor_sync(0xffffffffu, nv, o);
                     if (lane == 0) sMisc[12 + (e >> 5)] = nv;
@@ -1037,8 +1083,8 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
                 const int kk = p.m - 1;
                 const int kept = static_cast<int>(nv) <= kk ? static_cast<int>(nv) : kk;
                 if (static_cast<int>(nv) <= kk) {
-                    if (PAR) {
-                        if (nv > 0) epi_emit(sKeys, nb - 1, 0u, 0, bl, bd, sMisc, e);   // every unmasked one
+                    if (PAR || GAT) {
+                        if (nv > 0) epi_emit(sKeys, nsl, 0u, 0, bl, bd, sMisc, e, par, p.bf);   // every unmasked one
                     } else {
                         for (int i = e; i < kept; i += 128) {                         // every candidate
                             bl[i] = i;
@@ -1047,8 +1093,8 @@ __global__ void __launch_bounds__(score_threads(MODE, E4M3, D), two_per_sm_kind(
                     }
                 } else if (kk > 0) {
                     int take_eq;
-                    const uint32_t T = epi_threshold<PAR>(sKeys, nb - 1, kk, sHist, sMisc, e, &take_eq);
-                    epi_emit(sKeys, nb - 1, T, take_eq, bl, bd, sMisc, e);
+                    const uint32_t T = epi_threshold<PAR || GAT>(sKeys, nsl, kk, sHist, sMisc, e, &take_eq);
+                    epi_emit(sKeys, nsl, T, take_eq, bl, bd, sMisc, e, par, p.bf);
                 }
                 for (int i = kept + e; i < p.mm; i += 128) {
                     const int v = i == kept ? nb - 1 : -1;   // own block last
@@ -1264,6 +1310,9 @@ cudaError_t launch_score(int mode, bool e4m3, int d, const CUtensorMap& amap, co
         if (p.cp)
             return d == 128 ? launch_t<kScoreBlocks, false, 128, kBlocksShard>(amap, qmap, p, grid, s)
                             : launch_t<kScoreBlocks, false, 64, kBlocksShard>(amap, qmap, p, grid, s);
+        if (p.parent && p.parent_n)
+            return d == 128 ? launch_t<kScoreBlocks, false, 128, kBlocksGathered>(amap, qmap, p, grid, s)
+                            : launch_t<kScoreBlocks, false, 64, kBlocksGathered>(amap, qmap, p, grid, s);
         if (p.parent)
             return d == 128 ? launch_t<kScoreBlocks, false, 128, kBlocksMasked>(amap, qmap, p, grid, s)
                             : launch_t<kScoreBlocks, false, 64, kBlocksMasked>(amap, qmap, p, grid, s);

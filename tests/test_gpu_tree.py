@@ -77,6 +77,17 @@ def test_tree_matches_oracle(dtype, B, bf, W, m, k):
     assert check_tree(case, g, bf, W, m, k) <= 3
 
 
+def test_tree_gathered_level_matches_oracle():
+    """Kept superblocks of bf = 32 blocks covering under a quarter of the
+    blocks: the level under them loads and scores only their children (runs
+    of 32 representatives), d = 64; the counters report those children."""
+    case = make_case(batch=2, L=[20000, 9000], H=16, d=64, B=16, m=12, k=150, seed=79,
+                     positions=[np.array([19999, 12345, 40]), np.array([8999, 4096])])
+    kv = device_case(case)
+    g = run_tree(case, kv, 32, 8, 12, 150)
+    assert check_tree(case, g, 32, 8, 12, 150) <= 3
+
+
 def test_tree_max_pooling_matches_oracle():
     case = make_case(batch=2, L=[5000, 3000], H=32, d=128, B=64, m=10, k=256, seed=77,
                      positions=[np.array([4999, 2000]), np.array([2999, 64])])
