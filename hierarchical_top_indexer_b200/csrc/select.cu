@@ -560,6 +560,16 @@ __global__ void __launch_bounds__(NT, NT >= 1024 ? 1 : (NT >= 512 ? 2 : 4)) sele
     const int row = blockIdx.x;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int mode = MODE >= 0 ? MODE : p.mode;
+    // token rows: this thread's keys load before the row's plan is read (its
+    // slot count masks them later), so that the two L2 round trips overlap;
+    // the loads stay within the row's ldk slots
+    uint4 kpre[KPT / 4];
+    if (MODE == kSelHisaTokens) {
+        const uint4* g4 = reinterpret_cast<const uint4*>(p.keys + static_cast<size_t>(row) * p.ldk + tid * KPT);
+#pragma unroll
+        for (int q = 0; q < KPT / 4; ++q)
+            kpre[q] = tid * KPT + 4 * q < p.ldk ? __ldg(g4 + q) : make_uint4(0u, 0u, 0u, 0u);
+    }
 
     int n = 0, kk = p.k, b = 0, t = 0, nb = 0, cp_own = 0;
     bool bad = false;
@@ -653,7 +663,8 @@ __global__ void __launch_bounds__(NT, NT >= 1024 ? 1 : (NT >= 512 ? 2 : 4)) sele
 #pragma unroll
         for (int q = 0; q < KPT / 4; ++q) {
             uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (c0 + 4 * q < n) v = __ldg(g4 + q);   // L1 keeps the half of each sector the next load uses
+            if (MODE == kSelHisaTokens) v = kpre[q];
+            else if (c0 + 4 * q < n) v = __ldg(g4 + q);   // L1 keeps the half of each sector the next load uses
             x[4 * q] = c0 + 4 * q < n ? v.x : 0u;
             x[4 * q + 1] = c0 + 4 * q + 1 < n ? v.y : 0u;
             x[4 * q + 2] = c0 + 4 * q + 2 < n ? v.z : 0u;
