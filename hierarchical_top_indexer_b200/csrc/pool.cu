@@ -32,6 +32,27 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(KvView kv) {
     block_mean<D, E4M3, MAX, kPoolThreads>(kv, b, j, s0, cnt, partial, threadIdx.x, CtaSync{});
 }
 
+// e4m3 keys, blocks of one chunk: a CTA pools blocks 2x and 2x + 1, the
+// rows of both loaded before either is added (an e4m3 block is half the
+// bytes of a bf16 one, and four CTAs per SM would leave too few bytes in
+// flight).  Each block's arithmetic is block_mean's.
+template <int D, bool MAX>
+__global__ void __launch_bounds__(kPoolThreads) pool_pair_kernel(KvView kv) {
+    __shared__ __align__(16) float partial[PoolShape<D, true>::kGroups * D];
+    const int j = 2 * blockIdx.x;
+    const int b = blockIdx.y;
+    const int n = kv.len[b];
+    if (n < 0 || n > kv.cap) {
+        if (threadIdx.x == 0 && j == 0) set_status(kv.status, HISA_DEV_BAD_LEN);
+        return;
+    }
+    const int s0 = j * kv.B;
+    if (s0 >= n) return;
+    const int cnt0 = min(kv.B, n - s0);
+    const int cnt1 = j + 1 < kv.nblk && s0 + kv.B < n ? min(kv.B, n - s0 - kv.B) : 0;
+    block_mean_pair<D, true, MAX>(kv, b, j, s0, cnt0, cnt1, partial, threadIdx.x);
+}
+
 // STEP: the decode step's append (launched with programmatic dependent
 // launch): the next kernel, which scores this step's blocks, may start at once
 // (it reads the old length and takes the new key's position from it); the
@@ -97,6 +118,12 @@ cudaError_t launch_tail_t(const KvView& kv, cudaStream_t s) {
 
 template <int D, bool E4M3>
 cudaError_t launch_pool_t(const KvView& kv, cudaStream_t s) {
+    if (E4M3 && kv.B <= pool_chunk_rows<D, true>()) {
+        dim3 grid((kv.nblk + 1) / 2, kv.batch);
+        if (kv.pool_max) pool_pair_kernel<D, true><<<grid, kPoolThreads, 0, s>>>(kv);
+        else pool_pair_kernel<D, false><<<grid, kPoolThreads, 0, s>>>(kv);
+        return cudaGetLastError();
+    }
     dim3 grid(kv.nblk, kv.batch);
     if (kv.pool_max) pool_kernel<D, E4M3, true><<<grid, kPoolThreads, 0, s>>>(kv);
     else pool_kernel<D, E4M3, false><<<grid, kPoolThreads, 0, s>>>(kv);
