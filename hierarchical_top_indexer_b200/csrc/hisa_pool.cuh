@@ -177,13 +177,16 @@ __host__ __device__ constexpr int pool_chunk_rows() {
 
 // Blocks j and j + 1 of sequence b (cnt0 > 0 and cnt1 >= 0 keys, each at most
 // pool_chunk_rows: one chunk), with block_mean's arithmetic for each; the
-// rows of both are loaded before either is added, twice the bytes in flight.
+// rows of both are loaded before either is added, twice the bytes in flight,
+// and the two blocks' group sums (partial holds 2 x kGroups x D floats) are
+// reduced side by side, threads 0 .. NT/2 - 1 for the first block.
 template <int D, bool E4M3, bool MAX>
 __device__ void block_mean_pair(const KvView& kv, int b, int j, int s0, int cnt0, int cnt1, float* partial,
                                 int tid) {
     using S = PoolShape<D, E4M3>;
     constexpr int V = S::kVec;
     constexpr int kUnroll = !E4M3 ? 8 : 4;
+    static_assert(kPoolThreads / 2 >= D, "one reducing thread per element of each block");
     const int lane = tid % S::kLanes, grp = tid / S::kLanes;
     const int cnt[2] = {cnt0, cnt1};
     uint4 raw[2][kUnroll];
@@ -201,7 +204,6 @@ __device__ void block_mean_pair(const KvView& kv, int b, int j, int s0, int cnt0
     }
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
-        if (cnt[q] <= 0) break;
         float acc[V];
 #pragma unroll
         for (int e = 0; e < V; ++e) acc[e] = MAX ? -INFINITY : 0.f;
@@ -210,12 +212,14 @@ __device__ void block_mean_pair(const KvView& kv, int b, int j, int s0, int cnt0
             if (grp + i * S::kGroups >= cnt[q]) break;
             mean_add<D, E4M3, MAX>(raw[q][i], sc[q][i], acc);
         }
-        if (q) __syncthreads();   // the first block's sums are read before these overwrite them
 #pragma unroll
-        for (int e = 0; e < V; ++e) partial[grp * D + lane * V + e] = acc[e];
-        __syncthreads();
-        mean_finish<D, E4M3, MAX, kPoolThreads>(kv, b, j + q, cnt[q], partial, tid);
+        for (int e = 0; e < V; ++e) partial[(q * S::kGroups + grp) * D + lane * V + e] = acc[e];
     }
+    __syncthreads();
+    const int q = tid / (kPoolThreads / 2);
+    if (cnt[q] > 0)
+        mean_finish<D, E4M3, MAX, kPoolThreads / 2>(kv, b, j + q, cnt[q], partial + q * S::kGroups * D,
+                                                    tid - q * (kPoolThreads / 2));
 }
 
 

@@ -38,7 +38,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(KvView kv) {
 // flight).  Each block's arithmetic is block_mean's.
 template <int D, bool MAX>
 __global__ void __launch_bounds__(kPoolThreads) pool_pair_kernel(KvView kv) {
-    __shared__ __align__(16) float partial[PoolShape<D, true>::kGroups * D];
+    __shared__ __align__(16) float partial[2 * PoolShape<D, true>::kGroups * D];
     const int j = 2 * blockIdx.x;
     const int b = blockIdx.y;
     const int n = kv.len[b];
