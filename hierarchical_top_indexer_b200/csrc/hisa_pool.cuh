@@ -1,7 +1,7 @@
 // Block representatives (HISA: mean pooling of each block of B keys; gptget.net
-// summary, "Methodology"), shared by the pool / append kernels and by the
-// decode step fused into block scoring, so that every path computes a block's
-// representative with the same arithmetic and gets the same bits.
+// summary, "Methodology"), shared by the pool, append and trailing-block
+// kernels, so that every path computes a block's representative with the
+// same arithmetic and gets the same bits.
 #pragma once
 
 #include "hisa_kernels.cuh"

@@ -7,9 +7,9 @@
 // Makes Sparse Attention Actually Fast", "HISA's Approach") keeps the summary
 // current as tokens are appended; here only the trailing block changes.
 //
-// Both kernels (and the decode step fused into block scoring) run the same
-// block_mean routine with the same arithmetic, so an appended block equals a
-// from-scratch re-pool bit for bit.
+// Every kernel here (the decode step's append included) runs block_mean's
+// arithmetic, so an appended block equals a from-scratch re-pool bit for
+// bit.
 #include "hisa_pool.cuh"
 
 namespace hisa {
