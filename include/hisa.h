@@ -241,7 +241,13 @@ int hisa_select_inspect(const hisa_kv* kv, const uint16_t* Q, const float* w,
  *   counts [n_q, 3] out (or NULL), zeroed by the call: superblocks scored,
  *          blocks scored, token slots scored
  * W covering every superblock gives hisa_select's result.  kv2 may hold up to
- * 32768 superblocks per sequence (HISA_E_UNSUPPORTED beyond).
+ * 32768 superblocks per sequence (HISA_E_UNSUPPORTED beyond).  The block
+ * level reads and scores only the kept superblocks' children when they are
+ * at most a quarter of the blocks, W * bf <= 512, bf is a power of two from
+ * 8 to 128 and there are at most two rows per SM; otherwise it scores every
+ * visible block and masks the others.  Either way the results and the
+ * counters (which count the children below the own block, plus the own
+ * block) are the same.
  */
 size_t hisa_tree_workspace_bytes(const hisa_kv* kv, const hisa_kv* kv2, int n_q, int H, int W,
                                  int m, int k);
