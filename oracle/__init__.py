@@ -59,11 +59,13 @@ def _bind(lib):
     lib.hisa_oracle_topk_f32.argtypes = [P, I, I, I, P]
     lib.hisa_oracle_tree_select.argtypes = [P, P, I, I, I, I, I, I, I, P, P, P, P, P, I, I, I, I,
                                             I, I, P, P, P, P, P, P, P]
+    lib.hisa_oracle_levels_select.argtypes = [P, P, I, I, I, I, I, P, P, I, P, P, P, P, P, I, I,
+                                              I, I, P, P, P, P, P]
     lib.hisa_oracle_sparse_attn.argtypes = [P, I, P, P, P, I, I, I, P, P, I, I, ctypes.c_double, I,
                                             P, P]
     for f in ("hisa_oracle_pool", "hisa_oracle_select", "hisa_oracle_refine",
               "hisa_oracle_flat", "hisa_oracle_topk_f32", "hisa_oracle_tree_select",
-              "hisa_oracle_sparse_attn"):
+              "hisa_oracle_levels_select", "hisa_oracle_sparse_attn"):
         getattr(lib, f).restype = I
     return lib
 
@@ -171,6 +173,36 @@ def tree_select(cache: Cache, Q, w, q_seq, q_pos, B: int, bf: int, W: int, m: in
         raise ValueError(f"hisa_oracle_tree_select rc={rc}")
     return dict(idx=idx, score=score, sblocks=sblocks, nsblocks=nsblocks, blocks=blocks,
                 nblocks=nblocks, counts=counts)
+
+
+def levels_select(cache: Cache, Q, w, q_seq, q_pos, level_B, keep, k: int,
+                  threads: Optional[int] = None, lib=None, pool: str = "mean") -> dict:
+    """Search of any depth.  Level l (finest first) groups the keys into units
+    of level_B[l] tokens, each size a multiple of the one below; from the
+    coarsest level down, the own unit plus the best keep[l] - 1 candidates
+    (every visible unit at the top, the units inside the kept ones below)
+    are kept; then the tokens of the kept level-0 blocks (top k).  kept[l] is
+    [n_q, keep[l]] (ascending, -1 padded), nkept [n_q, levels], counts
+    [n_q, levels + 1] (units scored per level, then token slots)."""
+    lib = lib or load()
+    Q, w, q_seq, q_pos, n_q, H = _queries(Q, w, q_seq, q_pos)
+    nl = len(level_B)
+    lb = np.ascontiguousarray(level_B, np.int32)
+    kp = np.ascontiguousarray(keep, np.int32)
+    idx = np.empty((n_q, k), np.int32)
+    score = np.empty((n_q, k))
+    kept = np.empty((n_q, int(kp.sum())), np.int32)
+    nkept = np.empty((n_q, nl), np.int32)
+    counts = np.empty((n_q, nl + 1), np.int64)
+    rc = lib.hisa_oracle_levels_select(*cache.args(), nl, _p(lb), _p(kp), POOL_MODES[pool],
+                                       _p(cache.lens), _p(Q), _p(w), _p(q_seq), _p(q_pos), n_q, H, k,
+                                       threads or default_threads(), _p(idx), _p(score), _p(kept),
+                                       _p(nkept), _p(counts))
+    if rc:
+        raise ValueError(f"hisa_oracle_levels_select rc={rc}")
+    off = np.concatenate([[0], np.cumsum(kp)])
+    return dict(idx=idx, score=score, kept=[kept[:, off[l]:off[l + 1]] for l in range(nl)],
+                nkept=nkept, counts=counts)
 
 
 def hisa_refine(cache: Cache, Q, w, q_seq, q_pos, B: int, k: int, blocks, nblocks,

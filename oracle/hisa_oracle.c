@@ -20,7 +20,10 @@
  *        attention operator.
  *   The flat DSA scan (blog "Hierarchical Indexing Makes Sparse Attention
  *   Actually Fast", "How Fine-Grained Sparse Attention Works Today") scores
- *   every prefix token and keeps the top-k.
+ *   every prefix token and keeps the top-k.  The multi-level search (same
+ *   blog, "HISA's Approach") repeats steps 1-2 from the coarsest level of
+ *   a tree of growing units down, each level scoring only the units inside
+ *   the ones kept above it, before steps 3-4.
  *
  * The indexer score of a key x for one query row is
  *     score(q, x) = sum_h w_h * max(0, q_h . x)      over the H indexer heads,
@@ -239,6 +242,10 @@ typedef struct {
     /* tree: branching factor, superblocks kept, outputs */
     int bf, W;
     int32_t* sblocks; int32_t* nsblocks;
+    /* search of any depth: levels finest first (level 0 = blocks of B) */
+    int n_lv;
+    const int* lv_B; const int* lv_W;
+    int32_t* lv_kept; int32_t* lv_nkept; int lv_ld; int maxW; long lv_items;
 } job_t;
 
 static long row_position(const job_t* J, int i, int* b_out) {
@@ -430,6 +437,88 @@ static void tree_row(void* ctx, int i, void* scratch) {
     refine_blocks(J, i, b, t, q, w, chosen, n_chosen, items, x, idx, val, NULL);
 }
 
+/* Search of any depth (blog "Hierarchical Indexing Makes Sparse Attention
+ * Actually Fast", "HISA's Approach" and "The Complexity Win": the summary is
+ * a tree searched from the root down, the best branches kept at each level).
+ * Level l groups the keys into units of lv_B[l] tokens (lv_B[0] = B, each
+ * size a multiple of the one below), pooled from the keys like blocks.  From
+ * the coarsest level down: the candidates are every visible unit (coarsest
+ * level) or the visible units inside the units kept one level up; the own
+ * unit, the one holding the query position, is kept without being compared,
+ * together with the best lv_W[l] - 1 candidates by (score desc, id asc).
+ * The tokens of the kept level-0 blocks are then refined as in the
+ * two-stage search.  counts[l] is the units of level l scored (candidates
+ * plus the own unit), counts[n_lv] the token slots scored. */
+static void levels_row(void* ctx, int i, void* scratch) {
+    job_t* J = (job_t*)ctx;
+    int H = J->H, d = J->c.d, b;
+    long t = row_position(J, i, &b);
+    int32_t* idx = J->idx + (size_t)i * J->k;
+    double* val = J->score ? J->score + (size_t)i * J->k : NULL;
+    if (t < 0) {
+        J->bad = 1;
+        for (int r = 0; r < J->k; ++r) { idx[r] = -1; if (val) val[r] = NAN; }
+        return;
+    }
+    double* q = (double*)scratch;
+    double* w = q + (size_t)H * d;
+    double* mu = w + H;
+    double* x = mu + d;
+    scored_t* items = (scored_t*)(x + d);
+    int32_t* cur = (int32_t*)(items + J->lv_items);
+    int32_t* up = cur + J->maxW;                   /* the kept units one level up */
+    load_query(J, i, q, w);
+    long n_t = t + 1;
+    int n_up = 0;
+    for (int l = J->n_lv - 1; l >= 0; --l) {
+        long Bl = J->lv_B[l];
+        long nu = (n_t + Bl - 1) / Bl;             /* visible units; the own one is nu - 1 */
+        long nc = 0;
+        if (l == J->n_lv - 1) {
+            for (long j = 0; j < nu - 1; ++j) {
+                pool_block(&J->c, b, (int)Bl, j, n_t, mu, x, J->pool_mode);
+                items[nc].v = indexer_score(q, w, H, d, mu);
+                items[nc].i = j;
+                ++nc;
+            }
+        } else {
+            long bf = J->lv_B[l + 1] / Bl;         /* units of this level per unit above */
+            for (int r = 0; r < n_up; ++r)
+                for (long j = (long)up[r] * bf; j < (long)(up[r] + 1) * bf && j < nu - 1; ++j) {
+                    pool_block(&J->c, b, (int)Bl, j, n_t, mu, x, J->pool_mode);
+                    items[nc].v = indexer_score(q, w, H, d, mu);
+                    items[nc].i = j;
+                    ++nc;
+                }
+        }
+        int W = J->lv_W[l], n_keep;
+        if (nc + 1 <= W) {
+            n_keep = (int)nc + 1;
+            for (long r = 0; r < nc; ++r) cur[r] = (int32_t)items[r].i;
+        } else {
+            qsort(items, (size_t)nc, sizeof(scored_t), by_value_then_index);
+            n_keep = W;
+            for (int r = 0; r < W - 1; ++r) cur[r] = (int32_t)items[r].i;
+        }
+        cur[n_keep - 1] = (int32_t)(nu - 1);
+        for (int a = 1; a < n_keep; ++a)
+            for (int c2 = a; c2 > 0 && cur[c2 - 1] > cur[c2]; --c2) {
+                int32_t tmp = cur[c2]; cur[c2] = cur[c2 - 1]; cur[c2 - 1] = tmp;
+            }
+        if (J->lv_kept) {
+            int32_t* o = J->lv_kept + (size_t)i * J->lv_ld;
+            for (int j = 0; j < l; ++j) o += J->lv_W[j];
+            for (int r = 0; r < W; ++r) o[r] = r < n_keep ? cur[r] : -1;
+        }
+        if (J->lv_nkept) J->lv_nkept[(size_t)i * J->n_lv + l] = n_keep;
+        if (J->counts) J->counts[(size_t)i * (J->n_lv + 1) + l] = nc + 1;
+        int32_t* tmp = up; up = cur; cur = tmp;
+        n_up = n_keep;
+    }
+    if (J->counts) J->counts[(size_t)i * (J->n_lv + 1) + J->n_lv] = (int64_t)n_up * J->B;
+    refine_blocks(J, i, b, t, q, w, up, n_up, items, x, idx, val, NULL);
+}
+
 static void refine_row(void* ctx, int i, void* scratch) {
     job_t* J = (job_t*)ctx;
     int H = J->H, d = J->c.d, b;
@@ -552,6 +641,39 @@ int hisa_oracle_tree_select(const void* keys, const float* scale, int dtype, int
     J.blocks = blocks; J.nblocks = nblocks; J.counts = counts;
     long items = J.nbmax > (long)m * B ? J.nbmax : (long)m * B;
     int rc = for_rows(tree_row, &J, n_q, n_threads, row_scratch_bytes(H, d, items));
+    return rc ? rc : (J.bad ? 2 : 0);
+}
+
+int hisa_oracle_levels_select(const void* keys, const float* scale, int dtype, int batch, int cap,
+                              int d, int n_levels, const int* level_B, const int* keep,
+                              int pool_mode, const int32_t* lens, const uint16_t* Q, const float* w,
+                              const int32_t* q_seq, const int32_t* q_pos, int n_q, int H, int k,
+                              int n_threads, int32_t* idx, double* score, int32_t* kept,
+                              int32_t* nkept, int64_t* counts) {
+    if (check_cache(keys, scale, dtype, batch, cap, d) || n_levels < 1 || n_levels > 8 || !level_B ||
+        !keep || !lens || !Q || !w || !q_seq || n_q < 0 || H < 1 || k < 1 || !idx ||
+        (pool_mode != POOL_MEAN && pool_mode != POOL_MAX))
+        return 1;
+    int ld = 0, maxW = 0;
+    for (int l = 0; l < n_levels; ++l) {
+        if (level_B[l] < 1 || keep[l] < 1 || keep[l] > (1 << 20)) return 1;
+        if (l > 0 && level_B[l] % level_B[l - 1] != 0) return 1;
+        ld += keep[l];
+        if (keep[l] > maxW) maxW = keep[l];
+    }
+    job_t J;
+    memset(&J, 0, sizeof J);
+    J.c = (cache_t){keys, scale, dtype, batch, cap, d};
+    J.pool_mode = pool_mode;
+    J.B = level_B[0]; J.lens = lens; J.Q = Q; J.w = w; J.q_seq = q_seq; J.q_pos = q_pos;
+    J.n_q = n_q; J.H = H; J.m = keep[0]; J.k = k; J.nbmax = (cap + J.B - 1) / J.B;
+    J.idx = idx; J.score = score; J.counts = counts;
+    J.n_lv = n_levels; J.lv_B = level_B; J.lv_W = keep;
+    J.lv_kept = kept; J.lv_nkept = nkept; J.lv_ld = ld; J.maxW = maxW;
+    /* candidates at any level are at most the level-0 blocks; the tokens at most m * B */
+    J.lv_items = J.nbmax > (long)keep[0] * J.B ? J.nbmax : (long)keep[0] * J.B;
+    size_t bytes = row_scratch_bytes(H, d, J.lv_items) + 2 * sizeof(int32_t) * (size_t)maxW;
+    int rc = for_rows(levels_row, &J, n_q, n_threads, bytes);
     return rc ? rc : (J.bad ? 2 : 0);
 }
 

@@ -149,3 +149,42 @@ def tree_row(keys, key_scale, dtype, Q, w, b, t, i, B, bf, W, m, k, pool="mean")
     val = {s: v for v, s in toks}
     return dict(idx=kept, scores=[val[s] for s in kept], sblocks=skept, blocks=sorted(chosen),
                 counts=(ns, len(cand) + 1, len(chosen) * B))
+
+
+def levels_row(keys, key_scale, dtype, Q, w, b, t, i, level_B, keep, k, pool="mean"):
+    """Search of any depth by definition: level l (finest first) has units of
+    level_B[l] tokens; from the coarsest level down, keep the own unit plus
+    the best keep[l] - 1 candidates, the candidates being every visible unit
+    at the top and the visible units inside the kept units one level up
+    below it; then the top k tokens of the kept blocks."""
+    q, ww = query_values(Q, w, i)
+    n = t + 1
+    rep = block_max if pool == "max" else block_mean
+    nl = len(level_B)
+    kept, counts = [None] * nl, [0] * (nl + 1)
+    up = None
+    for lv in range(nl - 1, -1, -1):
+        U = level_B[lv]
+        nu = -(-n // U)
+        if up is None:
+            cand = list(range(nu - 1))
+        else:
+            bf = level_B[lv + 1] // U
+            cand = [j for p in up for j in range(p * bf, min((p + 1) * bf, nu - 1))]
+        S = {j: score(q, ww, rep(keys, key_scale, dtype, b, U, j, n)) for j in cand}
+        if len(cand) + 1 <= keep[lv]:
+            chosen = sorted(cand) + [nu - 1]
+        else:
+            chosen = keep_by_definition([(S[j], j) for j in cand], keep[lv] - 1) + [nu - 1]
+        kept[lv] = sorted(chosen)
+        counts[lv] = len(cand) + 1
+        up = kept[lv]
+    B = level_B[0]
+    toks = []
+    for j in up:
+        for s in range(j * B, min((j + 1) * B, n)):
+            toks.append((score(q, ww, key_values(keys, key_scale, dtype, b, s)), s))
+    counts[nl] = len(up) * B
+    sel = keep_by_definition(toks, k)
+    val = {s: v for v, s in toks}
+    return dict(idx=sel, scores=[val[s] for s in sel], kept=kept, counts=tuple(counts))

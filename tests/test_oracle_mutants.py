@@ -34,6 +34,12 @@ MUTANTS = {
                                        "skept[J->W - 1] = (int32_t)items[J->W - 1].i;"),
     "tree_children_skip_last": ("j < (long)(skept[r] + 1) * bf && j < nb - 1; ++j",
                                 "j < (long)(skept[r] + 1) * bf - 1 && j < nb - 1; ++j"),
+    "levels_own_unit_not_forced": ("cur[n_keep - 1] = (int32_t)(nu - 1);",
+                                   "cur[n_keep - 1] = (int32_t)(nu - 2 > 0 ? nu - 2 : 0);"),
+    "levels_children_skip_last": ("j < (long)(up[r] + 1) * bf && j < nu - 1; ++j",
+                                  "j < (long)(up[r] + 1) * bf - 1 && j < nu - 1; ++j"),
+    "levels_counts_miss_own_unit": ("J->counts[(size_t)i * (J->n_lv + 1) + l] = nc + 1;",
+                                    "J->counts[(size_t)i * (J->n_lv + 1) + l] = nc;"),
     "refine_cand_layout_transposed": ("if (cand) cand[(size_t)r * J->B + o] = v;",
                                       "if (cand) cand[(size_t)o * J->mm + r] = v;"),
     "refine_skips_last_given_block": ("for (int r = 0; r < nblk; ++r) {",
@@ -144,6 +150,19 @@ def _detects(lib) -> bool:
         if list(r["blocks"][i][:r["nblocks"][i]]) != ref["blocks"] or \
                 [x for x in r["idx"][i] if x >= 0] != ref["idx"]:
             return True
+    # the search of any depth against its brute force (kept units, counts, tokens)
+    c = make_case(batch=1, L=50, H=2, d=4, B=2, m=3, k=6, seed=314, positions=np.array([49, 31, 8]))
+    cache = oracle.Cache.of(c)
+    level_B, keep = [2, 4, 12], [3, 2, 2]
+    r = oracle.levels_select(cache, c.Q, c.w, c.q_seq, c.q_pos, level_B, keep, 6, threads=1, lib=lib)
+    for i in range(c.n_q):
+        ref = brute.levels_row(c.keys, c.key_scale, c.dtype, c.Q, c.w, int(c.q_seq[i]),
+                               int(c.q_pos[i]), i, level_B, keep, 6)
+        if [x for x in r["idx"][i] if x >= 0] != ref["idx"] or tuple(r["counts"][i]) != ref["counts"]:
+            return True
+        for lv in range(3):
+            if list(r["kept"][lv][i][:r["nkept"][i, lv]]) != ref["kept"][lv]:
+                return True
     return False
 
 
