@@ -39,7 +39,8 @@ HISA_DEV_BAD_QUERY, HISA_DEV_CAPACITY, HISA_DEV_BAD_LEN, HISA_DEV_TIMEOUT = 0x1,
 EXPORTS = ("hisa_pool_blocks", "hisa_append", "hisa_select_workspace_bytes", "hisa_select",
            "hisa_decode_step_workspace_bytes", "hisa_decode_step",
            "hisa_select_inspect", "hisa_select_static", "hisa_tree_workspace_bytes",
-           "hisa_tree_select", "hisa_pool_tail", "hisa_cp_workspace_bytes", "hisa_cp_blocks",
+           "hisa_tree_select", "hisa_pool_tail", "hisa_levels_workspace_bytes", "hisa_levels_select",
+           "hisa_cp_workspace_bytes", "hisa_cp_blocks",
            "hisa_cp_tokens", "hisa_merge_topk", "hisa_sparse_attn_workspace_bytes", "hisa_sparse_attn",
            "dsa_flat_workspace_bytes", "dsa_flat_select", "hisa_topk_f32",
            "hisa_profile_enable", "hisa_profile_read", "hisa_status_string", "hisa_last_cuda_error",
@@ -74,6 +75,10 @@ _lib.hisa_tree_workspace_bytes.restype = _Z
 _lib.hisa_tree_select.argtypes = [_KVP, _KVP, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P,
                                   _P, _P, _P, _Z, _P]
 _lib.hisa_pool_tail.argtypes = [_KVP, _P]
+_lib.hisa_levels_workspace_bytes.argtypes = [_P, _I, _P, _I, _I, _I]
+_lib.hisa_levels_workspace_bytes.restype = _Z
+_lib.hisa_levels_select.argtypes = [_P, _I, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _Z,
+                                    _P]
 _lib.hisa_cp_workspace_bytes.argtypes = [_KVP, ctypes.c_int32, _I, _I, _I, _I]
 _lib.hisa_cp_workspace_bytes.restype = _Z
 _lib.hisa_cp_blocks.argtypes = [_KVP, ctypes.c_int32, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _Z, _P]
@@ -98,7 +103,8 @@ _lib.hisa_last_cuda_error.argtypes = []
 _lib.hisa_last_cuda_error.restype = ctypes.c_char_p
 for _f in ("hisa_pool_blocks", "hisa_append", "hisa_select", "hisa_decode_step", "hisa_select_inspect",
            "hisa_select_static",
-           "hisa_tree_select", "hisa_pool_tail", "hisa_cp_blocks", "hisa_cp_tokens", "hisa_merge_topk",
+           "hisa_tree_select", "hisa_pool_tail", "hisa_levels_select", "hisa_cp_blocks", "hisa_cp_tokens",
+           "hisa_merge_topk",
            "hisa_sparse_attn", "dsa_flat_select", "hisa_topk_f32", "hisa_profile_enable", "hisa_profile_read"):
     getattr(_lib, _f).restype = _I
 
@@ -436,6 +442,58 @@ def hisa_tree_select(kv: KVCache, kv2: KVCache, Q, w, q_seq, q_pos, W: int, m: i
     if inspect:
         out["idx"] = idx
         return out
+    return idx
+
+
+def _levels_args(kvs, keep):
+    """Host arrays of the level indexes and kept counts (kept alive by the caller)."""
+    n = len(kvs)
+    if n != len(keep):
+        raise ValueError("hisa_levels_select: one keep count per level")
+    arr = (_KVP * n)(*[ctypes.pointer(kv._struct) for kv in kvs])
+    kp = (ctypes.c_int * n)(*[int(x) for x in keep])
+    return n, arr, kp
+
+
+def hisa_levels_workspace_bytes(kvs, keep, n_q: int, H: int, k: int) -> int:
+    n, arr, kp = _levels_args(kvs, keep)
+    return int(_lib.hisa_levels_workspace_bytes(ctypes.cast(arr, _P), n, ctypes.cast(kp, _P), n_q, H, k))
+
+
+def hisa_levels_select(kvs, Q, w, q_seq, q_pos, keep, k: int, inspect: bool = False,
+                       ws: Optional[torch.Tensor] = None, idx: Optional[torch.Tensor] = None,
+                       stream=None):
+    """Search of any depth.  kvs: indexes over the same keys, finest first
+    (kvs[0] the block index, each unit size a multiple of the one below, the
+    coarser ones made by superblock_index); keep[l]: units kept at level l.
+    Returns idx [n_q, k], or with inspect=True a dict with scores, the kept
+    units of every level (kept[l], nkept[l]) and the per-row work counters."""
+    kv = kvs[0]
+    Q, w, q_seq, q_pos = _queries(kv, Q, w, q_seq, q_pos)
+    n_q, H = Q.shape[0], Q.shape[1]
+    dev = kv.keys.device
+    _check_out("hisa_levels_select", kv, n_q, k, idx, None)
+    _check_ws("hisa_levels_select", kv, ws)
+    n, arr, kp = _levels_args(kvs, keep)
+    ws = workspace(hisa_levels_workspace_bytes(kvs, keep, n_q, H, k), dev) if ws is None else ws
+    idx = torch.empty((n_q, k), dtype=torch.int32, device=dev) if idx is None else idx
+    scores = kept = nkept = counts = None
+    kept_p = nkept_p = None
+    if inspect:
+        scores = torch.empty((n_q, k), dtype=torch.float32, device=dev)
+        kept = [torch.empty((n_q, min(int(keep[l]), kvs[l].nblk)), dtype=torch.int32, device=dev)
+                for l in range(n)]
+        nkept = [torch.empty(n_q, dtype=torch.int32, device=dev) for _ in range(n)]
+        counts = torch.empty((n_q, n + 1), dtype=torch.int64, device=dev)
+        kept_p = (_P * n)(*[t.data_ptr() for t in kept])
+        nkept_p = (_P * n)(*[t.data_ptr() for t in nkept])
+    _check("hisa_levels_select", _lib.hisa_levels_select(
+        ctypes.cast(arr, _P), n, ctypes.cast(kp, _P), _ptr(Q), _ptr(w), _ptr(q_seq), _ptr(q_pos), n_q,
+        H, k, _ptr(idx), _ptr(scores), ctypes.cast(kept_p, _P) if kept_p else None,
+        ctypes.cast(nkept_p, _P) if nkept_p else None, _ptr(counts), _ptr(ws), ws.numel(),
+        _stream(stream)))
+    if inspect:
+        return dict(idx=idx, scores=scores, kept=kept, nkept=nkept, counts=counts)
     return idx
 
 

@@ -621,6 +621,55 @@ int check_tree(const hisa_kv* kv, const hisa_kv* kv2, KvView* v, KvView* v2) {
     return HISA_OK;
 }
 
+// Search of any depth: level 0 (the block index) uses hisa_select's layout,
+// each coarser level l a score-key row, a kept list, its lengths and a plan.
+struct LevelsWs {
+    HisaWs L;
+    size_t bkeys[HISA_MAX_LEVELS], kept[HISA_MAX_LEVELS], nkept[HISA_MAX_LEVELS], plan[HISA_MAX_LEVELS];
+    int ldb[HISA_MAX_LEVELS], mm[HISA_MAX_LEVELS];
+    size_t total;
+};
+
+LevelsWs levels_ws(const KvView* v, int n, const int* keep, int n_q, int H) {
+    LevelsWs T;
+    std::memset(&T, 0, sizeof T);
+    T.L = hisa_ws(v[0], n_q, H, keep[0]);
+    T.mm[0] = T.L.mm;
+    T.ldb[0] = T.L.ldb;
+    Carve c;
+    c.off = T.L.total;
+    for (int l = 1; l < n; ++l) {
+        T.mm[l] = keep[l] < v[l].nblk ? keep[l] : v[l].nblk;
+        T.ldb[l] = static_cast<int>(round_up(v[l].nblk, 128));
+        T.bkeys[l] = c.take(static_cast<size_t>(n_q) * T.ldb[l] * 4);
+        T.kept[l] = c.take(static_cast<size_t>(n_q) * T.mm[l] * 4);
+        T.nkept[l] = c.take(static_cast<size_t>(n_q) * 4);
+        T.plan[l] = c.take(static_cast<size_t>(n_q) * 16);
+    }
+    T.total = c.off;
+    return T;
+}
+
+// Every level indexes kv[0]'s keys; each unit size is a multiple of the one
+// below; a level that parents another holds at most kParentBits units.
+int check_levels(const hisa_kv* const* kv, int n, const int* keep, KvView* v) {
+    if (!kv || !keep || n < 1 || n > HISA_MAX_LEVELS) return HISA_E_INVAL;
+    for (int l = 0; l < n; ++l) {
+        if (!kv[l] || keep[l] < 1) return HISA_E_INVAL;
+        int rc = check_kv(kv[l], &v[l]);
+        if (rc) return rc;
+        if (l == 0) continue;
+        const hisa_kv* a = kv[0];
+        const hisa_kv* b = kv[l];
+        if (b->keys != a->keys || b->key_scale != a->key_scale || b->len != a->len ||
+            b->batch != a->batch || b->cap != a->cap || b->d != a->d || b->dtype != a->dtype ||
+            b->pool != a->pool || b->B % kv[l - 1]->B != 0)
+            return HISA_E_INVAL;
+        if (v[l].nblk > kParentBits) return HISA_E_UNSUPPORTED;
+    }
+    return HISA_OK;
+}
+
 // Scratch of hisa_select_static: a file-scope device array, one per device
 // (the runtime gives every device's context its own copy when it loads this
 // module).  Its address is looked up once per device context and cached with
@@ -909,6 +958,68 @@ int hisa_tree_select(const hisa_kv* kv, const hisa_kv* kv2, const uint16_t* Q, c
     rc = block_stage(l1, Q, w, q_seq, q_pos, n_q, H, k, counts, 3, s);
     if (rc) return rc;
     return token_stage(v, T.L, base, Q, w, q_seq, q_pos, n_q, H, k, idx, scores, counts, 3, 1, 0, s);
+}
+
+size_t hisa_levels_workspace_bytes(const hisa_kv* const* kv, int n_levels, const int* keep, int n_q,
+                                   int H, int k) {
+    (void)k;
+    KvView v[HISA_MAX_LEVELS];
+    if (check_levels(kv, n_levels, keep, v) || n_q < 0 || H < 1 || H > 128) return 0;
+    return levels_ws(v, n_levels, keep, n_q, H).total;
+}
+
+int hisa_levels_select(const hisa_kv* const* kv, int n_levels, const int* keep, const uint16_t* Q,
+                       const float* w, const int32_t* q_seq, const int32_t* q_pos, int n_q, int H, int k,
+                       int32_t* idx, float* scores, int32_t* const* kept, int32_t* const* nkept,
+                       uint64_t* counts, void* ws, size_t ws_bytes, hisa_stream_t stream) {
+    KvView v[HISA_MAX_LEVELS];
+    int rc = check_levels(kv, n_levels, keep, v);
+    if (rc) return rc;
+    if (!select_block_size_ok(v[0].B)) return HISA_E_UNSUPPORTED;
+    rc = check_queries(Q, w, q_seq, n_q, H, k, idx);
+    if (rc) return rc;
+    if (n_q == 0) return HISA_OK;
+    const LevelsWs T = levels_ws(v, n_levels, keep, n_q, H);
+    if (!ws || !aligned(ws, 256) || ws_bytes < T.total) return HISA_E_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    const int cld = n_levels + 1;   // counts: units scored per level, then token slots
+    if (counts && cudaMemsetAsync(counts, 0, sizeof(uint64_t) * cld * n_q, s) != cudaSuccess)
+        return HISA_E_CUDA;
+    // from the coarsest level down: the own unit plus the best keep[l] - 1
+    // candidates, the candidates below the top being the children of the
+    // units kept one level up (gathered where gathered_level allows)
+    const int32_t* parent = nullptr;
+    const int32_t* parent_n = nullptr;
+    int parent_ld = 0;
+    for (int l = n_levels - 1; l >= 0; --l) {
+        BlockLevel lv;
+        std::memset(&lv, 0, sizeof lv);
+        lv.v = &v[l];
+        lv.m = keep[l];
+        lv.mm = T.mm[l];
+        lv.ldb = T.ldb[l];
+        lv.bkeys = reinterpret_cast<uint32_t*>(base + (l ? T.bkeys[l] : T.L.bkeys));
+        lv.blocks = reinterpret_cast<int32_t*>(base + (l ? T.kept[l] : T.L.blocks));
+        lv.nblocks = reinterpret_cast<int32_t*>(base + (l ? T.nkept[l] : T.L.nblocks));
+        lv.plan = reinterpret_cast<int4*>(base + (l ? T.plan[l] : T.L.plan));
+        lv.blocks_out = kept ? kept[l] : nullptr;
+        lv.nblocks_out = nkept ? nkept[l] : nullptr;
+        lv.counts_col = l;
+        if (parent) {
+            lv.parent = parent;
+            lv.parent_ld = parent_ld;
+            lv.bf = v[l + 1].B / v[l].B;
+            if (gathered_level(lv.bf, parent_ld, v[l].nblk, n_q)) lv.parent_n = parent_n;
+        }
+        rc = block_stage(lv, Q, w, q_seq, q_pos, n_q, H, k, counts, cld, s);
+        if (rc) return rc;
+        parent = lv.blocks;
+        parent_n = lv.nblocks;
+        parent_ld = lv.mm;
+    }
+    return token_stage(v[0], T.L, base, Q, w, q_seq, q_pos, n_q, H, k, idx, scores, counts, cld,
+                       n_levels - 1, 0, s);
 }
 
 // ---------------------------------------------------- context parallelism

@@ -266,6 +266,56 @@ int hisa_tree_select(const hisa_kv* kv, const hisa_kv* kv2, const uint16_t* Q, c
 int hisa_pool_tail(const hisa_kv* kv, hisa_stream_t stream);
 
 /*
+ * hisa_levels_select — search of any depth: n_levels levels of blocks, then
+ * tokens.  Blog "Hierarchical Indexing Makes Sparse Attention Actually
+ * Fast", "HISA's Approach" and "The Complexity Win": the cache summarised as
+ * a tree, searched from the root down with the best branches kept at every
+ * level, so that the summaries a query scores grow with the depth of the
+ * tree rather than with L/B.
+ *   kv      [n_levels] host array of indexes over the same keys (keys,
+ *           key_scale, len, batch, cap, d, dtype and pool equal to kv[0]'s),
+ *           finest first: kv[0] is the block index (its B is the token
+ *           block size, as hisa_select), kv[l]->B a multiple of kv[l-1]->B;
+ *           each built by hisa_pool_blocks and, after hisa_append on kv[0],
+ *           kept current by hisa_pool_tail(kv[l]); kv[l] for l >= 1 may hold
+ *           up to 32768 units per sequence (HISA_E_UNSUPPORTED beyond)
+ *   n_levels 1 .. HISA_MAX_LEVELS (1: hisa_select_inspect's result)
+ *   keep    [n_levels] host array, each >= 1: units kept per row at level l,
+ *           the own unit (the one holding the query position) plus the best
+ *           keep[l] - 1 candidates by (score desc, id asc); keep[0] is m
+ *   The candidates are every visible unit at the top level and, below it,
+ *   the visible units inside the units kept one level up (the own unit
+ *   apart).  A level reads and scores only those children when
+ *   hisa_tree_select's gathered conditions hold for it (branching factor a
+ *   power of two from 8 to 128, the kept units above times it at most 512
+ *   and at most a quarter of the level's units, at most two rows per SM);
+ *   otherwise it scores every visible unit and masks the others, with the
+ *   same results.
+ *   k, idx, scores  as hisa_select
+ *   kept    NULL, or a host array of n_levels device pointers, each NULL or
+ *           [n_q, min(keep[l], units of kv[l])] out: the kept units ascending,
+ *           -1 padded
+ *   nkept   NULL, or a host array of n_levels device pointers, each NULL or
+ *           [n_q] out: the units kept at level l
+ *   counts  [n_q, n_levels + 1] out (or NULL), zeroed by the call: the units
+ *           of each level scored (candidates plus the own unit), then the
+ *           token slots scored
+ * Two levels give hisa_tree_select's result (with its counts columns in
+ * the other order).  Errors: HISA_E_INVAL for a level that does not match
+ * kv[0] or a unit size that is not a multiple of the one below;
+ * HISA_E_WORKSPACE for ws smaller than hisa_levels_workspace_bytes (0 for
+ * invalid arguments); the other codes as hisa_select.
+ */
+#define HISA_MAX_LEVELS 8
+size_t hisa_levels_workspace_bytes(const hisa_kv* const* kv, int n_levels, const int* keep, int n_q,
+                                   int H, int k);
+int hisa_levels_select(const hisa_kv* const* kv, int n_levels, const int* keep, const uint16_t* Q,
+                       const float* w, const int32_t* q_seq, const int32_t* q_pos, int n_q, int H,
+                       int k, int32_t* idx, float* scores, int32_t* const* kept,
+                       int32_t* const* nkept, uint64_t* counts, void* ws, size_t ws_bytes,
+                       hisa_stream_t stream);
+
+/*
  * Context parallelism: one sequence longer than a GPU holds, split by token
  * range over R ranks.  The pages motivate contexts of 64K to 1M tokens and
  * beyond (blog "What This Means for Long-Context Inference"; gptget.net

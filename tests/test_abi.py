@@ -249,3 +249,46 @@ def test_decode_step_checks_before_any_launch(hisa):
     assert step(ws_bytes=16) == hisa.HISA_E_WORKSPACE
     need = lib.hisa_decode_step_workspace_bytes(ctypes.byref(kv), 64, 64, 2048)
     assert need == lib.hisa_select_workspace_bytes(ctypes.byref(kv), kv.batch, 64, 64, 2048) > 0
+
+
+def test_levels_entry_checks_and_workspace(hisa):
+    """hisa_levels_select refuses malformed level lists on the host, and its
+    workspace is hisa_select's for one level and hisa_tree_select's for two."""
+    lib = hisa.lib()
+    P = ctypes.c_void_p
+    KVP = ctypes.POINTER(hisa.hisa_kv)
+    base = dict(cap=32768, B=128)
+    kv0 = _kv(hisa, **base)
+    kv1 = _kv(hisa, **dict(base, B=1024))
+    kv2 = _kv(hisa, **dict(base, B=8192))
+
+    def arrays(kvs, keep):
+        arr = (KVP * len(kvs))(*[ctypes.pointer(k) for k in kvs])
+        return arr, (ctypes.c_int * len(keep))(*keep)
+
+    def sel(kvs, keep, n=None, n_q=4, ws=P(256), ws_bytes=1 << 30):
+        arr, kp = arrays(kvs, keep)
+        return lib.hisa_levels_select(ctypes.cast(arr, P), len(kvs) if n is None else n,
+                                      ctypes.cast(kp, P), P(16), P(16), P(16), None, n_q, 64, 16,
+                                      P(16), None, None, None, None, ws, ws_bytes, None)
+
+    def wsb(kvs, keep, n_q=64):
+        arr, kp = arrays(kvs, keep)
+        return lib.hisa_levels_workspace_bytes(ctypes.cast(arr, P), len(kvs), ctypes.cast(kp, P),
+                                               n_q, 64, 2048)
+
+    assert sel([kv0, kv1], [8, 4], n=0) == hisa.HISA_E_INVAL
+    assert sel([kv0] * 9, [8] * 9) == hisa.HISA_E_INVAL                      # above HISA_MAX_LEVELS
+    assert sel([kv0, kv1], [8, 0]) == hisa.HISA_E_INVAL                      # nothing kept
+    assert sel([kv0, _kv(hisa, **dict(base, B=1000))], [8, 4]) == hisa.HISA_E_INVAL   # not a multiple
+    assert sel([kv0, _kv(hisa, **dict(base, B=1024, keys=32))], [8, 4]) == hisa.HISA_E_INVAL
+    assert sel([kv0, kv1, _kv(hisa, **dict(base, B=512))], [8, 4, 2]) == hisa.HISA_E_INVAL
+    big = dict(cap=1 << 22, B=16)
+    assert sel([_kv(hisa, **big), _kv(hisa, **dict(big, B=64))], [8, 4]) == hisa.HISA_E_UNSUPPORTED
+    assert sel([kv0, kv1, kv2], [8, 4, 2], ws_bytes=16) == hisa.HISA_E_WORKSPACE
+    assert sel([kv0, kv1, kv2], [8, 4, 2], n_q=0) == hisa.HISA_OK
+    assert wsb([kv0], [64]) == lib.hisa_select_workspace_bytes(ctypes.byref(kv0), 64, 64, 64, 2048)
+    assert wsb([kv0, kv1], [64, 8]) == lib.hisa_tree_workspace_bytes(
+        ctypes.byref(kv0), ctypes.byref(kv1), 64, 64, 8, 64, 2048)
+    assert wsb([kv0, kv1, kv2], [64, 8, 2]) > wsb([kv0, kv1], [64, 8])
+    assert wsb([kv0, kv1], [64, 0]) == 0
