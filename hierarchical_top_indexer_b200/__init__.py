@@ -10,6 +10,12 @@ PyTorch fallback: if the library is missing, importing this package fails.
     kv.load(keys_bf16, lens)             # host or device tensors
     hisa.hisa_pool_blocks(kv)
     idx = hisa.hisa_select(kv, Q, w, q_seq, q_pos, m=64, k=2048)
+
+    # a deeper search: coarser indexes over the same keys, finest first
+    kvs = [kv] + [hisa.superblock_index(kv, f) for f in (8, 64)]
+    for c in kvs[1:]:
+        hisa.hisa_pool_blocks(c)
+    idx = hisa.hisa_levels_select(kvs, Q, w, q_seq, q_pos, keep=[64, 32, 8], k=2048)
 """
 from __future__ import annotations
 
