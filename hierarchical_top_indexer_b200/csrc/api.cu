@@ -54,7 +54,7 @@ bool make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, size_t
 // boxes of [1, 128, 64]: a box that runs past a sequence's nblk rows is
 // zero-filled there instead of reading the next sequence's rows.
 // boxes of `rows` representatives (128: a tile; bf: the children of one
-// superblock in the gathered level of the three-level search)
+// kept unit in a gathered level of the multi-level search)
 bool pooled_map(CUtensorMap* map, const KvView& v, int rows = 128) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
@@ -361,8 +361,8 @@ int prep_f8(const KvView& v, const uint16_t* Q, const float* w, int n_q, int H, 
     return HISA_OK;
 }
 
-// One block level: score the level's representatives (under the kept parent
-// superblocks, if any) and keep each row's own block plus the best m - 1
+// One block level: score the level's representatives (under the units kept
+// one level up, if any) and keep each row's own block plus the best m - 1
 // others into blocks [n_q, mm] / nblocks / plan.
 struct BlockLevel {
     const KvView* v;
@@ -741,8 +741,8 @@ int check_cp(const hisa_kv* kv, int32_t tok_off, KvView* v) {
     return HISA_OK;
 }
 
-// The level under the kept superblocks loads and scores only their children
-// when that is at most a quarter of the blocks (otherwise scoring every block
+// A level under kept units loads and scores only their children when that
+// is at most a quarter of its blocks (otherwise scoring every block
 // over all SMs and masking the others is as fast), a row's children fit one
 // fused CTA (at most kFuseMaxBlocks), runs of bf children start on whole
 // swizzle atoms (bf a power of two from 8 to 128) and there are at most two

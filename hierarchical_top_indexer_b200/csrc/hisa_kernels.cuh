@@ -45,9 +45,10 @@ struct ScoreParams {
     const int32_t* blocks;
     const int4* plan_in;
     int mm;
-    // kScoreBlocks under a kept-superblock list (three-level search): block
-    // c of a row is a candidate only if superblock c / bf is in the row's
-    // parent[row, 0 .. parent_ld) (-1 padded); null: every block is
+    // kScoreBlocks under the units kept one level up (multi-level search):
+    // block c of a row is a candidate only if unit c / bf of the level above
+    // (a superblock) is in the row's parent[row, 0 .. parent_ld) (-1
+    // padded); null: every block is
     const int32_t* parent;
     int parent_ld, bf;
     // with parent_n (the kept superblocks per row) the kernel loads and
