@@ -64,6 +64,11 @@ def _bad_calls(h, case, device):
                                         want_scores=True), big2))
     calls.append(("dsa_flat_select with a short idx",
                   lambda: h.dsa_flat_select(kv, Q, w, qs, qp, k, idx=short_idx), big))
+    calls.append(("hisa_levels_select with a short idx",
+                  lambda: h.hisa_levels_select([kv], Q, w, qs, qp, [m], k, idx=short_idx), big))
+    calls.append(("hisa_levels_select with one keep count for two levels",
+                  lambda: h.hisa_levels_select([kv, h.superblock_index(kv, 4)], Q, w, qs, qp, [m], k,
+                                               idx=idx_ok), big2))
     ws_f32 = torch.zeros(1 << 20, dtype=torch.float32, device=device)
     calls.append(("workspace not bytes",
                   lambda: h.hisa_select(kv, Q, w, qs, qp, m, k, ws=ws_f32, idx=idx_ok), big2))
@@ -85,14 +90,14 @@ def test_binding_refuses_bad_buffers_cpu_tensors():
     """Host tensors: every bad case must be refused in Python (the library is
     never reached, so no device is needed)."""
     import hierarchical_top_indexer_b200 as h
-    assert _run(h, _case(), "cpu") == 12
+    assert _run(h, _case(), "cpu") == 14
 
 
 @pytest.mark.gpu
 def test_binding_refuses_bad_buffers():
     import hierarchical_top_indexer_b200 as h
     case = _case()
-    assert _run(h, case, "cuda") == 12
+    assert _run(h, case, "cuda") == 14
     torch.cuda.synchronize()
     # and the well-formed call still works on the same tensors
     kv, Q, w, qs, qp = _args(h, case, "cuda")
