@@ -468,8 +468,9 @@ def _phase_ms(hisa, fn, phase, n):
 def run_workloads(args, dev, peaks):
     """Select-only timings on the other workloads: HISA against the flat scan
     (speedup, mean IoU) at 64K prefill and 128K e4m3 decode, the three-level
-    search at 128K, a block size / pooling sweep at 32K, and the streaming
-    append + select step at 128K.  Parity on these sizes is in the GPU tests."""
+    search at 128K, a block size / pooling sweep at 32K, the streaming
+    append + select step at 128K, and searches of three and four block
+    levels at 128K.  Parity on these sizes is in the GPU tests."""
     import torch
     import hierarchical_top_indexer_b200 as hisa
     from hisa_inputs import make_config
@@ -526,6 +527,7 @@ def run_workloads(args, dev, peaks):
     r["l2"] = "flushed between calls (cache 528 MiB)"
     out[case.name] = r
     out["tree_" + case.name] = run_tree(case, dev, n, flush, stream, r["hisa_ms_per_select"])
+    deep_case, deep_two_ms = case, r["hisa_ms_per_select"]
 
     # block size / kept-block count / pooling sweep at a fixed candidate
     # budget m * B = 8192 on the 32K decode workload: quality (IoU with the
@@ -588,6 +590,12 @@ def run_workloads(args, dev, peaks):
                       "l2": "cache (32 MiB) L2-resident; no flush: each step follows the last",
                       "step": "hisa_decode_step (1 key appended, 1 row selected), replayed from a "
                               "CUDA graph per step"}
+    # searches of three and four block levels at 128K (last, so that a
+    # failure is reported in the line rather than ending the run)
+    try:
+        out["levels_" + deep_case.name] = run_levels(deep_case, dev, n, flush, stream, deep_two_ms)
+    except Exception as e:  # noqa: BLE001
+        out["levels_" + deep_case.name] = {"error": f"{type(e).__name__}: {e}"}
     return out
 
 
@@ -678,6 +686,47 @@ def run_tree(case, dev, n, flush, stream, two_level_ms):
     return {"two_level_ms_per_select": two_level_ms,
             "two_level_scores_per_row": {"blocks": nb, "tokens": min(m, nb) * case.B},
             "levels": rows, "l2": "flushed between calls"}
+
+
+def run_levels(case, dev, n, flush, stream, two_level_ms):
+    """Searches of three and four block levels (hisa_levels_select; units of
+    1024 and 8192 tokens, or 1024, 4096 and 16384, above the workload's
+    blocks) against the flat scan on one workload: select time, units and
+    token slots scored per row, and mean IoU."""
+    import torch
+    import hierarchical_top_indexer_b200 as hisa
+
+    kv = hisa.KVCache.from_case(case, device=dev)
+    hisa.hisa_pool_blocks(kv)
+    Q = torch.from_numpy(case.Q.view(np.int16)).view(torch.bfloat16).to(dev)
+    w = torch.from_numpy(case.w).to(dev)
+    qs = torch.from_numpy(case.q_seq).to(dev)
+    n_q, H, m, k = case.n_q, case.H, case.m, case.k
+    fws = hisa.workspace(hisa.dsa_flat_workspace_bytes(kv, n_q, H, k), dev)
+    fidx = hisa.dsa_flat_select(kv, Q, w, qs, None, k, ws=fws).cpu().numpy()
+    del fws
+    rows = []
+    for factors, keep in (((8, 64), (m, 32, 8)), ((8, 32, 128), (m, 32, 16, 4))):
+        kvs = [kv] + [hisa.superblock_index(kv, f) for f in factors]
+        for c in kvs[1:]:
+            hisa.hisa_pool_blocks(c)
+        ws = hisa.workspace(hisa.hisa_levels_workspace_bytes(kvs, keep, n_q, H, k), dev)
+        idx = torch.empty((n_q, k), dtype=torch.int32, device=dev)
+        counts = hisa.hisa_levels_select(kvs, Q, w, qs, None, keep, k, inspect=True)["counts"]
+        per_row = counts.double().mean(0).cpu().tolist()
+        run = lambda: hisa.hisa_levels_select(kvs, Q, w, qs, None, keep, k, ws=ws, idx=idx)
+        ms = _median_ms(run, n, flush, stream)
+        mi = float(np.mean([iou(a, b) for a, b in zip(idx.cpu().numpy(), fidx)]))
+        assert kv.status_bits() == 0, f"device status {kv.status_bits():#x}"
+        rows.append({"unit_tokens": [case.B] + [case.B * f for f in factors], "keep": list(keep),
+                     "ms_per_select": ms, "selections_per_s": n_q / (ms / 1e3),
+                     "mean_iou_vs_flat": mi,
+                     "scored_per_row": {"units_per_level": per_row[:-1], "token_slots": per_row[-1]}})
+        del kvs, ws
+        torch.cuda.empty_cache()
+    del kv
+    torch.cuda.empty_cache()
+    return {"two_level_ms_per_select": two_level_ms, "searches": rows, "l2": "flushed between calls"}
 
 
 def run_select_only(args):
