@@ -271,6 +271,7 @@ static size_t row_scratch_bytes(int H, int d, long n_items) {
 static void refine_blocks(const job_t* J, int i, int b, long t, const double* q, const double* w,
                           const int32_t* blk, int nblk, scored_t* items, double* x,
                           int32_t* idx, double* val, double* cand) {
+    (void)i;
     long n = 0;
     for (int r = 0; r < nblk; ++r) {
         for (int o = 0; o < J->B; ++o) {
